@@ -1,0 +1,86 @@
+"""Pins of the attention oracle (c7, c8).
+
+* support recovery is exact: if the kept tokens contain the entmax support,
+  the sparse output equals the full-cache output bit for bit (pages, section 3);
+* the error bound ||o - o~|| <= 2 B delta when support tokens are dropped;
+* o equals P @ V computed by a matrix product (a different summation order);
+* softmax baseline: equal scores give the mean value vector; a dominating
+  score gives that token's value;
+* two tokens at alpha = 2 follow the textbook sparsemax closed form.
+"""
+import numpy as np
+import pytest
+
+from oracle import attend
+
+
+def _data(rng, n, d, G=4):
+    q = rng.standard_normal((G, d))
+    K = rng.standard_normal((n, d))
+    V = rng.standard_normal((n, d))
+    return q, K, V
+
+
+@pytest.mark.parametrize("alpha", [1.5, 2.0])
+def test_support_recovery_is_bitwise_exact(alpha):
+    rng = np.random.default_rng(40)
+    q, K, V = _data(rng, 512, 32)
+    scale = 1.0 / np.sqrt(32)
+    o_full, tau_full, P = attend.entmax_attention(q, K, V, alpha, scale)
+    support = np.nonzero(P.sum(axis=0) > 0)[0]
+    assert 0 < support.size < 512
+    extra = rng.choice(np.setdiff1d(np.arange(512), support), 40, replace=False)
+    keep = np.sort(np.concatenate([support, extra]))
+    o_sp, tau_sp, _ = attend.entmax_attention(q, K[keep], V[keep], alpha, scale)
+    assert np.array_equal(o_sp, o_full)
+    assert np.array_equal(tau_sp, tau_full)
+    assert np.all(attend.dropped_mass(P, keep) == 0)
+    assert np.all(attend.support_recall(P, keep) == 1)
+
+
+@pytest.mark.parametrize("alpha", [1.5, 2.0])
+def test_error_bound_when_support_is_dropped(alpha):
+    rng = np.random.default_rng(41)
+    q, K, V = _data(rng, 400, 16)
+    scale = 0.25
+    o_full, _, P = attend.entmax_attention(q, K, V, alpha, scale)
+    B = np.linalg.norm(V, axis=1).max()
+    for trial in range(5):
+        keep = np.sort(rng.choice(400, 250, replace=False))
+        o_sp, _, _ = attend.entmax_attention(q, K[keep], V[keep], alpha, scale)
+        delta = attend.dropped_mass(P, keep)
+        err = np.linalg.norm(o_sp - o_full, axis=1)
+        assert np.all(err <= 2 * B * delta + 1e-12)
+
+
+def test_output_is_p_times_v():
+    rng = np.random.default_rng(42)
+    q, K, V = _data(rng, 300, 24)
+    o, _, P = attend.entmax_attention(q, K, V, 1.5, 0.3)
+    np.testing.assert_allclose(o, P @ V, rtol=1e-12, atol=1e-12)
+
+
+def test_softmax_special_cases():
+    rng = np.random.default_rng(43)
+    V = rng.standard_normal((10, 8))
+    K = np.zeros((10, 8))
+    q = rng.standard_normal((2, 8))
+    np.testing.assert_allclose(attend.softmax_attention(q, K, V, 1.0), np.tile(V.mean(0), (2, 1)),
+                               rtol=1e-13, atol=1e-13)
+    K[3] = 1e3 * q[0]
+    o = attend.softmax_attention(q[:1], K, V, 1.0)
+    np.testing.assert_allclose(o[0], V[3], atol=1e-12)
+
+
+def test_two_token_sparsemax():
+    V = np.array([[1.0, 0.0], [0.0, 1.0]])
+    for a, b in [(0.2, 0.0), (0.0, 0.9), (3.0, 0.0)]:
+        K = np.array([[a], [b]])
+        q = np.array([[1.0]])
+        o, _, _ = attend.entmax_attention(q, K, V, 2.0, 1.0)
+        p1 = min(1.0, max(0.0, (a - b + 1.0) / 2.0))
+        np.testing.assert_allclose(o[0], [p1, 1.0 - p1], atol=1e-14)
+
+
+def test_token_indices_ragged():
+    assert list(attend.token_indices([2, 0], 37, 16)) == list(range(0, 16)) + list(range(32, 37))

@@ -1,0 +1,84 @@
+"""Pins of the Gaussian tau_hat oracle (c4, c5).
+
+* closed-form page expectations g against numerical integration (scipy quad)
+  and against Monte-Carlo (10^6 draws, 4-sigma bound), and against the worked
+  examples in tests/golden;
+* with one token per page and zero spread, F is the exact entmax mass, so
+  tau_hat must equal the exact entmax threshold of c1;
+* F is strictly decreasing and F(tau_hat) = 1;
+* the z table against sqrt(2 ln n).
+"""
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+from scipy.integrate import quad
+
+from oracle import entmax, gauss
+
+GOLD = json.load(open(os.path.join(os.path.dirname(__file__), "golden", "worked_examples.json")))
+
+
+@pytest.mark.parametrize("ex", GOLD["gauss_g"], ids=lambda e: "a%g_m%g_s%g" % (e["alpha"], e["m"], e["s"]))
+def test_g_worked_examples(ex):
+    val = gauss.g(ex["m"], ex["s"], ex["tau"], ex["alpha"])
+    assert abs(float(val) - ex["g"]) < 1e-14
+
+
+@pytest.mark.parametrize("alpha", [1.5, 2.0])
+def test_g_against_quadrature(alpha):
+    r = 1.0 / (alpha - 1.0)
+    for m, s, tau in [(0.3, 0.25, 0.9), (1.8, 0.15, 1.9), (-1.0, 2.0, 0.5), (0.0, 1e-3, -0.01),
+                      (2.0, 0.5, 0.0), (0.1, 0.3, 2.5)]:
+        dens = lambda x: math.exp(-0.5 * ((x - m) / s) ** 2) / (s * math.sqrt(2 * math.pi))  # noqa: E731
+        val, err = quad(lambda x: (x - tau) ** r * dens(x), tau, max(tau, m) + 40 * s,
+                        epsabs=1e-15, epsrel=1e-12, limit=400)
+        assert abs(float(gauss.g(m, s, tau, alpha)) - val) < 1e-10 + 1e-9 * abs(val)
+
+
+@pytest.mark.parametrize("alpha", [1.5, 2.0])
+def test_g_against_monte_carlo(alpha):
+    rng = np.random.default_rng(20)
+    r = 1.0 / (alpha - 1.0)
+    for m, s, tau in [(0.5, 0.4, 0.6), (0.0, 1.0, -0.3)]:
+        x = m + s * rng.standard_normal(1_000_000)
+        y = np.maximum(x - tau, 0.0) ** r
+        se = y.std() / math.sqrt(y.size)
+        assert abs(y.mean() - float(gauss.g(m, s, tau, alpha))) < 4 * se
+
+
+@pytest.mark.parametrize("alpha", [1.5, 2.0])
+def test_point_pages_reduce_to_exact_entmax(alpha):
+    rng = np.random.default_rng(21)
+    for n in (1, 5, 64, 1000):
+        s = rng.standard_normal(n)
+        tau = gauss.tau_hat(s, np.zeros(n), np.ones(n), alpha)
+        exact = entmax.tau_sort((alpha - 1.0) * s, alpha)
+        assert abs(tau - exact) < 1e-10
+
+
+@pytest.mark.parametrize("alpha", [1.5, 2.0])
+def test_F_decreasing_and_root(alpha):
+    rng = np.random.default_rng(22)
+    P = 500
+    m = rng.standard_normal(P)
+    v = (0.5 * rng.random(P)) ** 2
+    n = rng.integers(1, 65, P)
+    t = gauss.tau_hat(m, v, n, alpha)
+    assert abs(gauss.F(t, m, v, n, alpha) - 1.0) < 1e-9
+    grid = np.linspace(t - 2, t + 2, 81)
+    vals = [gauss.F(x, m, v, n, alpha) for x in grid]
+    assert all(a > b for a, b in zip(vals, vals[1:]))
+
+
+def test_z_table():
+    for e in GOLD["z_table"]:
+        assert abs(gauss.z_table(64)[e["n"]] - e["z"]) < 1e-15
+
+
+def test_est_max_single_token_equals_mean():
+    m = np.array([[0.3, -1.2]])
+    v = np.array([[0.0, 0.0]])
+    np.testing.assert_array_equal(gauss.est_max(m, v, np.array([[1, 1]]), 64), m)
