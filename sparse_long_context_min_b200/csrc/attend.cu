@@ -1,0 +1,987 @@
+// Exact alpha-entmax attention over gathered pages, and the full-cache
+// softmax (flash-decode) baseline.
+//
+// EntmaxKV (German technical summary, section 2.C): once candidate pages are
+// chosen, only their keys and values are loaded and alpha-entmax is computed
+// over that reduced set; the result is exact when the set holds the support.
+// Section 4 compares against full-cache entmax and full-cache softmax
+// (FlashDecoding) decoding.
+//
+// The threshold tau needs every candidate score before any weight is known,
+// so entmax attention runs as three kernels on the caller's stream:
+//   K pass   (qk_*):  split-KV CTAs gather key pages through the page table
+//                     (TMA tile loads into 128-byte-swizzled shared memory,
+//                     4-stage mbarrier pipeline), score the GQA head group
+//                     with mma.sync (keys bf16, query split into a bf16 high
+//                     and low part so the product keeps ~16 mantissa bits),
+//                     and write x = (alpha-1) * scale * q.k per listed token;
+//   tau solve (tau_): one CTA per (sequence, query head) keeps the scores
+//                     above max x - 1 (no other score can be in the support)
+//                     and runs Newton steps from the left on the restricted
+//                     normalisation equation until the support is stable,
+//                     then takes the closed form on that support in float64;
+//   V pass   (pv_*):  the same splits gather value pages, turn x into
+//                     p = [x - tau]_+^(1/(alpha-1)) (split bf16 high + low) and
+//                     accumulate P.V with mma.sync in fp32; the last CTA of a
+//                     (sequence, kv head) adds the split partials in split
+//                     order (deterministic).
+// The softmax baseline does K and V in one pass with an online softmax and a
+// log-sum-exp merge of the splits.
+//
+// fp32 caches (small configurations) take plain CUDA-core kernels that follow
+// the same split structure and workspace.
+#include "common.cuh"
+#include "kernels.cuh"
+
+namespace ekv {
+
+constexpr int kStagesQK = 4;
+constexpr int kStagesPV = 4;
+constexpr int kStagesSM = 3;
+constexpr int kPsPad = 8;   // padding (bf16 elements) of a row of the P tile
+
+struct Range {
+    int start, end;
+};
+
+EKV_DEV Range split_range(int cnt, int S, int s)
+{
+    const int per = (cnt + S - 1) / S;
+    const int start = min(cnt, s * per);
+    return {start, min(cnt, start + per)};
+}
+
+
+EKV_DEV int list_count(const AttnArgs& a, int b, int g, int P)
+{
+    if (!a.sel_count) return P;
+    int c = a.sel_count[(size_t)b * a.H_kv + g];
+    if (c < 0 || c > a.k_max) {
+        report(a.status, ENTMAXKV_DEVICE_BOUNDS);
+        c = max(0, min(c, a.k_max));
+    }
+    return c;
+}
+
+// Physical page of list entry idx of (b, g), or -1 when the entry or its page
+// id is out of range (reported when `rep`).
+EKV_DEV int resolve(const AttnArgs& a, int b, int g, int idx, int P, int& lp, bool rep)
+{
+    lp = a.sel ? a.sel[((size_t)b * a.H_kv + g) * a.k_max + idx] : idx;
+    if (lp < 0 || lp >= P) {
+        if (rep) report(a.status, ENTMAXKV_DEVICE_BOUNDS);
+        return -1;
+    }
+    const int phys = a.page_table[(size_t)b * a.max_pages + lp];
+    if (phys < 0 || phys >= a.num_phys) {
+        if (rep) report(a.status, ENTMAXKV_DEVICE_BOUNDS);
+        return -1;
+    }
+    return phys;
+}
+
+EKV_DEV uint8_t* align1024(uint8_t* p)
+{
+    return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
+}
+
+// Issue the TMA loads of pipeline stage `st` (pages start + st*PPS ...) of one
+// tensor into `dst`; returns the bytes expected.  Called by one thread.
+template <int D, int PS>
+EKV_DEV uint32_t issue_stage(const AttnArgs& a, const CUtensorMap* map, uint8_t* dst, uint64_t* bar, int b,
+                             int g, Range r, int st, int P)
+{
+    constexpr int PPS = kStageTok / PS;
+    int phys[PPS];
+    uint32_t bytes = 0;
+#pragma unroll
+    for (int i = 0; i < PPS; ++i) {
+        const int idx = r.start + st * PPS + i;
+        int lp;
+        phys[i] = idx < r.end ? resolve(a, b, g, idx, P, lp, true) : -1;
+        if (phys[i] >= 0) bytes += PS * D * 2;
+    }
+    mbar_arrive_expect_tx(bar, bytes);
+#pragma unroll
+    for (int i = 0; i < PPS; ++i) {
+        if (phys[i] < 0) continue;
+        const int y = (phys[i] * a.H_kv + g) * PS;
+#pragma unroll
+        for (int h = 0; h < D / 64; ++h) tma_load_2d(dst + h * (kStageTok * 128) + i * PS * 128, map, bar, h * 64, y);
+    }
+    return bytes;
+}
+
+// Query fragments (B operand of m16n8k16, k = head dim, n = 2*head + part).
+template <int D, int NT>
+EKV_DEV void load_q_frags(const AttnArgs& a, int b, int g, float mul, uint32_t (&bq)[NT][D / 16][2])
+{
+    const int lane = threadIdx.x & 31;
+    const int n = lane >> 2, c = lane & 3;
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+        const int head = 4 * nt + (n >> 1);
+        const int part = n & 1;
+        const float* qh = a.q + ((size_t)b * a.H_q + (size_t)g * a.G + head) * D;
+#pragma unroll
+        for (int j = 0; j < D / 16; ++j) {
+            uint32_t bits[4];
+            const int ks[4] = {16 * j + 2 * c, 16 * j + 2 * c + 1, 16 * j + 2 * c + 8, 16 * j + 2 * c + 9};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const float v = head < a.G ? qh[ks[e]] * mul : 0.f;
+                uint32_t hi, lo;
+                split_bf16(v, hi, lo);
+                bits[e] = part ? lo : hi;
+            }
+            bq[nt][j][0] = pack2(bits[0], bits[1]);
+            bq[nt][j][1] = pack2(bits[2], bits[3]);
+        }
+    }
+}
+
+// Zero the shared-memory rows of stage tokens that hold no valid token, so a
+// zero weight never meets a non-finite value.
+template <int D, int PS>
+EKV_DEV void zero_invalid_rows(const AttnArgs& a, uint8_t* stage, int b, int g, Range r, int st, int P, int L)
+{
+    const int tid = threadIdx.x;
+    const int t = tid & (kStageTok - 1);
+    const int half = tid >> 6;
+    if (half >= D / 64) return;
+    const int i = t / PS;
+    const int idx = r.start + st * (kStageTok / PS) + i;
+    bool valid = false;
+    if (idx < r.end) {
+        int lp;
+        const int phys = resolve(a, b, g, idx, P, lp, false);
+        valid = phys >= 0 && lp * PS + (t % PS) < L;
+    }
+    if (!valid) {
+        uint4* row = reinterpret_cast<uint4*>(stage + half * (kStageTok * 128) + t * 128);
+#pragma unroll
+        for (int k = 0; k < 8; ++k) row[k] = make_uint4(0, 0, 0, 0);
+    }
+}
+
+// ====================================================================== K pass
+template <int D, int PS, int NT>
+__global__ void __launch_bounds__(kThreads) qk_bf16_kernel(const __grid_constant__ CUtensorMap kmap, const AttnArgs a)
+{
+    constexpr int STAGE = kStageTok * D * 2;
+    constexpr int PPS = kStageTok / PS;
+    constexpr int KS = D / 16;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = align1024(smem_raw);
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kStagesQK * STAGE);
+    __shared__ int abort_flag;
+
+    const int b = blockIdx.z, g = blockIdx.y, s = blockIdx.x;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int L = a.seq_lens[b];
+    const int P = pages_of(L, PS, a.max_pages, a.status);
+    const int cnt = list_count(a, b, g, P);
+    if (s == 0 && tid == 0) a.counters[(size_t)b * a.H_kv + g] = 0;
+    const Range r = split_range(cnt, a.S, s);
+    if (r.end <= r.start) return;
+    const int nst = (r.end - r.start + PPS - 1) / PPS;
+
+    uint32_t bq[NT][KS][2];
+    load_q_frags<D, NT>(a, b, g, a.xscale, bq);
+
+    if (tid == 0) {
+        prefetch_tmap(&kmap);
+        for (int i = 0; i < kStagesQK; ++i) mbar_init(&bars[i], 1);
+        fence_mbar_init();
+        abort_flag = 0;
+    }
+    __syncthreads();
+    if (tid == 0)
+        for (int st = 0; st < min(kStagesQK, nst); ++st)
+            issue_stage<D, PS>(a, &kmap, smem + st * STAGE, &bars[st], b, g, r, st, P);
+
+    const uint32_t sbase = smem_addr(smem);
+    const size_t xstride = (size_t)a.k_max * PS;
+    for (int st = 0; st < nst; ++st) {
+        const int slot = st % kStagesQK;
+        if (!mbar_wait(&bars[slot], (st / kStagesQK) & 1, kWaitLimitNs)) {
+            abort_flag = 1;
+            report(a.status, ENTMAXKV_TIMEOUT);
+        }
+        __syncthreads();
+        if (abort_flag) {
+            if (tid == 0)
+                for (int k = st; k < min(st + kStagesQK, nst); ++k)
+                    mbar_wait(&bars[k % kStagesQK], (k / kStagesQK) & 1, kWaitLimitNs);
+            return;
+        }
+        const uint32_t base = sbase + slot * STAGE;
+        const int row0 = warp * 16;
+        float acc[NT][4];
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0.f;
+        const int arow = row0 + (lane & 7) + ((lane >> 3) & 1) * 8;
+#pragma unroll
+        for (int j = 0; j < KS; ++j) {
+            uint32_t af[4];
+            ldsm_x4(swz_addr(base, arow, 2 * j + (lane >> 4)), af);
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) mma_bf16(acc[nt], af, bq[nt][j][0], bq[nt][j][1]);
+        }
+        const int gi = lane >> 2, c = lane & 3;
+#pragma unroll
+        for (int rr = 0; rr < 2; ++rr) {
+            const int t = row0 + gi + 8 * rr;
+            const int idx = r.start + st * PPS + t / PS;
+            if (idx >= r.end) continue;
+            int lp;
+            const int phys = resolve(a, b, g, idx, P, lp, false);
+            const int prow = t % PS;
+            const bool valid = phys >= 0 && lp * PS + prow < L;
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) {
+                const int head = 4 * nt + c;
+                if (head < a.G) {
+                    const float x = valid ? acc[nt][2 * rr] + acc[nt][2 * rr + 1] : -INFINITY;
+                    a.xbuf[((size_t)b * a.H_q + (size_t)g * a.G + head) * xstride + (size_t)idx * PS + prow] = x;
+                }
+            }
+        }
+        __syncthreads();
+        if (tid == 0 && st + kStagesQK < nst)
+            issue_stage<D, PS>(a, &kmap, smem + slot * STAGE, &bars[slot], b, g, r, st + kStagesQK, P);
+    }
+}
+
+// fp32 cache: each thread scores (token, head) pairs of a page with a float64
+// dot product.
+template <int D>
+__global__ void __launch_bounds__(kThreads) qk_f32_kernel(const float* __restrict__ k_pool, int ps, const AttnArgs a)
+{
+    const int b = blockIdx.z, g = blockIdx.y, s = blockIdx.x, tid = threadIdx.x;
+    const int L = a.seq_lens[b];
+    const int P = pages_of(L, ps, a.max_pages, a.status);
+    const int cnt = list_count(a, b, g, P);
+    if (s == 0 && tid == 0) a.counters[(size_t)b * a.H_kv + g] = 0;
+    const Range r = split_range(cnt, a.S, s);
+    const size_t xstride = (size_t)a.k_max * ps;
+    const double xs = (double)a.xscale;
+    for (int idx = r.start; idx < r.end; ++idx) {
+        int lp;
+        const int phys = resolve(a, b, g, idx, P, lp, tid == 0);
+        for (int w = tid; w < ps * a.G; w += kThreads) {
+            const int t = w % ps, head = w / ps;
+            float x = -INFINITY;
+            if (phys >= 0 && lp * ps + t < L) {
+                const float* kr = k_pool + (((size_t)phys * a.H_kv + g) * ps + t) * D;
+                const float* qh = a.q + ((size_t)b * a.H_q + (size_t)g * a.G + head) * D;
+                double dot = 0.0;
+                for (int j = 0; j < D; ++j) dot = fma((double)qh[j], (double)kr[j], dot);
+                x = (float)(dot * xs);
+            }
+            a.xbuf[((size_t)b * a.H_q + (size_t)g * a.G + head) * xstride + (size_t)idx * ps + t] = x;
+        }
+    }
+}
+
+// ====================================================================== tau
+constexpr int kTauCap = 8192;
+constexpr int kTauBlock = 256;
+
+__global__ void __launch_bounds__(kTauBlock) tau_kernel(int ps, const AttnArgs a)
+{
+    __shared__ float cand[kTauCap];
+    __shared__ int ncand;
+    __shared__ double redd[kTauBlock / 32];
+    __shared__ float redf[kTauBlock / 32];
+    const int b = blockIdx.y, h = blockIdx.x, tid = threadIdx.x;
+    const int g = h / a.G;
+    const int L = a.seq_lens[b];
+    const int P = pages_of(L, ps, a.max_pages, a.status);
+    const int cnt = list_count(a, b, g, P);
+    const int n = cnt * ps;
+    const float* x = a.xbuf + ((size_t)b * a.H_q + h) * (size_t)a.k_max * ps;
+
+    float M = -INFINITY;
+    for (int i = tid; i < n; i += kTauBlock) M = fmaxf(M, x[i]);
+    M = block_max(M, redf);
+    if (M == -INFINITY) {
+        if (tid == 0) {
+            a.tau[(size_t)b * a.H_q + h] = INFINITY;
+            if (a.tau_out) a.tau_out[(size_t)b * a.H_q + h] = INFINITY;
+        }
+        return;
+    }
+    // no score at or below max - 1 can be in the support (tau >= max - 1)
+    const double thr = (double)M - 1.0;
+    if (tid == 0) ncand = 0;
+    __syncthreads();
+    for (int i = tid; i < n; i += kTauBlock) {
+        const float v = x[i];
+        if ((double)v > thr) {
+            const int k = atomicAdd(&ncand, 1);
+            if (k < kTauCap) cand[k] = v;
+        }
+    }
+    __syncthreads();
+    const bool spill = ncand > kTauCap;
+    const float* src = spill ? x : cand;
+    const int len = spill ? n : ncand;
+    const bool a2 = a.alpha == 2.0f;
+
+    double tau = thr;
+    for (int it = 0; it < 100; ++it) {
+        double k = 0.0, sx = 0.0, sxx = 0.0;
+        float minS = INFINITY, maxN = -INFINITY;
+        for (int i = tid; i < len; i += kTauBlock) {
+            const float v = src[i];
+            const double vd = (double)v;
+            if (!(vd > thr)) continue;
+            if (vd > tau) {
+                k += 1.0;
+                sx += vd;
+                sxx = fma(vd, vd, sxx);
+                minS = fminf(minS, v);
+            } else {
+                maxN = fmaxf(maxN, v);
+            }
+        }
+        k = block_sum(k, redd);
+        sx = block_sum(sx, redd);
+        sxx = block_sum(sxx, redd);
+        minS = block_min(minS, redf);
+        maxN = block_max(maxN, redf);
+        // closed form on the current support S = {x > tau}
+        double tcf;
+        bool ok;
+        if (a2) {
+            tcf = (sx - 1.0) / k;
+            ok = true;
+        } else {
+            const double mean = sx / k, msq = sxx / k;
+            const double disc = mean * mean - msq + 1.0 / k;
+            ok = disc >= 0.0;
+            tcf = ok ? mean - sqrt(disc) : 0.0;
+        }
+        if (ok && tcf < (double)minS && (double)maxN <= tcf) {
+            tau = tcf;
+            break;
+        }
+        // Newton step from tau on sum_S (x - tau)^r = 1
+        double nt;
+        if (a2) {
+            nt = tcf;
+        } else {
+            const double s1 = sx - k * tau;
+            const double s2 = sxx - 2.0 * tau * sx + k * tau * tau;
+            nt = tau + (s2 - 1.0) / (2.0 * s1);
+        }
+        if (!(nt != tau) || !isfinite(nt)) break;
+        tau = nt;
+    }
+    if (tid == 0) {
+        a.tau[(size_t)b * a.H_q + h] = (float)tau;
+        if (a.tau_out) a.tau_out[(size_t)b * a.H_q + h] = (float)tau;
+    }
+}
+
+// ====================================================================== split reduction
+// Each CTA has written its partial for (b, g); the last one to arrive sums the
+// partials in split order.
+template <int D, bool SOFTMAX>
+EKV_DEV void reduce_splits(const AttnArgs& a, int b, int g)
+{
+    __shared__ int is_last;
+    __threadfence();
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        const int t = atomicAdd(&a.counters[(size_t)b * a.H_kv + g], 1);
+        is_last = (t == a.S - 1);
+    }
+    __syncthreads();
+    if (!is_last) return;
+    __threadfence();
+    for (int i = threadIdx.x; i < a.G * D; i += blockDim.x) {
+        const int head = i / D, dd = i % D;
+        const size_t row = (size_t)b * a.H_q + (size_t)g * a.G + head;
+        float acc = 0.f;
+        if (!SOFTMAX) {
+            for (int s = 0; s < a.S; ++s) acc += __ldcg(&a.opart[(row * a.S + s) * D + dd]);
+            a.out[row * D + dd] = acc;
+        } else {
+            float Mx = -INFINITY;
+            for (int s = 0; s < a.S; ++s) Mx = fmaxf(Mx, __ldcg(&a.mlpart[(row * a.S + s) * 2]));
+            float l = 0.f;
+            if (Mx != -INFINITY) {
+                for (int s = 0; s < a.S; ++s) {
+                    const float ms = __ldcg(&a.mlpart[(row * a.S + s) * 2]);
+                    if (ms == -INFINITY) continue;
+                    const float w = expf(ms - Mx);
+                    l += w * __ldcg(&a.mlpart[(row * a.S + s) * 2 + 1]);
+                    acc += w * __ldcg(&a.opart[(row * a.S + s) * D + dd]);
+                }
+            }
+            a.out[row * D + dd] = l > 0.f ? acc / l : 0.f;
+        }
+    }
+    if (threadIdx.x == 0) a.counters[(size_t)b * a.H_kv + g] = 0;
+}
+
+// ====================================================================== V pass
+template <int D, int PS, int NT>
+__global__ void __launch_bounds__(kThreads) pv_bf16_kernel(const __grid_constant__ CUtensorMap vmap, const AttnArgs a)
+{
+    constexpr int STAGE = kStageTok * D * 2;
+    constexpr int PPS = kStageTok / PS;
+    constexpr int MTW = D / 64;           // 16-row m-tiles (head-dim rows) per warp
+    constexpr int PROW = kStageTok + kPsPad;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = align1024(smem_raw);
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kStagesPV * STAGE);
+    uint16_t* ps_tile = reinterpret_cast<uint16_t*>(smem + kStagesPV * STAGE + 64);   // [8*NT][PROW]
+    __shared__ int abort_flag;
+
+    const int b = blockIdx.z, g = blockIdx.y, s = blockIdx.x;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int L = a.seq_lens[b];
+    const int P = pages_of(L, PS, a.max_pages, a.status);
+    const int cnt = list_count(a, b, g, P);
+    const Range r = split_range(cnt, a.S, s);
+    const int nst = r.end > r.start ? (r.end - r.start + PPS - 1) / PPS : 0;
+    const bool a2 = a.alpha == 2.0f;
+    const size_t xstride = (size_t)a.k_max * PS;
+
+    float acc[NT][MTW][4];
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+        for (int m = 0; m < MTW; ++m) acc[nt][m][0] = acc[nt][m][1] = acc[nt][m][2] = acc[nt][m][3] = 0.f;
+
+    if (nst > 0) {
+        if (tid == 0) {
+            prefetch_tmap(&vmap);
+            for (int i = 0; i < kStagesPV; ++i) mbar_init(&bars[i], 1);
+            fence_mbar_init();
+            abort_flag = 0;
+        }
+        for (int i = tid; i < 8 * NT * PROW; i += kThreads) ps_tile[i] = 0;
+        __syncthreads();
+        if (tid == 0)
+            for (int st = 0; st < min(kStagesPV, nst); ++st)
+                issue_stage<D, PS>(a, &vmap, smem + st * STAGE, &bars[st], b, g, r, st, P);
+        // this thread's weights: token tid % 64, heads (tid / 64) * 2 * NT ...
+        const int ptok = tid & (kStageTok - 1);
+        const int hbase = (tid >> 6) * 2 * NT;
+        float tau_h[2 * NT];
+#pragma unroll
+        for (int k = 0; k < 2 * NT; ++k) {
+            const int head = hbase + k;
+            tau_h[k] = head < a.G ? a.tau[(size_t)b * a.H_q + g * a.G + head] : INFINITY;
+        }
+        const uint32_t sbase = smem_addr(smem);
+        const uint32_t pbase = smem_addr(ps_tile);
+        for (int st = 0; st < nst; ++st) {
+            const int slot = st % kStagesPV;
+            // weights of this stage (independent of the V tile; computed while it lands)
+            {
+                const int idx = r.start + st * PPS + ptok / PS;
+                const int prow = ptok % PS;
+#pragma unroll
+                for (int k = 0; k < 2 * NT; ++k) {
+                    const int head = hbase + k;
+                    float p = 0.f;
+                    if (head < a.G && idx < r.end) {
+                        const float xv = a.xbuf[((size_t)b * a.H_q + (size_t)g * a.G + head) * xstride + (size_t)idx * PS + prow];
+                        const float u = fmaxf(xv - tau_h[k], 0.f);
+                        p = a2 ? u : u * u;
+                    }
+                    uint32_t hi, lo;
+                    split_bf16(p, hi, lo);
+                    ps_tile[(2 * head) * PROW + ptok] = (uint16_t)hi;
+                    ps_tile[(2 * head + 1) * PROW + ptok] = (uint16_t)lo;
+                }
+            }
+            if (!mbar_wait(&bars[slot], (st / kStagesPV) & 1, kWaitLimitNs)) {
+                abort_flag = 1;
+                report(a.status, ENTMAXKV_TIMEOUT);
+            }
+            __syncthreads();
+            if (abort_flag) {
+                if (tid == 0)
+                    for (int k = st; k < min(st + kStagesPV, nst); ++k)
+                        mbar_wait(&bars[k % kStagesPV], (k / kStagesPV) & 1, kWaitLimitNs);
+                return;
+            }
+            zero_invalid_rows<D, PS>(a, smem + slot * STAGE, b, g, r, st, P, L);
+            __syncthreads();
+            const uint32_t base = sbase + slot * STAGE;
+            const int n = lane >> 2, c = lane & 3;
+#pragma unroll
+            for (int kk = 0; kk < kStageTok / 16; ++kk) {
+                uint32_t b0[NT], b1[NT];
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt) {
+                    const uint32_t pr = pbase + ((8 * nt + n) * PROW + 16 * kk + 2 * c) * 2;
+                    asm volatile("ld.shared.b32 %0, [%1];" : "=r"(b0[nt]) : "r"(pr));
+                    asm volatile("ld.shared.b32 %0, [%1];" : "=r"(b1[nt]) : "r"(pr + 16));
+                }
+                const int mi = lane >> 3;
+                const int trow = 16 * kk + (lane & 7) + 8 * (mi >> 1);
+#pragma unroll
+                for (int m = 0; m < MTW; ++m) {
+                    const int d0 = 16 * (warp * MTW + m);
+                    uint32_t af[4];
+                    ldsm_x4_t(swz_addr(base, trow, d0 / 8 + (mi & 1)), af);
+#pragma unroll
+                    for (int nt = 0; nt < NT; ++nt) mma_bf16(acc[nt][m], af, b0[nt], b1[nt]);
+                }
+            }
+            __syncthreads();
+            if (tid == 0 && st + kStagesPV < nst)
+                issue_stage<D, PS>(a, &vmap, smem + slot * STAGE, &bars[slot], b, g, r, st + kStagesPV, P);
+        }
+    }
+    // partial output of this split: o[head 4nt + c][d]
+    {
+        const int c = lane & 3, gi = lane >> 2;
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+            const int head = 4 * nt + c;
+            if (head >= a.G) continue;
+            const size_t row = ((size_t)b * a.H_q + (size_t)g * a.G + head) * a.S + s;
+#pragma unroll
+            for (int m = 0; m < MTW; ++m) {
+                const int d = 16 * (warp * MTW + m) + gi;
+                a.opart[row * D + d] = acc[nt][m][0] + acc[nt][m][1];
+                a.opart[row * D + d + 8] = acc[nt][m][2] + acc[nt][m][3];
+            }
+        }
+    }
+    reduce_splits<D, false>(a, b, g);
+}
+
+template <int D>
+__global__ void __launch_bounds__(kThreads) pv_f32_kernel(const float* __restrict__ v_pool, int ps, const AttnArgs a)
+{
+    const int b = blockIdx.z, g = blockIdx.y, s = blockIdx.x, tid = threadIdx.x;
+    const int L = a.seq_lens[b];
+    const int P = pages_of(L, ps, a.max_pages, a.status);
+    const int cnt = list_count(a, b, g, P);
+    const Range r = split_range(cnt, a.S, s);
+    const size_t xstride = (size_t)a.k_max * ps;
+    const bool a2 = a.alpha == 2.0f;
+    for (int w = tid; w < a.G * D; w += kThreads) {
+        const int head = w / D, dd = w % D;
+        const size_t row = (size_t)b * a.H_q + (size_t)g * a.G + head;
+        const float tau = a.tau[row];
+        double acc = 0.0;
+        for (int idx = r.start; idx < r.end; ++idx) {
+            int lp;
+            const int phys = resolve(a, b, g, idx, P, lp, false);
+            if (phys < 0) continue;
+            for (int t = 0; t < ps && lp * ps + t < L; ++t) {
+                const float xv = a.xbuf[row * xstride + (size_t)idx * ps + t];
+                const double u = fmax((double)xv - (double)tau, 0.0);
+                if (u > 0.0) {
+                    const double p = a2 ? u : u * u;
+                    acc = fma(p, (double)v_pool[(((size_t)phys * a.H_kv + g) * ps + t) * D + dd], acc);
+                }
+            }
+        }
+        a.opart[(row * a.S + s) * D + dd] = (float)acc;
+    }
+    reduce_splits<D, false>(a, b, g);
+}
+
+// ====================================================================== softmax
+template <int D, int PS, int NT>
+__global__ void __launch_bounds__(kThreads) softmax_bf16_kernel(const __grid_constant__ CUtensorMap kmap,
+                                                                const __grid_constant__ CUtensorMap vmap,
+                                                                const AttnArgs a)
+{
+    constexpr int STAGE = kStageTok * D * 2;
+    constexpr int PPS = kStageTok / PS;
+    constexpr int KS = D / 16;
+    constexpr int MTW = D / 64;
+    constexpr int PROW = kStageTok + kPsPad;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = align1024(smem_raw);
+    // stage i: K tile at 2i*STAGE, V tile at (2i+1)*STAGE
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + 2 * kStagesSM * STAGE);
+    uint16_t* ps_tile = reinterpret_cast<uint16_t*>(smem + 2 * kStagesSM * STAGE + 64);
+    __shared__ float wmax[4][4 * NT];
+    __shared__ int abort_flag;
+
+    const int b = blockIdx.z, g = blockIdx.y, s = blockIdx.x;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int gi = lane >> 2, c = lane & 3;
+    const int L = a.seq_lens[b];
+    const int P = pages_of(L, PS, a.max_pages, a.status);
+    const int cnt = list_count(a, b, g, P);
+    const Range r = split_range(cnt, a.S, s);
+    const int nst = r.end > r.start ? (r.end - r.start + PPS - 1) / PPS : 0;
+
+    float acc[NT][MTW][4];
+    float mrun[NT], lrun[NT];
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+        mrun[nt] = -INFINITY;
+        lrun[nt] = 0.f;
+#pragma unroll
+        for (int m = 0; m < MTW; ++m) acc[nt][m][0] = acc[nt][m][1] = acc[nt][m][2] = acc[nt][m][3] = 0.f;
+    }
+
+    if (nst > 0) {
+        uint32_t bq[NT][KS][2];
+        load_q_frags<D, NT>(a, b, g, a.xscale, bq);
+        if (tid == 0) {
+            prefetch_tmap(&kmap);
+            prefetch_tmap(&vmap);
+            for (int i = 0; i < kStagesSM; ++i) mbar_init(&bars[i], 1);
+            fence_mbar_init();
+            abort_flag = 0;
+        }
+        for (int i = tid; i < 8 * NT * PROW; i += kThreads) ps_tile[i] = 0;
+        __syncthreads();
+        auto issue = [&](int st) {
+            const int slot = st % kStagesSM;
+            // one barrier for both tiles: expect the sum of their bytes
+            constexpr int PPS_ = PPS;
+            int phys[PPS_];
+            uint32_t bytes = 0;
+#pragma unroll
+            for (int i = 0; i < PPS_; ++i) {
+                const int idx = r.start + st * PPS_ + i;
+                int lp;
+                phys[i] = idx < r.end ? resolve(a, b, g, idx, P, lp, true) : -1;
+                if (phys[i] >= 0) bytes += 2 * PS * D * 2;
+            }
+            mbar_arrive_expect_tx(&bars[slot], bytes);
+#pragma unroll
+            for (int i = 0; i < PPS_; ++i) {
+                if (phys[i] < 0) continue;
+                const int y = (phys[i] * a.H_kv + g) * PS;
+#pragma unroll
+                for (int h = 0; h < D / 64; ++h) {
+                    tma_load_2d(smem + (2 * slot) * STAGE + h * (kStageTok * 128) + i * PS * 128, &kmap, &bars[slot], h * 64, y);
+                    tma_load_2d(smem + (2 * slot + 1) * STAGE + h * (kStageTok * 128) + i * PS * 128, &vmap, &bars[slot], h * 64, y);
+                }
+            }
+        };
+        if (tid == 0)
+            for (int st = 0; st < min(kStagesSM, nst); ++st) issue(st);
+        const uint32_t sbase = smem_addr(smem);
+        const uint32_t pbase = smem_addr(ps_tile);
+        for (int st = 0; st < nst; ++st) {
+            const int slot = st % kStagesSM;
+            if (!mbar_wait(&bars[slot], (st / kStagesSM) & 1, kWaitLimitNs)) {
+                abort_flag = 1;
+                report(a.status, ENTMAXKV_TIMEOUT);
+            }
+            __syncthreads();
+            if (abort_flag) {
+                if (tid == 0)
+                    for (int k = st; k < min(st + kStagesSM, nst); ++k)
+                        mbar_wait(&bars[k % kStagesSM], (k / kStagesSM) & 1, kWaitLimitNs);
+                return;
+            }
+            const uint32_t kbase = sbase + (2 * slot) * STAGE;
+            const uint32_t vbase = sbase + (2 * slot + 1) * STAGE;
+            // scores of tokens row0+gi (+8), head 4nt + c
+            const int row0 = warp * 16;
+            float sc[NT][2];
+            {
+                float qa[NT][4];
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt) qa[nt][0] = qa[nt][1] = qa[nt][2] = qa[nt][3] = 0.f;
+                const int arow = row0 + (lane & 7) + ((lane >> 3) & 1) * 8;
+#pragma unroll
+                for (int j = 0; j < KS; ++j) {
+                    uint32_t af[4];
+                    ldsm_x4(swz_addr(kbase, arow, 2 * j + (lane >> 4)), af);
+#pragma unroll
+                    for (int nt = 0; nt < NT; ++nt) mma_bf16(qa[nt], af, bq[nt][j][0], bq[nt][j][1]);
+                }
+#pragma unroll
+                for (int rr = 0; rr < 2; ++rr) {
+                    const int t = row0 + gi + 8 * rr;
+                    const int idx = r.start + st * PPS + t / PS;
+                    bool valid = false;
+                    if (idx < r.end) {
+                        int lp;
+                        const int phys = resolve(a, b, g, idx, P, lp, false);
+                        valid = phys >= 0 && lp * PS + t % PS < L;
+                    }
+#pragma unroll
+                    for (int nt = 0; nt < NT; ++nt)
+                        sc[nt][rr] = (valid && 4 * nt + c < a.G) ? qa[nt][2 * rr] + qa[nt][2 * rr + 1] : -INFINITY;
+                }
+            }
+            // stage maximum per head (lanes with equal c share a head)
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) {
+                float mloc = fmaxf(sc[nt][0], sc[nt][1]);
+                mloc = fmaxf(mloc, __shfl_xor_sync(0xffffffffu, mloc, 4));
+                mloc = fmaxf(mloc, __shfl_xor_sync(0xffffffffu, mloc, 8));
+                mloc = fmaxf(mloc, __shfl_xor_sync(0xffffffffu, mloc, 16));
+                if (gi == 0) wmax[warp][4 * nt + c] = mloc;
+            }
+            zero_invalid_rows<D, PS>(a, smem + (2 * slot + 1) * STAGE, b, g, r, st, P, L);
+            __syncthreads();
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) {
+                const int hh = 4 * nt + c;
+                const float smax = fmaxf(fmaxf(wmax[0][hh], wmax[1][hh]), fmaxf(wmax[2][hh], wmax[3][hh]));
+                const float mnew = fmaxf(mrun[nt], smax);
+                const float corr = (mnew == -INFINITY) ? 1.f : expf(mrun[nt] - mnew);
+                mrun[nt] = mnew;
+                lrun[nt] *= corr;
+#pragma unroll
+                for (int m = 0; m < MTW; ++m) {
+                    acc[nt][m][0] *= corr; acc[nt][m][1] *= corr;
+                    acc[nt][m][2] *= corr; acc[nt][m][3] *= corr;
+                }
+#pragma unroll
+                for (int rr = 0; rr < 2; ++rr) {
+                    const float p = (sc[nt][rr] == -INFINITY) ? 0.f : expf(sc[nt][rr] - mnew);
+                    lrun[nt] += p;
+                    uint32_t hi, lo;
+                    split_bf16(p, hi, lo);
+                    const int t = row0 + gi + 8 * rr;
+                    ps_tile[(2 * hh) * PROW + t] = (uint16_t)hi;
+                    ps_tile[(2 * hh + 1) * PROW + t] = (uint16_t)lo;
+                }
+            }
+            __syncthreads();
+#pragma unroll
+            for (int kk = 0; kk < kStageTok / 16; ++kk) {
+                uint32_t b0[NT], b1[NT];
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt) {
+                    const uint32_t pr = pbase + ((8 * nt + gi) * PROW + 16 * kk + 2 * c) * 2;
+                    asm volatile("ld.shared.b32 %0, [%1];" : "=r"(b0[nt]) : "r"(pr));
+                    asm volatile("ld.shared.b32 %0, [%1];" : "=r"(b1[nt]) : "r"(pr + 16));
+                }
+                const int mi = lane >> 3;
+                const int trow = 16 * kk + (lane & 7) + 8 * (mi >> 1);
+#pragma unroll
+                for (int m = 0; m < MTW; ++m) {
+                    const int d0 = 16 * (warp * MTW + m);
+                    uint32_t af[4];
+                    ldsm_x4_t(swz_addr(vbase, trow, d0 / 8 + (mi & 1)), af);
+#pragma unroll
+                    for (int nt = 0; nt < NT; ++nt) mma_bf16(acc[nt][m], af, b0[nt], b1[nt]);
+                }
+            }
+            __syncthreads();
+            if (tid == 0 && st + kStagesSM < nst) issue(st + kStagesSM);
+        }
+    }
+    // running sums: lanes with equal c, all warps
+    __shared__ float lsum[4][4 * NT];
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+        float l = lrun[nt];
+        l += __shfl_xor_sync(0xffffffffu, l, 4);
+        l += __shfl_xor_sync(0xffffffffu, l, 8);
+        l += __shfl_xor_sync(0xffffffffu, l, 16);
+        if (gi == 0) lsum[warp][4 * nt + c] = l;
+    }
+    __syncthreads();
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+        const int head = 4 * nt + c;
+        if (head >= a.G) continue;
+        const size_t row = ((size_t)b * a.H_q + (size_t)g * a.G + head) * a.S + s;
+#pragma unroll
+        for (int m = 0; m < MTW; ++m) {
+            const int d = 16 * (warp * MTW + m) + gi;
+            a.opart[row * D + d] = acc[nt][m][0] + acc[nt][m][1];
+            a.opart[row * D + d + 8] = acc[nt][m][2] + acc[nt][m][3];
+        }
+        if (warp == 0 && gi == 0) {
+            a.mlpart[row * 2] = mrun[nt];
+            a.mlpart[row * 2 + 1] = lsum[0][head] + lsum[1][head] + lsum[2][head] + lsum[3][head];
+        }
+    }
+    reduce_splits<D, true>(a, b, g);
+}
+
+template <int D>
+__global__ void __launch_bounds__(kThreads) softmax_f32_kernel(const float* __restrict__ k_pool,
+                                                               const float* __restrict__ v_pool, int ps,
+                                                               const AttnArgs a)
+{
+    __shared__ float sc[64 * 8];
+    const int b = blockIdx.z, g = blockIdx.y, s = blockIdx.x, tid = threadIdx.x;
+    const int L = a.seq_lens[b];
+    const int P = pages_of(L, ps, a.max_pages, a.status);
+    const int cnt = list_count(a, b, g, P);
+    const Range r = split_range(cnt, a.S, s);
+    // thread w < G*D owns (head, d) pairs w, w + kThreads, ...
+    constexpr int PER = (8 * D + kThreads - 1) / kThreads;
+    float m[PER], l[PER];
+    double o[PER];
+    for (int k = 0; k < PER; ++k) { m[k] = -INFINITY; l[k] = 0.f; o[k] = 0.0; }
+    for (int idx = r.start; idx < r.end; ++idx) {
+        int lp;
+        const int phys = resolve(a, b, g, idx, P, lp, tid == 0);
+        __syncthreads();
+        for (int w = tid; w < ps * a.G; w += kThreads) {
+            const int t = w % ps, head = w / ps;
+            float x = -INFINITY;
+            if (phys >= 0 && lp * ps + t < L) {
+                const float* kr = k_pool + (((size_t)phys * a.H_kv + g) * ps + t) * D;
+                const float* qh = a.q + ((size_t)b * a.H_q + (size_t)g * a.G + head) * D;
+                double dot = 0.0;
+                for (int j = 0; j < D; ++j) dot = fma((double)qh[j], (double)kr[j], dot);
+                x = (float)(dot * (double)a.xscale);
+            }
+            sc[head * 64 + t] = x;
+        }
+        __syncthreads();
+        for (int k = 0; k < PER; ++k) {
+            const int w = tid + k * kThreads;
+            if (w >= a.G * D) break;
+            const int head = w / D, dd = w % D;
+            for (int t = 0; t < ps; ++t) {
+                const float x = sc[head * 64 + t];
+                if (x == -INFINITY) continue;
+                const float mn = fmaxf(m[k], x);
+                const float corr = m[k] == -INFINITY ? 0.f : expf(m[k] - mn);
+                const float p = expf(x - mn);
+                l[k] = l[k] * corr + p;
+                o[k] = o[k] * corr + (double)p * (double)v_pool[(((size_t)phys * a.H_kv + g) * ps + t) * D + dd];
+                m[k] = mn;
+            }
+        }
+    }
+    for (int k = 0; k < PER; ++k) {
+        const int w = tid + k * kThreads;
+        if (w >= a.G * D) break;
+        const int head = w / D, dd = w % D;
+        const size_t row = ((size_t)b * a.H_q + (size_t)g * a.G + head) * a.S + s;
+        a.opart[row * D + dd] = (float)o[k];
+        if (dd == 0) {
+            a.mlpart[row * 2] = m[k];
+            a.mlpart[row * 2 + 1] = l[k];
+        }
+    }
+    reduce_splits<D, true>(a, b, g);
+}
+
+// ====================================================================== self test
+__global__ void selftest_timeout_kernel(uint64_t limit_ns, int32_t* status)
+{
+    __shared__ uint64_t bar;
+    if (threadIdx.x == 0) {
+        mbar_init(&bar, 2);   // two arrivals expected, only one ever comes
+        fence_mbar_init();
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) mbar_arrive(&bar);
+    if (!mbar_wait(&bar, 0, limit_ns)) {
+        if (threadIdx.x == 0) report(status, ENTMAXKV_TIMEOUT);
+    }
+}
+
+// ====================================================================== launch
+template <int D, int PS, int NT>
+static int launch_entmax_bf16(const AttnArgs& a, int B, const CUtensorMap* kmap, const CUtensorMap* vmap,
+                              cudaStream_t stream)
+{
+    dim3 grid(a.S, a.H_kv, B);
+    const int qk_smem = kStagesQK * kStageTok * D * 2 + 1024 + 64;
+    const int pv_smem = kStagesPV * kStageTok * D * 2 + 1024 + 64 + 8 * NT * (kStageTok + kPsPad) * 2;
+    if (ensure_smem((const void*)qk_bf16_kernel<D, PS, NT>, qk_smem)) return ENTMAXKV_CUDA_ERROR;
+    if (ensure_smem((const void*)pv_bf16_kernel<D, PS, NT>, pv_smem)) return ENTMAXKV_CUDA_ERROR;
+    qk_bf16_kernel<D, PS, NT><<<grid, kThreads, qk_smem, stream>>>(*kmap, a);
+    if (cudaGetLastError() != cudaSuccess) return ENTMAXKV_CUDA_ERROR;
+    tau_kernel<<<dim3(a.H_q, B), kTauBlock, 0, stream>>>(PS, a);
+    if (cudaGetLastError() != cudaSuccess) return ENTMAXKV_CUDA_ERROR;
+    pv_bf16_kernel<D, PS, NT><<<grid, kThreads, pv_smem, stream>>>(*vmap, a);
+    return cudaGetLastError() == cudaSuccess ? ENTMAXKV_OK : ENTMAXKV_CUDA_ERROR;
+}
+
+template <int D>
+static int launch_entmax_f32(const entmaxkv_pool& pool, const AttnArgs& a, int B, cudaStream_t stream)
+{
+    dim3 grid(a.S, a.H_kv, B);
+    qk_f32_kernel<D><<<grid, kThreads, 0, stream>>>((const float*)pool.k_pool, pool.ps, a);
+    if (cudaGetLastError() != cudaSuccess) return ENTMAXKV_CUDA_ERROR;
+    tau_kernel<<<dim3(a.H_q, B), kTauBlock, 0, stream>>>(pool.ps, a);
+    if (cudaGetLastError() != cudaSuccess) return ENTMAXKV_CUDA_ERROR;
+    pv_f32_kernel<D><<<grid, kThreads, 0, stream>>>((const float*)pool.v_pool, pool.ps, a);
+    return cudaGetLastError() == cudaSuccess ? ENTMAXKV_OK : ENTMAXKV_CUDA_ERROR;
+}
+
+int launch_entmax_attend(const entmaxkv_pool& pool, const AttnArgs& a, int B, const CUtensorMap* kmap,
+                         const CUtensorMap* vmap, cudaStream_t stream)
+{
+    if (pool.dtype == ENTMAXKV_F32) {
+        return pool.d == 128 ? launch_entmax_f32<128>(pool, a, B, stream) : launch_entmax_f32<64>(pool, a, B, stream);
+    }
+    const bool g8 = a.G == 8;
+    if (pool.d == 128) {
+        if (pool.ps == 64) return g8 ? launch_entmax_bf16<128, 64, 2>(a, B, kmap, vmap, stream)
+                                     : launch_entmax_bf16<128, 64, 1>(a, B, kmap, vmap, stream);
+        return g8 ? launch_entmax_bf16<128, 16, 2>(a, B, kmap, vmap, stream)
+                  : launch_entmax_bf16<128, 16, 1>(a, B, kmap, vmap, stream);
+    }
+    if (pool.ps == 64) return g8 ? launch_entmax_bf16<64, 64, 2>(a, B, kmap, vmap, stream)
+                                 : launch_entmax_bf16<64, 64, 1>(a, B, kmap, vmap, stream);
+    return g8 ? launch_entmax_bf16<64, 16, 2>(a, B, kmap, vmap, stream)
+              : launch_entmax_bf16<64, 16, 1>(a, B, kmap, vmap, stream);
+}
+
+template <int D, int PS, int NT>
+static int launch_softmax_bf16(const AttnArgs& a, int B, const CUtensorMap* kmap, const CUtensorMap* vmap,
+                               cudaStream_t stream)
+{
+    dim3 grid(a.S, a.H_kv, B);
+    const int smem = 2 * kStagesSM * kStageTok * D * 2 + 1024 + 64 + 8 * NT * (kStageTok + kPsPad) * 2;
+    if (ensure_smem((const void*)softmax_bf16_kernel<D, PS, NT>, smem)) return ENTMAXKV_CUDA_ERROR;
+    softmax_bf16_kernel<D, PS, NT><<<grid, kThreads, smem, stream>>>(*kmap, *vmap, a);
+    return cudaGetLastError() == cudaSuccess ? ENTMAXKV_OK : ENTMAXKV_CUDA_ERROR;
+}
+
+__global__ void zero_counters_kernel(int32_t* counters, int n)
+{
+    const int i = blockIdx.x * blockDim.x + threadIdx.x;
+    if (i < n) counters[i] = 0;
+}
+
+int launch_softmax_attend(const entmaxkv_pool& pool, const AttnArgs& a, int B, const CUtensorMap* kmap,
+                          const CUtensorMap* vmap, cudaStream_t stream)
+{
+    const int n = B * a.H_kv;
+    zero_counters_kernel<<<(n + 255) / 256, 256, 0, stream>>>(a.counters, n);
+    if (cudaGetLastError() != cudaSuccess) return ENTMAXKV_CUDA_ERROR;
+    if (pool.dtype == ENTMAXKV_F32) {
+        dim3 grid(a.S, a.H_kv, B);
+        if (pool.d == 128)
+            softmax_f32_kernel<128><<<grid, kThreads, 0, stream>>>((const float*)pool.k_pool, (const float*)pool.v_pool, pool.ps, a);
+        else
+            softmax_f32_kernel<64><<<grid, kThreads, 0, stream>>>((const float*)pool.k_pool, (const float*)pool.v_pool, pool.ps, a);
+        return cudaGetLastError() == cudaSuccess ? ENTMAXKV_OK : ENTMAXKV_CUDA_ERROR;
+    }
+    const bool g8 = a.G == 8;
+    if (pool.d == 128) {
+        if (pool.ps == 64) return g8 ? launch_softmax_bf16<128, 64, 2>(a, B, kmap, vmap, stream)
+                                     : launch_softmax_bf16<128, 64, 1>(a, B, kmap, vmap, stream);
+        return g8 ? launch_softmax_bf16<128, 16, 2>(a, B, kmap, vmap, stream)
+                  : launch_softmax_bf16<128, 16, 1>(a, B, kmap, vmap, stream);
+    }
+    if (pool.ps == 64) return g8 ? launch_softmax_bf16<64, 64, 2>(a, B, kmap, vmap, stream)
+                                 : launch_softmax_bf16<64, 64, 1>(a, B, kmap, vmap, stream);
+    return g8 ? launch_softmax_bf16<64, 16, 2>(a, B, kmap, vmap, stream)
+              : launch_softmax_bf16<64, 16, 1>(a, B, kmap, vmap, stream);
+}
+
+int launch_selftest_timeout(int64_t limit_ns, int32_t* status, cudaStream_t stream)
+{
+    selftest_timeout_kernel<<<1, 32, 0, stream>>>((uint64_t)limit_ns, status);
+    return cudaGetLastError() == cudaSuccess ? ENTMAXKV_OK : ENTMAXKV_CUDA_ERROR;
+}
+
+}  // namespace ekv

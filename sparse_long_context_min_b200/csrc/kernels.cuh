@@ -1,0 +1,63 @@
+// Host-side launch entry points of the kernels (internal to the library).
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include <cmath>
+
+#include "entmaxkv.h"
+
+namespace ekv {
+
+// Arguments shared by the attention kernels (passed by value).
+struct AttnArgs {
+    const float* q;                // [B][H_q][d]
+    int H_q, H_kv, G;
+    const int32_t* page_table;     // [B][max_pages]
+    int max_pages;
+    const int32_t* seq_lens;       // [B]
+    const int32_t* sel;            // [B][H_kv][k_max], NULL = every page in order
+    const int32_t* sel_count;      // [B][H_kv], NULL = P_b
+    int k_max;                     // row length of sel and of the score buffer (in pages)
+    int num_phys;
+    int S;                         // splits per (sequence, kv head)
+    float alpha;
+    float xscale;                  // (alpha - 1) * scale, or scale for softmax
+    float* xbuf;                   // [B][H_q][k_max * ps] scores x of the listed tokens
+    float* tau;                    // [B][H_q]
+    float* opart;                  // [B][H_q][S][d] partial outputs
+    float* mlpart;                 // [B][H_q][S][2] softmax running max and sum
+    int32_t* counters;             // [B][H_kv] arrival counters of the split reduction
+    float* out;                    // [B][H_q][d]
+    float* tau_out;                // [B][H_q] or NULL
+    int32_t* status;
+};
+
+int launch_append(const entmaxkv_pool& pool, const void* k_new, const void* v_new, int n_new,
+                  const int32_t* page_table, int max_pages, int32_t* seq_lens, int B, int32_t* status,
+                  cudaStream_t stream);
+
+int launch_score(const entmaxkv_pool& pool, const float* q, int H_q, const int32_t* page_table,
+                 int max_pages, const int32_t* seq_lens, int B, int mode, float scale, float* ub, float* m,
+                 float* v, float* est, int32_t* status, cudaStream_t stream);
+
+int launch_select(int mode, const float* ub, const float* m, const float* v, const float* est,
+                  const int32_t* seq_lens, int ps, int B, int H_q, int H_kv, int max_pages, int budget,
+                  float budget_frac, float alpha, float delta, int k_max, int32_t* sel, int32_t* sel_count,
+                  float* tau_hat, int32_t* status, cudaStream_t stream);
+
+// entmax attention over the listed pages (sparse, or full when a.sel == NULL)
+int launch_entmax_attend(const entmaxkv_pool& pool, const AttnArgs& a, int B, const CUtensorMap* kmap,
+                         const CUtensorMap* vmap, cudaStream_t stream);
+
+int launch_softmax_attend(const entmaxkv_pool& pool, const AttnArgs& a, int B, const CUtensorMap* kmap,
+                          const CUtensorMap* vmap, cudaStream_t stream);
+
+int launch_selftest_timeout(int64_t limit_ns, int32_t* status, cudaStream_t stream);
+
+// set the dynamic shared memory limit of a kernel once per device
+int ensure_smem(const void* func, int bytes);
+
+}  // namespace ekv

@@ -1,0 +1,115 @@
+"""Decode-step driver: buffers plus the ordered C-ABI calls of one EntmaxKV step.
+
+    append (optional) -> score_pages -> select -> sparse_attend
+
+Host orchestration only -- it allocates device buffers with torch once and
+issues the library calls in order on one stream; every step of the path runs
+in the CUDA library.
+"""
+import math
+
+import torch
+
+from . import binding as B
+from .workloads import Workload
+
+
+def build_pool(wl: Workload, device="cuda", status=None):
+    """Allocate the pool of a workload and fill it sequence by sequence with
+    entmaxkv_append_metadata (whole-sequence appends build every page).
+    Returns (pool, seq_lens tensor on device)."""
+    cfg = wl.cfg
+    pool = B.Pool.allocate(wl.num_phys, cfg.H_kv, cfg.ps, cfg.d, cfg.dtype, device)
+    seq_lens = torch.zeros(cfg.B, dtype=torch.int32, device=device)
+    st = torch.zeros(1, dtype=torch.int32, device=device) if status is None else status
+    pt = wl.page_table.to(device)
+    for b in range(cfg.B):
+        k, v = wl.sequence(b)
+        k = k.to(device).unsqueeze(0).contiguous()
+        v = v.to(device).unsqueeze(0).contiguous()
+        B.append_metadata(pool, k, v, pt[b:b + 1], seq_lens[b:b + 1], st)
+        del k, v
+    if status is None:
+        torch.cuda.synchronize()
+        if int(st.item()) != 0:
+            raise B.EntmaxKVError(int(st.item()), "build_pool")
+    return pool, seq_lens
+
+
+class DecodeStep:
+    """One decode step of a configuration: scores, selects and attends.
+
+    mode "topk" (budget pages or budget_frac) or "gauss" (alpha, delta).
+    """
+
+    def __init__(self, pool, page_table, seq_lens, H_q, mode="topk", budget=-1, budget_frac=0.0,
+                 alpha=1.5, delta=0.5, extra_pages=0):
+        self.pool, self.page_table, self.seq_lens = pool, page_table, seq_lens
+        self.B = seq_lens.shape[0]
+        self.H_q, self.H_kv = H_q, pool.H_kv
+        self.max_pages = page_table.shape[1]
+        self.mode, self.budget, self.budget_frac = mode, budget, budget_frac
+        self.alpha, self.delta = alpha, delta
+        self.scale = 1.0 / math.sqrt(pool.d)
+        dev = pool.k_pool.device
+        f32 = dict(dtype=torch.float32, device=dev)
+        i32 = dict(dtype=torch.int32, device=dev)
+        if mode == "topk":
+            self.k_max = budget if budget >= 0 else int(math.ceil(float(torch.tensor(budget_frac,
+                                                                                       dtype=torch.float32))
+                                                                   * self.max_pages))
+            self.k_max = max(1, self.k_max)
+            self.ub = torch.empty(self.B, self.H_kv, self.max_pages, **f32)
+            self.m = self.v = self.est = self.tau_hat = None
+        else:
+            self.k_max = self.max_pages
+            self.ub = None
+            self.m = torch.empty(self.B, H_q, self.max_pages, **f32)
+            self.v = torch.empty_like(self.m)
+            self.est = torch.empty_like(self.m)
+            self.tau_hat = torch.empty(self.B, H_q, **f32)
+        self.sel = torch.empty(self.B, self.H_kv, self.k_max, **i32)
+        self.sel_count = torch.empty(self.B, self.H_kv, **i32)
+        self.out = torch.empty(self.B, H_q, pool.d, **f32)
+        self.tau = torch.empty(self.B, H_q, **f32)
+        ws = B.workspace_size(B.OP_SPARSE_ATTEND, self.B, H_q, self.H_kv, self.max_pages, self.k_max,
+                              pool.ps, pool.d)
+        self.workspace = torch.empty(max(ws, 256), dtype=torch.uint8, device=dev)
+        self.status = torch.zeros(1, **i32)
+
+    def score(self, q, stream=None):
+        if self.mode == "topk":
+            B.score_pages(self.pool, q, self.page_table, self.seq_lens, B.SCORE_BBOX, self.scale, self.status,
+                          ub=self.ub, stream=stream)
+        else:
+            B.score_pages(self.pool, q, self.page_table, self.seq_lens, B.SCORE_GAUSS, self.scale, self.status,
+                          m=self.m, v=self.v, est_max=self.est, stream=stream)
+
+    def choose(self, stream=None):
+        if self.mode == "topk":
+            B.select(B.SELECT_TOPK, self.seq_lens, self.pool.ps, self.H_q, self.H_kv, self.max_pages, self.k_max,
+                     self.sel, self.sel_count, self.status, ub=self.ub, budget=self.budget,
+                     budget_frac=self.budget_frac, stream=stream)
+        else:
+            B.select(B.SELECT_GAUSS, self.seq_lens, self.pool.ps, self.H_q, self.H_kv, self.max_pages,
+                     self.k_max, self.sel, self.sel_count, self.status, m=self.m, v=self.v, est_max=self.est,
+                     alpha=self.alpha, delta=self.delta, tau_hat=self.tau_hat, stream=stream)
+
+    def attend(self, q, stream=None):
+        B.sparse_attend(self.pool, q, self.page_table, self.seq_lens, self.sel, self.sel_count, self.alpha,
+                        self.scale, self.out, self.workspace, self.status, tau_out=self.tau, stream=stream)
+
+    def __call__(self, q, k_new=None, v_new=None, stream=None):
+        """One step; appends (k_new, v_new) [B, H_kv, 1, d] first when given."""
+        if k_new is not None:
+            B.append_metadata(self.pool, k_new, v_new, self.page_table, self.seq_lens, self.status, stream=stream)
+        self.score(q, stream)
+        self.choose(stream)
+        self.attend(q, stream)
+        return self.out
+
+    def check(self):
+        torch.cuda.synchronize()
+        code = int(self.status.item())
+        if code:
+            raise B.EntmaxKVError(code, "decode step (device status)")

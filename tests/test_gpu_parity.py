@@ -1,0 +1,402 @@
+"""GPU parity of every step of the decode path against the CPU oracle.
+
+Every call goes through the C ABI (sparse_long_context_min_b200.binding).
+Sizes span several pipeline stages, several splits and a ragged last page;
+the oracle side is computed from the generator's tensors only.
+"""
+import math
+from dataclasses import replace
+
+import numpy as np
+import pytest
+import torch
+
+import helpers as H
+from oracle import attend, select
+from sparse_long_context_min_b200 import binding as B
+from sparse_long_context_min_b200 import workloads
+from sparse_long_context_min_b200.step import DecodeStep, build_pool
+
+pytestmark = pytest.mark.gpu
+
+
+def _wl(n, lengths=None, B_=None, **kw):
+    cfg = workloads.config(n, B=B_)
+    if lengths is not None:
+        cfg = replace(cfg, B=len(lengths), lengths=list(lengths))
+    if kw:
+        cfg = replace(cfg, **kw)
+    return workloads.Workload(cfg, device="cuda")
+
+
+def _status():
+    return torch.zeros(1, dtype=torch.int32, device="cuda")
+
+
+def _assert_ok(st):
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0, B.status_string(int(st.item()))
+
+
+# (config, lengths) cases: fp32 tiny, bf16 d=128 ps=64 with ragged pages, permuted pool
+CASES = {
+    "tiny": (1, [4096 + 5]),
+    "llama": (2, [16384 + 1]),
+    "ragged": (5, [5000, 12345, 777]),
+}
+
+
+@pytest.fixture(scope="module", params=list(CASES))
+def built(request):
+    n, lens = CASES[request.param]
+    wl = _wl(n, lens)
+    pool, seq_lens = build_pool(wl)
+    oseqs = [H.OracleSeq(wl, b) for b in range(wl.cfg.B)]
+    return wl, pool, seq_lens, oseqs
+
+
+def test_append_metadata_bitexact(built):
+    wl, pool, seq_lens, oseqs = built
+    cfg = wl.cfg
+    assert seq_lens.cpu().tolist() == cfg.lengths
+    pt = wl.page_table.cpu()
+    for b, o in enumerate(oseqs):
+        P = cfg.pages(b)
+        phys = pt[b, :P].long()
+        for g in range(cfg.H_kv):
+            m = o.meta(g)
+            assert np.array_equal(pool.kmin[phys, g].float().cpu().numpy(), m["kmin"])
+            assert np.array_equal(pool.kmax[phys, g].float().cpu().numpy(), m["kmax"])
+            assert np.array_equal(pool.mean[phys, g].cpu().numpy(), m["mean"])
+            assert np.array_equal(pool.m2[phys, g].cpu().numpy(), m["m2"])
+            # pool contents are the appended tokens
+            kp = pool.k_pool[phys, g].float().cpu().numpy().reshape(P * cfg.ps, cfg.d)[:o.L]
+            assert np.array_equal(kp, o.keys[g])
+        assert np.array_equal(pool.count[phys].cpu().numpy(), o.meta(0)["count"])
+
+
+def test_append_one_token_at_a_time_matches_whole_pages():
+    wl = _wl(2, [200])
+    cfg = wl.cfg
+    pool_a, _ = build_pool(wl)
+    pool_b = B.Pool.allocate(wl.num_phys, cfg.H_kv, cfg.ps, cfg.d, cfg.dtype)
+    seq = torch.zeros(1, dtype=torch.int32, device="cuda")
+    st = _status()
+    k, v = wl.sequence(0)
+    pt = wl.page_table
+    for t in range(0, 200, 7):            # chunks of 7 tokens cross page boundaries
+        kk = k[:, t:t + 7].unsqueeze(0).contiguous()
+        vv = v[:, t:t + 7].unsqueeze(0).contiguous()
+        B.append_metadata(pool_b, kk, vv, pt, seq, st)
+    _assert_ok(st)
+    assert int(seq.item()) == 200
+    for name in ("kmin", "kmax", "mean", "m2", "count", "k_pool", "v_pool"):
+        a, b_ = getattr(pool_a, name), getattr(pool_b, name)
+        assert torch.equal(a, b_), name
+
+
+def test_score_bbox_bitexact(built):
+    wl, pool, seq_lens, oseqs = built
+    cfg = wl.cfg
+    st = _status()
+    ub = torch.empty(cfg.B, cfg.H_kv, wl.max_pages, device="cuda")
+    B.score_pages(pool, wl.q, wl.page_table, seq_lens, B.SCORE_BBOX, H.scale32(cfg), st, ub=ub)
+    _assert_ok(st)
+    ub = ub.cpu().numpy()
+    for b, o in enumerate(oseqs):
+        P = cfg.pages(b)
+        for g in range(cfg.H_kv):
+            assert np.array_equal(ub[b, g, :P], o.ubg(g)), (b, g)
+            assert np.all(ub[b, g, P:] == -np.inf)
+
+
+@pytest.mark.parametrize("frac", [1 / 32, 1 / 8])
+def test_topk_selection_bitexact(built, frac):
+    wl, pool, seq_lens, oseqs = built
+    cfg = wl.cfg
+    step = DecodeStep(pool, wl.page_table, seq_lens, cfg.H_q, "topk", budget_frac=frac, alpha=cfg.alpha)
+    step.score(wl.q)
+    step.choose()
+    step.check()
+    sel, cnt = step.sel.cpu().numpy(), step.sel_count.cpu().numpy()
+    for b, o in enumerate(oseqs):
+        for g in range(cfg.H_kv):
+            ref = o.topk(g, -1, frac)
+            assert cnt[b, g] == len(ref)
+            assert np.array_equal(sel[b, g, :cnt[b, g]], ref), (b, g)
+
+
+def test_topk_ties_signed_zeros_and_budgets():
+    """select() on a hand-made bound array with heavy ties, +-0 and every budget regime."""
+    rng = np.random.default_rng(7)
+    P, Bn, Hkv = 3000, 3, 2
+    vals = np.array([-1.0, -0.0, 0.0, 0.25, 0.25, 2.0, 5.5], dtype=np.float32)
+    ub = vals[rng.integers(0, len(vals), (Bn, Hkv, P))]
+    ub[1, 1] = rng.standard_normal(P).astype(np.float32)
+    ub[2] = 0.25                                  # all equal
+    seq_lens = torch.tensor([P * 16, P * 16 - 15, 40 * 16], dtype=torch.int32, device="cuda")
+    for budget in (0, 1, 7, 300, 2999, 3000, 5000):
+        k_max = max(1, budget)
+        sel = torch.full((Bn, Hkv, k_max), -7, dtype=torch.int32, device="cuda")
+        cnt = torch.empty(Bn, Hkv, dtype=torch.int32, device="cuda")
+        st = _status()
+        B.select(B.SELECT_TOPK, seq_lens, 16, Hkv * 4, Hkv, P, k_max, sel, cnt, st,
+                 ub=torch.from_numpy(ub).cuda(), budget=budget)
+        _assert_ok(st)
+        for b in range(Bn):
+            Pb = (int(seq_lens[b]) + 15) // 16
+            for g in range(Hkv):
+                ref = select.topk(ub[b, g, :Pb], select.budget_pages(Pb, budget, 0.0))
+                c = int(cnt[b, g])
+                assert c == len(ref)
+                assert np.array_equal(sel[b, g, :c].cpu().numpy(), ref), (budget, b, g)
+
+
+def test_score_gauss_bitexact(built):
+    wl, pool, seq_lens, oseqs = built
+    cfg = wl.cfg
+    st = _status()
+    shape = (cfg.B, cfg.H_q, wl.max_pages)
+    m = torch.empty(shape, device="cuda")
+    v = torch.empty(shape, device="cuda")
+    e = torch.empty(shape, device="cuda")
+    B.score_pages(pool, wl.q, wl.page_table, seq_lens, B.SCORE_GAUSS, H.scale32(cfg), st, m=m, v=v, est_max=e)
+    _assert_ok(st)
+    m, v, e = m.cpu().numpy(), v.cpu().numpy(), e.cpu().numpy()
+    G = cfg.G
+    for b, o in enumerate(oseqs):
+        P = cfg.pages(b)
+        for g in range(cfg.H_kv):
+            rm, rv, re = o.gauss(g)
+            sl = slice(g * G, (g + 1) * G)
+            assert np.array_equal(m[b, sl, :P], rm)
+            assert np.array_equal(v[b, sl, :P], rv)
+            assert np.array_equal(e[b, sl, :P], re)
+            assert np.all(e[b, sl, P:] == -np.inf)
+
+
+@pytest.mark.parametrize("alpha", [1.5, 2.0])
+@pytest.mark.parametrize("delta", [0.0, 0.5])
+def test_gauss_selection(alpha, delta):
+    wl = _wl(3, [8192 + 20, 4096 + 1])
+    cfg = wl.cfg
+    pool, seq_lens = build_pool(wl)
+    step = DecodeStep(pool, wl.page_table, seq_lens, cfg.H_q, "gauss", alpha=alpha, delta=delta)
+    step.score(wl.q)
+    step.choose()
+    step.check()
+    tau_gpu = step.tau_hat.cpu().numpy()
+    sel, cnt = step.sel.cpu().numpy(), step.sel_count.cpu().numpy()
+    G = cfg.G
+    for b in range(cfg.B):
+        o = H.OracleSeq(wl, b)
+        for g in range(cfg.H_kv):
+            ref = o.tau_hat(g, alpha)
+            got = tau_gpu[b, g * G:(g + 1) * G].astype(np.float64)
+            assert np.all(np.abs(got - ref) <= H.TAU_HAT_TOL * np.maximum(1.0, np.abs(ref))), (got, ref)
+            # the replica's keep rule with the oracle threshold: every decision
+            # outside the threshold's uncertainty band must match
+            _, _, est = o.gauss(g)
+            band = np.abs(got - ref) + 1e-6 * np.maximum(1.0, np.abs(ref))
+            margin = (alpha - 1.0) * est.astype(np.float64) - (ref[:, None] - delta)
+            must_keep = np.nonzero(np.any(margin > band[:, None], axis=0))[0]
+            must_drop = np.nonzero(np.all(margin < -band[:, None], axis=0))[0]
+            kept = set(sel[b, g, :cnt[b, g]].tolist())
+            assert set(must_keep.tolist()) <= kept
+            assert not (set(must_drop.tolist()) & kept)
+            assert list(sel[b, g, :cnt[b, g]]) == sorted(kept)
+
+
+def test_sparse_attend_against_oracle(built):
+    wl, pool, seq_lens, oseqs = built
+    cfg = wl.cfg
+    step = DecodeStep(pool, wl.page_table, seq_lens, cfg.H_q, "topk", budget_frac=1 / 16, alpha=cfg.alpha)
+    # selection from the oracle, handed to the GPU as input
+    sel = torch.zeros_like(step.sel)
+    cnt = torch.zeros_like(step.sel_count)
+    refs = {}
+    for b, o in enumerate(oseqs):
+        for g in range(cfg.H_kv):
+            pages = o.topk(g, -1, 1 / 16)
+            # add a few low-bound pages so the set is not only the best ones
+            P = cfg.pages(b)
+            extra = [p for p in range(0, P, 7) if p not in set(pages)][:3]
+            pages = np.array(sorted(set(pages.tolist()) | set(extra)))[:step.k_max]
+            sel[b, g, :len(pages)] = torch.from_numpy(pages.astype(np.int32))
+            cnt[b, g] = len(pages)
+            refs[b, g] = o.attention(g, pages, cfg.alpha)
+    st = _status()
+    out = torch.empty_like(step.out)
+    tau = torch.empty_like(step.tau)
+    B.sparse_attend(pool, wl.q, wl.page_table, seq_lens, sel, cnt, cfg.alpha, H.scale32(cfg), out,
+                    step.workspace, st, tau_out=tau)
+    _assert_ok(st)
+    out, tau = out.cpu().numpy(), tau.cpu().numpy()
+    G = cfg.G
+    for (b, g), (o_ref, t_ref) in refs.items():
+        H.compare_out(out[b, g * G:(g + 1) * G], o_ref, cfg.dtype)
+        assert np.all(np.abs(tau[b, g * G:(g + 1) * G] - t_ref) <= 1e-5 * np.maximum(1, np.abs(t_ref)))
+
+
+def test_decode_step_end_to_end(built):
+    """score -> select -> attend on the GPU against the oracle's own pipeline."""
+    wl, pool, seq_lens, oseqs = built
+    cfg = wl.cfg
+    step = DecodeStep(pool, wl.page_table, seq_lens, cfg.H_q, "topk", budget_frac=1 / 16, alpha=cfg.alpha)
+    step(wl.q)
+    step.check()
+    sel, cnt = step.sel.cpu().numpy(), step.sel_count.cpu().numpy()
+    out = step.out.cpu().numpy()
+    G = cfg.G
+    for b, o in enumerate(oseqs):
+        for g in range(cfg.H_kv):
+            pages = o.topk(g, -1, 1 / 16)
+            assert np.array_equal(sel[b, g, :cnt[b, g]], pages)
+            o_ref, _ = o.attention(g, pages, cfg.alpha)
+            H.compare_out(out[b, g * G:(g + 1) * G], o_ref, cfg.dtype)
+
+
+def test_full_entmax_and_softmax(built):
+    wl, pool, seq_lens, oseqs = built
+    cfg = wl.cfg
+    st = _status()
+    out = torch.empty(cfg.B, cfg.H_q, cfg.d, device="cuda")
+    tau = torch.empty(cfg.B, cfg.H_q, device="cuda")
+    ws = torch.empty(B.workspace_size(B.OP_FULL_ENTMAX, cfg.B, cfg.H_q, cfg.H_kv, wl.max_pages, 0, cfg.ps,
+                                      cfg.d), dtype=torch.uint8, device="cuda")
+    B.full_entmax_decode(pool, wl.q, wl.page_table, seq_lens, cfg.alpha, H.scale32(cfg), out, ws, st, tau_out=tau)
+    out_s = torch.empty_like(out)
+    ws_s = torch.empty(B.workspace_size(B.OP_FULL_SOFTMAX, cfg.B, cfg.H_q, cfg.H_kv, wl.max_pages, 0, cfg.ps,
+                                        cfg.d), dtype=torch.uint8, device="cuda")
+    B.full_softmax_decode(pool, wl.q, wl.page_table, seq_lens, H.scale32(cfg), out_s, ws_s, st)
+    _assert_ok(st)
+    out, out_s = out.cpu().numpy(), out_s.cpu().numpy()
+    G = cfg.G
+    for b, o in enumerate(oseqs):
+        P = cfg.pages(b)
+        for g in range(cfg.H_kv):
+            o_ref, _ = o.attention(g, np.arange(P), cfg.alpha)
+            H.compare_out(out[b, g * G:(g + 1) * G], o_ref, cfg.dtype)
+            s_ref = attend.softmax_attention(o.qgroup(g), o.keys[g], o.values[g], 1.0 / math.sqrt(cfg.d))
+            H.compare_out(out_s[b, g * G:(g + 1) * G], s_ref, cfg.dtype)
+
+
+def test_support_recovery_on_gpu():
+    """If the kept pages hold the support, sparse == full (oracle: bitwise)."""
+    wl = _wl(2, [8192 + 33])
+    cfg = wl.cfg
+    pool, seq_lens = build_pool(wl)
+    o = H.OracleSeq(wl, 0)
+    G = cfg.G
+    sel = torch.zeros(1, cfg.H_kv, wl.max_pages, dtype=torch.int32, device="cuda")
+    cnt = torch.zeros(1, cfg.H_kv, dtype=torch.int32, device="cuda")
+    for g in range(cfg.H_kv):
+        _, _, pm = attend.entmax_attention(o.qgroup(g), o.keys[g], o.values[g], cfg.alpha, 1 / math.sqrt(cfg.d))
+        sup_pages = set((np.nonzero(pm.sum(axis=0) > 0)[0] // cfg.ps).tolist())
+        pages = sorted(sup_pages | {0, cfg.pages(0) - 1})
+        sel[0, g, :len(pages)] = torch.tensor(pages, dtype=torch.int32)
+        cnt[0, g] = len(pages)
+    st = _status()
+    ws = torch.empty(B.workspace_size(B.OP_SPARSE_ATTEND, 1, cfg.H_q, cfg.H_kv, wl.max_pages, wl.max_pages,
+                                      cfg.ps, cfg.d), dtype=torch.uint8, device="cuda")
+    out = torch.empty(1, cfg.H_q, cfg.d, device="cuda")
+    B.sparse_attend(pool, wl.q, wl.page_table, seq_lens, sel, cnt, cfg.alpha, H.scale32(cfg), out, ws, st)
+    wsf = torch.empty(B.workspace_size(B.OP_FULL_ENTMAX, 1, cfg.H_q, cfg.H_kv, wl.max_pages, 0, cfg.ps, cfg.d),
+                      dtype=torch.uint8, device="cuda")
+    full = torch.empty_like(out)
+    B.full_entmax_decode(pool, wl.q, wl.page_table, seq_lens, cfg.alpha, H.scale32(cfg), full, wsf, st)
+    _assert_ok(st)
+    for g in range(cfg.H_kv):
+        pages = sel[0, g, :cnt[0, g]].cpu().numpy()
+        o_sp, _ = o.attention(g, pages, cfg.alpha)
+        o_full, _ = o.attention(g, np.arange(cfg.pages(0)), cfg.alpha)
+        assert np.array_equal(o_sp, o_full)            # oracle: exact
+    assert torch.allclose(out, full, rtol=0, atol=H.BF16_ATOL)
+
+
+def test_edge_cases_empty_sequence_and_full_budget():
+    wl = _wl(2, [0, 64 * 5 + 1, 64])
+    cfg = wl.cfg
+    pool, seq_lens = build_pool(wl)
+    step = DecodeStep(pool, wl.page_table, seq_lens, cfg.H_q, "topk", budget=1000 if wl.max_pages >= 1000 else
+                      wl.max_pages, alpha=cfg.alpha)
+    step(wl.q)
+    step.check()
+    cnt = step.sel_count.cpu().numpy()
+    assert np.all(cnt[0] == 0)
+    assert np.all(cnt[1] == 6) and np.all(cnt[2] == 1)
+    out, tau = step.out.cpu().numpy(), step.tau.cpu().numpy()
+    assert np.all(out[0] == 0) and np.all(np.isinf(tau[0]))
+    for b in (1, 2):
+        o = H.OracleSeq(wl, b)
+        for g in range(cfg.H_kv):
+            o_ref, _ = o.attention(g, np.arange(cfg.pages(b)), cfg.alpha)
+            H.compare_out(out[b, g * cfg.G:(g + 1) * cfg.G], o_ref, cfg.dtype)
+
+
+def test_bad_page_id_reports_bounds():
+    wl = _wl(2, [1000])
+    pool, seq_lens = build_pool(wl)
+    pt = wl.page_table.clone()
+    pt[0, 3] = wl.num_phys + 11
+    st = _status()
+    ub = torch.empty(1, wl.cfg.H_kv, wl.max_pages, device="cuda")
+    B.score_pages(pool, wl.q, pt, seq_lens, B.SCORE_BBOX, H.scale32(wl.cfg), st, ub=ub)
+    torch.cuda.synchronize()
+    assert int(st.item()) == B.DEVICE_BOUNDS
+
+
+def test_host_validation_rejects_bad_arguments():
+    wl = _wl(2, [100])
+    pool, seq_lens = build_pool(wl)
+    st = _status()
+    out = torch.empty(1, wl.cfg.H_q, wl.cfg.d, device="cuda")
+    small = torch.empty(16, dtype=torch.uint8, device="cuda")
+    with pytest.raises(B.EntmaxKVError) as e:
+        B.full_entmax_decode(pool, wl.q, wl.page_table, seq_lens, 1.5, 0.1, out, small, st)
+    assert e.value.code == B.WORKSPACE
+    with pytest.raises(B.EntmaxKVError) as e:
+        B.full_entmax_decode(pool, wl.q, wl.page_table, seq_lens, 3.0, 0.1, out, small, st)
+    assert e.value.code == B.UNSUPPORTED
+
+
+def test_bounded_wait_times_out_and_context_survives():
+    st = _status()
+    B.selftest_timeout(2_000_000, st)     # 2 ms
+    torch.cuda.synchronize()
+    assert int(st.item()) == B.TIMEOUT
+    x = torch.arange(10, device="cuda").sum()
+    assert int(x.item()) == 45
+
+
+def test_decode_appends_then_step():
+    """Config 5 shape: ragged batch, permuted pages, one token appended per step."""
+    wl = _wl(5, [3000, 700, 64 * 9])
+    cfg = wl.cfg
+    pool, seq_lens = build_pool(wl)
+    step = DecodeStep(pool, wl.page_table, seq_lens, cfg.H_q, "topk", budget_frac=1 / 16, alpha=cfg.alpha)
+    toks = []
+    for t in range(3):
+        k, v, q = wl.decode_token(t)
+        step(q, k, v)
+        toks.append((k, v, q))
+    step.check()
+    lens = [L + 3 for L in cfg.lengths]
+    assert seq_lens.cpu().tolist() == lens
+    out = step.out.cpu().numpy()
+    q_last = toks[-1][2].cpu().numpy()
+    G = cfg.G
+    for b in range(cfg.B):
+        keys, vals = H.host_sequence(wl, b)
+        keys = np.concatenate([keys] + [t[0][b].float().cpu().numpy() for t in toks], axis=1)
+        vals = np.concatenate([vals] + [t[1][b].float().cpu().numpy() for t in toks], axis=1)
+        from oracle import replica
+        for g in range(cfg.H_kv):
+            meta = replica.page_meta(keys[g], cfg.ps)
+            qg = q_last[b, g * G:(g + 1) * G]
+            _, ubg = replica.bound(qg, meta["kmin"], meta["kmax"], H.scale32(cfg))
+            P = (lens[b] + cfg.ps - 1) // cfg.ps
+            pages = select.topk(ubg, select.budget_pages(P, -1, 1 / 16))
+            tok = attend.token_indices(pages, lens[b], cfg.ps)
+            o_ref, _, _ = attend.entmax_attention(qg, keys[g][tok], vals[g][tok], cfg.alpha, 1 / math.sqrt(cfg.d))
+            H.compare_out(out[b, g * G:(g + 1) * G], o_ref, cfg.dtype)
