@@ -1,0 +1,457 @@
+"""Benchmark: one EntmaxKV decode step at 1M-token context on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+
+A step is the whole decode path on one batch: append the step's token (KV
+write + page metadata), score every page (bounding-box bound), select the top
+1/64 of pages per kv head, and run exact 1.5-entmax attention over the
+selected pages.  Workload: B=1 sequence of 2^20 tokens per GPU, 32 query / 8
+kv heads, head dim 128, pages of 64, bf16 cache (synthetic clustered keys with
+planted tokens).  L2 is flushed (a 256 MiB write) between timed steps, outside
+the per-step CUDA events.  Rank 0 prints one JSON line.
+
+--impl reference times the CPU oracle on the host cores instead (rank 0 only).
+"""
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "sparse entmax decode µs/step @1M ctx; achieved HBM GB/s vs 8 TB/s roofline"
+HBM_NOMINAL_GBS = 8000.0
+PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
+FALLBACK_HBM_GBS = 6650.0
+MiB = 1 << 20
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="native", choices=["native", "reference"])
+    ap.add_argument("--context", type=int, default=1 << 20, help="tokens per sequence (default 2^20)")
+    ap.add_argument("--no-baselines", action="store_true", help="skip the full-cache and Gaussian timings")
+    ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline leg")
+    return ap.parse_args()
+
+
+def hbm_peak():
+    try:
+        with open(PEAKS_FILE) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+# ---------------------------------------------------------------- distributed
+def dist_init(n):
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=torch.device("cuda", local))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(0)
+    return rank, world, local
+
+
+def barrier(world):
+    if world > 1:
+        torch.distributed.barrier()
+
+
+def max_over_ranks(x, world):
+    if world == 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ---------------------------------------------------------------- clocks
+class Clocks:
+    """nvidia-smi samples of SM clock and throttle reasons while running."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index):
+        self.dev = device_index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.dev), "--query-gpu=" + self.FIELDS, "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        self.lines = []
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except Exception:
+                self.proc.kill()
+                out = ""
+            self.lines = [l for l in out.splitlines() if l.strip()]
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for l in getattr(self, "lines", []):
+            f = [x.strip() for x in l.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = float(f[2])
+            except ValueError:
+                continue
+            for name, val in zip(names, f[5:9]):
+                if val.lower() == "active":
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ---------------------------------------------------------------- workload
+def make_workload(context, rank):
+    import dataclasses
+    from sparse_long_context_min_b200 import workloads
+    cfg = workloads.config(4)
+    cfg = dataclasses.replace(cfg, lengths=[context], seed=cfg.seed + 100 * rank, decode_steps=256)
+    return workloads.Workload(cfg, device="cuda")
+
+
+def algorithmic_bytes(cfg, k_pages, v_pages, mode):
+    """Bytes one step must move: metadata of every page, keys of the selected
+    pages, values of the selected pages that hold weight, the appended token
+    with its metadata row, the page table and the outputs."""
+    d, ps, Hkv, Hq, B = cfg.d, cfg.ps, cfg.H_kv, cfg.H_q, cfg.B
+    P = sum(cfg.pages(b) for b in range(B))
+    elt = 2 if cfg.dtype == torch.bfloat16 else 4
+    if mode == "topk":
+        meta = P * Hkv * d * 2 * elt + B * Hkv * P * 4            # kmin, kmax read; ub written
+    else:
+        meta = P * Hkv * d * 2 * 4 + 3 * B * Hq * P * 4           # mean, m2 read; m, v, est written
+    kv = (k_pages + v_pages) * ps * d * elt                       # K of selected, V of weighted pages
+    append = B * Hkv * d * (2 * elt + 2 * (2 * elt + 2 * 4))      # token write + metadata row r/w
+    table = B * P * 4
+    out = B * Hq * d * 4
+    return {"score": meta + table, "attend": kv, "total": meta + kv + append + table + out}
+
+
+def score_bytes(cfg, mode):
+    return algorithmic_bytes(cfg, 0, 0, mode)["score"]
+
+
+# ---------------------------------------------------------------- native arm
+def run_native(args, rank, world, local):
+    import numpy as np
+    from sparse_long_context_min_b200 import binding as BND
+    from sparse_long_context_min_b200.step import DecodeStep, GraphedStep, build_pool
+
+    torch.manual_seed(0)
+    wl = make_workload(args.context, rank)
+    cfg = wl.cfg
+    pool, seq_lens = build_pool(wl)
+    torch.cuda.synchronize()
+    stream = torch.cuda.current_stream()
+    flush = torch.empty(256 * MiB, dtype=torch.uint8, device="cuda")
+    K, W = args.steps, args.warmup
+    total_steps = W + K
+
+    def one_mode(mode, budget_frac=1 / 64, delta=0.5, steps=None, warm=None):
+        """K graphed steps; returns per-step us, mean stage us, mean selected
+        and loaded-value page-heads per step."""
+        steps = K if steps is None else steps
+        warm = W if warm is None else warm
+        st = DecodeStep(pool, wl.page_table, seq_lens, cfg.H_q, mode, budget_frac=budget_frac, alpha=cfg.alpha,
+                        delta=delta)
+        gs = GraphedStep(st, append=True, stage_events=True)
+        toks = [wl.decode_token(i) for i in range(warm + steps)]
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        step_us, stages, sel, vp = [], [], [], []
+        for i in range(warm + steps):
+            k, v, q = toks[i]
+            gs.q.copy_(q)
+            gs.k.copy_(k)
+            gs.v.copy_(v)
+            st.v_pages.zero_()
+            flush.fill_(i & 0xFF)
+            e0.record(stream)
+            gs.replay()
+            e1.record(stream)
+            torch.cuda.synchronize()
+            if i >= warm:
+                step_us.append(e0.elapsed_time(e1) * 1e3)
+                stages.append(gs.stage_us())
+                sel.append(int(st.sel_count.sum().item()))
+                vp.append(int(st.v_pages.sum().item()))
+        st.check()
+        stage = {n: statistics.mean(x[n] for x in stages) for n in GraphedStep.STAGES} if stages[0] else {}
+        return step_us, stage, statistics.mean(sel), statistics.mean(vp)
+
+    # ---- headline: top-k 1/64, timed K steps bracketed by barrier + sync
+    clocks = Clocks(local)
+    barrier(world)
+    torch.cuda.synchronize()
+    with clocks:
+        step_us, stage, sel_total, v_total = one_mode("topk")
+    torch.cuda.synchronize()
+    barrier(world)
+    mean_us = statistics.mean(step_us)
+    mean_us_all = max_over_ranks(mean_us, world)
+    score_us = max_over_ranks(stage["score"], world)
+    by = algorithmic_bytes(cfg, sel_total, v_total, "topk")
+    peak, peak_kind = hbm_peak()
+
+    # ---- e2e through the C ABI with host buffers (copies inside the timed region)
+    e2e_us, h2d, d2h = run_e2e(wl, pool, seq_lens, K, W, flush)
+    e2e_us = max_over_ranks(e2e_us, world)
+
+    extra = {}
+    if not args.no_baselines:
+        g_us, g_stage, g_sel, g_v = one_mode("gauss", steps=max(3, K // 4), warm=3)
+        extra["gauss_value_pages"] = round(g_v, 1)
+        extra["gauss_us_per_step"] = round(max_over_ranks(statistics.mean(g_us), world), 2)
+        extra["gauss_selected_pages"] = round(g_sel, 1)
+        extra["gauss_stage_us"] = {k: round(v, 2) for k, v in g_stage.items()}
+        fe, fs = run_full(wl, pool, seq_lens, flush)
+        fe, fs = max_over_ranks(fe, world), max_over_ranks(fs, world)
+        extra["full_entmax_us"] = round(fe, 1)
+        extra["full_softmax_us"] = round(fs, 1)
+        extra["topk_speedup_vs_full_entmax"] = round(fe / mean_us_all, 2)
+        extra["topk_speedup_vs_full_softmax"] = round(fs / mean_us_all, 2)
+        extra["gauss_speedup_vs_full_entmax"] = round(fe / extra["gauss_us_per_step"], 2)
+        extra["gauss_speedup_vs_full_softmax"] = round(fs / extra["gauss_us_per_step"], 2)
+
+    cpu = None
+    if rank == 0 and not args.no_cpu:
+        cpu = cpu_baseline(wl, pool, budget_frac=1 / 64, seconds=8.0)
+
+    n_launch = 7   # append + advance, score, select, qk + tau + pv (one graph replay)
+    step_gbs = by["total"] / (mean_us_all * 1e-6) / 1e9
+    score_gbs = by["score"] / (score_us * 1e-6) / 1e9
+    clk = clocks.summary()
+    line = {
+        "metric": METRIC,
+        "value": round(mean_us_all, 2),
+        "unit": "us/step",
+        "n_gpus": world,
+        "steps": K,
+        "warmup": W,
+        "ms_per_step": round(mean_us_all / 1e3, 5),
+        "higher_is_better": False,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic (seeded clustered-page keys, planted tokens; no dataset)",
+        "config": {
+            "workload": "million-token decode: B=1 x 2^20 tokens per GPU, 32/8 heads, d=128, page 64, bf16 KV, "
+                        "alpha=1.5, top-k 1/64 of pages (256), append 1 token per step",
+            "global_batch": world,
+            "seq_len": cfg.lengths[0],
+            "parallelism": "replicas: one independent sequence per GPU" if world > 1 else "single GPU",
+            "l2": "flushed between steps (256 MiB write outside the step events)",
+            "selected_pages_per_step": round(sel_total, 1),
+            "value_pages_loaded_per_step": round(v_total, 1),
+            "algorithmic_bytes_per_step": by["total"],
+            "achieved_gbs_step": round(step_gbs, 1),
+            "frac_of_8tbs": round(step_gbs / HBM_NOMINAL_GBS, 4),
+            "frac_of_measured_hbm": round(step_gbs / peak, 4),
+            "stage_us": {k: round(v, 2) for k, v in stage.items()},
+            **extra,
+        },
+        "roofline": {
+            "kernel": "score_bbox_kernel (entmaxkv_score_pages, bbox)",
+            "bound": "hbm",
+            "achieved": round(score_gbs, 1),
+            "peak": peak,
+            "peak_kind": peak_kind,
+            "unit": "GB/s",
+            "frac": round(score_gbs / peak, 4),
+            "traffic": None,
+            "bytes_per_launch": by["score"],
+        },
+        "e2e": {"value": round(e2e_us, 2), "unit": "us/step", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h},
+        "gpu_launches": n_launch * K,
+        "clocks": clk,
+    }
+    if cpu is not None:
+        line["cpu_baseline"] = cpu
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+def run_e2e(wl, pool, seq_lens, K, W, flush):
+    """Same step through the public API (the graphed step) with the step's
+    inputs in pinned host memory: H2D of q and the new token and D2H of the
+    output inside the events."""
+    from sparse_long_context_min_b200.step import DecodeStep, GraphedStep
+    cfg = wl.cfg
+    stream = torch.cuda.current_stream()
+    st = DecodeStep(pool, wl.page_table, seq_lens, cfg.H_q, "topk", budget_frac=1 / 64, alpha=cfg.alpha)
+    gs = GraphedStep(st, append=True, stage_events=False)
+    host = []
+    for i in range(W + K):
+        k, v, q = wl.decode_token(10_000 + i)
+        host.append((k.cpu().pin_memory(), v.cpu().pin_memory(), q.cpu().pin_memory()))
+    out_h = torch.empty(st.out.shape, dtype=st.out.dtype).pin_memory()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    for i in range(W + K):
+        flush.fill_(i & 0xFF)
+        j = i - W
+        if j >= 0:
+            ev[j][0].record(stream)
+        k, v, q = host[i]
+        gs.k.copy_(k, non_blocking=True)
+        gs.v.copy_(v, non_blocking=True)
+        gs.q.copy_(q, non_blocking=True)
+        gs.replay()
+        out_h.copy_(st.out, non_blocking=True)
+        if j >= 0:
+            ev[j][1].record(stream)
+    torch.cuda.synchronize()
+    st.check()
+    us = statistics.mean(a.elapsed_time(b) * 1e3 for a, b in ev)
+    h2d = sum(t.numel() * t.element_size() for t in host[0])
+    d2h = out_h.numel() * out_h.element_size()
+    return us, h2d, d2h
+
+
+def run_full(wl, pool, seq_lens, flush, reps=5, warm=3):
+    """Full-cache entmax and softmax decode over every page (the baselines)."""
+    from sparse_long_context_min_b200 import binding as BND
+    cfg = wl.cfg
+    stream = torch.cuda.current_stream()
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    out = torch.empty(cfg.B, cfg.H_q, cfg.d, device="cuda")
+    res = []
+    for op in (BND.OP_FULL_ENTMAX, BND.OP_FULL_SOFTMAX):
+        ws = torch.empty(BND.workspace_size(op, cfg.B, cfg.H_q, cfg.H_kv, wl.max_pages, 0, cfg.ps, cfg.d),
+                         dtype=torch.uint8, device="cuda")
+        times = []
+        for i in range(warm + reps):
+            flush.fill_(i & 0xFF)
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            if op == BND.OP_FULL_ENTMAX:
+                BND.full_entmax_decode(pool, wl.q, wl.page_table, seq_lens, cfg.alpha, cfg.scale, out, ws, st)
+            else:
+                BND.full_softmax_decode(pool, wl.q, wl.page_table, seq_lens, cfg.scale, out, ws, st)
+            b.record(stream)
+            if i >= warm:
+                times.append((a, b))
+        torch.cuda.synchronize()
+        if int(st.item()):
+            raise BND.EntmaxKVError(int(st.item()), "full-cache baseline")
+        res.append(statistics.mean(a.elapsed_time(b) * 1e3 for a, b in times))
+        del ws
+    return res[0], res[1]
+
+
+# ---------------------------------------------------------------- oracle timing
+def oracle_sample(wl, g, budget_frac, meta, keys, vals):
+    """The oracle's sparse step for kv head g: replica bounds, top-k, entmax attention."""
+    from oracle import attend, replica, select
+    cfg = wl.cfg
+    qg = wl.q[0, g * cfg.G:(g + 1) * cfg.G].cpu().numpy()
+    _, ubg = replica.bound(qg, meta["kmin"], meta["kmax"], float(torch.tensor(cfg.scale, dtype=torch.float32)))
+    pages = select.topk(ubg, select.budget_pages(len(ubg), -1, budget_frac))
+    tok = attend.token_indices(pages, cfg.lengths[0], cfg.ps)
+    o, tau, _ = attend.entmax_attention(qg, keys[tok], vals[tok], cfg.alpha, 1.0 / math.sqrt(cfg.d))
+    return o
+
+
+def cpu_baseline(wl, pool, budget_frac, seconds):
+    """Time the oracle (as it stands) on the host cores: one kv head's share of
+    the sparse step, repeated for about `seconds`, scaled to the 8 heads."""
+    from oracle import replica
+    cfg = wl.cfg
+    keys, vals = wl.sequence(0, heads=[0])
+    keys = keys[0].float().cpu().numpy()
+    vals = vals[0].float().cpu().numpy()
+    meta = replica.page_meta(keys, cfg.ps)          # metadata exists before a decode step
+    t0 = time.perf_counter()
+    n = 0
+    while True:
+        oracle_sample(wl, 0, budget_frac, meta, keys, vals)
+        n += 1
+        if time.perf_counter() - t0 > seconds:
+            break
+    per_head = (time.perf_counter() - t0) / n
+    us = per_head * cfg.H_kv * 1e6
+    return {"value": round(us, 1), "unit": "us/step", "cores": 1, "kind": "oracle",
+            "sample": "kv head 0 of 8 (4 query heads): replica bounds over all 16384 pages, top-k, float64 "
+                      "entmax attention over the 256 kept pages; %d repetitions, scaled x8 to a full step" % n}
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return
+    if torch.cuda.is_available():
+        torch.cuda.set_device(0)
+    wl = make_workload(args.context, 0)
+    from oracle import replica
+    cfg = wl.cfg
+    keys, vals = wl.sequence(0, heads=[0])
+    keys = keys[0].float().cpu().numpy()
+    vals = vals[0].float().cpu().numpy()
+    meta = replica.page_meta(keys, cfg.ps)
+    for _ in range(args.warmup):
+        oracle_sample(wl, 0, 1 / 64, meta, keys, vals)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        oracle_sample(wl, 0, 1 / 64, meta, keys, vals)
+    per = (time.perf_counter() - t0) / args.steps * cfg.H_kv * 1e6
+    sample = ("kv head 0 of 8 per step (replica bounds over all pages, top-k, float64 entmax attention over "
+              "the kept pages), scaled x8")
+    line = {"metric": METRIC, "value": round(per, 1), "unit": "us/step", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": round(per / 1e3, 3), "higher_is_better": False,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": "million-token decode: B=1 x 2^20 tokens, 32/8 heads, d=128, page 64, "
+                                   "alpha=1.5, top-k 1/64", "seq_len": cfg.lengths[0]},
+            "impl": "reference",
+            "cpu_baseline": {"value": round(per, 1), "unit": "us/step", "cores": 1, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": round(per, 1), "unit": "us/step", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse()
+    rank, world, local = dist_init(args.gpus)
+    try:
+        if args.impl == "reference":
+            run_reference(args, rank, world)
+        else:
+            run_native(args, rank, world, local)
+    finally:
+        if world > 1:
+            torch.distributed.barrier()
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -177,24 +177,31 @@ ENTMAXKV_API int entmaxkv_select(int32_t mode, const float* ub, const float* m, 
  *   so that sum_i [x_i - tau]_+^(1/(alpha-1)) = 1, out[b][h] = sum_i p_i v_i.
  *   out [B][H_q][d] fp32; tau_out [B][H_q] fp32 (may be NULL).  A head with
  *   no valid token gets out = 0 and tau = +INFINITY.
+ *   Value rows are loaded only for pages holding a token with p > 0 for some
+ *   head of the group (the weights are exactly zero elsewhere, German summary
+ *   section 3: tokens outside the support carry no mass).  v_pages
+ *   [B][H_kv] int32 (may be NULL): the number of value pages loaded is ADDED
+ *   to it (the caller zeroes it).
  *   workspace: entmaxkv_workspace_size(ENTMAXKV_OP_SPARSE_ATTEND, ...) bytes.
  */
 ENTMAXKV_API int entmaxkv_sparse_attend(const entmaxkv_pool* pool, const float* q, int32_t H_q,
                            const int32_t* page_table, int32_t max_pages, const int32_t* seq_lens,
                            int32_t B, const int32_t* sel, const int32_t* sel_count, int32_t k_max,
-                           float alpha, float scale, float* out, float* tau_out, void* workspace,
-                           size_t ws_bytes, int32_t* status, void* stream);
+                           float alpha, float scale, float* out, float* tau_out, int32_t* v_pages,
+                           void* workspace, size_t ws_bytes, int32_t* status, void* stream);
 
 /*
  * Full-cache alpha-entmax decode: entmaxkv_sparse_attend over every page of
  * every sequence (German summary, section 4: the full-cache entmax decoding
- * baseline).  workspace: ENTMAXKV_OP_FULL_ENTMAX.
+ * baseline).  Every key is read; value pages are read where they hold weight,
+ * as in entmaxkv_sparse_attend (v_pages likewise, may be NULL).
+ * workspace: ENTMAXKV_OP_FULL_ENTMAX.
  */
 ENTMAXKV_API int entmaxkv_full_entmax_decode(const entmaxkv_pool* pool, const float* q, int32_t H_q,
                                 const int32_t* page_table, int32_t max_pages,
                                 const int32_t* seq_lens, int32_t B, float alpha, float scale,
-                                float* out, float* tau_out, void* workspace, size_t ws_bytes,
-                                int32_t* status, void* stream);
+                                float* out, float* tau_out, int32_t* v_pages, void* workspace,
+                                size_t ws_bytes, int32_t* status, void* stream);
 
 /*
  * Full-cache softmax decode, split over the cache with a log-sum-exp merge

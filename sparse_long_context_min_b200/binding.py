@@ -58,8 +58,8 @@ def lib():
         L.entmaxkv_append_metadata.argtypes = [PP, P, P, I, P, I, P, I, P, P]
         L.entmaxkv_score_pages.argtypes = [PP, P, I, P, I, P, I, I, F, P, P, P, P, P, P]
         L.entmaxkv_select.argtypes = [I, P, P, P, P, P, I, I, I, I, I, I, F, F, F, I, P, P, P, P, S, P, P]
-        L.entmaxkv_sparse_attend.argtypes = [PP, P, I, P, I, P, I, P, P, I, F, F, P, P, P, S, P, P]
-        L.entmaxkv_full_entmax_decode.argtypes = [PP, P, I, P, I, P, I, F, F, P, P, P, S, P, P]
+        L.entmaxkv_sparse_attend.argtypes = [PP, P, I, P, I, P, I, P, P, I, F, F, P, P, P, P, S, P, P]
+        L.entmaxkv_full_entmax_decode.argtypes = [PP, P, I, P, I, P, I, F, F, P, P, P, P, S, P, P]
         L.entmaxkv_full_softmax_decode.argtypes = [PP, P, I, P, I, P, I, F, P, P, S, P, P]
         L.entmaxkv_workspace_size.argtypes = [I, I, I, I, I, I, I, I]
         L.entmaxkv_workspace_size.restype = ctypes.c_size_t
@@ -153,20 +153,20 @@ def workspace_size(op, B, H_q, H_kv, max_pages, k_max, ps, d):
 
 
 def sparse_attend(pool, q, page_table, seq_lens, sel, sel_count, alpha, scale, out, workspace, status,
-                  tau_out=None, stream=None):
+                  tau_out=None, v_pages=None, stream=None):
     B, H_q, _ = q.shape
     _check(lib().entmaxkv_sparse_attend(pool.c, _p(q), H_q, _p(page_table), page_table.shape[1],
                                         _p(seq_lens), B, _p(sel), _p(sel_count), sel.shape[2], alpha,
-                                        scale, _p(out), _p(tau_out), _p(workspace),
+                                        scale, _p(out), _p(tau_out), _p(v_pages), _p(workspace),
                                         workspace.numel() * workspace.element_size(), _p(status),
                                         _stream(stream)), "sparse_attend")
 
 
 def full_entmax_decode(pool, q, page_table, seq_lens, alpha, scale, out, workspace, status,
-                       tau_out=None, stream=None):
+                       tau_out=None, v_pages=None, stream=None):
     B, H_q, _ = q.shape
     _check(lib().entmaxkv_full_entmax_decode(pool.c, _p(q), H_q, _p(page_table), page_table.shape[1],
-                                             _p(seq_lens), B, alpha, scale, _p(out), _p(tau_out),
+                                             _p(seq_lens), B, alpha, scale, _p(out), _p(tau_out), _p(v_pages),
                                              _p(workspace), workspace.numel() * workspace.element_size(),
                                              _p(status), _stream(stream)), "full_entmax_decode")
 

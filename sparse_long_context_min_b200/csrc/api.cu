@@ -117,7 +117,7 @@ static int num_splits(int B, int H_kv, int list_pages)
 
 struct AttnLayout {
     int S;
-    size_t xbuf, opart, mlpart, tau, counters, total;
+    size_t xbuf, opart, mlpart, lmax, tau, counters, total;
 };
 
 static AttnLayout attn_layout(int op, int B, int H_q, int H_kv, int max_pages, int k_max, int ps, int d)
@@ -132,6 +132,8 @@ static AttnLayout attn_layout(int op, int B, int H_q, int H_kv, int max_pages, i
     off += round256((size_t)B * H_q * L.S * d * sizeof(float));
     L.mlpart = off;
     if (op == ENTMAXKV_OP_FULL_SOFTMAX) off += round256((size_t)B * H_q * L.S * 2 * sizeof(float));
+    L.lmax = off;
+    if (op != ENTMAXKV_OP_FULL_SOFTMAX) off += round256((size_t)B * H_q * L.S * sizeof(float));
     L.tau = off;
     off += round256((size_t)B * H_q * sizeof(float));
     L.counters = off;
@@ -143,7 +145,8 @@ static AttnLayout attn_layout(int op, int B, int H_q, int H_kv, int max_pages, i
 static int attend_common(int op, const entmaxkv_pool* pool, const float* q, int H_q, const int32_t* page_table,
                          int max_pages, const int32_t* seq_lens, int B, const int32_t* sel,
                          const int32_t* sel_count, int k_max, float alpha, float scale, float* out,
-                         float* tau_out, void* workspace, size_t ws_bytes, int32_t* status, void* stream)
+                         float* tau_out, int32_t* v_pages, void* workspace, size_t ws_bytes, int32_t* status,
+                         void* stream)
 {
     int rc = check_pool(pool, true, false);
     if (rc) return rc;
@@ -176,6 +179,8 @@ static int attend_common(int op, const entmaxkv_pool* pool, const float* q, int 
     a.xbuf = reinterpret_cast<float*>(ws + lay.xbuf);
     a.opart = reinterpret_cast<float*>(ws + lay.opart);
     a.mlpart = reinterpret_cast<float*>(ws + lay.mlpart);
+    a.lmax = reinterpret_cast<float*>(ws + lay.lmax);
+    a.vpages = v_pages;
     a.tau = reinterpret_cast<float*>(ws + lay.tau);
     a.counters = reinterpret_cast<int32_t*>(ws + lay.counters);
     a.out = out;
@@ -266,19 +271,22 @@ int entmaxkv_select(int32_t mode, const float* ub, const float* m, const float* 
 int entmaxkv_sparse_attend(const entmaxkv_pool* pool, const float* q, int32_t H_q, const int32_t* page_table,
                            int32_t max_pages, const int32_t* seq_lens, int32_t B, const int32_t* sel,
                            const int32_t* sel_count, int32_t k_max, float alpha, float scale, float* out,
-                           float* tau_out, void* workspace, size_t ws_bytes, int32_t* status, void* stream)
+                           float* tau_out, int32_t* v_pages, void* workspace, size_t ws_bytes, int32_t* status,
+                           void* stream)
 {
     return attend_common(ENTMAXKV_OP_SPARSE_ATTEND, pool, q, H_q, page_table, max_pages, seq_lens, B, sel,
-                         sel_count, k_max, alpha, scale, out, tau_out, workspace, ws_bytes, status, stream);
+                         sel_count, k_max, alpha, scale, out, tau_out, v_pages, workspace, ws_bytes, status,
+                         stream);
 }
 
 int entmaxkv_full_entmax_decode(const entmaxkv_pool* pool, const float* q, int32_t H_q,
                                 const int32_t* page_table, int32_t max_pages, const int32_t* seq_lens, int32_t B,
-                                float alpha, float scale, float* out, float* tau_out, void* workspace,
-                                size_t ws_bytes, int32_t* status, void* stream)
+                                float alpha, float scale, float* out, float* tau_out, int32_t* v_pages,
+                                void* workspace, size_t ws_bytes, int32_t* status, void* stream)
 {
     return attend_common(ENTMAXKV_OP_FULL_ENTMAX, pool, q, H_q, page_table, max_pages, seq_lens, B, nullptr,
-                         nullptr, max_pages, alpha, scale, out, tau_out, workspace, ws_bytes, status, stream);
+                         nullptr, max_pages, alpha, scale, out, tau_out, v_pages, workspace, ws_bytes, status,
+                         stream);
 }
 
 int entmaxkv_full_softmax_decode(const entmaxkv_pool* pool, const float* q, int32_t H_q,
@@ -287,7 +295,8 @@ int entmaxkv_full_softmax_decode(const entmaxkv_pool* pool, const float* q, int3
                                  void* stream)
 {
     return attend_common(ENTMAXKV_OP_FULL_SOFTMAX, pool, q, H_q, page_table, max_pages, seq_lens, B, nullptr,
-                         nullptr, max_pages, 1.5f, scale, out, nullptr, workspace, ws_bytes, status, stream);
+                         nullptr, max_pages, 1.5f, scale, out, nullptr, nullptr, workspace, ws_bytes, status,
+                         stream);
 }
 
 size_t entmaxkv_workspace_size(int32_t op, int32_t B, int32_t H_q, int32_t H_kv, int32_t max_pages, int32_t k_max,

@@ -165,6 +165,32 @@ EKV_DEV void zero_invalid_rows(const AttnArgs& a, uint8_t* stage, int b, int g, 
 }
 
 // ====================================================================== K pass
+// Per-head maximum over lanes with equal (lane & 3): xor over lane bits 2..4.
+EKV_DEV float group_lane_max(float v)
+{
+    v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 4));
+    v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 8));
+    v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 16));
+    return v;
+}
+
+// Write this split's maximum score of every head of the group (all threads
+// call; `wm` is shared [4][8]).
+EKV_DEV void write_split_max(const AttnArgs& a, int b, int g, int s, const float* run, int NT, float (*wm)[8])
+{
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, c = lane & 3;
+    for (int nt = 0; nt < NT; ++nt) {
+        const float m = group_lane_max(run[nt]);
+        if (lane < 4) wm[warp][4 * nt + c] = m;
+    }
+    __syncthreads();
+    if (threadIdx.x < a.G) {
+        const int h = threadIdx.x;
+        const float m = fmaxf(fmaxf(wm[0][h], wm[1][h]), fmaxf(wm[2][h], wm[3][h]));
+        a.lmax[((size_t)b * a.H_q + (size_t)g * a.G + h) * a.S + s] = m;
+    }
+}
+
 template <int D, int PS, int NT>
 __global__ void __launch_bounds__(kThreads) qk_bf16_kernel(const __grid_constant__ CUtensorMap kmap, const AttnArgs a)
 {
@@ -175,6 +201,7 @@ __global__ void __launch_bounds__(kThreads) qk_bf16_kernel(const __grid_constant
     uint8_t* smem = align1024(smem_raw);
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kStagesQK * STAGE);
     __shared__ int abort_flag;
+    __shared__ float wm[4][8];
 
     const int b = blockIdx.z, g = blockIdx.y, s = blockIdx.x;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -183,22 +210,29 @@ __global__ void __launch_bounds__(kThreads) qk_bf16_kernel(const __grid_constant
     const int cnt = list_count(a, b, g, P);
     if (s == 0 && tid == 0) a.counters[(size_t)b * a.H_kv + g] = 0;
     const Range r = split_range(cnt, a.S, s);
-    if (r.end <= r.start) return;
-    const int nst = (r.end - r.start + PPS - 1) / PPS;
+    const int nst = r.end > r.start ? (r.end - r.start + PPS - 1) / PPS : 0;
 
+    // start the key loads first; the query fragments are prepared meanwhile
+    if (tid == 0) {
+        abort_flag = 0;
+        if (nst > 0) {
+            prefetch_tmap(&kmap);
+            for (int i = 0; i < kStagesQK; ++i) mbar_init(&bars[i], 1);
+            fence_mbar_init();
+            for (int st = 0; st < min(kStagesQK, nst); ++st)
+                issue_stage<D, PS>(a, &kmap, smem + st * STAGE, &bars[st], b, g, r, st, P);
+        }
+    }
+    float run[NT];
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) run[nt] = -INFINITY;
+    if (nst == 0) {
+        write_split_max(a, b, g, s, run, NT, wm);
+        return;
+    }
     uint32_t bq[NT][KS][2];
     load_q_frags<D, NT>(a, b, g, a.xscale, bq);
-
-    if (tid == 0) {
-        prefetch_tmap(&kmap);
-        for (int i = 0; i < kStagesQK; ++i) mbar_init(&bars[i], 1);
-        fence_mbar_init();
-        abort_flag = 0;
-    }
     __syncthreads();
-    if (tid == 0)
-        for (int st = 0; st < min(kStagesQK, nst); ++st)
-            issue_stage<D, PS>(a, &kmap, smem + st * STAGE, &bars[st], b, g, r, st, P);
 
     const uint32_t sbase = smem_addr(smem);
     const size_t xstride = (size_t)a.k_max * PS;
@@ -243,6 +277,7 @@ __global__ void __launch_bounds__(kThreads) qk_bf16_kernel(const __grid_constant
                 const int head = 4 * nt + c;
                 if (head < a.G) {
                     const float x = valid ? acc[nt][2 * rr] + acc[nt][2 * rr + 1] : -INFINITY;
+                    run[nt] = fmaxf(run[nt], x);
                     a.xbuf[((size_t)b * a.H_q + (size_t)g * a.G + head) * xstride + (size_t)idx * PS + prow] = x;
                 }
             }
@@ -251,6 +286,7 @@ __global__ void __launch_bounds__(kThreads) qk_bf16_kernel(const __grid_constant
         if (tid == 0 && st + kStagesQK < nst)
             issue_stage<D, PS>(a, &kmap, smem + slot * STAGE, &bars[slot], b, g, r, st + kStagesQK, P);
     }
+    write_split_max(a, b, g, s, run, NT, wm);
 }
 
 // fp32 cache: each thread scores (token, head) pairs of a page with a float64
@@ -258,11 +294,14 @@ __global__ void __launch_bounds__(kThreads) qk_bf16_kernel(const __grid_constant
 template <int D>
 __global__ void __launch_bounds__(kThreads) qk_f32_kernel(const float* __restrict__ k_pool, int ps, const AttnArgs a)
 {
+    __shared__ unsigned int hmax[8];
     const int b = blockIdx.z, g = blockIdx.y, s = blockIdx.x, tid = threadIdx.x;
     const int L = a.seq_lens[b];
     const int P = pages_of(L, ps, a.max_pages, a.status);
     const int cnt = list_count(a, b, g, P);
     if (s == 0 && tid == 0) a.counters[(size_t)b * a.H_kv + g] = 0;
+    if (tid < 8) hmax[tid] = ordered_key(-INFINITY);
+    __syncthreads();
     const Range r = split_range(cnt, a.S, s);
     const size_t xstride = (size_t)a.k_max * ps;
     const double xs = (double)a.xscale;
@@ -278,50 +317,91 @@ __global__ void __launch_bounds__(kThreads) qk_f32_kernel(const float* __restric
                 double dot = 0.0;
                 for (int j = 0; j < D; ++j) dot = fma((double)qh[j], (double)kr[j], dot);
                 x = (float)(dot * xs);
+                atomicMax(&hmax[head], ordered_key(x));
             }
             a.xbuf[((size_t)b * a.H_q + (size_t)g * a.G + head) * xstride + (size_t)idx * ps + t] = x;
         }
     }
+    __syncthreads();
+    if (tid < a.G) {
+        const unsigned int k = hmax[tid];
+        const float m = __uint_as_float((k & 0x80000000u) ? (k & 0x7FFFFFFFu) : ~k);
+        a.lmax[((size_t)b * a.H_q + (size_t)g * a.G + tid) * a.S + s] = m;
+    }
 }
 
 // ====================================================================== tau
+// One CTA per (sequence, query head).  The maximum score M comes from the
+// split maxima of the K pass; tau >= M - 1 (the top score alone has mass
+// >= 1 there), so only scores above M - 1 can carry weight.  They are
+// compacted in one vectorised pass, then Newton steps from the left (never
+// past the root: the mass is convex and decreasing in tau) shrink the support
+// {x > tau} until the closed form on it is consistent.
 constexpr int kTauCap = 8192;
-constexpr int kTauBlock = 256;
+constexpr int kTauBlock = 512;
+constexpr int kTauWarps = kTauBlock / 32;
 
 __global__ void __launch_bounds__(kTauBlock) tau_kernel(int ps, const AttnArgs a)
 {
     __shared__ float cand[kTauCap];
     __shared__ int ncand;
-    __shared__ double redd[kTauBlock / 32];
-    __shared__ float redf[kTauBlock / 32];
-    const int b = blockIdx.y, h = blockIdx.x, tid = threadIdx.x;
+    __shared__ float redm[kTauWarps];
+    __shared__ double redd[2][kTauWarps][3];
+    __shared__ float redf[2][kTauWarps][2];
+    const int b = blockIdx.y, h = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int g = h / a.G;
     const int L = a.seq_lens[b];
     const int P = pages_of(L, ps, a.max_pages, a.status);
     const int cnt = list_count(a, b, g, P);
     const int n = cnt * ps;
-    const float* x = a.xbuf + ((size_t)b * a.H_q + h) * (size_t)a.k_max * ps;
+    const size_t row = (size_t)b * a.H_q + h;
+    const float* x = a.xbuf + row * (size_t)a.k_max * ps;
 
     float M = -INFINITY;
-    for (int i = tid; i < n; i += kTauBlock) M = fmaxf(M, x[i]);
-    M = block_max(M, redf);
-    if (M == -INFINITY) {
+    for (int s = tid; s < a.S; s += kTauBlock) M = fmaxf(M, a.lmax[row * a.S + s]);
+    M = block_max(M, redm);
+    if (!(M > -INFINITY)) {
         if (tid == 0) {
-            a.tau[(size_t)b * a.H_q + h] = INFINITY;
-            if (a.tau_out) a.tau_out[(size_t)b * a.H_q + h] = INFINITY;
+            a.tau[row] = INFINITY;
+            if (a.tau_out) a.tau_out[row] = INFINITY;
         }
         return;
     }
-    // no score at or below max - 1 can be in the support (tau >= max - 1)
     const double thr = (double)M - 1.0;
     if (tid == 0) ncand = 0;
     __syncthreads();
-    for (int i = tid; i < n; i += kTauBlock) {
-        const float v = x[i];
-        if ((double)v > thr) {
-            const int k = atomicAdd(&ncand, 1);
-            if (k < kTauCap) cand[k] = v;
+    // compaction of {x > M - 1}: 4 float4 per lane per round, warp-aggregated slots
+    const float4* x4 = reinterpret_cast<const float4*>(x);
+    const int n4 = n >> 2;
+    for (int base = warp * 32 * 4; base < n4; base += kTauBlock * 4) {
+        float v[16];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int i = base + u * 32 + lane;
+            const float4 f = i < n4 ? x4[i] : make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY);
+            v[4 * u] = f.x; v[4 * u + 1] = f.y; v[4 * u + 2] = f.z; v[4 * u + 3] = f.w;
         }
+        int c = 0;
+#pragma unroll
+        for (int e = 0; e < 16; ++e) c += (double)v[e] > thr;
+        int incl = c;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int t = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += t;
+        }
+        const int tot = __shfl_sync(0xffffffffu, incl, 31);
+        if (tot == 0) continue;
+        int wbase = 0;
+        if (lane == 31) wbase = atomicAdd(&ncand, tot);
+        wbase = __shfl_sync(0xffffffffu, wbase, 31);
+        int pos = wbase + incl - c;
+#pragma unroll
+        for (int e = 0; e < 16; ++e)
+            if ((double)v[e] > thr) {
+                if (pos < kTauCap) cand[pos] = v[e];
+                ++pos;
+            }
     }
     __syncthreads();
     const bool spill = ncand > kTauCap;
@@ -346,11 +426,31 @@ __global__ void __launch_bounds__(kTauBlock) tau_kernel(int ps, const AttnArgs a
                 maxN = fmaxf(maxN, v);
             }
         }
-        k = block_sum(k, redd);
-        sx = block_sum(sx, redd);
-        sxx = block_sum(sxx, redd);
-        minS = block_min(minS, redf);
-        maxN = block_max(maxN, redf);
+        k = warp_sum(k);
+        sx = warp_sum(sx);
+        sxx = warp_sum(sxx);
+        minS = warp_min(minS);
+        maxN = warp_max(maxN);
+        const int bb = it & 1;
+        if (lane == 0) {
+            redd[bb][warp][0] = k;
+            redd[bb][warp][1] = sx;
+            redd[bb][warp][2] = sxx;
+            redf[bb][warp][0] = minS;
+            redf[bb][warp][1] = maxN;
+        }
+        __syncthreads();
+        k = sx = sxx = 0.0;
+        minS = INFINITY;
+        maxN = -INFINITY;
+#pragma unroll
+        for (int w = 0; w < kTauWarps; ++w) {
+            k += redd[bb][w][0];
+            sx += redd[bb][w][1];
+            sxx += redd[bb][w][2];
+            minS = fminf(minS, redf[bb][w][0]);
+            maxN = fmaxf(maxN, redf[bb][w][1]);
+        }
         // closed form on the current support S = {x > tau}
         double tcf;
         bool ok;
@@ -367,7 +467,7 @@ __global__ void __launch_bounds__(kTauBlock) tau_kernel(int ps, const AttnArgs a
             tau = tcf;
             break;
         }
-        // Newton step from tau on sum_S (x - tau)^r = 1
+        // Newton step on sum_S (x - tau)^r = 1
         double nt;
         if (a2) {
             nt = tcf;
@@ -380,8 +480,8 @@ __global__ void __launch_bounds__(kTauBlock) tau_kernel(int ps, const AttnArgs a
         tau = nt;
     }
     if (tid == 0) {
-        a.tau[(size_t)b * a.H_q + h] = (float)tau;
-        if (a.tau_out) a.tau_out[(size_t)b * a.H_q + h] = (float)tau;
+        a.tau[row] = (float)tau;
+        if (a.tau_out) a.tau_out[row] = (float)tau;
     }
 }
 
@@ -428,6 +528,13 @@ EKV_DEV void reduce_splits(const AttnArgs& a, int b, int g)
 }
 
 // ====================================================================== V pass
+// Only pages holding a token with p > 0 for some head of the group are
+// loaded: p = [x - tau]_+^(1/(alpha-1)) is exactly zero elsewhere, so the
+// result is unchanged (support-aware value loading).  The split's pages are
+// scanned in windows; each window's active pages are compacted into a list
+// that feeds the TMA pipeline.
+constexpr int kActWin = 512;
+
 template <int D, int PS, int NT>
 __global__ void __launch_bounds__(kThreads) pv_bf16_kernel(const __grid_constant__ CUtensorMap vmap, const AttnArgs a)
 {
@@ -440,6 +547,10 @@ __global__ void __launch_bounds__(kThreads) pv_bf16_kernel(const __grid_constant
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kStagesPV * STAGE);
     uint16_t* ps_tile = reinterpret_cast<uint16_t*>(smem + kStagesPV * STAGE + 64);   // [8*NT][PROW]
     __shared__ int abort_flag;
+    __shared__ int act[kActWin];
+    __shared__ unsigned char flag[kActWin];
+    __shared__ int nact;
+    __shared__ float tau_s[8];
 
     const int b = blockIdx.z, g = blockIdx.y, s = blockIdx.x;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -447,9 +558,9 @@ __global__ void __launch_bounds__(kThreads) pv_bf16_kernel(const __grid_constant
     const int P = pages_of(L, PS, a.max_pages, a.status);
     const int cnt = list_count(a, b, g, P);
     const Range r = split_range(cnt, a.S, s);
-    const int nst = r.end > r.start ? (r.end - r.start + PPS - 1) / PPS : 0;
     const bool a2 = a.alpha == 2.0f;
     const size_t xstride = (size_t)a.k_max * PS;
+    const size_t row0h = (size_t)b * a.H_q + (size_t)g * a.G;
 
     float acc[NT][MTW][4];
 #pragma unroll
@@ -457,51 +568,110 @@ __global__ void __launch_bounds__(kThreads) pv_bf16_kernel(const __grid_constant
 #pragma unroll
         for (int m = 0; m < MTW; ++m) acc[nt][m][0] = acc[nt][m][1] = acc[nt][m][2] = acc[nt][m][3] = 0.f;
 
-    if (nst > 0) {
-        if (tid == 0) {
-            prefetch_tmap(&vmap);
-            for (int i = 0; i < kStagesPV; ++i) mbar_init(&bars[i], 1);
-            fence_mbar_init();
-            abort_flag = 0;
-        }
-        for (int i = tid; i < 8 * NT * PROW; i += kThreads) ps_tile[i] = 0;
+    if (tid < 8) tau_s[tid] = tid < a.G ? a.tau[row0h + tid] : INFINITY;
+    if (tid == 0) {
+        abort_flag = 0;
+        prefetch_tmap(&vmap);
+        for (int i = 0; i < kStagesPV; ++i) mbar_init(&bars[i], 1);
+        fence_mbar_init();
+    }
+    for (int i = tid; i < 8 * NT * PROW; i += kThreads) ps_tile[i] = 0;
+    __syncthreads();
+    const uint32_t sbase = smem_addr(smem);
+    const uint32_t pbase = smem_addr(ps_tile);
+    int gst = 0;          // stages issued so far (barrier phase bookkeeping)
+    int loaded = 0;
+
+    for (int w0 = r.start; w0 < r.end; w0 += kActWin) {
+        const int wn = min(kActWin, r.end - w0);
+        // --- which pages of the window hold weight
+        for (int i = tid; i < wn; i += kThreads) flag[i] = 0;
         __syncthreads();
-        if (tid == 0)
-            for (int st = 0; st < min(kStagesPV, nst); ++st)
-                issue_stage<D, PS>(a, &vmap, smem + st * STAGE, &bars[st], b, g, r, st, P);
-        // this thread's weights: token tid % 64, heads (tid / 64) * 2 * NT ...
-        const int ptok = tid & (kStageTok - 1);
-        const int hbase = (tid >> 6) * 2 * NT;
-        float tau_h[2 * NT];
-#pragma unroll
-        for (int k = 0; k < 2 * NT; ++k) {
-            const int head = hbase + k;
-            tau_h[k] = head < a.G ? a.tau[(size_t)b * a.H_q + g * a.G + head] : INFINITY;
+        {
+            constexpr int Q = PS / 4;           // float4 per (page, head)
+            const int items = wn * a.G * Q;
+            for (int it = tid; it < items; it += kThreads) {
+                const int j = it / (a.G * Q), rem = it % (a.G * Q);
+                const int h = rem / Q, q4 = rem % Q;
+                const float4 v = *reinterpret_cast<const float4*>(
+                    a.xbuf + (row0h + h) * xstride + (size_t)(w0 + j) * PS + 4 * q4);
+                const float t = tau_s[h];
+                if (v.x > t || v.y > t || v.z > t || v.w > t) flag[j] = 1;
+            }
         }
-        const uint32_t sbase = smem_addr(smem);
-        const uint32_t pbase = smem_addr(ps_tile);
+        __syncthreads();
+        if (warp == 0) {   // ordered compaction of the flags
+            int base = 0;
+            for (int i0 = 0; i0 < wn; i0 += 32) {
+                const bool f = (i0 + lane < wn) && flag[i0 + lane];
+                const unsigned m = __ballot_sync(0xffffffffu, f);
+                if (f) act[base + __popc(m & ((1u << lane) - 1u))] = w0 + i0 + lane;
+                base += __popc(m);
+            }
+            if (lane == 0) nact = base;
+        }
+        __syncthreads();
+        const int na = nact;
+        loaded += na;
+        const int nst = (na + PPS - 1) / PPS;
+        if (nst == 0) continue;
+        // --- pipeline over the active pages
+        auto issue = [&](int st, int slot_) {
+            uint8_t* dst = smem + slot_ * STAGE;
+            int phys[PPS];
+            uint32_t bytes = 0;
+#pragma unroll
+            for (int i = 0; i < PPS; ++i) {
+                const int ai = st * PPS + i;
+                int lp;
+                phys[i] = ai < na ? resolve(a, b, g, act[ai], P, lp, true) : -1;
+                if (phys[i] >= 0) bytes += PS * D * 2;
+            }
+            mbar_arrive_expect_tx(&bars[slot_], bytes);
+#pragma unroll
+            for (int i = 0; i < PPS; ++i) {
+                if (phys[i] < 0) continue;
+                const int y = (phys[i] * a.H_kv + g) * PS;
+#pragma unroll
+                for (int hh = 0; hh < D / 64; ++hh)
+                    tma_load_2d(dst + hh * (kStageTok * 128) + i * PS * 128, &vmap, &bars[slot_], hh * 64, y);
+            }
+        };
+        if (tid == 0)
+            for (int st = 0; st < min(kStagesPV, nst); ++st) issue(st, (gst + st) % kStagesPV);
         for (int st = 0; st < nst; ++st) {
-            const int slot = st % kStagesPV;
-            // weights of this stage (independent of the V tile; computed while it lands)
+            const int gs = gst + st;
+            const int slot = gs % kStagesPV;
+            // weights of this stage: token tid % 64, heads (tid / 64) * 2 * NT ...
             {
-                const int idx = r.start + st * PPS + ptok / PS;
-                const int prow = ptok % PS;
+                const int t = tid & (kStageTok - 1);
+                const int ai = st * PPS + t / PS;
+                const int prow = t % PS;
+                int idx = -1;
+                bool valid = false;
+                if (ai < na) {
+                    idx = act[ai];
+                    int lp;
+                    const int phys = resolve(a, b, g, idx, P, lp, false);
+                    valid = phys >= 0 && lp * PS + prow < L;
+                }
+                const int hbase = (tid >> 6) * 2 * NT;
 #pragma unroll
                 for (int k = 0; k < 2 * NT; ++k) {
                     const int head = hbase + k;
                     float p = 0.f;
-                    if (head < a.G && idx < r.end) {
-                        const float xv = a.xbuf[((size_t)b * a.H_q + (size_t)g * a.G + head) * xstride + (size_t)idx * PS + prow];
-                        const float u = fmaxf(xv - tau_h[k], 0.f);
+                    if (head < a.G && valid) {
+                        const float xv = a.xbuf[(row0h + head) * xstride + (size_t)idx * PS + prow];
+                        const float u = fmaxf(xv - tau_s[head], 0.f);
                         p = a2 ? u : u * u;
                     }
                     uint32_t hi, lo;
                     split_bf16(p, hi, lo);
-                    ps_tile[(2 * head) * PROW + ptok] = (uint16_t)hi;
-                    ps_tile[(2 * head + 1) * PROW + ptok] = (uint16_t)lo;
+                    ps_tile[(2 * head) * PROW + t] = (uint16_t)hi;
+                    ps_tile[(2 * head + 1) * PROW + t] = (uint16_t)lo;
                 }
             }
-            if (!mbar_wait(&bars[slot], (st / kStagesPV) & 1, kWaitLimitNs)) {
+            if (!mbar_wait(&bars[slot], (gs / kStagesPV) & 1, kWaitLimitNs)) {
                 abort_flag = 1;
                 report(a.status, ENTMAXKV_TIMEOUT);
             }
@@ -509,10 +679,28 @@ __global__ void __launch_bounds__(kThreads) pv_bf16_kernel(const __grid_constant
             if (abort_flag) {
                 if (tid == 0)
                     for (int k = st; k < min(st + kStagesPV, nst); ++k)
-                        mbar_wait(&bars[k % kStagesPV], (k / kStagesPV) & 1, kWaitLimitNs);
+                        mbar_wait(&bars[(gst + k) % kStagesPV], ((gst + k) / kStagesPV) & 1, kWaitLimitNs);
                 return;
             }
-            zero_invalid_rows<D, PS>(a, smem + slot * STAGE, b, g, r, st, P, L);
+            // rows without a valid token are zeroed so zero weights never meet garbage
+            {
+                const int t = tid & (kStageTok - 1);
+                const int half = tid >> 6;
+                if (half < D / 64) {
+                    const int ai = st * PPS + t / PS;
+                    bool valid = false;
+                    if (ai < na) {
+                        int lp;
+                        const int phys = resolve(a, b, g, act[ai], P, lp, false);
+                        valid = phys >= 0 && lp * PS + (t % PS) < L;
+                    }
+                    if (!valid) {
+                        uint4* rowp = reinterpret_cast<uint4*>(smem + slot * STAGE + half * (kStageTok * 128) + t * 128);
+#pragma unroll
+                        for (int k = 0; k < 8; ++k) rowp[k] = make_uint4(0, 0, 0, 0);
+                    }
+                }
+            }
             __syncthreads();
             const uint32_t base = sbase + slot * STAGE;
             const int n = lane >> 2, c = lane & 3;
@@ -537,10 +725,11 @@ __global__ void __launch_bounds__(kThreads) pv_bf16_kernel(const __grid_constant
                 }
             }
             __syncthreads();
-            if (tid == 0 && st + kStagesPV < nst)
-                issue_stage<D, PS>(a, &vmap, smem + slot * STAGE, &bars[slot], b, g, r, st + kStagesPV, P);
+            if (tid == 0 && st + kStagesPV < nst) issue(st + kStagesPV, (gs + kStagesPV) % kStagesPV);
         }
+        gst += nst;
     }
+    if (tid == 0 && a.vpages) atomicAdd(&a.vpages[(size_t)b * a.H_kv + g], loaded);
     // partial output of this split: o[head 4nt + c][d]
     {
         const int c = lane & 3, gi = lane >> 2;
@@ -548,7 +737,7 @@ __global__ void __launch_bounds__(kThreads) pv_bf16_kernel(const __grid_constant
         for (int nt = 0; nt < NT; ++nt) {
             const int head = 4 * nt + c;
             if (head >= a.G) continue;
-            const size_t row = ((size_t)b * a.H_q + (size_t)g * a.G + head) * a.S + s;
+            const size_t row = (row0h + head) * a.S + s;
 #pragma unroll
             for (int m = 0; m < MTW; ++m) {
                 const int d = 16 * (warp * MTW + m) + gi;
@@ -589,6 +778,22 @@ __global__ void __launch_bounds__(kThreads) pv_f32_kernel(const float* __restric
             }
         }
         a.opart[(row * a.S + s) * D + dd] = (float)acc;
+    }
+    if (tid == 0 && a.vpages) {   // pages of this split holding weight for some head
+        int n = 0;
+        for (int idx = r.start; idx < r.end; ++idx) {
+            int lp;
+            if (resolve(a, b, g, idx, P, lp, false) < 0) continue;
+            bool any = false;
+            for (int head = 0; head < a.G && !any; ++head) {
+                const size_t row = (size_t)b * a.H_q + (size_t)g * a.G + head;
+                const float tau = a.tau[row];
+                for (int t = 0; t < ps && lp * ps + t < L; ++t)
+                    if (a.xbuf[row * xstride + (size_t)idx * ps + t] > tau) { any = true; break; }
+            }
+            n += any;
+        }
+        atomicAdd(&a.vpages[(size_t)b * a.H_kv + g], n);
     }
     reduce_splits<D, false>(a, b, g);
 }

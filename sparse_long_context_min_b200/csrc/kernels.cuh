@@ -29,6 +29,8 @@ struct AttnArgs {
     float* tau;                    // [B][H_q]
     float* opart;                  // [B][H_q][S][d] partial outputs
     float* mlpart;                 // [B][H_q][S][2] softmax running max and sum
+    float* lmax;                   // [B][H_q][S] largest score of each split (K pass)
+    int32_t* vpages;               // [B][H_kv] value pages loaded (V pass adds), or NULL
     int32_t* counters;             // [B][H_kv] arrival counters of the split reduction
     float* out;                    // [B][H_q][d]
     float* tau_out;                // [B][H_q] or NULL

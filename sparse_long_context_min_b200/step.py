@@ -76,6 +76,7 @@ class DecodeStep:
                               pool.ps, pool.d)
         self.workspace = torch.empty(max(ws, 256), dtype=torch.uint8, device=dev)
         self.status = torch.zeros(1, **i32)
+        self.v_pages = torch.zeros(self.B, self.H_kv, **i32)     # value pages loaded, accumulated
 
     def score(self, q, stream=None):
         if self.mode == "topk":
@@ -97,7 +98,8 @@ class DecodeStep:
 
     def attend(self, q, stream=None):
         B.sparse_attend(self.pool, q, self.page_table, self.seq_lens, self.sel, self.sel_count, self.alpha,
-                        self.scale, self.out, self.workspace, self.status, tau_out=self.tau, stream=stream)
+                        self.scale, self.out, self.workspace, self.status, tau_out=self.tau,
+                        v_pages=self.v_pages, stream=stream)
 
     def __call__(self, q, k_new=None, v_new=None, stream=None):
         """One step; appends (k_new, v_new) [B, H_kv, 1, d] first when given."""
@@ -113,3 +115,94 @@ class DecodeStep:
         code = int(self.status.item())
         if code:
             raise B.EntmaxKVError(code, "decode step (device status)")
+
+
+class _CudaRT:
+    """Event-record nodes inside a captured graph (cudaEventRecordWithFlags with
+    cudaEventRecordExternal) so stage boundaries can be timed during replay."""
+
+    def __init__(self):
+        import ctypes
+        self.ct = ctypes
+        self.rt = ctypes.CDLL("libcudart.so.12")
+        self.rt.cudaEventCreateWithFlags.argtypes = [ctypes.POINTER(ctypes.c_void_p), ctypes.c_uint]
+        self.rt.cudaEventRecordWithFlags.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_uint]
+        self.rt.cudaEventElapsedTime.argtypes = [ctypes.POINTER(ctypes.c_float), ctypes.c_void_p, ctypes.c_void_p]
+        self.rt.cudaEventDestroy.argtypes = [ctypes.c_void_p]
+
+    def event(self):
+        e = self.ct.c_void_p()
+        if self.rt.cudaEventCreateWithFlags(self.ct.byref(e), 0) != 0:
+            raise RuntimeError("cudaEventCreateWithFlags failed")
+        return e
+
+    def record_node(self, e, stream):
+        rc = self.rt.cudaEventRecordWithFlags(e, self.ct.c_void_p(stream.cuda_stream), 1)
+        if rc != 0:
+            raise RuntimeError("cudaEventRecordWithFlags failed (%d)" % rc)
+
+    def elapsed_ms(self, a, b):
+        ms = self.ct.c_float()
+        rc = self.rt.cudaEventElapsedTime(self.ct.byref(ms), a, b)
+        return None if rc != 0 else ms.value
+
+
+class GraphedStep:
+    """A DecodeStep captured once into a CUDA graph.
+
+    The step's inputs live in static device buffers (q, k, v): copy the new
+    query and token into them, then replay().  With stage_events=True the
+    graph also records an event node between stages; stage_us() returns the
+    last replay's per-stage durations (append, score, select, attend) in us.
+    """
+
+    STAGES = ("append", "score", "select", "attend")
+
+    def __init__(self, step: DecodeStep, append=True, stage_events=True):
+        self.step = step
+        pool = step.pool
+        dev = pool.k_pool.device
+        self.q = torch.zeros(step.B, step.H_q, pool.d, dtype=torch.float32, device=dev)
+        self.k = torch.zeros(step.B, step.H_kv, 1, pool.d, dtype=pool.k_pool.dtype, device=dev)
+        self.v = torch.zeros_like(self.k)
+        self.append = append
+        self.rt = _CudaRT() if stage_events else None
+        self.ev = [self.rt.event() for _ in range(5)] if stage_events else None
+        side = torch.cuda.Stream(device=dev)
+        side.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(side):          # warm-up outside capture (no append)
+            step.score(self.q)
+            step.choose()
+            step.attend(self.q)
+        torch.cuda.current_stream().wait_stream(side)
+        torch.cuda.synchronize()
+        self.graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(self.graph):
+            cs = torch.cuda.current_stream()
+            self._mark(0, cs)
+            if append:
+                B.append_metadata(pool, self.k, self.v, step.page_table, step.seq_lens, step.status)
+            self._mark(1, cs)
+            step.score(self.q)
+            self._mark(2, cs)
+            step.choose()
+            self._mark(3, cs)
+            step.attend(self.q)
+            self._mark(4, cs)
+
+    def _mark(self, i, stream):
+        if self.ev is not None:
+            self.rt.record_node(self.ev[i], stream)
+
+    def replay(self):
+        self.graph.replay()
+        return self.step.out
+
+    def stage_us(self):
+        if self.ev is None:
+            return None
+        out = {}
+        for i, name in enumerate(self.STAGES):
+            ms = self.rt.elapsed_ms(self.ev[i], self.ev[i + 1])
+            out[name] = None if ms is None else ms * 1e3
+        return out

@@ -228,14 +228,25 @@ def test_sparse_attend_against_oracle(built):
     st = _status()
     out = torch.empty_like(step.out)
     tau = torch.empty_like(step.tau)
+    vp = torch.zeros(cfg.B, cfg.H_kv, dtype=torch.int32, device="cuda")
     B.sparse_attend(pool, wl.q, wl.page_table, seq_lens, sel, cnt, cfg.alpha, H.scale32(cfg), out,
-                    step.workspace, st, tau_out=tau)
+                    step.workspace, st, tau_out=tau, v_pages=vp)
     _assert_ok(st)
-    out, tau = out.cpu().numpy(), tau.cpu().numpy()
+    out, tau, vp = out.cpu().numpy(), tau.cpu().numpy(), vp.cpu().numpy()
     G = cfg.G
     for (b, g), (o_ref, t_ref) in refs.items():
         H.compare_out(out[b, g * G:(g + 1) * G], o_ref, cfg.dtype)
         assert np.all(np.abs(tau[b, g * G:(g + 1) * G] - t_ref) <= 1e-5 * np.maximum(1, np.abs(t_ref)))
+        # value pages loaded = selected pages holding a token with p > 0 (within a band
+        # for tokens whose score sits on the threshold)
+        o = oseqs[b]
+        pages = sel[b, g, :cnt[b, g]].cpu().numpy()
+        tok = attend.token_indices(pages, o.L, cfg.ps)
+        x = (cfg.alpha - 1) * (o.keys[g][tok] @ o.qgroup(g).astype(np.float64).T) / math.sqrt(cfg.d)
+        page_of = tok // cfg.ps
+        sure = set(page_of[np.any(x > t_ref[None, :] + 1e-4, axis=1)].tolist())
+        maybe = set(page_of[np.any(x > t_ref[None, :] - 1e-4, axis=1)].tolist())
+        assert len(sure) <= vp[b, g] <= len(maybe), (len(sure), vp[b, g], len(maybe))
 
 
 def test_decode_step_end_to_end(built):
@@ -400,3 +411,28 @@ def test_decode_appends_then_step():
             tok = attend.token_indices(pages, lens[b], cfg.ps)
             o_ref, _, _ = attend.entmax_attention(qg, keys[g][tok], vals[g][tok], cfg.alpha, 1 / math.sqrt(cfg.d))
             H.compare_out(out[b, g * G:(g + 1) * G], o_ref, cfg.dtype)
+
+
+def test_graphed_step_equals_eager_step():
+    from sparse_long_context_min_b200.step import GraphedStep
+    wl = _wl(2, [5000])
+    cfg = wl.cfg
+    pool_a, lens_a = build_pool(wl)
+    pool_b, lens_b = build_pool(wl)
+    eager = DecodeStep(pool_a, wl.page_table, lens_a, cfg.H_q, "topk", budget_frac=1 / 16, alpha=cfg.alpha)
+    graphed = GraphedStep(DecodeStep(pool_b, wl.page_table, lens_b, cfg.H_q, "topk", budget_frac=1 / 16,
+                                     alpha=cfg.alpha))
+    for t in range(3):
+        k, v, q = wl.decode_token(t)
+        eager(q, k, v)
+        graphed.q.copy_(q)
+        graphed.k.copy_(k)
+        graphed.v.copy_(v)
+        graphed.replay()
+        torch.cuda.synchronize()
+        assert torch.equal(eager.out, graphed.step.out)
+        assert torch.equal(lens_a, lens_b)
+    eager.check()
+    graphed.step.check()
+    stages = graphed.stage_us()
+    assert set(stages) == set(GraphedStep.STAGES)
