@@ -125,16 +125,20 @@ ENTMAXKV_API int entmaxkv_append_metadata(const entmaxkv_pool* pool, const void*
  * section 2.A).
  *   q     : [B][H_q][d] fp32 query.
  *   scale : score scale (1/sqrt(d) for standard attention); s = scale * q.k.
+ *   Every sum over d below is taken in one fixed fp32 order, because
+ *   selection is decided on these values: d is cut into 8 consecutive slices
+ *   of d/8 coordinates, each slice is a chain of fused multiply-adds from 0 in
+ *   ascending d, and the slice sums are combined as
+ *   ((S0 + S1) + (S2 + S3)) + ((S4 + S5) + (S6 + S7)).
  *   mode ENTMAXKV_SCORE_BBOX: ub [B][H_kv][max_pages] fp32, the bounding-box
  *     bound of the group, UBg = max over the group's heads of
- *     scale * sum_d q_d (q_d >= 0 ? kmax_d : kmin_d), each head's sum taken as
- *     fp32 fused multiply-adds in ascending d from 0; -0 becomes +0.
+ *     scale * sum_d q_d (q_d >= 0 ? kmax_d : kmin_d); -0 becomes +0.
  *     m, v, est_max are ignored (may be NULL).
  *   mode ENTMAXKV_SCORE_GAUSS: m, v, est_max [B][H_q][max_pages] fp32, the
- *     Gaussian page model of each query head: m = scale * sum fma(q_d, mean_d),
- *     v = (sum fma(q_d*q_d, m2_d) / n) * scale^2, est_max = fma(sqrt(v), z_n, m)
- *     with z_n = fp32(sqrt(2 ln n)) for n >= 2 and z_1 = 0, n the page's tokens
- *     (sums in ascending d from 0).  ub is ignored.
+ *     Gaussian page model of each query head: m = scale * sum_d q_d mean_d,
+ *     v = ((sum_d (q_d*q_d) m2_d) / n) * scale^2, est_max = fma(sqrt(v), z_n, m)
+ *     with z_n = fp32(sqrt(2 ln n)) for n >= 2 and z_1 = 0, n the page's
+ *     tokens.  ub is ignored.
  *   Entries p >= P_b are written as -INFINITY (v as 0).
  */
 ENTMAXKV_API int entmaxkv_score_pages(const entmaxkv_pool* pool, const float* q, int32_t H_q,

@@ -2,7 +2,9 @@
 
 The fp32 canonical-order replicas decide page selection in the same precision
 and order as the GPU kernels must (see the comment at the top of
-replica_f32.c for the exact operation order).  ``build()`` compiles the C file
+replica_f32.c for the exact operation order: Welford metadata in token order;
+dot products over d as 8 consecutive slices of serial fmaf chains combined by a
+fixed pairwise tree).  ``build()`` compiles the C file
 with gcc; it is called lazily on first use.
 """
 
@@ -82,6 +84,8 @@ def bound(q, kmin, kmax, scale):
     kmin = _f32(kmin)
     kmax = _f32(kmax)
     G, d = q.shape
+    if d % 8:
+        raise ValueError("the canonical order splits d into 8 slices: d must be a multiple of 8")
     P = kmin.shape[0]
     ub = np.zeros((G, P), dtype=np.float32)
     ubg = np.zeros(P, dtype=np.float32)
@@ -108,6 +112,8 @@ def gauss(q, mean, m2, count, scale, ps):
     if count.size and (count.min() < 1 or count.max() > ps):
         raise ValueError("page counts must lie in [1, ps]")
     G, d = q.shape
+    if d % 8:
+        raise ValueError("the canonical order splits d into 8 slices: d must be a multiple of 8")
     P = mean.shape[0]
     z = z_table_f32(ps)
     m = np.zeros((G, P), dtype=np.float32)

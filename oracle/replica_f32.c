@@ -16,11 +16,15 @@
  *            d1 = x - mean;  mean = mean + d1 / n;  d2 = x - mean;
  *            m2 = fmaf(d1, d2, m2);
  *            kmin = (x < kmin) ? x : kmin;  kmax = (x > kmax) ? x : kmax
- *  - bounding-box bound of one page for head h (d ascending):
- *        acc = 0;  acc = fmaf(q[d], q[d] >= 0 ? kmax[d] : kmin[d], acc)
- *        UB_h = acc * scale;  UBg = max over the group's heads; -0 -> +0
- *  - Gaussian page estimate for head h (d ascending):
- *        ma = sum fmaf(q[d], mean[d], .);   va = sum fmaf(q[d]*q[d], m2[d], .)
+ *  - dot products over d (the bound's sum and the Gaussian sums) split d into
+ *    8 consecutive slices of d/8 coordinates; each slice is a chain of fmaf
+ *    from 0 in ascending d, and the slice sums S0..S7 are combined as
+ *        ((S0 + S1) + (S2 + S3)) + ((S4 + S5) + (S6 + S7))
+ *  - bounding-box bound of one page for head h, with terms
+ *        q[d] * (q[d] >= 0 ? kmax[d] : kmin[d]):
+ *        UB_h = dot * scale;  UBg = max over the group's heads; -0 -> +0
+ *  - Gaussian page estimate for head h:
+ *        ma = dot of q[d] * mean[d];   va = dot of (q[d]*q[d]) * m2[d]
  *        m = ma * scale;  v = (va / n) * (scale * scale)
  *        est = fmaf(sqrtf(v), z[n], m)
  *
@@ -65,22 +69,33 @@ void replica_page_meta(const float* keys, int64_t L, int d, int ps,
     }
 }
 
+/* The fixed combination of the 8 slice sums. */
+static float tree8(const float* s)
+{
+    return ((s[0] + s[1]) + (s[2] + s[3])) + ((s[4] + s[5]) + (s[6] + s[7]));
+}
+
 /* Bounding-box bounds of P pages for the G heads of one group.
  * q: [G][d]; kmin/kmax: [P][d]; ub: [G][P] (may be NULL); ubg: [P]. */
 void replica_bound(const float* q, int G, int d,
                    const float* kmin, const float* kmax, int64_t P,
                    float scale, float* ub, float* ubg)
 {
+    const int w = d / 8;
     for (int64_t p = 0; p < P; ++p) {
         float best = 0.0f;
         for (int h = 0; h < G; ++h) {
-            float acc = 0.0f;
-            for (int j = 0; j < d; ++j) {
-                float qd = q[h * d + j];
-                float sel = (qd >= 0.0f) ? kmax[p * d + j] : kmin[p * d + j];
-                acc = fmaf(qd, sel, acc);
+            float s[8];
+            for (int k = 0; k < 8; ++k) {
+                float acc = 0.0f;
+                for (int j = k * w; j < (k + 1) * w; ++j) {
+                    float qd = q[h * d + j];
+                    float sel = (qd >= 0.0f) ? kmax[p * d + j] : kmin[p * d + j];
+                    acc = fmaf(qd, sel, acc);
+                }
+                s[k] = acc;
             }
-            float u = acc * scale;
+            float u = tree8(s) * scale;
             if (ub) ub[h * P + p] = u;
             if (h == 0 || u > best) best = u;
         }
@@ -98,18 +113,24 @@ void replica_gauss(const float* q, int G, int d,
                    float* m, float* v, float* est)
 {
     float scale2 = scale * scale;
+    const int w = d / 8;
     for (int h = 0; h < G; ++h) {
         for (int64_t p = 0; p < P; ++p) {
-            float ma = 0.0f, va = 0.0f;
-            for (int j = 0; j < d; ++j) {
-                float qd = q[h * d + j];
-                float q2 = qd * qd;
-                ma = fmaf(qd, mean[p * d + j], ma);
-                va = fmaf(q2, m2[p * d + j], va);
+            float sm[8], sv[8];
+            for (int k = 0; k < 8; ++k) {
+                float ma = 0.0f, va = 0.0f;
+                for (int j = k * w; j < (k + 1) * w; ++j) {
+                    float qd = q[h * d + j];
+                    float q2 = qd * qd;
+                    ma = fmaf(qd, mean[p * d + j], ma);
+                    va = fmaf(q2, m2[p * d + j], va);
+                }
+                sm[k] = ma;
+                sv[k] = va;
             }
             int32_t n = count[p];
-            float mm = ma * scale;
-            float vv = (va / (float)n) * scale2;
+            float mm = tree8(sm) * scale;
+            float vv = (tree8(sv) / (float)n) * scale2;
             m[h * P + p] = mm;
             v[h * P + p] = vv;
             est[h * P + p] = fmaf(sqrtf(vv), z[n], mm);

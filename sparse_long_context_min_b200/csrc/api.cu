@@ -11,11 +11,14 @@
 namespace ekv {
 
 // ------------------------------------------------------------------ devices
-static int sm_count()
+int num_sms()
 {
+    static int cache[64] = {0};
     int dev = 0, n = 148;
     if (cudaGetDevice(&dev) != cudaSuccess) return n;
+    if (dev >= 0 && dev < 64 && cache[dev] > 0) return cache[dev];
     if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) n = 148;
+    if (dev >= 0 && dev < 64) cache[dev] = n;
     return n;
 }
 
@@ -108,7 +111,7 @@ static size_t round256(size_t x) { return (x + 255) & ~size_t(255); }
 static int num_splits(int B, int H_kv, int list_pages)
 {
     const long long units = (long long)B * H_kv;
-    long long S = (2ll * sm_count() + units - 1) / (units > 0 ? units : 1);
+    long long S = (2ll * num_sms() + units - 1) / (units > 0 ? units : 1);
     if (S > list_pages) S = list_pages;
     if (S > 1024) S = 1024;
     if (S < 1) S = 1;

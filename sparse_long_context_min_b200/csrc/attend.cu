@@ -65,7 +65,7 @@ EKV_DEV int list_count(const AttnArgs& a, int b, int g, int P)
 
 // Physical page of list entry idx of (b, g), or -1 when the entry or its page
 // id is out of range (reported when `rep`).
-EKV_DEV int resolve(const AttnArgs& a, int b, int g, int idx, int P, int& lp, bool rep)
+EKV_DEV int resolve_g(const AttnArgs& a, int b, int g, int idx, int P, int& lp, bool rep)
 {
     lp = a.sel ? a.sel[((size_t)b * a.H_kv + g) * a.k_max + idx] : idx;
     if (lp < 0 || lp >= P) {
@@ -80,9 +80,40 @@ EKV_DEV int resolve(const AttnArgs& a, int b, int g, int idx, int P, int& lp, bo
     return phys;
 }
 
-EKV_DEV uint8_t* align1024(uint8_t* p)
+// Page ids of a CTA's split, resolved once into shared memory so that the
+// copy pipeline never waits on a dependent chain of global loads (list entry,
+// then page table) before issuing a stage.  Every attention kernel calls
+// tab_fill first; splits longer than the table resolve from global memory.
+constexpr int kTabCap = 1024;
+__shared__ int tab_phys[kTabCap];
+__shared__ int tab_lp[kTabCap];
+__shared__ int tab_base, tab_n;
+
+EKV_DEV void tab_fill(const AttnArgs& a, int b, int g, Range r, int P)
 {
-    return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
+    const int n = r.end > r.start ? r.end - r.start : 0;
+    if (threadIdx.x == 0) {
+        tab_base = r.start;
+        tab_n = n <= kTabCap ? n : 0;
+    }
+    if (n <= kTabCap)
+        for (int i = threadIdx.x; i < n; i += blockDim.x) {
+            int lp;
+            const int ph = resolve_g(a, b, g, r.start + i, P, lp, true);
+            tab_phys[i] = ph;
+            tab_lp[i] = lp;
+        }
+    __syncthreads();
+}
+
+EKV_DEV int resolve(const AttnArgs& a, int b, int g, int idx, int P, int& lp, bool rep)
+{
+    const int j = idx - tab_base;
+    if (j >= 0 && j < tab_n) {
+        lp = tab_lp[j];
+        return tab_phys[j];
+    }
+    return resolve_g(a, b, g, idx, P, lp, rep);
 }
 
 // Issue the TMA loads of pipeline stage `st` (pages start + st*PPS ...) of one
@@ -161,6 +192,7 @@ EKV_DEV void zero_invalid_rows(const AttnArgs& a, uint8_t* stage, int b, int g, 
         uint4* row = reinterpret_cast<uint4*>(stage + half * (kStageTok * 128) + t * 128);
 #pragma unroll
         for (int k = 0; k < 8; ++k) row[k] = make_uint4(0, 0, 0, 0);
+        fence_proxy_async();
     }
 }
 
@@ -194,11 +226,12 @@ EKV_DEV void write_split_max(const AttnArgs& a, int b, int g, int s, const float
 template <int D, int PS, int NT>
 __global__ void __launch_bounds__(kThreads) qk_bf16_kernel(const __grid_constant__ CUtensorMap kmap, const AttnArgs a)
 {
+    pdl_enter();
     constexpr int STAGE = kStageTok * D * 2;
     constexpr int PPS = kStageTok / PS;
     constexpr int KS = D / 16;
     extern __shared__ uint8_t smem_raw[];
-    uint8_t* smem = align1024(smem_raw);
+    uint8_t* smem = smem_align<1024>(smem_raw);
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kStagesQK * STAGE);
     __shared__ int abort_flag;
     __shared__ float wm[4][8];
@@ -211,6 +244,7 @@ __global__ void __launch_bounds__(kThreads) qk_bf16_kernel(const __grid_constant
     if (s == 0 && tid == 0) a.counters[(size_t)b * a.H_kv + g] = 0;
     const Range r = split_range(cnt, a.S, s);
     const int nst = r.end > r.start ? (r.end - r.start + PPS - 1) / PPS : 0;
+    tab_fill(a, b, g, r, P);
 
     // start the key loads first; the query fragments are prepared meanwhile
     if (tid == 0) {
@@ -294,6 +328,7 @@ __global__ void __launch_bounds__(kThreads) qk_bf16_kernel(const __grid_constant
 template <int D>
 __global__ void __launch_bounds__(kThreads) qk_f32_kernel(const float* __restrict__ k_pool, int ps, const AttnArgs a)
 {
+    pdl_enter();
     __shared__ unsigned int hmax[8];
     const int b = blockIdx.z, g = blockIdx.y, s = blockIdx.x, tid = threadIdx.x;
     const int L = a.seq_lens[b];
@@ -301,8 +336,8 @@ __global__ void __launch_bounds__(kThreads) qk_f32_kernel(const float* __restric
     const int cnt = list_count(a, b, g, P);
     if (s == 0 && tid == 0) a.counters[(size_t)b * a.H_kv + g] = 0;
     if (tid < 8) hmax[tid] = ordered_key(-INFINITY);
-    __syncthreads();
     const Range r = split_range(cnt, a.S, s);
+    tab_fill(a, b, g, r, P);
     const size_t xstride = (size_t)a.k_max * ps;
     const double xs = (double)a.xscale;
     for (int idx = r.start; idx < r.end; ++idx) {
@@ -334,20 +369,65 @@ __global__ void __launch_bounds__(kThreads) qk_f32_kernel(const float* __restric
 // One CTA per (sequence, query head).  The maximum score M comes from the
 // split maxima of the K pass; tau >= M - 1 (the top score alone has mass
 // >= 1 there), so only scores above M - 1 can carry weight.  They are
-// compacted in one vectorised pass, then Newton steps from the left (never
-// past the root: the mass is convex and decreasing in tau) shrink the support
-// {x > tau} until the closed form on it is consistent.
-constexpr int kTauCap = 8192;
+// compacted in one vectorised pass.  A 2048-bin histogram of them over
+// [M - 1, M] then brackets tau: at every bin edge t the counts give a lower
+// and an upper bound of F(t) = sum (x - t)_+^(1/(alpha-1)) (each value lies
+// within its bin), so tau lies between the last edge with F_lower >= 1 and
+// the first edge with F_upper < 1, a few bins apart.  Newton steps from that
+// lower edge (never past the root: F is convex and decreasing) then shrink
+// the support {x > tau} until the closed form on it is consistent, usually
+// in one to three passes.
 constexpr int kTauBlock = 512;
 constexpr int kTauWarps = kTauBlock / 32;
+constexpr int kTauBins = 2048;
+constexpr int kTauCap = 32768;                         // candidates kept in shared memory
+constexpr int kTauSmem = kTauCap * 4 + kTauBins * 4 + 64;
+
+// block-wide sum of 3 doubles and min/max of 2 floats; double-buffered scratch
+struct TauRed {
+    double d[2][kTauWarps][3];
+    float f[2][kTauWarps][2];
+};
+
+EKV_DEV void tau_reduce(TauRed& R, int it, double (&v)[3], float& mn, float& mx)
+{
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, bb = it & 1;
+#pragma unroll
+    for (int i = 0; i < 3; ++i) v[i] = warp_sum(v[i]);
+    mn = warp_min(mn);
+    mx = warp_max(mx);
+    if (lane == 0) {
+        R.d[bb][warp][0] = v[0];
+        R.d[bb][warp][1] = v[1];
+        R.d[bb][warp][2] = v[2];
+        R.f[bb][warp][0] = mn;
+        R.f[bb][warp][1] = mx;
+    }
+    __syncthreads();
+    v[0] = v[1] = v[2] = 0.0;
+    mn = INFINITY;
+    mx = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < kTauWarps; ++w) {
+        v[0] += R.d[bb][w][0];
+        v[1] += R.d[bb][w][1];
+        v[2] += R.d[bb][w][2];
+        mn = fminf(mn, R.f[bb][w][0]);
+        mx = fmaxf(mx, R.f[bb][w][1]);
+    }
+}
 
 __global__ void __launch_bounds__(kTauBlock) tau_kernel(int ps, const AttnArgs a)
 {
-    __shared__ float cand[kTauCap];
+    pdl_enter();
+    extern __shared__ uint8_t tau_smem[];
+    float* cand = reinterpret_cast<float*>(tau_smem);
+    int* hist = reinterpret_cast<int*>(tau_smem + kTauCap * 4);
     __shared__ int ncand;
     __shared__ float redm[kTauWarps];
-    __shared__ double redd[2][kTauWarps][3];
-    __shared__ float redf[2][kTauWarps][2];
+    __shared__ TauRed R;
+    __shared__ double scan[kTauWarps][5];
+    __shared__ double brk[2][kTauWarps];
     const int b = blockIdx.y, h = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int g = h / a.G;
     const int L = a.seq_lens[b];
@@ -356,6 +436,7 @@ __global__ void __launch_bounds__(kTauBlock) tau_kernel(int ps, const AttnArgs a
     const int n = cnt * ps;
     const size_t row = (size_t)b * a.H_q + h;
     const float* x = a.xbuf + row * (size_t)a.k_max * ps;
+    const bool a2 = a.alpha == 2.0f;
 
     float M = -INFINITY;
     for (int s = tid; s < a.S; s += kTauBlock) M = fmaxf(M, a.lmax[row * a.S + s]);
@@ -369,8 +450,9 @@ __global__ void __launch_bounds__(kTauBlock) tau_kernel(int ps, const AttnArgs a
     }
     const double thr = (double)M - 1.0;
     if (tid == 0) ncand = 0;
+    for (int i = tid; i < kTauBins; i += kTauBlock) hist[i] = 0;
     __syncthreads();
-    // compaction of {x > M - 1}: 4 float4 per lane per round, warp-aggregated slots
+    // --- compaction of {x > M - 1} (4 float4 per lane per round) + histogram
     const float4* x4 = reinterpret_cast<const float4*>(x);
     const int n4 = n >> 2;
     for (int base = warp * 32 * 4; base < n4; base += kTauBlock * 4) {
@@ -383,7 +465,13 @@ __global__ void __launch_bounds__(kTauBlock) tau_kernel(int ps, const AttnArgs a
         }
         int c = 0;
 #pragma unroll
-        for (int e = 0; e < 16; ++e) c += (double)v[e] > thr;
+        for (int e = 0; e < 16; ++e) {
+            const double d = (double)v[e] - thr;
+            if (d > 0.0) {
+                ++c;
+                atomicAdd(&hist[min(kTauBins - 1, (int)(d * kTauBins))], 1);
+            }
+        }
         int incl = c;
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
@@ -404,54 +492,119 @@ __global__ void __launch_bounds__(kTauBlock) tau_kernel(int ps, const AttnArgs a
             }
     }
     __syncthreads();
+    // --- bracket tau from the histogram.  Bin j holds values in
+    // [e_j - eps, e_{j+1} + eps], e_j = thr + j / NB.  With lo_j = e_j - eps and
+    // hi_j = e_{j+1} + eps:
+    //   F(e_i) >= sum_{j > i}  c_j (lo_j - e_i)^r      (F_lower)
+    //   F(e_i) <= sum_{j >= i-1} c_j (hi_j - e_i)^r    (F_upper)
+    // expanded in suffix sums of c_j, c_j a_j, c_j a_j^2 (a = lo or hi).
+    constexpr int BPT = kTauBins / kTauBlock;            // bins per thread (4)
+    const double w = 1.0 / kTauBins;
+    const double eps = 4e-7 * fmax(1.0, fabs((double)M));
+    double loc[5] = {0, 0, 0, 0, 0};                     // c, c lo, c lo^2, c hi, c hi^2 over my bins
+    const int j0 = tid * BPT;
+#pragma unroll
+    for (int k = 0; k < BPT; ++k) {
+        const int j = j0 + k;
+        const double c = (double)hist[j];
+        const double lo = thr + j * w - eps, hi = thr + (j + 1) * w + eps;
+        loc[0] += c;
+        loc[1] += c * lo;
+        loc[2] += c * lo * lo;
+        loc[3] += c * hi;
+        loc[4] += c * hi * hi;
+    }
+    // exclusive suffix scan over threads (bins above mine): reverse warp scan + warp totals
+    double suf[5];
+#pragma unroll
+    for (int i = 0; i < 5; ++i) {
+        double v = loc[i];
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const double t = __shfl_down_sync(0xffffffffu, v, o);
+            if (lane + o < 32) v += t;
+        }
+        suf[i] = v;                                      // inclusive suffix within the warp
+    }
+    if (lane == 0)
+#pragma unroll
+        for (int i = 0; i < 5; ++i) scan[warp][i] = suf[i];
+    __syncthreads();
+#pragma unroll
+    for (int i = 0; i < 5; ++i) {
+        double above = 0.0;
+        for (int ww = warp + 1; ww < kTauWarps; ++ww) above += scan[ww][i];
+        suf[i] = suf[i] - loc[i] + above;                // exclusive: bins of threads above
+    }
+    // walk my bins from the top keeping suffix sums; evaluate both bounds at each edge
+    double best_lo = thr, best_hi = (double)M;
+    {
+        double S[5];
+#pragma unroll
+        for (int i = 0; i < 5; ++i) S[i] = suf[i];        // sums over bins > my last bin
+        for (int k = BPT - 1; k >= 0; --k) {
+            const int j = j0 + k;                         // edge e_j (lower edge of bin j)
+            const double c = (double)hist[j];
+            const double lo = thr + j * w - eps, hi = thr + (j + 1) * w + eps;
+            const double e = thr + j * w;
+            // F_lower(e_j): bins > j  (S excludes bin j)
+            const double flo = a2 ? (S[1] - e * S[0]) : (S[2] - 2.0 * e * S[1] + e * e * S[0]);
+            // F_upper(e_j): bins >= j-1 (add bin j and bin j-1)
+            double c1 = S[0] + c, h1 = S[3] + c * hi, h2 = S[4] + c * hi * hi;
+            if (j > 0) {
+                const double cm = (double)hist[j - 1];
+                const double him = thr + j * w + eps;
+                c1 += cm;
+                h1 += cm * him;
+                h2 += cm * him * him;
+            }
+            const double fhi = a2 ? (h1 - e * c1) : (h2 - 2.0 * e * h1 + e * e * c1);
+            if (flo >= 1.0) best_lo = fmax(best_lo, e);
+            if (fhi < 1.0) best_hi = fmin(best_hi, e);
+            S[0] += c;
+            S[1] += c * lo;
+            S[2] += c * lo * lo;
+            S[3] += c * hi;
+            S[4] += c * hi * hi;
+        }
+    }
+    best_lo = warp_max_d(best_lo);
+    best_hi = warp_min_d(best_hi);
+    if (lane == 0) {
+        brk[0][warp] = best_lo;
+        brk[1][warp] = best_hi;
+    }
+    __syncthreads();
+    double lo_t = thr, hi_t = (double)M;
+    for (int ww = 0; ww < kTauWarps; ++ww) {
+        lo_t = fmax(lo_t, brk[0][ww]);
+        hi_t = fmin(hi_t, brk[1][ww]);
+    }
+    (void)hi_t;
     const bool spill = ncand > kTauCap;
     const float* src = spill ? x : cand;
     const int len = spill ? n : ncand;
-    const bool a2 = a.alpha == 2.0f;
 
-    double tau = thr;
+    // --- Newton / closed form over {x > lo_t}
+    double tau = lo_t;
     for (int it = 0; it < 100; ++it) {
-        double k = 0.0, sx = 0.0, sxx = 0.0;
+        double v[3] = {0.0, 0.0, 0.0};
         float minS = INFINITY, maxN = -INFINITY;
         for (int i = tid; i < len; i += kTauBlock) {
-            const float v = src[i];
-            const double vd = (double)v;
-            if (!(vd > thr)) continue;
+            const float f = src[i];
+            const double vd = (double)f;
+            if (!(vd > lo_t)) continue;
             if (vd > tau) {
-                k += 1.0;
-                sx += vd;
-                sxx = fma(vd, vd, sxx);
-                minS = fminf(minS, v);
+                v[0] += 1.0;
+                v[1] += vd;
+                v[2] = fma(vd, vd, v[2]);
+                minS = fminf(minS, f);
             } else {
-                maxN = fmaxf(maxN, v);
+                maxN = fmaxf(maxN, f);
             }
         }
-        k = warp_sum(k);
-        sx = warp_sum(sx);
-        sxx = warp_sum(sxx);
-        minS = warp_min(minS);
-        maxN = warp_max(maxN);
-        const int bb = it & 1;
-        if (lane == 0) {
-            redd[bb][warp][0] = k;
-            redd[bb][warp][1] = sx;
-            redd[bb][warp][2] = sxx;
-            redf[bb][warp][0] = minS;
-            redf[bb][warp][1] = maxN;
-        }
-        __syncthreads();
-        k = sx = sxx = 0.0;
-        minS = INFINITY;
-        maxN = -INFINITY;
-#pragma unroll
-        for (int w = 0; w < kTauWarps; ++w) {
-            k += redd[bb][w][0];
-            sx += redd[bb][w][1];
-            sxx += redd[bb][w][2];
-            minS = fminf(minS, redf[bb][w][0]);
-            maxN = fmaxf(maxN, redf[bb][w][1]);
-        }
-        // closed form on the current support S = {x > tau}
+        tau_reduce(R, it, v, minS, maxN);
+        const double k = v[0], sx = v[1], sxx = v[2];
         double tcf;
         bool ok;
         if (a2) {
@@ -463,11 +616,12 @@ __global__ void __launch_bounds__(kTauBlock) tau_kernel(int ps, const AttnArgs a
             ok = disc >= 0.0;
             tcf = ok ? mean - sqrt(disc) : 0.0;
         }
-        if (ok && tcf < (double)minS && (double)maxN <= tcf) {
+        // consistent support: every kept value above tcf, every dropped one at or
+        // below it (values at or below lo_t are below tau as well)
+        if (ok && tcf < (double)minS && (double)maxN <= tcf && tcf >= lo_t) {
             tau = tcf;
             break;
         }
-        // Newton step on sum_S (x - tau)^r = 1
         double nt;
         if (a2) {
             nt = tcf;
@@ -506,7 +660,17 @@ EKV_DEV void reduce_splits(const AttnArgs& a, int b, int g)
         const size_t row = (size_t)b * a.H_q + (size_t)g * a.G + head;
         float acc = 0.f;
         if (!SOFTMAX) {
-            for (int s = 0; s < a.S; ++s) acc += __ldcg(&a.opart[(row * a.S + s) * D + dd]);
+            // loads issued 8 at a time, added in split order (deterministic)
+            const float* src = a.opart + row * a.S * D + dd;
+            int s = 0;
+            for (; s + 8 <= a.S; s += 8) {
+                float t[8];
+#pragma unroll
+                for (int u = 0; u < 8; ++u) t[u] = __ldcg(src + (size_t)(s + u) * D);
+#pragma unroll
+                for (int u = 0; u < 8; ++u) acc += t[u];
+            }
+            for (; s < a.S; ++s) acc += __ldcg(src + (size_t)s * D);
             a.out[row * D + dd] = acc;
         } else {
             float Mx = -INFINITY;
@@ -538,12 +702,13 @@ constexpr int kActWin = 512;
 template <int D, int PS, int NT>
 __global__ void __launch_bounds__(kThreads) pv_bf16_kernel(const __grid_constant__ CUtensorMap vmap, const AttnArgs a)
 {
+    pdl_enter();
     constexpr int STAGE = kStageTok * D * 2;
     constexpr int PPS = kStageTok / PS;
     constexpr int MTW = D / 64;           // 16-row m-tiles (head-dim rows) per warp
     constexpr int PROW = kStageTok + kPsPad;
     extern __shared__ uint8_t smem_raw[];
-    uint8_t* smem = align1024(smem_raw);
+    uint8_t* smem = smem_align<1024>(smem_raw);
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kStagesPV * STAGE);
     uint16_t* ps_tile = reinterpret_cast<uint16_t*>(smem + kStagesPV * STAGE + 64);   // [8*NT][PROW]
     __shared__ int abort_flag;
@@ -568,6 +733,7 @@ __global__ void __launch_bounds__(kThreads) pv_bf16_kernel(const __grid_constant
 #pragma unroll
         for (int m = 0; m < MTW; ++m) acc[nt][m][0] = acc[nt][m][1] = acc[nt][m][2] = acc[nt][m][3] = 0.f;
 
+    tab_fill(a, b, g, r, P);
     if (tid < 8) tau_s[tid] = tid < a.G ? a.tau[row0h + tid] : INFINITY;
     if (tid == 0) {
         abort_flag = 0;
@@ -698,6 +864,7 @@ __global__ void __launch_bounds__(kThreads) pv_bf16_kernel(const __grid_constant
                         uint4* rowp = reinterpret_cast<uint4*>(smem + slot * STAGE + half * (kStageTok * 128) + t * 128);
 #pragma unroll
                         for (int k = 0; k < 8; ++k) rowp[k] = make_uint4(0, 0, 0, 0);
+                        fence_proxy_async();
                     }
                 }
             }
@@ -752,11 +919,13 @@ __global__ void __launch_bounds__(kThreads) pv_bf16_kernel(const __grid_constant
 template <int D>
 __global__ void __launch_bounds__(kThreads) pv_f32_kernel(const float* __restrict__ v_pool, int ps, const AttnArgs a)
 {
+    pdl_enter();
     const int b = blockIdx.z, g = blockIdx.y, s = blockIdx.x, tid = threadIdx.x;
     const int L = a.seq_lens[b];
     const int P = pages_of(L, ps, a.max_pages, a.status);
     const int cnt = list_count(a, b, g, P);
     const Range r = split_range(cnt, a.S, s);
+    tab_fill(a, b, g, r, P);
     const size_t xstride = (size_t)a.k_max * ps;
     const bool a2 = a.alpha == 2.0f;
     for (int w = tid; w < a.G * D; w += kThreads) {
@@ -804,13 +973,14 @@ __global__ void __launch_bounds__(kThreads) softmax_bf16_kernel(const __grid_con
                                                                 const __grid_constant__ CUtensorMap vmap,
                                                                 const AttnArgs a)
 {
+    pdl_enter();
     constexpr int STAGE = kStageTok * D * 2;
     constexpr int PPS = kStageTok / PS;
     constexpr int KS = D / 16;
     constexpr int MTW = D / 64;
     constexpr int PROW = kStageTok + kPsPad;
     extern __shared__ uint8_t smem_raw[];
-    uint8_t* smem = align1024(smem_raw);
+    uint8_t* smem = smem_align<1024>(smem_raw);
     // stage i: K tile at 2i*STAGE, V tile at (2i+1)*STAGE
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + 2 * kStagesSM * STAGE);
     uint16_t* ps_tile = reinterpret_cast<uint16_t*>(smem + 2 * kStagesSM * STAGE + 64);
@@ -825,6 +995,7 @@ __global__ void __launch_bounds__(kThreads) softmax_bf16_kernel(const __grid_con
     const int cnt = list_count(a, b, g, P);
     const Range r = split_range(cnt, a.S, s);
     const int nst = r.end > r.start ? (r.end - r.start + PPS - 1) / PPS : 0;
+    tab_fill(a, b, g, r, P);
 
     float acc[NT][MTW][4];
     float mrun[NT], lrun[NT];
@@ -1017,12 +1188,14 @@ __global__ void __launch_bounds__(kThreads) softmax_f32_kernel(const float* __re
                                                                const float* __restrict__ v_pool, int ps,
                                                                const AttnArgs a)
 {
+    pdl_enter();
     __shared__ float sc[64 * 8];
     const int b = blockIdx.z, g = blockIdx.y, s = blockIdx.x, tid = threadIdx.x;
     const int L = a.seq_lens[b];
     const int P = pages_of(L, ps, a.max_pages, a.status);
     const int cnt = list_count(a, b, g, P);
     const Range r = split_range(cnt, a.S, s);
+    tab_fill(a, b, g, r, P);
     // thread w < G*D owns (head, d) pairs w, w + kThreads, ...
     constexpr int PER = (8 * D + kThreads - 1) / kThreads;
     float m[PER], l[PER];
@@ -1078,6 +1251,7 @@ __global__ void __launch_bounds__(kThreads) softmax_f32_kernel(const float* __re
 // ====================================================================== self test
 __global__ void selftest_timeout_kernel(uint64_t limit_ns, int32_t* status)
 {
+    pdl_enter();
     __shared__ uint64_t bar;
     if (threadIdx.x == 0) {
         mbar_init(&bar, 2);   // two arrivals expected, only one ever comes
@@ -1100,11 +1274,12 @@ static int launch_entmax_bf16(const AttnArgs& a, int B, const CUtensorMap* kmap,
     const int pv_smem = kStagesPV * kStageTok * D * 2 + 1024 + 64 + 8 * NT * (kStageTok + kPsPad) * 2;
     if (ensure_smem((const void*)qk_bf16_kernel<D, PS, NT>, qk_smem)) return ENTMAXKV_CUDA_ERROR;
     if (ensure_smem((const void*)pv_bf16_kernel<D, PS, NT>, pv_smem)) return ENTMAXKV_CUDA_ERROR;
-    qk_bf16_kernel<D, PS, NT><<<grid, kThreads, qk_smem, stream>>>(*kmap, a);
+    launch_pdl(qk_bf16_kernel<D, PS, NT>, dim3(grid), dim3(kThreads), qk_smem, stream, *kmap, a);
     if (cudaGetLastError() != cudaSuccess) return ENTMAXKV_CUDA_ERROR;
-    tau_kernel<<<dim3(a.H_q, B), kTauBlock, 0, stream>>>(PS, a);
+    if (ensure_smem((const void*)tau_kernel, kTauSmem)) return ENTMAXKV_CUDA_ERROR;
+    launch_pdl(tau_kernel, dim3(dim3(a.H_q, B)), dim3(kTauBlock), kTauSmem, stream, PS, a);
     if (cudaGetLastError() != cudaSuccess) return ENTMAXKV_CUDA_ERROR;
-    pv_bf16_kernel<D, PS, NT><<<grid, kThreads, pv_smem, stream>>>(*vmap, a);
+    launch_pdl(pv_bf16_kernel<D, PS, NT>, dim3(grid), dim3(kThreads), pv_smem, stream, *vmap, a);
     return cudaGetLastError() == cudaSuccess ? ENTMAXKV_OK : ENTMAXKV_CUDA_ERROR;
 }
 
@@ -1112,11 +1287,12 @@ template <int D>
 static int launch_entmax_f32(const entmaxkv_pool& pool, const AttnArgs& a, int B, cudaStream_t stream)
 {
     dim3 grid(a.S, a.H_kv, B);
-    qk_f32_kernel<D><<<grid, kThreads, 0, stream>>>((const float*)pool.k_pool, pool.ps, a);
+    launch_pdl(qk_f32_kernel<D>, dim3(grid), dim3(kThreads), 0, stream, (const float*)pool.k_pool, pool.ps, a);
     if (cudaGetLastError() != cudaSuccess) return ENTMAXKV_CUDA_ERROR;
-    tau_kernel<<<dim3(a.H_q, B), kTauBlock, 0, stream>>>(pool.ps, a);
+    if (ensure_smem((const void*)tau_kernel, kTauSmem)) return ENTMAXKV_CUDA_ERROR;
+    launch_pdl(tau_kernel, dim3(dim3(a.H_q, B)), dim3(kTauBlock), kTauSmem, stream, pool.ps, a);
     if (cudaGetLastError() != cudaSuccess) return ENTMAXKV_CUDA_ERROR;
-    pv_f32_kernel<D><<<grid, kThreads, 0, stream>>>((const float*)pool.v_pool, pool.ps, a);
+    launch_pdl(pv_f32_kernel<D>, dim3(grid), dim3(kThreads), 0, stream, (const float*)pool.v_pool, pool.ps, a);
     return cudaGetLastError() == cudaSuccess ? ENTMAXKV_OK : ENTMAXKV_CUDA_ERROR;
 }
 
@@ -1146,12 +1322,13 @@ static int launch_softmax_bf16(const AttnArgs& a, int B, const CUtensorMap* kmap
     dim3 grid(a.S, a.H_kv, B);
     const int smem = 2 * kStagesSM * kStageTok * D * 2 + 1024 + 64 + 8 * NT * (kStageTok + kPsPad) * 2;
     if (ensure_smem((const void*)softmax_bf16_kernel<D, PS, NT>, smem)) return ENTMAXKV_CUDA_ERROR;
-    softmax_bf16_kernel<D, PS, NT><<<grid, kThreads, smem, stream>>>(*kmap, *vmap, a);
+    launch_pdl(softmax_bf16_kernel<D, PS, NT>, dim3(grid), dim3(kThreads), smem, stream, *kmap, *vmap, a);
     return cudaGetLastError() == cudaSuccess ? ENTMAXKV_OK : ENTMAXKV_CUDA_ERROR;
 }
 
 __global__ void zero_counters_kernel(int32_t* counters, int n)
 {
+    pdl_enter();
     const int i = blockIdx.x * blockDim.x + threadIdx.x;
     if (i < n) counters[i] = 0;
 }
@@ -1160,14 +1337,14 @@ int launch_softmax_attend(const entmaxkv_pool& pool, const AttnArgs& a, int B, c
                           const CUtensorMap* vmap, cudaStream_t stream)
 {
     const int n = B * a.H_kv;
-    zero_counters_kernel<<<(n + 255) / 256, 256, 0, stream>>>(a.counters, n);
+    launch_pdl(zero_counters_kernel, dim3((n + 255) / 256), dim3(256), 0, stream, a.counters, n);
     if (cudaGetLastError() != cudaSuccess) return ENTMAXKV_CUDA_ERROR;
     if (pool.dtype == ENTMAXKV_F32) {
         dim3 grid(a.S, a.H_kv, B);
         if (pool.d == 128)
-            softmax_f32_kernel<128><<<grid, kThreads, 0, stream>>>((const float*)pool.k_pool, (const float*)pool.v_pool, pool.ps, a);
+            launch_pdl(softmax_f32_kernel<128>, dim3(grid), dim3(kThreads), 0, stream, (const float*)pool.k_pool, (const float*)pool.v_pool, pool.ps, a);
         else
-            softmax_f32_kernel<64><<<grid, kThreads, 0, stream>>>((const float*)pool.k_pool, (const float*)pool.v_pool, pool.ps, a);
+            launch_pdl(softmax_f32_kernel<64>, dim3(grid), dim3(kThreads), 0, stream, (const float*)pool.k_pool, (const float*)pool.v_pool, pool.ps, a);
         return cudaGetLastError() == cudaSuccess ? ENTMAXKV_OK : ENTMAXKV_CUDA_ERROR;
     }
     const bool g8 = a.G == 8;
@@ -1185,7 +1362,7 @@ int launch_softmax_attend(const entmaxkv_pool& pool, const AttnArgs& a, int B, c
 
 int launch_selftest_timeout(int64_t limit_ns, int32_t* status, cudaStream_t stream)
 {
-    selftest_timeout_kernel<<<1, 32, 0, stream>>>((uint64_t)limit_ns, status);
+    launch_pdl(selftest_timeout_kernel, dim3(1), dim3(32), 0, stream, (uint64_t)limit_ns, status);
     return cudaGetLastError() == cudaSuccess ? ENTMAXKV_OK : ENTMAXKV_CUDA_ERROR;
 }
 

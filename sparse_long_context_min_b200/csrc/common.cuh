@@ -114,6 +114,22 @@ EKV_DEV void tma_load_2d(void* dst, const CUtensorMap* map, uint64_t* bar, int x
         : "memory");
 }
 
+// 1-D bulk copy global -> shared (both 16-byte aligned, bytes a multiple of 16),
+// completion counted on `bar` in bytes.
+EKV_DEV void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar)
+{
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+                 ::"r"(smem_addr(dst)), "l"(src), "r"(bytes), "r"(smem_addr(bar))
+                 : "memory");
+}
+
+// Order this thread's generic-proxy shared-memory writes before later
+// async-proxy (TMA) accesses of the same memory.
+EKV_DEV void fence_proxy_async()
+{
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
 EKV_DEV void prefetch_tmap(const CUtensorMap* map)
 {
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
@@ -127,6 +143,30 @@ EKV_DEV uint32_t swz_addr(uint32_t base, int row, int chunk)
     const int half = chunk >> 3;
     const int c = chunk & 7;
     return base + half * (kStageTok * 128) + row * 128 + ((c ^ (row & 7)) << 4);
+}
+
+// Round a dynamic shared-memory base up to `align` bytes by offsetting from
+// the shared array itself (keeps the pointer in the shared address space, so
+// the compiler emits shared loads/stores instead of generic ones).
+template <int ALIGN>
+EKV_DEV uint8_t* smem_align(uint8_t* base)
+{
+    const uint32_t a = smem_addr(base);
+    return base + ((ALIGN - (a & (ALIGN - 1))) & (ALIGN - 1));
+}
+
+EKV_DEV uint4 lds128(uint32_t addr)
+{
+    uint4 v;
+    asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr));
+    return v;
+}
+
+EKV_DEV float4 lds128f(uint32_t addr)
+{
+    float4 v;
+    asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];" : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w) : "r"(addr));
+    return v;
 }
 
 // ---------------------------------------------------------------- tensor cores
@@ -167,6 +207,20 @@ EKV_DEV float warp_max(float v)
 {
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+    return v;
+}
+
+EKV_DEV double warp_max_d(double v)
+{
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v = fmax(v, __shfl_xor_sync(0xffffffffu, v, o));
+    return v;
+}
+
+EKV_DEV double warp_min_d(double v)
+{
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v = fmin(v, __shfl_xor_sync(0xffffffffu, v, o));
     return v;
 }
 
@@ -225,6 +279,17 @@ EKV_DEV uint32_t ordered_key(float f)
 }
 
 EKV_DEV int ceil_div(int a, int b) { return (a + b - 1) / b; }
+
+// Programmatic dependent launch: every kernel of the library starts with
+// pdl_enter(), which lets the next kernel in the stream begin launching and
+// then waits until the previous grid has completed and its writes are
+// visible.  Every CTA calls it before anything else, so completion stays
+// transitive along the stream.
+EKV_DEV void pdl_enter()
+{
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+}
 
 // Pages of a sequence of L tokens, clipped to the page-table row length; a
 // longer sequence is reported as ENTMAXKV_DEVICE_BOUNDS.

@@ -6,6 +6,7 @@
 #include <stdint.h>
 
 #include <cmath>
+#include <utility>
 
 #include "entmaxkv.h"
 
@@ -61,5 +62,26 @@ int launch_selftest_timeout(int64_t limit_ns, int32_t* status, cudaStream_t stre
 
 // set the dynamic shared memory limit of a kernel once per device
 int ensure_smem(const void* func, int bytes);
+
+// SM count of the current device
+int num_sms();
+
+// Launch with programmatic stream serialization (the kernel calls pdl_enter()).
+template <typename... KArgs, typename... Args>
+static cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                              Args&&... args)
+{
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+}
 
 }  // namespace ekv

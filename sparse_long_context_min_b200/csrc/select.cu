@@ -65,6 +65,7 @@ topk_kernel(const float* __restrict__ ub, const int32_t* __restrict__ seq_lens, 
             int max_pages, int budget, float budget_frac, int k_max, int32_t* __restrict__ sel,
             int32_t* __restrict__ sel_count, int32_t* status)
 {
+    pdl_enter();
     __shared__ TopkShared sh;
     const int b = blockIdx.y, g = blockIdx.x, tid = threadIdx.x;
     const int L = seq_lens[b];
@@ -227,6 +228,172 @@ topk_kernel(const float* __restrict__ ub, const int32_t* __restrict__ seq_lens, 
     }
 }
 
+// Register-resident variant: thread t holds keys [t*KPT, (t+1)*KPT) (ordered
+// integer form, -0 as +0); the same bucket narrowing and index-ordered
+// emission as topk_kernel, without returning to memory between passes.
+template <int KPT>
+__global__ void __launch_bounds__(kSelThreads, 1)
+topk_reg_kernel(const float* __restrict__ ub, const int32_t* __restrict__ seq_lens, int ps, int H_kv,
+                int max_pages, int budget, float budget_frac, int k_max, int32_t* __restrict__ sel,
+                int32_t* __restrict__ sel_count, int32_t* status)
+{
+    pdl_enter();
+    __shared__ TopkShared sh;
+    const int b = blockIdx.y, g = blockIdx.x, tid = threadIdx.x;
+    const int L = seq_lens[b];
+    const int P = pages_of(L, ps, max_pages, status);
+    int k = budget >= 0 ? budget : (int)ceil((double)budget_frac * (double)P);
+    k = min(k, P);
+    if (k > k_max) {
+        if (tid == 0) report(status, ENTMAXKV_DEVICE_BOUNDS);
+        k = k_max;
+    }
+    const float* keys = ub + ((size_t)b * H_kv + g) * max_pages;
+    int32_t* out = sel + ((size_t)b * H_kv + g) * k_max;
+    if (k <= 0 || k >= P) {
+        const int n = k <= 0 ? 0 : P;
+        for (int i = tid; i < n; i += kSelThreads) out[i] = i;
+        if (tid == 0) sel_count[(size_t)b * H_kv + g] = n;
+        return;
+    }
+    // keys of this thread (absent entries become the smallest float)
+    const int i0 = tid * KPT;
+    float kv[KPT];
+#pragma unroll
+    for (int e = 0; e < KPT; ++e) {
+        const int i = i0 + e;
+        float v = i < P ? __ldg(keys + i) : -INFINITY;
+        if (v == 0.f) v = 0.f;
+        kv[e] = v;
+    }
+    auto inr = [&](int e, float lo, float hi) { return i0 + e < P && kv[e] >= lo && kv[e] <= hi; };
+
+    float lo_v = -INFINITY, hi_v = INFINITY;
+    int need = k;
+    bool done = false;
+    unsigned int thr_key = 0;
+    int thr_idx = 0;
+    for (int round = 0; round < 8 && !done; ++round) {
+        float mn = INFINITY, mx = -INFINITY;
+#pragma unroll
+        for (int e = 0; e < KPT; ++e)
+            if (inr(e, lo_v, hi_v)) {
+                mn = fminf(mn, kv[e]);
+                mx = fmaxf(mx, kv[e]);
+            }
+        mn = block_min(mn, sh.redf);
+        mx = block_max(mx, sh.redf);
+        if (mn == mx) {
+            thr_key = ordered_key(mn);
+            int c = 0;
+#pragma unroll
+            for (int e = 0; e < KPT; ++e) c += inr(e, mn, mn);
+            const int incl = block_scan_incl(c, sh.wsum);
+            int before = incl - c;
+#pragma unroll
+            for (int e = 0; e < KPT; ++e)
+                if (inr(e, mn, mn)) {
+                    if (before == need - 1) sh.thr_idx = i0 + e;
+                    ++before;
+                }
+            __syncthreads();
+            thr_idx = sh.thr_idx;
+            done = true;
+            break;
+        }
+        const float w = (float)kBins / (mx - mn);
+        for (int i = tid; i < kBins; i += kSelThreads) sh.hist[i] = 0;
+        __syncthreads();
+        // bucket of key e in this round (-1 when outside the range); recomputed, not stored
+        auto bucket = [&](int e) { return inr(e, mn, mx) ? (int)fminf((kv[e] - mn) * w, (float)(kBins - 1)) : -1; };
+#pragma unroll
+        for (int e = 0; e < KPT; ++e) {
+            const int bk = bucket(e);
+            if (bk >= 0) atomicAdd(&sh.hist[bk], 1);
+        }
+        __syncthreads();
+        const int bA = kBins - 1 - 2 * tid, bB = bA - 1;
+        const int cA = sh.hist[bA], cB = sh.hist[bB];
+        const int incl = block_scan_incl(cA + cB, sh.wsum);
+        const int above = incl - cA - cB;
+        if (above < need && need <= above + cA) {
+            sh.bucket = bA;
+            sh.need = need - above;
+        } else if (above + cA < need && need <= above + cA + cB) {
+            sh.bucket = bB;
+            sh.need = need - above - cA;
+        }
+        __syncthreads();
+        const int T = sh.bucket;
+        need = sh.need;
+        float bmn = INFINITY, bmx = -INFINITY;
+#pragma unroll
+        for (int e = 0; e < KPT; ++e)
+            if (bucket(e) == T) {
+                bmn = fminf(bmn, kv[e]);
+                bmx = fmaxf(bmx, kv[e]);
+            }
+        bmn = block_min(bmn, sh.redf);
+        bmx = block_max(bmx, sh.redf);
+        lo_v = bmn;
+        hi_v = bmx;
+        const int cnt = sh.hist[T];
+        if (cnt <= kRankCap && bmn != bmx) {
+            if (tid == 0) sh.ncand = 0;
+            __syncthreads();
+#pragma unroll
+            for (int e = 0; e < KPT; ++e)
+                if (bucket(e) == T) {
+                    const int slot = atomicAdd(&sh.ncand, 1);
+                    if (slot < kRankCap)
+                        sh.cand[slot] = ((unsigned long long)ordered_key(kv[e]) << 32) |
+                                        (unsigned long long)(0xFFFFFFFFu - (unsigned)(i0 + e));
+                }
+            __syncthreads();
+            const int nc = min(sh.ncand, kRankCap);
+            if (tid < nc) {
+                const unsigned long long me = sh.cand[tid];
+                int rank = 0;
+                for (int j = 0; j < nc; ++j) rank += (sh.cand[j] > me);
+                if (rank == need - 1) {
+                    sh.thr_key = (unsigned)(me >> 32);
+                    sh.thr_idx = (int)(0xFFFFFFFFu - (unsigned)(me & 0xFFFFFFFFull));
+                }
+            }
+            __syncthreads();
+            thr_key = sh.thr_key;
+            thr_idx = sh.thr_idx;
+            done = true;
+        }
+        __syncthreads();
+    }
+    if (!done) {
+        if (tid == 0) report(status, ENTMAXKV_DEVICE_BOUNDS);
+        thr_key = 0xFFFFFFFFu;
+        thr_idx = -1;
+    }
+    int c = 0;
+#pragma unroll
+    for (int e = 0; e < KPT; ++e) {
+        const unsigned kk = ordered_key(kv[e]);
+        c += (i0 + e < P) && ((kk > thr_key) || (kk == thr_key && i0 + e <= thr_idx));
+    }
+    const int incl = block_scan_incl(c, sh.wsum);
+    int pos = incl - c;
+#pragma unroll
+    for (int e = 0; e < KPT; ++e) {
+        const unsigned kk = ordered_key(kv[e]);
+        if ((i0 + e < P) && ((kk > thr_key) || (kk == thr_key && i0 + e <= thr_idx))) {
+            if (pos < k_max) out[pos] = i0 + e;
+            ++pos;
+        }
+    }
+    if (tid == kSelThreads - 1) {
+        if (incl != k) report(status, ENTMAXKV_DEVICE_BOUNDS);
+        sel_count[(size_t)b * H_kv + g] = min(incl, k_max);
+    }
+}
+
 // ---------------------------------------------------------------- Gaussian
 //
 // tau_hat per (sequence, query head): root of
@@ -263,6 +430,7 @@ __global__ void __launch_bounds__(kTauThreads)
 gauss_tau_kernel(const float* __restrict__ m, const float* __restrict__ v, const int32_t* __restrict__ seq_lens,
                  int ps, int H_q, int max_pages, float alpha, float* __restrict__ tau_hat)
 {
+    pdl_enter();
     __shared__ double red[kTauThreads / 32];
     __shared__ float redf[kTauThreads / 32];
     const int b = blockIdx.y, h = blockIdx.x, tid = threadIdx.x;
@@ -312,6 +480,7 @@ gauss_keep_kernel(const float* __restrict__ est, const float* __restrict__ tau_h
                   float alpha, float delta, int k_max, int32_t* __restrict__ sel, int32_t* __restrict__ sel_count,
                   int32_t* status)
 {
+    pdl_enter();
     __shared__ int wsum[32];
     const int b = blockIdx.y, g = blockIdx.x, tid = threadIdx.x;
     const int L = seq_lens[b];
@@ -354,15 +523,30 @@ int launch_select(int mode, const float* ub, const float* m, const float* v, con
                   float* tau_hat, int32_t* status, cudaStream_t stream)
 {
     if (mode == ENTMAXKV_SELECT_TOPK) {
-        topk_kernel<<<dim3(H_kv, B), kSelThreads, 0, stream>>>(ub, seq_lens, ps, H_kv, max_pages, budget,
-                                                               budget_frac, k_max, sel, sel_count, status);
+        // every sequence has at most max_pages pages: pick the register width from it
+        const dim3 grid(H_kv, B), block(kSelThreads);
+        if (max_pages <= 4 * kSelThreads)
+            launch_pdl(topk_reg_kernel<4>, grid, block, 0, stream, ub, seq_lens, ps, H_kv, max_pages, budget,
+                       budget_frac, k_max, sel, sel_count, status);
+        else if (max_pages <= 8 * kSelThreads)
+            launch_pdl(topk_reg_kernel<8>, grid, block, 0, stream, ub, seq_lens, ps, H_kv, max_pages, budget,
+                       budget_frac, k_max, sel, sel_count, status);
+        else if (max_pages <= 16 * kSelThreads)
+            launch_pdl(topk_reg_kernel<16>, grid, block, 0, stream, ub, seq_lens, ps, H_kv, max_pages, budget,
+                       budget_frac, k_max, sel, sel_count, status);
+        else if (max_pages <= 20 * kSelThreads)
+            launch_pdl(topk_reg_kernel<20>, grid, block, 0, stream, ub, seq_lens, ps, H_kv, max_pages, budget,
+                       budget_frac, k_max, sel, sel_count, status);
+        else
+            launch_pdl(topk_kernel, grid, block, 0, stream, ub, seq_lens, ps, H_kv, max_pages, budget, budget_frac,
+                       k_max, sel, sel_count, status);
     } else {
-        gauss_tau_kernel<<<dim3(H_q, B), kTauThreads, 0, stream>>>(m, v, seq_lens, ps, H_q, max_pages, alpha,
+        launch_pdl(gauss_tau_kernel, dim3(dim3(H_q, B)), dim3(kTauThreads), 0, stream, m, v, seq_lens, ps, H_q, max_pages, alpha,
                                                                    tau_hat);
         if (cudaGetLastError() != cudaSuccess) return ENTMAXKV_CUDA_ERROR;
         const int G = H_q / H_kv;
 #define EKV_KEEP(GG)                                                                                    \
-    gauss_keep_kernel<GG><<<dim3(H_kv, B), kSelThreads, 0, stream>>>(est, tau_hat, seq_lens, ps, H_q, \
+    launch_pdl(gauss_keep_kernel<GG>, dim3(dim3(H_kv, B)), dim3(kSelThreads), 0, stream, est, tau_hat, seq_lens, ps, H_q, \
                                                                      H_kv, max_pages, alpha, delta,    \
                                                                      k_max, sel, sel_count, status)
         switch (G) {
