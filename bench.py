@@ -27,6 +27,11 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 METRIC = "sparse entmax decode µs/step @1M ctx; achieved HBM GB/s vs 8 TB/s roofline"
+# DRAM bytes the scoring kernel read per (page, kv head) metadata row in an ncu
+# capture of the 2^18-token case (16,824,064 bytes for 4097 pages x 8 heads);
+# scaled by rows to the bench launch.  Must be re-measured when the scoring
+# kernel changes.
+SCORE_DRAM_BYTES_PER_ROW = 16824064 / (4097 * 8)
 HBM_NOMINAL_GBS = 8000.0
 PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
 FALLBACK_HBM_GBS = 6650.0
@@ -73,10 +78,11 @@ def barrier(world):
         torch.distributed.barrier()
 
 
-def max_over_ranks(x, world):
+def max_over_ranks(x, world, device="cuda"):
+    """The slowest rank's value (timings are reported as the max over ranks)."""
     if world == 1:
         return x
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    t = torch.tensor([x], dtype=torch.float64, device=device)
     torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
     return float(t.item())
 
@@ -133,12 +139,14 @@ class Clocks:
 
 
 # ---------------------------------------------------------------- workload
-def make_workload(context, rank):
+def make_workload(context, rank, device="cuda", appends=256):
+    """Rank r decodes its own independent sequence (seed offset by r); the page
+    table leaves room for `appends` decode tokens."""
     import dataclasses
     from sparse_long_context_min_b200 import workloads
     cfg = workloads.config(4)
-    cfg = dataclasses.replace(cfg, lengths=[context], seed=cfg.seed + 100 * rank, decode_steps=256)
-    return workloads.Workload(cfg, device="cuda")
+    cfg = dataclasses.replace(cfg, lengths=[context], seed=cfg.seed + 100 * rank, decode_steps=appends)
+    return workloads.Workload(cfg, device=device)
 
 
 def algorithmic_bytes(cfg, k_pages, v_pages, mode):
@@ -170,7 +178,9 @@ def run_native(args, rank, world, local):
     from sparse_long_context_min_b200.step import DecodeStep, GraphedStep, build_pool
 
     torch.manual_seed(0)
-    wl = make_workload(args.context, rank)
+    # tokens appended during the run: top-k (two graphs) + e2e + Gaussian (two graphs)
+    appends = 3 * (args.steps + args.warmup) + 2 * (max(3, args.steps // 4) + 3) + 64
+    wl = make_workload(args.context, rank, appends=appends)
     cfg = wl.cfg
     pool, seq_lens = build_pool(wl)
     torch.cuda.synchronize()
@@ -298,7 +308,8 @@ def run_native(args, rank, world, local):
             "peak_kind": peak_kind,
             "unit": "GB/s",
             "frac": round(score_gbs / peak, 4),
-            "traffic": None,
+            "traffic": round(SCORE_DRAM_BYTES_PER_ROW * sum(cfg.pages(b) for b in range(cfg.B)) * cfg.H_kv),
+            "traffic_note": "ncu dram__bytes_read+write of the 2^18-token case scaled by rows",
             "bytes_per_launch": by["score"],
         },
         "e2e": {"value": round(e2e_us, 2), "unit": "us/step", "h2d_bytes_per_step": h2d,
