@@ -58,7 +58,8 @@ typedef enum {
     ENTMAXKV_CUDA_ERROR = 3,     /* a CUDA runtime call or launch failed */
     ENTMAXKV_TIMEOUT = 4,        /* a bounded device wait ran out (device status) */
     ENTMAXKV_DEVICE_BOUNDS = 5,  /* a page id or index failed its device check */
-    ENTMAXKV_WORKSPACE = 6       /* workspace pointer NULL or ws_bytes too small */
+    ENTMAXKV_WORKSPACE = 6,      /* workspace pointer NULL or ws_bytes too small */
+    ENTMAXKV_STATIC_LIMIT = 7    /* needs more scratch than the built-in buffer holds */
 } entmaxkv_status;
 
 typedef enum { ENTMAXKV_F32 = 0, ENTMAXKV_BF16 = 1 } entmaxkv_dtype;
@@ -193,6 +194,34 @@ ENTMAXKV_API int entmaxkv_sparse_attend(const entmaxkv_pool* pool, const float* 
                            int32_t B, const int32_t* sel, const int32_t* sel_count, int32_t k_max,
                            float alpha, float scale, float* out, float* tau_out, int32_t* v_pages,
                            void* workspace, size_t ws_bytes, int32_t* status, void* stream);
+
+/*
+ * entmaxkv_sparse_attend for callers that cannot allocate device memory.  The
+ * paper has no counterpart: this is a deployment convenience.  Some callers
+ * may not call cudaMalloc when they decode -- code under CUDA stream capture
+ * (allocation is not allowed while capturing), hosts whose own allocator owns
+ * all device memory, latency-critical loops where an allocation or free would
+ * synchronise the device.  This call takes its scratch memory from a buffer
+ * built into the library (ENTMAXKV_STATIC_SCRATCH_BYTES, 16 MiB, held on every
+ * GPU that loads the library until the process exits) instead of a workspace.
+ *   Arguments, layouts and results are those of entmaxkv_sparse_attend.
+ *   Returns ENTMAXKV_STATIC_LIMIT, launching nothing, when
+ *   entmaxkv_workspace_size(ENTMAXKV_OP_SPARSE_ATTEND, ...) exceeds the buffer
+ *   (e.g. about 5 sequences of 2^20 tokens at a 1/64 budget with 32 query
+ *   heads of 128 dims).
+ *   The first call on a device looks up the buffer's device address on that
+ *   device (make it before any stream capture).  All calls share the buffer,
+ *   which keeps the last call's contents; the kernels reset what must start
+ *   at zero themselves.  Calls whose work overlaps on the GPU (other streams,
+ *   other threads) race on the buffer: serialise them.
+ */
+#define ENTMAXKV_STATIC_SCRATCH_BYTES ((size_t)16 << 20)
+ENTMAXKV_API int entmaxkv_sparse_attend_static(const entmaxkv_pool* pool, const float* q, int32_t H_q,
+                                  const int32_t* page_table, int32_t max_pages,
+                                  const int32_t* seq_lens, int32_t B, const int32_t* sel,
+                                  const int32_t* sel_count, int32_t k_max, float alpha, float scale,
+                                  float* out, float* tau_out, int32_t* v_pages, int32_t* status,
+                                  void* stream);
 
 /*
  * Full-cache alpha-entmax decode: entmaxkv_sparse_attend over every page of

@@ -14,7 +14,8 @@ import torch
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "_lib", "libentmaxkv.so")
 
-OK, INVALID_ARG, UNSUPPORTED, CUDA_ERROR, TIMEOUT, DEVICE_BOUNDS, WORKSPACE = range(7)
+OK, INVALID_ARG, UNSUPPORTED, CUDA_ERROR, TIMEOUT, DEVICE_BOUNDS, WORKSPACE, STATIC_LIMIT = range(8)
+STATIC_SCRATCH_BYTES = 16 << 20
 F32, BF16 = 0, 1
 SCORE_BBOX, SCORE_GAUSS = 0, 1
 SELECT_TOPK, SELECT_GAUSS = 0, 1
@@ -24,7 +25,7 @@ OP_SELECT, OP_SPARSE_ATTEND, OP_FULL_ENTMAX, OP_FULL_SOFTMAX = range(4)
 SYMBOLS = (
     "entmaxkv_append_metadata", "entmaxkv_score_pages", "entmaxkv_select", "entmaxkv_sparse_attend",
     "entmaxkv_full_entmax_decode", "entmaxkv_full_softmax_decode", "entmaxkv_workspace_size",
-    "entmaxkv_status_string", "entmaxkv_selftest_timeout",
+    "entmaxkv_status_string", "entmaxkv_selftest_timeout", "entmaxkv_sparse_attend_static",
 )
 
 
@@ -66,6 +67,7 @@ def lib():
         L.entmaxkv_status_string.argtypes = [I]
         L.entmaxkv_status_string.restype = ctypes.c_char_p
         L.entmaxkv_selftest_timeout.argtypes = [ctypes.c_int64, P, P]
+        L.entmaxkv_sparse_attend_static.argtypes = [PP, P, I, P, I, P, I, P, P, I, F, F, P, P, P, P, P]
         for name in SYMBOLS:
             if name not in ("entmaxkv_workspace_size", "entmaxkv_status_string"):
                 getattr(L, name).restype = ctypes.c_int
@@ -160,6 +162,16 @@ def sparse_attend(pool, q, page_table, seq_lens, sel, sel_count, alpha, scale, o
                                         scale, _p(out), _p(tau_out), _p(v_pages), _p(workspace),
                                         workspace.numel() * workspace.element_size(), _p(status),
                                         _stream(stream)), "sparse_attend")
+
+
+def sparse_attend_static(pool, q, page_table, seq_lens, sel, sel_count, alpha, scale, out, status,
+                         tau_out=None, v_pages=None, stream=None):
+    """sparse_attend with the library's built-in scratch buffer (no workspace)."""
+    B, H_q, _ = q.shape
+    _check(lib().entmaxkv_sparse_attend_static(pool.c, _p(q), H_q, _p(page_table), page_table.shape[1],
+                                               _p(seq_lens), B, _p(sel), _p(sel_count), sel.shape[2], alpha,
+                                               scale, _p(out), _p(tau_out), _p(v_pages), _p(status),
+                                               _stream(stream)), "sparse_attend_static")
 
 
 def full_entmax_decode(pool, q, page_table, seq_lens, alpha, scale, out, workspace, status,

@@ -323,6 +323,7 @@ const char* entmaxkv_status_string(int32_t code)
         case ENTMAXKV_TIMEOUT: return "bounded device wait timed out";
         case ENTMAXKV_DEVICE_BOUNDS: return "device index check failed (page id, list entry or count out of range)";
         case ENTMAXKV_WORKSPACE: return "workspace missing, misaligned or too small";
+        case ENTMAXKV_STATIC_LIMIT: return "problem needs more scratch than the built-in buffer holds";
         default: return "unknown status";
     }
 }
