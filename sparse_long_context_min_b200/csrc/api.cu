@@ -120,7 +120,7 @@ static int num_splits(int B, int H_kv, int list_pages)
 
 struct AttnLayout {
     int S;
-    size_t xbuf, opart, mlpart, lmax, tau, counters, total;
+    size_t xbuf, cmax, opart, mlpart, lmax, tau, counters, total;
 };
 
 static AttnLayout attn_layout(int op, int B, int H_q, int H_kv, int max_pages, int k_max, int ps, int d)
@@ -131,6 +131,8 @@ static AttnLayout attn_layout(int op, int B, int H_q, int H_kv, int max_pages, i
     size_t off = 0;
     L.xbuf = off;
     if (op != ENTMAXKV_OP_FULL_SOFTMAX) off += round256((size_t)B * H_q * list * ps * sizeof(float));
+    L.cmax = off;
+    if (op != ENTMAXKV_OP_FULL_SOFTMAX) off += round256((size_t)B * H_q * list * ((ps + 15) / 16) * sizeof(float));
     L.opart = off;
     off += round256((size_t)B * H_q * L.S * d * sizeof(float));
     L.mlpart = off;
@@ -180,6 +182,7 @@ static int attend_common(int op, const entmaxkv_pool* pool, const float* q, int 
     a.xscale = op == ENTMAXKV_OP_FULL_SOFTMAX ? scale : (alpha - 1.0f) * scale;
     char* ws = static_cast<char*>(workspace);
     a.xbuf = reinterpret_cast<float*>(ws + lay.xbuf);
+    a.cmax = reinterpret_cast<float*>(ws + lay.cmax);
     a.opart = reinterpret_cast<float*>(ws + lay.opart);
     a.mlpart = reinterpret_cast<float*>(ws + lay.mlpart);
     a.lmax = reinterpret_cast<float*>(ws + lay.lmax);

@@ -270,6 +270,7 @@ __global__ void __launch_bounds__(kThreads) qk_bf16_kernel(const __grid_constant
 
     const uint32_t sbase = smem_addr(smem);
     const size_t xstride = (size_t)a.k_max * PS;
+    const size_t cstride = (size_t)a.k_max * (PS / 16);
     for (int st = 0; st < nst; ++st) {
         const int slot = st % kStagesQK;
         if (!mbar_wait(&bars[slot], (st / kStagesQK) & 1, kWaitLimitNs)) {
@@ -296,24 +297,37 @@ __global__ void __launch_bounds__(kThreads) qk_bf16_kernel(const __grid_constant
 #pragma unroll
             for (int nt = 0; nt < NT; ++nt) mma_bf16(acc[nt], af, bq[nt][j][0], bq[nt][j][1]);
         }
+        // the warp's 16 rows lie in one page (16 divides PS): one list entry
         const int gi = lane >> 2, c = lane & 3;
-#pragma unroll
-        for (int rr = 0; rr < 2; ++rr) {
-            const int t = row0 + gi + 8 * rr;
-            const int idx = r.start + st * PPS + t / PS;
-            if (idx >= r.end) continue;
+        const int idx = r.start + st * PPS + row0 / PS;
+        if (idx < r.end) {
             int lp;
             const int phys = resolve(a, b, g, idx, P, lp, false);
-            const int prow = t % PS;
-            const bool valid = phys >= 0 && lp * PS + prow < L;
+            float cm[NT];
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) cm[nt] = -INFINITY;
+#pragma unroll
+            for (int rr = 0; rr < 2; ++rr) {
+                const int prow = (row0 + gi + 8 * rr) % PS;
+                const bool valid = phys >= 0 && lp * PS + prow < L;
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt) {
+                    const int head = 4 * nt + c;
+                    const float x = valid ? acc[nt][2 * rr] + acc[nt][2 * rr + 1] : -INFINITY;
+                    cm[nt] = fmaxf(cm[nt], x);
+                    if (head < a.G)
+                        a.xbuf[((size_t)b * a.H_q + (size_t)g * a.G + head) * xstride + (size_t)idx * PS + prow] = x;
+                }
+            }
+            // chunk maxima: the V pass decides from these which pages hold weight
 #pragma unroll
             for (int nt = 0; nt < NT; ++nt) {
+                const float m = group_lane_max(cm[nt]);
+                run[nt] = fmaxf(run[nt], m);
                 const int head = 4 * nt + c;
-                if (head < a.G) {
-                    const float x = valid ? acc[nt][2 * rr] + acc[nt][2 * rr + 1] : -INFINITY;
-                    run[nt] = fmaxf(run[nt], x);
-                    a.xbuf[((size_t)b * a.H_q + (size_t)g * a.G + head) * xstride + (size_t)idx * PS + prow] = x;
-                }
+                if (gi == 0 && head < a.G)
+                    a.cmax[((size_t)b * a.H_q + (size_t)g * a.G + head) * cstride + (size_t)idx * (PS / 16) +
+                           (row0 % PS) / 16] = m;
             }
         }
         __syncthreads();
@@ -426,8 +440,8 @@ __global__ void __launch_bounds__(kTauBlock) tau_kernel(int ps, const AttnArgs a
     __shared__ int ncand;
     __shared__ float redm[kTauWarps];
     __shared__ TauRed R;
-    __shared__ double scan[kTauWarps][5];
-    __shared__ double brk[2][kTauWarps];
+    __shared__ double scan[kTauWarps][3];
+    __shared__ double brk[1][kTauWarps];
     const int b = blockIdx.y, h = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int g = h / a.G;
     const int L = a.seq_lens[b];
@@ -452,20 +466,22 @@ __global__ void __launch_bounds__(kTauBlock) tau_kernel(int ps, const AttnArgs a
     if (tid == 0) ncand = 0;
     for (int i = tid; i < kTauBins; i += kTauBlock) hist[i] = 0;
     __syncthreads();
-    // --- compaction of {x > M - 1} (4 float4 per lane per round) + histogram
+    // --- compaction of {x > M - 1} + histogram.  Every thread issues all its
+    // loads of a round (8 float4) before using any of them.
     const float4* x4 = reinterpret_cast<const float4*>(x);
     const int n4 = n >> 2;
-    for (int base = warp * 32 * 4; base < n4; base += kTauBlock * 4) {
-        float v[16];
+    constexpr int U = 8;
+    for (int base = warp * 32 * U; base < n4; base += kTauBlock * U) {
+        float v[4 * U];
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
+        for (int u = 0; u < U; ++u) {
             const int i = base + u * 32 + lane;
             const float4 f = i < n4 ? x4[i] : make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY);
             v[4 * u] = f.x; v[4 * u + 1] = f.y; v[4 * u + 2] = f.z; v[4 * u + 3] = f.w;
         }
         int c = 0;
 #pragma unroll
-        for (int e = 0; e < 16; ++e) {
+        for (int e = 0; e < 4 * U; ++e) {
             const double d = (double)v[e] - thr;
             if (d > 0.0) {
                 ++c;
@@ -485,102 +501,74 @@ __global__ void __launch_bounds__(kTauBlock) tau_kernel(int ps, const AttnArgs a
         wbase = __shfl_sync(0xffffffffu, wbase, 31);
         int pos = wbase + incl - c;
 #pragma unroll
-        for (int e = 0; e < 16; ++e)
+        for (int e = 0; e < 4 * U; ++e)
             if ((double)v[e] > thr) {
                 if (pos < kTauCap) cand[pos] = v[e];
                 ++pos;
             }
     }
     __syncthreads();
-    // --- bracket tau from the histogram.  Bin j holds values in
-    // [e_j - eps, e_{j+1} + eps], e_j = thr + j / NB.  With lo_j = e_j - eps and
-    // hi_j = e_{j+1} + eps:
-    //   F(e_i) >= sum_{j > i}  c_j (lo_j - e_i)^r      (F_lower)
-    //   F(e_i) <= sum_{j >= i-1} c_j (hi_j - e_i)^r    (F_upper)
-    // expanded in suffix sums of c_j, c_j a_j, c_j a_j^2 (a = lo or hi).
+    // --- lower bracket of tau from the histogram.  Bin j holds values in
+    // [e_j, e_{j+1}], e_j = thr + j / NB (exact: x and thr are floats, the
+    // difference and the scaling by a power of two are exact in double), so
+    //   F(e_i) >= sum_{j > i} c_j (e_j - eps - e_i)^r = F_lower(e_i)
+    // expanded in suffix sums of c_j, c_j a_j, c_j a_j^2 with a_j = e_j - eps.
+    // tau >= the largest edge with F_lower >= 1 (and >= thr).
     constexpr int BPT = kTauBins / kTauBlock;            // bins per thread (4)
     const double w = 1.0 / kTauBins;
     const double eps = 4e-7 * fmax(1.0, fabs((double)M));
-    double loc[5] = {0, 0, 0, 0, 0};                     // c, c lo, c lo^2, c hi, c hi^2 over my bins
+    double loc[3] = {0, 0, 0};
     const int j0 = tid * BPT;
 #pragma unroll
     for (int k = 0; k < BPT; ++k) {
         const int j = j0 + k;
         const double c = (double)hist[j];
-        const double lo = thr + j * w - eps, hi = thr + (j + 1) * w + eps;
+        const double lo = thr + j * w - eps;
         loc[0] += c;
         loc[1] += c * lo;
         loc[2] += c * lo * lo;
-        loc[3] += c * hi;
-        loc[4] += c * hi * hi;
     }
-    // exclusive suffix scan over threads (bins above mine): reverse warp scan + warp totals
-    double suf[5];
+    double suf[3];
 #pragma unroll
-    for (int i = 0; i < 5; ++i) {
+    for (int i = 0; i < 3; ++i) {
         double v = loc[i];
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
             const double t = __shfl_down_sync(0xffffffffu, v, o);
             if (lane + o < 32) v += t;
         }
-        suf[i] = v;                                      // inclusive suffix within the warp
+        suf[i] = v;
     }
     if (lane == 0)
 #pragma unroll
-        for (int i = 0; i < 5; ++i) scan[warp][i] = suf[i];
+        for (int i = 0; i < 3; ++i) scan[warp][i] = suf[i];
     __syncthreads();
 #pragma unroll
-    for (int i = 0; i < 5; ++i) {
+    for (int i = 0; i < 3; ++i) {
         double above = 0.0;
         for (int ww = warp + 1; ww < kTauWarps; ++ww) above += scan[ww][i];
-        suf[i] = suf[i] - loc[i] + above;                // exclusive: bins of threads above
+        suf[i] = suf[i] - loc[i] + above;                // bins of the threads above mine
     }
-    // walk my bins from the top keeping suffix sums; evaluate both bounds at each edge
-    double best_lo = thr, best_hi = (double)M;
+    double best_lo = thr;
     {
-        double S[5];
-#pragma unroll
-        for (int i = 0; i < 5; ++i) S[i] = suf[i];        // sums over bins > my last bin
+        double S0 = suf[0], S1 = suf[1], S2 = suf[2];     // sums over bins > my last bin
         for (int k = BPT - 1; k >= 0; --k) {
-            const int j = j0 + k;                         // edge e_j (lower edge of bin j)
-            const double c = (double)hist[j];
-            const double lo = thr + j * w - eps, hi = thr + (j + 1) * w + eps;
+            const int j = j0 + k;
             const double e = thr + j * w;
-            // F_lower(e_j): bins > j  (S excludes bin j)
-            const double flo = a2 ? (S[1] - e * S[0]) : (S[2] - 2.0 * e * S[1] + e * e * S[0]);
-            // F_upper(e_j): bins >= j-1 (add bin j and bin j-1)
-            double c1 = S[0] + c, h1 = S[3] + c * hi, h2 = S[4] + c * hi * hi;
-            if (j > 0) {
-                const double cm = (double)hist[j - 1];
-                const double him = thr + j * w + eps;
-                c1 += cm;
-                h1 += cm * him;
-                h2 += cm * him * him;
-            }
-            const double fhi = a2 ? (h1 - e * c1) : (h2 - 2.0 * e * h1 + e * e * c1);
+            const double flo = a2 ? (S1 - e * S0) : (S2 - 2.0 * e * S1 + e * e * S0);
             if (flo >= 1.0) best_lo = fmax(best_lo, e);
-            if (fhi < 1.0) best_hi = fmin(best_hi, e);
-            S[0] += c;
-            S[1] += c * lo;
-            S[2] += c * lo * lo;
-            S[3] += c * hi;
-            S[4] += c * hi * hi;
+            const double c = (double)hist[j];
+            const double lo = e - eps;
+            S0 += c;
+            S1 += c * lo;
+            S2 += c * lo * lo;
         }
     }
     best_lo = warp_max_d(best_lo);
-    best_hi = warp_min_d(best_hi);
-    if (lane == 0) {
-        brk[0][warp] = best_lo;
-        brk[1][warp] = best_hi;
-    }
+    if (lane == 0) brk[0][warp] = best_lo;
     __syncthreads();
-    double lo_t = thr, hi_t = (double)M;
-    for (int ww = 0; ww < kTauWarps; ++ww) {
-        lo_t = fmax(lo_t, brk[0][ww]);
-        hi_t = fmin(hi_t, brk[1][ww]);
-    }
-    (void)hi_t;
+    double lo_t = thr;
+    for (int ww = 0; ww < kTauWarps; ++ww) lo_t = fmax(lo_t, brk[0][ww]);
     const bool spill = ncand > kTauCap;
     const float* src = spill ? x : cand;
     const int len = spill ? n : ncand;
@@ -655,24 +643,39 @@ EKV_DEV void reduce_splits(const AttnArgs& a, int b, int g)
     __syncthreads();
     if (!is_last) return;
     __threadfence();
-    for (int i = threadIdx.x; i < a.G * D; i += blockDim.x) {
-        const int head = i / D, dd = i % D;
-        const size_t row = (size_t)b * a.H_q + (size_t)g * a.G + head;
-        float acc = 0.f;
-        if (!SOFTMAX) {
-            // loads issued 8 at a time, added in split order (deterministic)
-            const float* src = a.opart + row * a.S * D + dd;
-            int s = 0;
-            for (; s + 8 <= a.S; s += 8) {
-                float t[8];
+    if (!SOFTMAX) {
+        // four outputs per thread; up to 16 partials in flight, added in split
+        // order (deterministic)
+        for (int i = threadIdx.x; i < a.G * D / 4; i += blockDim.x) {
+            const int head = 4 * i / D, dd = 4 * i % D;
+            const size_t row = (size_t)b * a.H_q + (size_t)g * a.G + head;
+            const float4* src = reinterpret_cast<const float4*>(a.opart + row * a.S * D + dd);
+            float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+            for (int s0 = 0; s0 < a.S; s0 += 16) {
+                float4 t[16];
 #pragma unroll
-                for (int u = 0; u < 8; ++u) t[u] = __ldcg(src + (size_t)(s + u) * D);
+                for (int u = 0; u < 16; ++u)
+                    if (s0 + u < a.S) t[u] = __ldcg(src + (size_t)(s0 + u) * (D / 4));
 #pragma unroll
-                for (int u = 0; u < 8; ++u) acc += t[u];
+                for (int u = 0; u < 16; ++u)
+                    if (s0 + u < a.S) {
+                        acc.x += t[u].x;
+                        acc.y += t[u].y;
+                        acc.z += t[u].z;
+                        acc.w += t[u].w;
+                    }
             }
-            for (; s < a.S; ++s) acc += __ldcg(src + (size_t)s * D);
-            a.out[row * D + dd] = acc;
-        } else {
+            float* o = a.out + row * D + dd;
+            o[0] = acc.x;
+            o[1] = acc.y;
+            o[2] = acc.z;
+            o[3] = acc.w;
+        }
+    } else {
+        for (int i = threadIdx.x; i < a.G * D; i += blockDim.x) {
+            const int head = i / D, dd = i % D;
+            const size_t row = (size_t)b * a.H_q + (size_t)g * a.G + head;
+            float acc = 0.f;
             float Mx = -INFINITY;
             for (int s = 0; s < a.S; ++s) Mx = fmaxf(Mx, __ldcg(&a.mlpart[(row * a.S + s) * 2]));
             float l = 0.f;
@@ -754,15 +757,24 @@ __global__ void __launch_bounds__(kThreads) pv_bf16_kernel(const __grid_constant
         for (int i = tid; i < wn; i += kThreads) flag[i] = 0;
         __syncthreads();
         {
-            constexpr int Q = PS / 4;           // float4 per (page, head)
-            const int items = wn * a.G * Q;
+            constexpr int C = PS / 16;          // 16-token chunk maxima per page
+            const size_t cstride = (size_t)a.k_max * C;
+            const int items = wn * a.G;
             for (int it = tid; it < items; it += kThreads) {
-                const int j = it / (a.G * Q), rem = it % (a.G * Q);
-                const int h = rem / Q, q4 = rem % Q;
-                const float4 v = *reinterpret_cast<const float4*>(
-                    a.xbuf + (row0h + h) * xstride + (size_t)(w0 + j) * PS + 4 * q4);
-                const float t = tau_s[h];
-                if (v.x > t || v.y > t || v.z > t || v.w > t) flag[j] = 1;
+                const int j = it / a.G, h = it % a.G;
+                const float* cp = a.cmax + (row0h + h) * cstride + (size_t)(w0 + j) * C;
+                float m = -INFINITY;
+                if constexpr (C % 4 == 0) {
+#pragma unroll
+                    for (int k = 0; k < C; k += 4) {
+                        const float4 v = *reinterpret_cast<const float4*>(cp + k);
+                        m = fmaxf(m, fmaxf(fmaxf(v.x, v.y), fmaxf(v.z, v.w)));
+                    }
+                } else {
+#pragma unroll
+                    for (int k = 0; k < C; ++k) m = fmaxf(m, cp[k]);
+                }
+                if (m > tau_s[h]) flag[j] = 1;
             }
         }
         __syncthreads();

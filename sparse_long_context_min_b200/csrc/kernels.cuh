@@ -27,6 +27,7 @@ struct AttnArgs {
     float alpha;
     float xscale;                  // (alpha - 1) * scale, or scale for softmax
     float* xbuf;                   // [B][H_q][k_max * ps] scores x of the listed tokens
+    float* cmax;                   // [B][H_q][k_max * ps / 16] largest x of each 16-token chunk (bf16 K pass)
     float* tau;                    // [B][H_q]
     float* opart;                  // [B][H_q][S][d] partial outputs
     float* mlpart;                 // [B][H_q][S][2] softmax running max and sum
