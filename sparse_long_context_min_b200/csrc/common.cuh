@@ -270,6 +270,60 @@ EKV_DEV float block_min(float v, float* red)
     return t;
 }
 
+// ---------------------------------------------------------------- clusters
+// Thread-block clusters: the CTAs of a cluster are co-scheduled on one GPC and
+// read each other's shared memory (distributed shared memory).  A CTA may
+// touch another CTA's shared memory only after a cluster barrier that both
+// have passed, and must not exit while another CTA may still read its own.
+EKV_DEV uint32_t cluster_rank()
+{
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+EKV_DEV void cluster_arrive() { asm volatile("barrier.cluster.arrive.release;" ::: "memory"); }
+EKV_DEV void cluster_wait() { asm volatile("barrier.cluster.wait.acquire;" ::: "memory"); }
+EKV_DEV void cluster_sync()
+{
+    cluster_arrive();
+    cluster_wait();
+}
+// Address, in the cluster's shared window, of this CTA's shared variable `p`
+// as held by the CTA of rank `rank`.
+EKV_DEV uint32_t dsmem(const void* p, uint32_t rank)
+{
+    uint32_t r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(smem_addr(p)), "r"(rank));
+    return r;
+}
+EKV_DEV float ld_dsmem_f32(uint32_t a)
+{
+    float v;
+    asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(a) : "memory");
+    return v;
+}
+EKV_DEV int ld_dsmem_s32(uint32_t a)
+{
+    int v;
+    asm volatile("ld.shared::cluster.s32 %0, [%1];" : "=r"(v) : "r"(a) : "memory");
+    return v;
+}
+EKV_DEV uint4 ld_dsmem_v4(uint32_t a)
+{
+    uint4 v;
+    asm volatile("ld.shared::cluster.v4.u32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "r"(a)
+                 : "memory");
+    return v;
+}
+EKV_DEV unsigned long long ld_dsmem_u64(uint32_t a)
+{
+    unsigned long long v;
+    asm volatile("ld.shared::cluster.u64 %0, [%1];" : "=l"(v) : "r"(a) : "memory");
+    return v;
+}
+
 // Ordered integer key of a float: larger float -> larger key; -0 maps like +0.
 EKV_DEV uint32_t ordered_key(float f)
 {

@@ -228,36 +228,73 @@ topk_kernel(const float* __restrict__ ub, const int32_t* __restrict__ seq_lens, 
     }
 }
 
-// Register-resident variant: thread t holds keys [t*KPT, (t+1)*KPT) (ordered
-// integer form, -0 as +0); the same bucket narrowing and index-ordered
-// emission as topk_kernel, without returning to memory between passes.
+// Cluster variant: the keys of one (sequence, kv head) are spread over a
+// cluster of kTopkCTAs CTAs, thread t of CTA r holding keys
+// [(r*kCThreads + t)*KPT, ... + KPT) in registers, so that every pass over the
+// keys runs on kTopkCTAs SMs.  Each round publishes per-CTA partial results
+// (range, histogram, candidates, counts) in shared memory and every CTA reads
+// all of them through distributed shared memory, so all CTAs take identical
+// decisions and meet the same cluster barriers.
+//  round: [min, max] of the keys in play; if equal, the keys in play are
+//         tied and the `need` lowest indices among them are kept; otherwise
+//         a 2048-bin histogram over a linear map of [min, max] gives the
+//         bucket T holding the need-th key; if T holds at most kCCap keys
+//         they are gathered and ranked exactly, else the next round
+//         narrows to T.
+//  emit:  kept pages in page order, offset by the kept counts of the CTAs
+//         of lower rank.
+constexpr int kTopkCTAs = 8;
+constexpr int kCThreads = 512;
+constexpr int kCBins = 2048;     // 4 per thread
+constexpr int kCCap = 1024;
+constexpr int kCRounds = 32;     // each round shrinks the range >= 2048x: covers every float range
+
+struct TopkClusterShared {
+    __align__(16) int hist[kCBins];          // this CTA's histogram of the round
+    unsigned long long lc[kCCap];            // this CTA's keys of the threshold bucket
+    unsigned long long mc[kCCap];            // the whole cluster's, merged
+    int wsum[32];
+    float redf[2][32];
+    float pub_mm[2];                         // this CTA's range of the keys in play
+    float g_mm[2];
+    int lcn;                                 // entries of lc
+    int pub_tie;                             // this CTA's tied keys (tie round)
+    int pub_kept;                            // this CTA's kept keys
+    int mc_off[kTopkCTAs + 1];
+    int before, total;
+    int T, need, cT;
+    unsigned int thr_key;
+    int thr_idx;
+};
+
 template <int KPT>
-__global__ void __launch_bounds__(kSelThreads, 1)
-topk_reg_kernel(const float* __restrict__ ub, const int32_t* __restrict__ seq_lens, int ps, int H_kv,
-                int max_pages, int budget, float budget_frac, int k_max, int32_t* __restrict__ sel,
-                int32_t* __restrict__ sel_count, int32_t* status)
+__global__ void __launch_bounds__(kCThreads)
+topk_cluster_kernel(const float* __restrict__ ub, const int32_t* __restrict__ seq_lens, int ps, int H_kv,
+                    int max_pages, int budget, float budget_frac, int k_max, int32_t* __restrict__ sel,
+                    int32_t* __restrict__ sel_count, int32_t* status)
 {
     pdl_enter();
-    __shared__ TopkShared sh;
-    const int b = blockIdx.y, g = blockIdx.x, tid = threadIdx.x;
+    __shared__ TopkClusterShared sh;
+    constexpr int C = kTopkCTAs;
+    const int r = (int)cluster_rank();
+    const int b = blockIdx.y, g = blockIdx.x / C, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int L = seq_lens[b];
-    const int P = pages_of(L, ps, max_pages, status);
+    const int P = pages_of(L, ps, max_pages, r == 0 ? status : nullptr);
     int k = budget >= 0 ? budget : (int)ceil((double)budget_frac * (double)P);
     k = min(k, P);
     if (k > k_max) {
-        if (tid == 0) report(status, ENTMAXKV_DEVICE_BOUNDS);
+        if (tid == 0 && r == 0) report(status, ENTMAXKV_DEVICE_BOUNDS);
         k = k_max;
     }
     const float* keys = ub + ((size_t)b * H_kv + g) * max_pages;
     int32_t* out = sel + ((size_t)b * H_kv + g) * k_max;
-    if (k <= 0 || k >= P) {
+    if (k <= 0 || k >= P) {   // the same on every CTA of the cluster: no barrier is met
         const int n = k <= 0 ? 0 : P;
-        for (int i = tid; i < n; i += kSelThreads) out[i] = i;
-        if (tid == 0) sel_count[(size_t)b * H_kv + g] = n;
+        for (int i = r * kCThreads + tid; i < n; i += C * kCThreads) out[i] = i;
+        if (tid == 0 && r == 0) sel_count[(size_t)b * H_kv + g] = n;
         return;
     }
-    // keys of this thread (absent entries become the smallest float)
-    const int i0 = tid * KPT;
+    const int i0 = (r * kCThreads + tid) * KPT;
     float kv[KPT];
 #pragma unroll
     for (int e = 0; e < KPT; ++e) {
@@ -266,95 +303,155 @@ topk_reg_kernel(const float* __restrict__ ub, const int32_t* __restrict__ seq_le
         if (v == 0.f) v = 0.f;
         kv[e] = v;
     }
-    auto inr = [&](int e, float lo, float hi) { return i0 + e < P && kv[e] >= lo && kv[e] <= hi; };
-
-    float lo_v = -INFINITY, hi_v = INFINITY;
+    // keys in play: valid, inside [lo_v, hi_v] and in bucket pT of the previous
+    // round's map (pmn, pw); round 0 takes every valid key
+    float lo_v = -INFINITY, hi_v = INFINITY, pmn = 0.f, pw = 0.f;
+    int pT = -1;
+    auto bucket_of = [](float v, float mn, float w) { return (int)fminf((v - mn) * w, (float)(kCBins - 1)); };
+    auto inplay = [&](int e) {
+        if (!(i0 + e < P && kv[e] >= lo_v && kv[e] <= hi_v)) return false;
+        return pT < 0 || bucket_of(kv[e], pmn, pw) == pT;
+    };
     int need = k;
-    bool done = false;
-    unsigned int thr_key = 0;
-    int thr_idx = 0;
-    for (int round = 0; round < 8 && !done; ++round) {
+    int mode = 0;           // 0 searching, 1 threshold (thr_key, thr_idx), 2 tie (thr_idx per thread)
+    unsigned int thr_key = 0xFFFFFFFFu;
+    int thr_idx = -1;
+    for (int round = 0; round < kCRounds && mode == 0; ++round) {
+        // --- range of the keys in play, over the cluster
         float mn = INFINITY, mx = -INFINITY;
 #pragma unroll
         for (int e = 0; e < KPT; ++e)
-            if (inr(e, lo_v, hi_v)) {
+            if (inplay(e)) {
                 mn = fminf(mn, kv[e]);
                 mx = fmaxf(mx, kv[e]);
             }
-        mn = block_min(mn, sh.redf);
-        mx = block_max(mx, sh.redf);
+        mn = warp_min(mn);
+        mx = warp_max(mx);
+        if (lane == 0) {
+            sh.redf[0][warp] = mn;
+            sh.redf[1][warp] = mx;
+        }
+        __syncthreads();
+        if (warp == 0) {
+            float a = lane < kCThreads / 32 ? sh.redf[0][lane] : INFINITY;
+            float c = lane < kCThreads / 32 ? sh.redf[1][lane] : -INFINITY;
+            a = warp_min(a);
+            c = warp_max(c);
+            if (lane == 0) {
+                sh.pub_mm[0] = a;
+                sh.pub_mm[1] = c;
+            }
+        }
+        cluster_sync();
+        if (warp == 0) {
+            float a = lane < C ? ld_dsmem_f32(dsmem(&sh.pub_mm[0], lane)) : INFINITY;
+            float c = lane < C ? ld_dsmem_f32(dsmem(&sh.pub_mm[1], lane)) : -INFINITY;
+            a = warp_min(a);
+            c = warp_max(c);
+            if (lane == 0) {
+                sh.g_mm[0] = a;
+                sh.g_mm[1] = c;
+            }
+        }
+        __syncthreads();
+        mn = sh.g_mm[0];
+        mx = sh.g_mm[1];
         if (mn == mx) {
+            // every key in play equals mn: keep the `need` lowest indices of them
             thr_key = ordered_key(mn);
             int c = 0;
 #pragma unroll
-            for (int e = 0; e < KPT; ++e) c += inr(e, mn, mn);
+            for (int e = 0; e < KPT; ++e) c += inplay(e);
             const int incl = block_scan_incl(c, sh.wsum);
-            int before = incl - c;
+            if (tid == kCThreads - 1) sh.pub_tie = incl;
+            cluster_sync();
+            if (warp == 0) {
+                int v = lane < r ? ld_dsmem_s32(dsmem(&sh.pub_tie, lane)) : 0;
+                v = warp_sum(v);
+                if (lane == 0) sh.before = v;
+            }
+            __syncthreads();
+            int rk = sh.before + incl - c;
 #pragma unroll
             for (int e = 0; e < KPT; ++e)
-                if (inr(e, mn, mn)) {
-                    if (before == need - 1) sh.thr_idx = i0 + e;
-                    ++before;
+                if (inplay(e)) {
+                    if (rk < need) thr_idx = i0 + e;   // ascending: the last kept one
+                    ++rk;
                 }
-            __syncthreads();
-            thr_idx = sh.thr_idx;
-            done = true;
+            mode = 2;
             break;
         }
-        const float w = (float)kBins / (mx - mn);
-        for (int i = tid; i < kBins; i += kSelThreads) sh.hist[i] = 0;
+        // --- histogram; this CTA's is read by the cluster after the barrier
+        const float w = (float)kCBins / (mx - mn);
+        for (int i = tid; i < kCBins; i += kCThreads) sh.hist[i] = 0;
         __syncthreads();
-        // bucket of key e in this round (-1 when outside the range); recomputed, not stored
-        auto bucket = [&](int e) { return inr(e, mn, mx) ? (int)fminf((kv[e] - mn) * w, (float)(kBins - 1)) : -1; };
-#pragma unroll
-        for (int e = 0; e < KPT; ++e) {
-            const int bk = bucket(e);
-            if (bk >= 0) atomicAdd(&sh.hist[bk], 1);
-        }
-        __syncthreads();
-        const int bA = kBins - 1 - 2 * tid, bB = bA - 1;
-        const int cA = sh.hist[bA], cB = sh.hist[bB];
-        const int incl = block_scan_incl(cA + cB, sh.wsum);
-        const int above = incl - cA - cB;
-        if (above < need && need <= above + cA) {
-            sh.bucket = bA;
-            sh.need = need - above;
-        } else if (above + cA < need && need <= above + cA + cB) {
-            sh.bucket = bB;
-            sh.need = need - above - cA;
-        }
-        __syncthreads();
-        const int T = sh.bucket;
-        need = sh.need;
-        float bmn = INFINITY, bmx = -INFINITY;
 #pragma unroll
         for (int e = 0; e < KPT; ++e)
-            if (bucket(e) == T) {
-                bmn = fminf(bmn, kv[e]);
-                bmx = fmaxf(bmx, kv[e]);
+            if (inplay(e)) atomicAdd(&sh.hist[bucket_of(kv[e], mn, w)], 1);
+        cluster_sync();
+        // thread t sums bins jb..jb+3 over the cluster (thread 0 the top four)
+        const int jb = kCBins - 4 * (tid + 1);
+        int hs[4] = {0, 0, 0, 0};
+#pragma unroll
+        for (int q = 0; q < C; ++q) {
+            const uint4 v = ld_dsmem_v4(dsmem(&sh.hist[jb], q));
+            hs[0] += (int)v.x;
+            hs[1] += (int)v.y;
+            hs[2] += (int)v.z;
+            hs[3] += (int)v.w;
+        }
+        const int s4 = hs[0] + hs[1] + hs[2] + hs[3];
+        const int incl = block_scan_incl(s4, sh.wsum);
+        int above = incl - s4;   // keys in bins above jb + 3
+#pragma unroll
+        for (int u = 3; u >= 0; --u) {
+            if (above < need && need <= above + hs[u]) {
+                sh.T = jb + u;
+                sh.need = need - above;
+                sh.cT = hs[u];
             }
-        bmn = block_min(bmn, sh.redf);
-        bmx = block_max(bmx, sh.redf);
-        lo_v = bmn;
-        hi_v = bmx;
-        const int cnt = sh.hist[T];
-        if (cnt <= kRankCap && bmn != bmx) {
-            if (tid == 0) sh.ncand = 0;
+            above += hs[u];
+        }
+        __syncthreads();
+        const int T = sh.T;
+        need = sh.need;
+        const int cT = sh.cT;
+        if (cT <= kCCap) {
+            // --- gather bucket T's keys from the cluster and rank them exactly
+            if (tid == 0) sh.lcn = 0;
             __syncthreads();
 #pragma unroll
             for (int e = 0; e < KPT; ++e)
-                if (bucket(e) == T) {
-                    const int slot = atomicAdd(&sh.ncand, 1);
-                    if (slot < kRankCap)
-                        sh.cand[slot] = ((unsigned long long)ordered_key(kv[e]) << 32) |
-                                        (unsigned long long)(0xFFFFFFFFu - (unsigned)(i0 + e));
+                if (inplay(e) && bucket_of(kv[e], mn, w) == T) {
+                    const int slot = atomicAdd(&sh.lcn, 1);
+                    sh.lc[slot] = ((unsigned long long)ordered_key(kv[e]) << 32) |
+                                  (unsigned long long)(0xFFFFFFFFu - (unsigned)(i0 + e));
                 }
+            cluster_sync();
+            if (warp == 0) {
+                const int n = lane < C ? ld_dsmem_s32(dsmem(&sh.lcn, lane)) : 0;
+                int x = n;
+#pragma unroll
+                for (int o = 1; o < 32; o <<= 1) {
+                    const int t = __shfl_up_sync(0xffffffffu, x, o);
+                    if (lane >= o) x += t;
+                }
+                if (lane < C) sh.mc_off[lane + 1] = x;
+                if (lane == 0) sh.mc_off[0] = 0;
+            }
             __syncthreads();
-            const int nc = min(sh.ncand, kRankCap);
-            if (tid < nc) {
-                const unsigned long long me = sh.cand[tid];
+#pragma unroll 1
+            for (int q = 0; q < C; ++q) {
+                const int o = sh.mc_off[q], n = sh.mc_off[q + 1] - o;
+                const uint32_t base = dsmem(&sh.lc[0], q);
+                for (int j = tid; j < n; j += kCThreads) sh.mc[o + j] = ld_dsmem_u64(base + 8u * (uint32_t)j);
+            }
+            __syncthreads();
+            const int nc = sh.mc_off[C];
+            for (int j = tid; j < nc; j += kCThreads) {
+                const unsigned long long me = sh.mc[j];
                 int rank = 0;
-                for (int j = 0; j < nc; ++j) rank += (sh.cand[j] > me);
+                for (int jj = 0; jj < nc; ++jj) rank += (sh.mc[jj] > me);
                 if (rank == need - 1) {
                     sh.thr_key = (unsigned)(me >> 32);
                     sh.thr_idx = (int)(0xFFFFFFFFu - (unsigned)(me & 0xFFFFFFFFull));
@@ -363,15 +460,18 @@ topk_reg_kernel(const float* __restrict__ ub, const int32_t* __restrict__ seq_le
             __syncthreads();
             thr_key = sh.thr_key;
             thr_idx = sh.thr_idx;
-            done = true;
+            mode = 1;
+        } else {
+            lo_v = mn;
+            hi_v = mx;
+            pmn = mn;
+            pw = w;
+            pT = T;
         }
-        __syncthreads();
     }
-    if (!done) {
-        if (tid == 0) report(status, ENTMAXKV_DEVICE_BOUNDS);
-        thr_key = 0xFFFFFFFFu;
-        thr_idx = -1;
-    }
+    if (mode == 0 && tid == 0 && r == 0) report(status, ENTMAXKV_DEVICE_BOUNDS);   // keeps nothing
+
+    // --- emit the kept pages in page order
     int c = 0;
 #pragma unroll
     for (int e = 0; e < KPT; ++e) {
@@ -379,7 +479,20 @@ topk_reg_kernel(const float* __restrict__ ub, const int32_t* __restrict__ seq_le
         c += (i0 + e < P) && ((kk > thr_key) || (kk == thr_key && i0 + e <= thr_idx));
     }
     const int incl = block_scan_incl(c, sh.wsum);
-    int pos = incl - c;
+    if (tid == kCThreads - 1) sh.pub_kept = incl;
+    cluster_sync();
+    if (warp == 0) {
+        const int v = lane < C ? ld_dsmem_s32(dsmem(&sh.pub_kept, lane)) : 0;
+        const int before = warp_sum(lane < r ? v : 0);
+        const int total = warp_sum(v);
+        if (lane == 0) {
+            sh.before = before;
+            sh.total = total;
+        }
+    }
+    __syncthreads();
+    cluster_arrive();   // this CTA reads no other CTA's shared memory from here on
+    int pos = sh.before + incl - c;
 #pragma unroll
     for (int e = 0; e < KPT; ++e) {
         const unsigned kk = ordered_key(kv[e]);
@@ -388,19 +501,22 @@ topk_reg_kernel(const float* __restrict__ ub, const int32_t* __restrict__ seq_le
             ++pos;
         }
     }
-    if (tid == kSelThreads - 1) {
-        if (incl != k) report(status, ENTMAXKV_DEVICE_BOUNDS);
-        sel_count[(size_t)b * H_kv + g] = min(incl, k_max);
+    if (tid == 0 && r == 0) {
+        if (sh.total != k) report(status, ENTMAXKV_DEVICE_BOUNDS);
+        sel_count[(size_t)b * H_kv + g] = min(sh.total, k_max);
     }
+    cluster_wait();     // no CTA leaves while another may still read its shared memory
 }
 
 // ---------------------------------------------------------------- Gaussian
 //
 // tau_hat per (sequence, query head): root of
-//   F(tau) = sum_p n_p E[((alpha-1) s_p - tau)_+^(1/(alpha-1))] - 1,
-// s_p ~ N(m_p, v_p), by bracketed Newton steps (F is convex and decreasing,
-// so a Newton step from the left never passes the root); a step that leaves
-// the bracket is replaced by bisection.
+//   F(tau) = sum_p n_p E[((alpha-1) s_p - tau)_+^(1/(alpha-1))] = 1,
+// s_p ~ N(m_p, v_p), by safeguarded Newton steps on log F (each term is
+// log-concave in tau, so the steps behave like Newton on a near-quadratic
+// function even where F spans many orders of magnitude); every evaluation
+// narrows a bracket [lo, hi] with F(lo) >= 1 > F(hi), and a step that leaves
+// it is replaced by bisection (or by doubling while no upper end is known).
 
 constexpr int kTauThreads = 512;
 
@@ -466,8 +582,17 @@ gauss_tau_kernel(const float* __restrict__ m, const float* __restrict__ v, const
         dF = block_sum(dF, red);
         if (F >= 1.0) lo = tau; else hi = tau;
         if (fabs(F - 1.0) < 1e-7 || (hi - lo) < 1e-7 * fmax(1.0, fabs(tau))) break;
-        double nt = dF > 0.0 ? tau + (F - 1.0) / dF : INFINITY;
-        if (!(nt > lo && nt < hi)) nt = isinf(hi) ? lo + fmax(1.0, 2.0 * (tau - lo + 0.5)) : 0.5 * (lo + hi);
+        // Newton step on log F: far left of the root F is exponential-like and a
+        // step on F itself would gain one e-fold at a time
+        double nt = (F > 0.0 && dF > 0.0) ? tau + F * log(F) / dF : INFINITY;
+        if (!(nt > lo && nt < hi)) {
+            nt = isinf(hi) ? lo + fmax(1.0, 2.0 * (tau - lo + 0.5)) : 0.5 * (lo + hi);
+        } else if (fabs(nt - tau) < 1e-6 * fmax(1.0, fabs(tau))) {
+            // the terms are evaluated in float: F is not known to better than
+            // about 1e-6 relative, so a smaller step is converged
+            tau = nt;
+            break;
+        }
         tau = nt;
     }
     if (tid == 0) tau_hat[(size_t)b * H_q + h] = (float)tau;
@@ -524,21 +649,19 @@ int launch_select(int mode, const float* ub, const float* m, const float* v, con
 {
     if (mode == ENTMAXKV_SELECT_TOPK) {
         // every sequence has at most max_pages pages: pick the register width from it
-        const dim3 grid(H_kv, B), block(kSelThreads);
-        if (max_pages <= 4 * kSelThreads)
-            launch_pdl(topk_reg_kernel<4>, grid, block, 0, stream, ub, seq_lens, ps, H_kv, max_pages, budget,
-                       budget_frac, k_max, sel, sel_count, status);
-        else if (max_pages <= 8 * kSelThreads)
-            launch_pdl(topk_reg_kernel<8>, grid, block, 0, stream, ub, seq_lens, ps, H_kv, max_pages, budget,
-                       budget_frac, k_max, sel, sel_count, status);
-        else if (max_pages <= 16 * kSelThreads)
-            launch_pdl(topk_reg_kernel<16>, grid, block, 0, stream, ub, seq_lens, ps, H_kv, max_pages, budget,
-                       budget_frac, k_max, sel, sel_count, status);
-        else if (max_pages <= 20 * kSelThreads)
-            launch_pdl(topk_reg_kernel<20>, grid, block, 0, stream, ub, seq_lens, ps, H_kv, max_pages, budget,
-                       budget_frac, k_max, sel, sel_count, status);
+        const dim3 grid(H_kv * kTopkCTAs, B), block(kCThreads);
+        constexpr int per = kTopkCTAs * kCThreads;
+#define EKV_TOPK(KPT) \
+    launch_pdl_cluster(topk_cluster_kernel<KPT>, grid, block, kTopkCTAs, 0, stream, ub, seq_lens, ps, H_kv, max_pages, \
+                       budget, budget_frac, k_max, sel, sel_count, status)
+        if (max_pages <= per) EKV_TOPK(1);
+        else if (max_pages <= 2 * per) EKV_TOPK(2);
+        else if (max_pages <= 4 * per) EKV_TOPK(4);
+        else if (max_pages <= 8 * per) EKV_TOPK(8);
+        else if (max_pages <= 16 * per) EKV_TOPK(16);
+#undef EKV_TOPK
         else
-            launch_pdl(topk_kernel, grid, block, 0, stream, ub, seq_lens, ps, H_kv, max_pages, budget, budget_frac,
+            launch_pdl(topk_kernel, dim3(H_kv, B), dim3(kSelThreads), 0, stream, ub, seq_lens, ps, H_kv, max_pages, budget, budget_frac,
                        k_max, sel, sel_count, status);
     } else {
         launch_pdl(gauss_tau_kernel, dim3(dim3(H_q, B)), dim3(kTauThreads), 0, stream, m, v, seq_lens, ps, H_q, max_pages, alpha,

@@ -152,6 +152,38 @@ def test_topk_ties_signed_zeros_and_budgets():
                 assert np.array_equal(sel[b, g, :c].cpu().numpy(), ref), (budget, b, g)
 
 
+def _topk_cases():
+    rng = np.random.default_rng(11)
+    big_tie = np.full(5000, 0.25, np.float32)
+    big_tie[rng.permutation(5000)[:100]] = 1.0          # threshold inside > 1024 equal keys
+    outlier = rng.random(5000).astype(np.float32)
+    outlier[17] = 1e6                                    # first bucket map squeezes the rest into one bucket
+    dense = (1.0 + np.arange(3000, dtype=np.float32) * np.float32(2.0 ** -22)).astype(np.float32)
+    dense[5] = -1e30
+    rng.shuffle(dense)                                   # 3000 distinct keys a few ulps apart
+    wide = rng.standard_normal(60000).astype(np.float32) # several keys per thread
+    return {"big_tie": big_tie, "outlier": outlier, "dense": dense, "wide": wide}
+
+
+@pytest.mark.parametrize("case", ["big_tie", "outlier", "dense", "wide"])
+def test_topk_narrowing_rounds(case):
+    """Key sets whose threshold bucket holds more than the exact-rank capacity,
+    so the selection narrows over several rounds (or ends in a tie round)."""
+    keys = _topk_cases()[case]
+    P = len(keys)
+    ub = torch.from_numpy(keys).reshape(1, 1, P).cuda()
+    seq_lens = torch.tensor([P * 16], dtype=torch.int32, device="cuda")
+    for budget in (1, 300, 2500, P - 1):
+        sel = torch.full((1, 1, budget), -7, dtype=torch.int32, device="cuda")
+        cnt = torch.empty(1, 1, dtype=torch.int32, device="cuda")
+        st = _status()
+        B.select(B.SELECT_TOPK, seq_lens, 16, 4, 1, P, budget, sel, cnt, st, ub=ub, budget=budget)
+        _assert_ok(st)
+        ref = select.topk(keys, budget)
+        assert int(cnt[0, 0]) == len(ref)
+        assert np.array_equal(sel[0, 0].cpu().numpy()[:len(ref)], ref), (case, budget)
+
+
 def test_score_gauss_bitexact(built):
     wl, pool, seq_lens, oseqs = built
     cfg = wl.cfg
