@@ -270,6 +270,21 @@ EKV_DEV float block_min(float v, float* red)
     return t;
 }
 
+// ---------------------------------------------------------------- cp.async
+// Per-thread asynchronous 16-byte global -> shared copies (L1 bypassed); a
+// thread waits only for its own groups, so a thread that reads back nothing
+// but what it copied itself needs no block barrier.
+EKV_DEV void cp_async16(uint32_t dst, const void* src)
+{
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
+EKV_DEV void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+EKV_DEV void cp_async_wait()
+{
+    asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
 // ---------------------------------------------------------------- clusters
 // Thread-block clusters: the CTAs of a cluster are co-scheduled on one GPC and
 // read each other's shared memory (distributed shared memory).  A CTA may

@@ -7,13 +7,14 @@
 //
 // Streaming kernel: eight threads share a metadata row (one page, one kv
 // head), thread k owning the k-th of 8 consecutive d-slices with its slice of
-// the query group held in registers.  Each thread reads its slice with 16-byte
-// loads, prefetching the next row while it computes the current one, forms
-// its slice sum as a chain of fp32 fused multiply-adds in ascending d, and the
-// 8 slice sums are combined by a fixed xor-shuffle tree
-// ((S0+S1)+(S2+S3))+((S4+S5)+(S6+S7)).  No shared memory, no block barrier:
-// at this size (tens of MB per call) fixed per-stage overheads cost more than
-// they hide.
+// the query group held in registers.  Each thread streams its own slices
+// through a private ring of shared-memory stages filled by 16-byte cp.async
+// copies kScoreStages - 1 rows ahead (the page-table entry of a row is loaded
+// one row earlier still), so the copies in flight are not bounded by
+// registers and no block barrier is ever needed.  A thread forms its slice
+// sum as a chain of fp32 fused multiply-adds in ascending d, and the 8 slice
+// sums are combined by a fixed xor-shuffle tree
+// ((S0+S1)+(S2+S3))+((S4+S5)+(S6+S7)).
 // That is the canonical order of entmaxkv.h: selection is decided on these
 // fp32 values, so nothing else may be fused or reordered (explicit
 // round-to-nearest intrinsics throughout).
@@ -25,6 +26,7 @@
 namespace ekv {
 
 constexpr int kScoreCTA = 512;
+constexpr int kScoreStages = 4;
 
 struct ZTable {
     float z[65];
@@ -42,6 +44,8 @@ struct ScoreShape {
     static constexpr int TPR = 8 * HS;                     // threads per row group
     static constexpr int CTA = (GAUSS || NV > 2) ? 256 : kScoreCTA;
     static constexpr int RG = CTA / TPR;                   // row groups per CTA
+    // shared memory: [stage][vector a|b][16-byte chunk][thread] + n[stage][thread]
+    static constexpr int SMEM = kScoreStages * (2 * NV * CTA * 16 + CTA * 4);
 };
 
 template <typename T>
@@ -95,11 +99,10 @@ EKV_DEV float slice_tree(float v)
     return v;
 }
 
-// Streaming kernel without shared memory or block barriers.  A row group of
-// 8 (or 16) threads owns one kv head g for the whole launch and walks the
-// (sequence, page) items j = first, first + step, ... of that head; thread k
-// of the group owns d-slice k.  The page id and the metadata slices of the
-// next item are loaded while the current one is computed.
+// A row group of 8 (or 16) threads owns one kv head g for the whole launch
+// and walks the (sequence, page) items j = first, first + step, ... of that
+// head; thread k of the group owns d-slice k.  Item j is page j % max_pages of
+// sequence j / max_pages, so its page-table entry is page_table[j].
 template <typename T, int D, int G, bool GAUSS>
 __global__ void __launch_bounds__(ScoreShape<T, D, G, GAUSS>::CTA, 1)
 score_kernel(const ScoreArgs a, const ZTable zt)
@@ -108,6 +111,8 @@ score_kernel(const ScoreArgs a, const ZTable zt)
     using S = ScoreShape<T, D, G, GAUSS>;
     using E = typename std::conditional<GAUSS, float, T>::type;
     using V = RowVec<E>;
+    constexpr int NST = kScoreStages;
+    extern __shared__ uint4 score_smem[];
     const int tid = threadIdx.x;
     const int w = tid % S::TPR, ks = w & 7, hs = w >> 3;
     const int rg = blockIdx.x * S::RG + tid / S::TPR;      // global row group
@@ -123,57 +128,63 @@ score_kernel(const ScoreArgs a, const ZTable zt)
     const uint8_t* basea = static_cast<const uint8_t*>(a.row_a) + (size_t)g * S::ROWB + ks * S::SLB;
     const uint8_t* baseb = static_cast<const uint8_t*>(a.row_b) + (size_t)g * S::ROWB + ks * S::SLB;
     const size_t pstride = (size_t)a.H_kv * S::ROWB;       // bytes between physical pages
+    const uint32_t sbase = smem_addr(score_smem);
+    // 16-byte chunk c of vector v (0: a, 1: b) of stage `slot`, this thread
+    auto chunk = [&](int slot, int v, int c) -> uint32_t {
+        return sbase + (uint32_t)((((slot * 2 + v) * S::NV + c) * S::CTA + tid) * 16);
+    };
+    int* nrow = reinterpret_cast<int*>(score_smem + NST * 2 * S::NV * S::CTA);   // [NST][CTA]
+
+    auto pt_load = [&](int j) -> int { return (valid_rg && j < items) ? __ldg(&a.page_table[j]) : -1; };
+    // copy item j's slices into stage `slot` (pt = its page-table entry); one group per call
+    auto issue = [&](int slot, int j, int pt) {
+        int n = 0;
+        if (valid_rg && j < items) {
+            const int b = j / a.max_pages, p = j - b * a.max_pages;
+            const int L = __ldg(&a.seq_lens[b]);
+            const int P = pages_of(L, a.ps, a.max_pages, a.status);
+            if (p < P) {
+                if (pt < 0 || pt >= a.num_phys) {
+                    if (w == 0) report(a.status, ENTMAXKV_DEVICE_BOUNDS);
+                } else {
+                    n = min(a.ps, L - p * a.ps);
+                    const uint8_t* pa = basea + (size_t)pt * pstride;
+                    const uint8_t* pb = baseb + (size_t)pt * pstride;
+#pragma unroll
+                    for (int c = 0; c < S::NV; ++c) {
+                        cp_async16(chunk(slot, 0, c), pa + 16 * c);
+                        cp_async16(chunk(slot, 1, c), pb + 16 * c);
+                    }
+                }
+            }
+        }
+        nrow[slot * S::CTA + tid] = n;
+        cp_async_commit();
+    };
+
+    // prologue: items 0 .. NST-2 in flight, the page-table entry of item NST-1 loading
+#pragma unroll
+    for (int t = 0; t < NST - 1; ++t) issue(t, first + t * step, pt_load(first + t * step));
+    int pt_next = pt_load(first + (NST - 1) * step);
 
     float qreg[S::HPT][S::SW];
     int qb = -1;
-    // item j -> (b, p, n, phys); phys < 0 for absent pages
-    auto info = [&](int j, int& b, int& p, int& n, int& phys) {
-        b = j / a.max_pages;
-        p = j - b * a.max_pages;
-        const int L = __ldg(&a.seq_lens[b]);
-        const int P = pages_of(L, a.ps, a.max_pages, a.status);
-        n = 0;
-        phys = -1;
-        if (p < P) {
-            phys = __ldg(&a.page_table[(size_t)b * a.max_pages + p]);
-            if (phys < 0 || phys >= a.num_phys) {
-                if (w == 0) report(a.status, ENTMAXKV_DEVICE_BOUNDS);
-                phys = -1;
-            } else {
-                n = min(a.ps, L - p * a.ps);
-            }
-        }
-    };
-    auto fetch = [&](int phys, uint4 (&ra)[S::NV], uint4 (&rb)[S::NV]) {
-        if (phys >= 0) {
-            const uint4* pa = reinterpret_cast<const uint4*>(basea + (size_t)phys * pstride);
-            const uint4* pb = reinterpret_cast<const uint4*>(baseb + (size_t)phys * pstride);
-#pragma unroll
-            for (int c = 0; c < S::NV; ++c) {
-                ra[c] = __ldg(pa + c);
-                rb[c] = __ldg(pb + c);
-            }
-        }
-    };
-
-    int b = 0, p = 0, n = 0, phys = -1;
-    uint4 ca[S::NV], cb[S::NV];
-    if (valid_rg && first < items) {
-        info(first, b, p, n, phys);
-        fetch(phys, ca, cb);
-    }
     // the trip count is uniform per warp (the shuffles below need every lane)
-    for (int j = first;; j += step) {
+    for (int t = 0;; ++t) {
+        const int j = first + t * step;
         const bool live = valid_rg && j < items;
         if (!__any_sync(0xffffffffu, live)) break;
-        // prefetch the next item
-        int b2 = 0, p2 = 0, n2 = 0, phys2 = -1;
-        uint4 na[S::NV], nb[S::NV];
-        if (valid_rg && j + step < items) {
-            info(j + step, b2, p2, n2, phys2);
-            fetch(phys2, na, nb);
+        const int slot = t % NST;
+        {   // keep NST - 1 items in flight
+            const int jn = j + (NST - 1) * step;
+            const int pt = pt_next;
+            pt_next = pt_load(jn + step);
+            issue((t + NST - 1) % NST, jn, pt);
         }
-        if (!live) n = 0;
+        cp_async_wait<NST - 1>();                          // this item's copies have landed
+        const int b = live ? j / a.max_pages : 0;
+        const int p = j - b * a.max_pages;
+        const int n = live ? nrow[slot * S::CTA + tid] : 0;
         if (live && b != qb) {
             const float* qg = a.q + ((size_t)b * a.H_q + (size_t)g * G + hs * S::HPT) * D + ks * S::SW;
 #pragma unroll
@@ -192,8 +203,8 @@ score_kernel(const ScoreArgs a, const ZTable zt)
 #pragma unroll
             for (int c = 0; c < S::NV; ++c) {
                 float fa[V::N], fb[V::N];
-                V::widen(ca[c], fa);
-                V::widen(cb[c], fb);
+                V::widen(lds128(chunk(slot, 0, c)), fa);
+                V::widen(lds128(chunk(slot, 1, c)), fb);
 #pragma unroll
                 for (int e = 0; e < V::N; ++e) {
 #pragma unroll
@@ -243,12 +254,278 @@ score_kernel(const ScoreArgs a, const ZTable zt)
                 }
             }
         }
-        b = b2; p = p2; n = n2; phys = phys2;
-#pragma unroll
-        for (int c = 0; c < S::NV; ++c) {
-            ca[c] = na[c];
-            cb[c] = nb[c];
+    }
+    cp_async_wait<0>();   // nothing may still be writing this CTA's shared memory at exit
+}
+
+// ---------------------------------------------------------------- bf16 boxes
+// Bounding-box scores of a bf16 cache, the scoring pass of every top-k decode
+// step.  Same canonical order as score_kernel; the work is split by role.
+//  * One producer warp walks the CTA's contiguous run of pages in chunks of
+//    PPS pages: it resolves each page (page-table entries loaded 32 at a time,
+//    ahead of use), writes (sequence, page, tokens) of the chunk's pages into
+//    the stage header and copies each page's k_min and k_max blocks (all kv
+//    heads, contiguous in the pool) with bulk copies (TMA) whose bytes
+//    complete the stage's `full` mbarrier.  It refills a stage once all
+//    consumer warps have arrived on its `empty` mbarrier.
+//  * kWsConsumers consumer warps each own kWsRounds x RPW fixed (page slot,
+//    kv head) rows of every stage, all of the same kv heads, so their query
+//    registers never change within a sequence.
+//    The head-dependent choice of k_max or k_min is a byte permute of the two
+//    packed bf16 words (one selector per head and word, built when the query
+//    is loaded), and two query heads advance their fma chains in one packed
+//    f32x2 fma (each lane an IEEE fma with round-to-nearest, as fmaf).
+// Every wait is bounded; a CTA meets one block barrier, after the barriers
+// are initialised.
+constexpr int kWsStages = 3;
+constexpr int kWsConsumers = 8;
+constexpr int kWsRounds = 4;    // row sets per stage and consumer warp
+
+template <int D, int G>
+struct BoxWsShape {
+    static constexpr int SW = D / 8;                  // coordinates per slice
+    static constexpr int WPS = SW / 2;                // packed bf16 words per slice
+    static constexpr int NV = SW * 2 / 16;            // 16-byte chunks per slice and vector
+    static constexpr int HPT = G >= 2 ? 2 : 1;        // query heads per thread
+    static constexpr int HS = G / HPT;                // threads sharing a slice
+    static constexpr int TPR = 8 * HS;                // threads per row (<= 32)
+    static constexpr int RPW = 32 / TPR;              // rows per consumer warp
+    static constexpr int SET = kWsConsumers * RPW;    // rows of one round of the consumer warps
+    static constexpr int SLOTS = kWsRounds * SET;     // rows per stage (= pages per stage x H_kv)
+    static constexpr int CTA = 32 * (kWsConsumers + 1);
+    static constexpr int ROWB = D * 2;                // bytes of one metadata vector
+    static constexpr int STAGEB = SLOTS * 2 * ROWB;   // k_min and k_max of every row of a stage
+    static constexpr int DATA = kWsStages * STAGEB;
+    // header per stage: SLOTS int4 {sequence or -1, page, tokens, 0}; then full[], empty[]
+    static constexpr int SMEM = DATA + kWsStages * SLOTS * 16 + kWsStages * 16;
+};
+
+EKV_DEV uint64_t pack2(float lo, float hi)
+{
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+    return r;
+}
+EKV_DEV void unpack2(uint64_t v, float& lo, float& hi)
+{
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+// two independent fmas, acc.lane = fma(x.lane, y.lane, acc.lane), round to nearest
+EKV_DEV void fma2(uint64_t& acc, uint64_t x, uint64_t y)
+{
+    asm("fma.rn.f32x2 %0, %1, %2, %0;" : "+l"(acc) : "l"(x), "l"(y));
+}
+
+template <int D, int G>
+__global__ void __launch_bounds__(BoxWsShape<D, G>::CTA, 2) score_box16_kernel(const ScoreArgs a)
+{
+    pdl_enter();
+    using S = BoxWsShape<D, G>;
+    constexpr int NST = kWsStages;
+    extern __shared__ __align__(128) uint8_t box_smem[];
+    int4* info = reinterpret_cast<int4*>(box_smem + S::DATA);                     // [NST][SLOTS]
+    uint64_t* full = reinterpret_cast<uint64_t*>(box_smem + S::DATA + NST * S::SLOTS * 16);
+    uint64_t* empty = full + NST;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int PPS = S::SLOTS / a.H_kv;                   // pages per stage (host checks H_kv | SLOTS)
+    const long long items = (long long)a.B * a.max_pages;
+    const long long nchunks = (items + PPS - 1) / PPS;
+    const long long per = (nchunks + gridDim.x - 1) / gridDim.x;
+    const long long c0 = blockIdx.x * per;
+    const int K = (int)max(0ll, min(nchunks, c0 + per) - c0);   // chunks of this CTA
+    const size_t vecb = (size_t)a.H_kv * S::ROWB;        // one page's block of one vector
+    if (tid == 0) {
+        for (int i = 0; i < NST; ++i) {
+            mbar_init(&full[i], 1);
+            mbar_init(&empty[i], kWsConsumers);
         }
+        fence_mbar_init();
+    }
+    __syncthreads();
+
+    if (warp == kWsConsumers) {
+        // ------------------------------------------------ producer
+        const long long j0 = c0 * PPS;                   // first item of the CTA
+        auto pt_load = [&](long long j) -> int {
+            return j < items && j < (c0 + K) * PPS ? __ldg(&a.page_table[j]) : -1;
+        };
+        int cur = pt_load(j0 + lane);                    // entries of items j0 + 32m + lane
+        int nxt = pt_load(j0 + 32 + lane);
+        int lb = -1, lL = 0, lP = 0;
+        const int per_batch = 32 / PPS;                  // chunks per batch of entries
+        // lane i < PPS walks items j = (c0 + k) * PPS + i as (sequence bb, page pp)
+        long long jl = c0 * PPS + lane;
+        int bb = (int)(jl / a.max_pages), pp = (int)(jl - (long long)bb * a.max_pages);
+        for (int k = 0; k < K; ++k) {
+            const int s = k % NST;
+            if (k >= NST && !mbar_wait(&empty[s], ((k / NST) - 1) & 1, kWaitLimitNs)) {
+                if (lane == 0) report(a.status, ENTMAXKV_TIMEOUT);
+                break;
+            }
+            const int kb = k % per_batch;
+            const int pt = __shfl_sync(0xffffffffu, cur, kb * PPS + (lane < PPS ? lane : 0));
+            if (kb == per_batch - 1) {
+                cur = nxt;
+                nxt = pt_load(j0 + (long long)(k + 1 + per_batch) * PPS + lane);
+            }
+            int n = 0;
+            if (lane < PPS) {
+                const bool in = jl < items;
+                if (in) {
+                    if (bb != lb) {
+                        lb = bb;
+                        lL = __ldg(&a.seq_lens[bb]);
+                        lP = pages_of(lL, a.ps, a.max_pages, a.status);
+                    }
+                    if (pp < lP) {
+                        if (pt < 0 || pt >= a.num_phys) report(a.status, ENTMAXKV_DEVICE_BOUNDS);
+                        else n = min(a.ps, lL - pp * a.ps);
+                    }
+                }
+                info[s * S::SLOTS + lane] = make_int4(in ? bb : -1, pp, n, 0);
+            }
+            jl += PPS;
+            pp += PPS;
+            while (pp >= a.max_pages) {
+                pp -= a.max_pages;
+                ++bb;
+            }
+            const unsigned copies = __ballot_sync(0xffffffffu, lane < PPS && n > 0);
+            __syncwarp();                                // header writes before the arrive
+            if (lane == 0) mbar_arrive_expect_tx(&full[s], (uint32_t)(__popc(copies) * 2 * vecb));
+            if (lane < PPS && n > 0) {
+                uint8_t* dst = box_smem + s * S::STAGEB + lane * 2 * vecb;
+                const size_t off = (size_t)pt * vecb;
+                bulk_load(dst, static_cast<const uint8_t*>(a.row_a) + off, (uint32_t)vecb, &full[s]);
+                bulk_load(dst + vecb, static_cast<const uint8_t*>(a.row_b) + off, (uint32_t)vecb, &full[s]);
+            }
+        }
+        return;   // the consumers keep the CTA alive until every copy has been consumed
+    }
+
+    // ---------------------------------------------------- consumers
+    const int w = lane % S::TPR, ks = w & 7, hs = w >> 3;
+    const int rw = lane / S::TPR;
+    const int slot = warp * S::RPW + rw;                 // row of round 0; round r adds r * SET
+    const int g = slot % a.H_kv, pi = slot / a.H_kv;     // kv head and page of this row (round 0)
+    const int ppr = S::SET / a.H_kv;                     // pages per round (host checks H_kv | SET)
+    const uint32_t rowoff = (uint32_t)(pi * 2 * vecb + g * S::ROWB + ks * S::SW * 2);
+    const uint32_t sbase = smem_addr(box_smem);
+    uint64_t qp[S::SW];                                  // (head 0, head 1) query pairs per coordinate
+    float qs[S::SW];                                     // single head (HPT == 1)
+    uint32_t sel[S::HPT][S::WPS];                        // byte-permute selectors
+    int qb = -1;
+    const float scale = a.scale;
+    for (int k = 0; k < K; ++k) {
+        const int s = k % NST;
+        const bool ok = mbar_wait(&full[s], (k / NST) & 1, kWaitLimitNs);
+        if (!__all_sync(0xffffffffu, ok)) {
+            if (lane == 0) report(a.status, ENTMAXKV_TIMEOUT);
+            break;
+        }
+#pragma unroll
+        for (int r = 0; r < kWsRounds; ++r) {
+            const int4 inf = info[s * S::SLOTS + pi + r * ppr];
+            const int b = inf.x, p = inf.y, n = inf.z;
+            if (b >= 0 && b != qb) {
+                const float* qg = a.q + ((size_t)b * a.H_q + (size_t)g * G + hs * S::HPT) * D + ks * S::SW;
+                float qv[S::HPT][S::SW];
+#pragma unroll
+                for (int i = 0; i < S::HPT; ++i)
+#pragma unroll
+                    for (int e = 0; e < S::SW; e += 4) {
+                        const float4 f = __ldg(reinterpret_cast<const float4*>(qg + (size_t)i * D + e));
+                        qv[i][e] = f.x; qv[i][e + 1] = f.y; qv[i][e + 2] = f.z; qv[i][e + 3] = f.w;
+                    }
+#pragma unroll
+                for (int i = 0; i < S::HPT; ++i)
+#pragma unroll
+                    for (int kk = 0; kk < S::WPS; ++kk)   // k_max (second operand) where q >= 0, else k_min
+                        sel[i][kk] = (qv[i][2 * kk] >= 0.f ? 0x0054u : 0x0010u) | (qv[i][2 * kk + 1] >= 0.f ? 0x7600u : 0x3200u);
+#pragma unroll
+                for (int e = 0; e < S::SW; ++e) {
+                    if (S::HPT == 2) qp[e] = pack2(qv[0][e], qv[S::HPT - 1][e]);
+                    else qs[e] = qv[0][e];
+                }
+                qb = b;
+            }
+            float acc[S::HPT];
+#pragma unroll
+            for (int i = 0; i < S::HPT; ++i) acc[i] = 0.f;
+            if (n > 0) {
+                const uint32_t src = sbase + (uint32_t)(s * S::STAGEB) + rowoff + (uint32_t)(r * ppr * 2 * vecb);
+                uint64_t acc2 = pack2(0.f, 0.f);
+#pragma unroll
+                for (int c = 0; c < S::NV; ++c) {
+                    const uint4 va = lds128(src + 16 * c);
+                    const uint4 vb = lds128(src + (uint32_t)vecb + 16 * c);
+                    const uint32_t wa[4] = {va.x, va.y, va.z, va.w};
+                    const uint32_t wb[4] = {vb.x, vb.y, vb.z, vb.w};
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk) {
+                        const int wd = 4 * c + kk, e = 2 * wd;
+                        if (S::HPT == 2) {
+                            const uint32_t d0 = __byte_perm(wa[kk], wb[kk], sel[0][wd]);
+                            const uint32_t d1 = __byte_perm(wa[kk], wb[kk], sel[S::HPT - 1][wd]);
+                            fma2(acc2, qp[e], pack2(__uint_as_float(d0 << 16), __uint_as_float(d1 << 16)));
+                            fma2(acc2, qp[e + 1],
+                                 pack2(__uint_as_float(d0 & 0xFFFF0000u), __uint_as_float(d1 & 0xFFFF0000u)));
+                        } else {
+                            const uint32_t d0 = __byte_perm(wa[kk], wb[kk], sel[0][wd]);
+                            acc[0] = __fmaf_rn(qs[e], __uint_as_float(d0 << 16), acc[0]);
+                            acc[0] = __fmaf_rn(qs[e + 1], __uint_as_float(d0 & 0xFFFF0000u), acc[0]);
+                        }
+                    }
+                }
+                if (S::HPT == 2) unpack2(acc2, acc[0], acc[S::HPT - 1]);
+            }
+            float best = -INFINITY;
+#pragma unroll
+            for (int i = 0; i < S::HPT; ++i) {
+                const float u = __fmul_rn(slice_tree(acc[i]), scale);
+                if (i == 0 || u > best) best = u;
+            }
+            if (S::HS > 1) best = fmaxf(best, __shfl_xor_sync(0xffffffffu, best, 8));
+            if (S::HS > 2) best = fmaxf(best, __shfl_xor_sync(0xffffffffu, best, 16));
+            if (best == 0.f) best = 0.f;   // -0 -> +0
+            if (b >= 0 && w == 0) a.ub[((size_t)b * a.H_kv + g) * a.max_pages + p] = n > 0 ? best : -INFINITY;
+        }
+        __syncwarp();                                    // every lane is done with stage s
+        if (lane == 0) mbar_arrive(&empty[s]);
+    }
+}
+
+template <int D, int G>
+static int launch_box16(const ScoreArgs& a, cudaStream_t stream)
+{
+    using S = BoxWsShape<D, G>;
+    static int occ[64] = {0};                              // resident CTAs per SM, per device
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev < 0 || dev >= 64) dev = 0;
+    if (ensure_smem((const void*)score_box16_kernel<D, G>, S::SMEM)) return ENTMAXKV_CUDA_ERROR;
+    if (occ[dev] == 0) {
+        int n = 1;
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, score_box16_kernel<D, G>, S::CTA, S::SMEM) !=
+                cudaSuccess || n < 1)
+            n = 1;
+        occ[dev] = n;
+    }
+    const int pps = S::SLOTS / a.H_kv;
+    const long long chunks = ((long long)a.B * a.max_pages + pps - 1) / pps;
+    const int grid = (int)std::max<long long>(1, std::min<long long>(chunks, (long long)occ[dev] * num_sms()));
+    launch_pdl(score_box16_kernel<D, G>, dim3(grid), dim3(S::CTA), S::SMEM, stream, a);
+    return cudaGetLastError() == cudaSuccess ? ENTMAXKV_OK : ENTMAXKV_CUDA_ERROR;
+}
+
+template <int D>
+static int dispatch_box16(int G, const ScoreArgs& a, cudaStream_t st)
+{
+    switch (G) {
+        case 1: return launch_box16<D, 1>(a, st);
+        case 2: return launch_box16<D, 2>(a, st);
+        case 4: return launch_box16<D, 4>(a, st);
+        default: return launch_box16<D, 8>(a, st);
     }
 }
 
@@ -260,9 +537,10 @@ static int launch_score_t(const ScoreArgs& a, const ZTable& zt, cudaStream_t str
     int dev = 0;
     cudaGetDevice(&dev);
     if (dev < 0 || dev >= 64) dev = 0;
+    if (ensure_smem((const void*)score_kernel<T, D, G, GAUSS>, S::SMEM)) return ENTMAXKV_CUDA_ERROR;
     if (occ[dev] == 0) {
         int n = 1;
-        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, score_kernel<T, D, G, GAUSS>, S::CTA, 0) !=
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, score_kernel<T, D, G, GAUSS>, S::CTA, S::SMEM) !=
                 cudaSuccess || n < 1)
             n = 1;
         occ[dev] = n;
@@ -271,7 +549,7 @@ static int launch_score_t(const ScoreArgs& a, const ZTable& zt, cudaStream_t str
     const long long want = (rows + S::RG - 1) / S::RG;
     const int grid = (int)std::max<long long>(1, std::min<long long>(want, (long long)occ[dev] * num_sms()));
     if ((long long)grid * S::RG < a.H_kv) return ENTMAXKV_UNSUPPORTED;   // at least one group per kv head
-    launch_pdl(score_kernel<T, D, G, GAUSS>, dim3(grid), dim3(S::CTA), 0, stream, a, zt);
+    launch_pdl(score_kernel<T, D, G, GAUSS>, dim3(grid), dim3(S::CTA), S::SMEM, stream, a, zt);
     return cudaGetLastError() == cudaSuccess ? ENTMAXKV_OK : ENTMAXKV_CUDA_ERROR;
 }
 
@@ -314,9 +592,15 @@ int launch_score(const entmaxkv_pool& pool, const float* q, int H_q, const int32
     if (mode == ENTMAXKV_SCORE_BBOX) {
         a.row_a = pool.kmin;
         a.row_b = pool.kmax;
-        if (pool.dtype == ENTMAXKV_BF16)
+        if (pool.dtype == ENTMAXKV_BF16) {
+            // the role-split kernel needs H_kv to divide the rows of a round and
+            // at most 32 pages per stage (one producer lane each)
+            const int set = kWsConsumers * (32 / (8 * (G >= 2 ? G / 2 : 1)));
+            if (set % pool.H_kv == 0 && kWsRounds * set / pool.H_kv <= 32)
+                return pool.d == 128 ? dispatch_box16<128>(G, a, stream) : dispatch_box16<64>(G, a, stream);
             return pool.d == 128 ? dispatch_g<uint16_t, 128, false>(G, a, zt, stream)
                                  : dispatch_g<uint16_t, 64, false>(G, a, zt, stream);
+        }
         return pool.d == 128 ? dispatch_g<float, 128, false>(G, a, zt, stream)
                              : dispatch_g<float, 64, false>(G, a, zt, stream);
     }

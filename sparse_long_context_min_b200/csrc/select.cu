@@ -542,34 +542,58 @@ EKV_DEV void gauss_term(float mp, float sp, float tau, bool a2, float& g, float&
     }
 }
 
+// The pages of one (sequence, query head) are split over a cluster of
+// kGaussTauCTAs CTAs; every evaluation of F and F' is summed per CTA, the
+// per-CTA sums are exchanged through distributed shared memory (double
+// buffered by iteration parity) and added in rank order by every CTA, so all
+// CTAs hold the same values and take the same steps.
+constexpr int kGaussTauCTAs = 4;
+
 __global__ void __launch_bounds__(kTauThreads)
 gauss_tau_kernel(const float* __restrict__ m, const float* __restrict__ v, const int32_t* __restrict__ seq_lens,
                  int ps, int H_q, int max_pages, float alpha, float* __restrict__ tau_hat)
 {
     pdl_enter();
-    __shared__ double red[kTauThreads / 32];
-    __shared__ float redf[kTauThreads / 32];
-    const int b = blockIdx.y, h = blockIdx.x, tid = threadIdx.x;
+    constexpr int C = kGaussTauCTAs, NW = kTauThreads / 32;
+    __shared__ double red[2][NW];
+    __shared__ float redf[NW];
+    __shared__ double pub[2][2];          // this CTA's (F, F') of the iterations of each parity
+    __shared__ float pub_mx;
+    __shared__ double gsum[2];
+    __shared__ float gmx;
+    const int r = (int)cluster_rank();
+    const int b = blockIdx.y, h = blockIdx.x / C, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int L = seq_lens[b];
     const int P = pages_of(L, ps, max_pages, nullptr);
     const float am1 = alpha - 1.0f;
     const bool a2 = alpha == 2.0f;
     const float* mh = m + ((size_t)b * H_q + h) * max_pages;
     const float* vh = v + ((size_t)b * H_q + h) * max_pages;
-    if (P == 0) {
-        if (tid == 0) tau_hat[(size_t)b * H_q + h] = INFINITY;
+    if (P == 0) {   // the same on every CTA of the cluster: no barrier is met
+        if (tid == 0 && r == 0) tau_hat[(size_t)b * H_q + h] = INFINITY;
         return;
     }
+    const int chunk = (P + C - 1) / C;
+    const int p0 = min(P, r * chunk), p1 = min(P, p0 + chunk);
+
     float mx = -INFINITY;
-    for (int p = tid; p < P; p += kTauThreads) mx = fmaxf(mx, am1 * mh[p]);
+    for (int p = p0 + tid; p < p1; p += kTauThreads) mx = fmaxf(mx, am1 * mh[p]);
     mx = block_max(mx, redf);
-    double lo = (double)mx - 1.0;   // F(lo) >= 1 (Jensen: the top page alone gives >= 1)
+    if (tid == 0) pub_mx = mx;
+    cluster_sync();
+    if (warp == 0) {
+        float x = lane < C ? ld_dsmem_f32(dsmem(&pub_mx, lane)) : -INFINITY;
+        x = warp_max(x);
+        if (lane == 0) gmx = x;
+    }
+    __syncthreads();
+    double lo = (double)gmx - 1.0;   // F(lo) >= 1 (Jensen: the top page alone gives >= 1)
     double hi = INFINITY;
     double tau = lo;
     for (int it = 0; it < 60; ++it) {
         double F = 0.0, dF = 0.0;
         const float tf = (float)tau;
-        for (int p = tid; p < P; p += kTauThreads) {
+        for (int p = p0 + tid; p < p1; p += kTauThreads) {
             const float mp = am1 * mh[p];
             const float sp = am1 * sqrtf(fmaxf(vh[p], 0.f));
             const int n = min(ps, L - p * ps);
@@ -578,8 +602,36 @@ gauss_tau_kernel(const float* __restrict__ m, const float* __restrict__ v, const
             F += (double)n * gv;
             dF += (double)n * dg;
         }
-        F = block_sum(F, red);
-        dF = block_sum(dF, red);
+        F = warp_sum(F);
+        dF = warp_sum(dF);
+        if (lane == 0) {
+            red[0][warp] = F;
+            red[1][warp] = dF;
+        }
+        __syncthreads();
+        const int par = it & 1;
+        if (tid == 0) {
+            double f = 0.0, df = 0.0;
+            for (int w = 0; w < NW; ++w) {
+                f += red[0][w];
+                df += red[1][w];
+            }
+            pub[par][0] = f;
+            pub[par][1] = df;
+        }
+        cluster_sync();
+        if (tid == 0) {
+            double f = 0.0, df = 0.0;
+            for (int q = 0; q < C; ++q) {   // rank order: the same sums on every CTA
+                f += __longlong_as_double((long long)ld_dsmem_u64(dsmem(&pub[par][0], q)));
+                df += __longlong_as_double((long long)ld_dsmem_u64(dsmem(&pub[par][1], q)));
+            }
+            gsum[0] = f;
+            gsum[1] = df;
+        }
+        __syncthreads();
+        F = gsum[0];
+        dF = gsum[1];
         if (F >= 1.0) lo = tau; else hi = tau;
         if (fabs(F - 1.0) < 1e-7 || (hi - lo) < 1e-7 * fmax(1.0, fabs(tau))) break;
         // Newton step on log F: far left of the root F is exponential-like and a
@@ -595,51 +647,101 @@ gauss_tau_kernel(const float* __restrict__ m, const float* __restrict__ v, const
         }
         tau = nt;
     }
-    if (tid == 0) tau_hat[(size_t)b * H_q + h] = (float)tau;
+    if (tid == 0 && r == 0) tau_hat[(size_t)b * H_q + h] = (float)tau;
+    cluster_sync();   // no CTA leaves while another may still read its shared memory
 }
 
+// Keep rule: page p is kept when (alpha-1) * est_p >= tau_hat_h - delta for
+// some query head h of the group (fp32, as entmaxkv.h states).  The pages of
+// one (sequence, kv head) are split over a cluster of kTopkCTAs CTAs; kept
+// counts are exchanged through distributed shared memory so that each CTA
+// writes its kept pages at the right offset, in page order.  Flags of a tile
+// are computed with coalesced loads, then each thread emits 8 consecutive
+// pages.
+constexpr int kKeepThreads = 256;
+
 template <int G>
-__global__ void __launch_bounds__(kSelThreads)
+__global__ void __launch_bounds__(kKeepThreads)
 gauss_keep_kernel(const float* __restrict__ est, const float* __restrict__ tau_hat,
                   const int32_t* __restrict__ seq_lens, int ps, int H_q, int H_kv, int max_pages,
                   float alpha, float delta, int k_max, int32_t* __restrict__ sel, int32_t* __restrict__ sel_count,
                   int32_t* status)
 {
     pdl_enter();
+    constexpr int C = kTopkCTAs, TILE = kKeepThreads * 8;
+    __shared__ __align__(16) uint8_t flags[TILE];
     __shared__ int wsum[32];
-    const int b = blockIdx.y, g = blockIdx.x, tid = threadIdx.x;
+    __shared__ int pub_cnt;
+    __shared__ int s_before, s_total, s_tile;
+    const int r = (int)cluster_rank();
+    const int b = blockIdx.y, g = blockIdx.x / C, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int L = seq_lens[b];
-    const int P = pages_of(L, ps, max_pages, status);
+    const int P = pages_of(L, ps, max_pages, r == 0 ? status : nullptr);
     const float am1 = alpha - 1.0f;
     float rhs[G];
 #pragma unroll
     for (int h = 0; h < G; ++h) rhs[h] = __fsub_rn(tau_hat[(size_t)b * H_q + g * G + h], delta);
     const float* e0 = est + ((size_t)b * H_q + (size_t)g * G) * max_pages;
-    const int per = (P + kSelThreads - 1) / kSelThreads;
-    const int i0 = tid * per, i1 = min(P, i0 + per);
+    auto keep = [&](int p) {
+        bool k = false;
+#pragma unroll
+        for (int h = 0; h < G; ++h) k |= __fmul_rn(am1, e0[(size_t)h * max_pages + p]) >= rhs[h];
+        return k;
+    };
+    const int chunk = (P + C - 1) / C;
+    const int p0 = min(P, r * chunk), p1 = min(P, p0 + chunk);
+
     int c = 0;
-    for (int i = i0; i < i1; ++i) {
-        bool keep = false;
+    for (int t0 = p0; t0 < p1; t0 += TILE)
 #pragma unroll
-        for (int h = 0; h < G; ++h) keep |= __fmul_rn(am1, e0[(size_t)h * max_pages + i]) >= rhs[h];
-        c += keep;
-    }
-    const int incl = block_scan_incl(c, wsum);
-    int pos = incl - c;
-    int32_t* out = sel + ((size_t)b * H_kv + g) * k_max;
-    for (int i = i0; i < i1; ++i) {
-        bool keep = false;
-#pragma unroll
-        for (int h = 0; h < G; ++h) keep |= __fmul_rn(am1, e0[(size_t)h * max_pages + i]) >= rhs[h];
-        if (keep) {
-            if (pos < k_max) out[pos] = i;
-            ++pos;
+        for (int e = 0; e < 8; ++e) {
+            const int p = t0 + e * kKeepThreads + tid;
+            if (p < p1) c += keep(p);
+        }
+    c = block_sum(c, wsum);
+    if (tid == 0) pub_cnt = c;
+    cluster_sync();
+    if (warp == 0) {
+        const int x = lane < C ? ld_dsmem_s32(dsmem(&pub_cnt, lane)) : 0;
+        const int before = warp_sum(lane < r ? x : 0);
+        const int total = warp_sum(x);
+        if (lane == 0) {
+            s_before = before;
+            s_total = total;
         }
     }
-    if (tid == kSelThreads - 1) {
-        if (incl > k_max) report(status, ENTMAXKV_DEVICE_BOUNDS);
-        sel_count[(size_t)b * H_kv + g] = min(incl, k_max);
+    __syncthreads();
+    cluster_arrive();   // this CTA reads no other CTA's shared memory from here on
+    int32_t* out = sel + ((size_t)b * H_kv + g) * k_max;
+    int pos = s_before;
+    for (int t0 = p0; t0 < p1; t0 += TILE) {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+            const int p = t0 + e * kKeepThreads + tid;
+            flags[e * kKeepThreads + tid] = p < p1 && keep(p);
+        }
+        __syncthreads();
+        const uint2 f8 = *reinterpret_cast<const uint2*>(&flags[tid * 8]);
+        const int n = __popc(f8.x) + __popc(f8.y);   // flags are 0 or 1
+        const int incl = block_scan_incl(n, wsum);
+        if (tid == kKeepThreads - 1) s_tile = incl;
+        int q = pos + incl - n;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+            const uint32_t word = e < 4 ? f8.x : f8.y;
+            if ((word >> (8 * (e & 3))) & 1u) {
+                if (q < k_max) out[q] = t0 + tid * 8 + e;
+                ++q;
+            }
+        }
+        __syncthreads();
+        pos += s_tile;
     }
+    if (tid == 0 && r == 0) {
+        if (s_total > k_max) report(status, ENTMAXKV_DEVICE_BOUNDS);
+        sel_count[(size_t)b * H_kv + g] = min(s_total, k_max);
+    }
+    cluster_wait();     // no CTA leaves while another may still read its shared memory
 }
 
 int launch_select(int mode, const float* ub, const float* m, const float* v, const float* est,
@@ -664,14 +766,13 @@ int launch_select(int mode, const float* ub, const float* m, const float* v, con
             launch_pdl(topk_kernel, dim3(H_kv, B), dim3(kSelThreads), 0, stream, ub, seq_lens, ps, H_kv, max_pages, budget, budget_frac,
                        k_max, sel, sel_count, status);
     } else {
-        launch_pdl(gauss_tau_kernel, dim3(dim3(H_q, B)), dim3(kTauThreads), 0, stream, m, v, seq_lens, ps, H_q, max_pages, alpha,
-                                                                   tau_hat);
+        launch_pdl_cluster(gauss_tau_kernel, dim3(H_q * kGaussTauCTAs, B), dim3(kTauThreads), kGaussTauCTAs, 0, stream,
+                           m, v, seq_lens, ps, H_q, max_pages, alpha, tau_hat);
         if (cudaGetLastError() != cudaSuccess) return ENTMAXKV_CUDA_ERROR;
         const int G = H_q / H_kv;
-#define EKV_KEEP(GG)                                                                                    \
-    launch_pdl(gauss_keep_kernel<GG>, dim3(dim3(H_kv, B)), dim3(kSelThreads), 0, stream, est, tau_hat, seq_lens, ps, H_q, \
-                                                                     H_kv, max_pages, alpha, delta,    \
-                                                                     k_max, sel, sel_count, status)
+#define EKV_KEEP(GG)                                                                                            \
+    launch_pdl_cluster(gauss_keep_kernel<GG>, dim3(H_kv * kTopkCTAs, B), dim3(kKeepThreads), kTopkCTAs, 0, stream, \
+                       est, tau_hat, seq_lens, ps, H_q, H_kv, max_pages, alpha, delta, k_max, sel, sel_count, status)
         switch (G) {
             case 1: EKV_KEEP(1); break;
             case 2: EKV_KEEP(2); break;

@@ -152,6 +152,42 @@ def test_topk_ties_signed_zeros_and_budgets():
                 assert np.array_equal(sel[b, g, :c].cpu().numpy(), ref), (budget, b, g)
 
 
+# bf16 cache shapes besides the benchmark's (G = 4, d = 128, pages of 64):
+# one, two and eight query heads per kv head, d = 64, pages of 16
+SHAPES = {
+    "g1_d64_ps16": dict(H_q=8, H_kv=8, d=64, ps=16),
+    "g2_d64_ps16": dict(H_q=16, H_kv=8, d=64, ps=16),
+    "g8_d128_ps64": dict(H_q=64, H_kv=8, d=128, ps=64),
+    "g4_d64_ps64": dict(H_q=32, H_kv=8, d=64, ps=64),
+    "g8_d64_ps16": dict(H_q=32, H_kv=4, d=64, ps=16),
+    "g2_d128_ps16": dict(H_q=8, H_kv=4, d=128, ps=16),
+}
+
+
+@pytest.mark.parametrize("shape", list(SHAPES))
+def test_head_and_page_shapes(shape):
+    wl = _wl(2, [3001, 1234], **SHAPES[shape])
+    cfg = wl.cfg
+    pool, seq_lens = build_pool(wl)
+    step = DecodeStep(pool, wl.page_table, seq_lens, cfg.H_q, "topk", budget_frac=1 / 8, alpha=cfg.alpha)
+    step.score(wl.q)
+    step.choose()
+    step.attend(wl.q)
+    step.check()
+    ub, sel, cnt = step.ub.cpu().numpy(), step.sel.cpu().numpy(), step.sel_count.cpu().numpy()
+    out = step.out.cpu().numpy()
+    G = cfg.G
+    for b in range(cfg.B):
+        o = H.OracleSeq(wl, b)
+        P = cfg.pages(b)
+        for g in range(cfg.H_kv):
+            assert np.array_equal(ub[b, g, :P], o.ubg(g)), (b, g)
+            ref = o.topk(g, -1, 1 / 8)
+            assert np.array_equal(sel[b, g, :cnt[b, g]], ref), (b, g)
+            o_ref, _ = o.attention(g, ref, cfg.alpha)
+            H.compare_out(out[b, g * G:(g + 1) * G], o_ref, cfg.dtype)
+
+
 def _topk_cases():
     rng = np.random.default_rng(11)
     big_tie = np.full(5000, 0.25, np.float32)
