@@ -325,8 +325,9 @@ def run_native(args, rank, world, local):
 
 def run_e2e(wl, pool, seq_lens, K, W, flush):
     """Same step through the public API (the graphed step) with the step's
-    inputs in pinned host memory: H2D of q and the new token and D2H of the
-    output inside the events."""
+    inputs in pinned host memory: one H2D copy of q and the new token (packed
+    by GraphedStep.pack_host) and one D2H copy of the output inside the
+    events."""
     from sparse_long_context_min_b200.step import DecodeStep, GraphedStep
     cfg = wl.cfg
     stream = torch.cuda.current_stream()
@@ -335,7 +336,7 @@ def run_e2e(wl, pool, seq_lens, K, W, flush):
     host = []
     for i in range(W + K):
         k, v, q = wl.decode_token(10_000 + i)
-        host.append((k.cpu().pin_memory(), v.cpu().pin_memory(), q.cpu().pin_memory()))
+        host.append(gs.pack_host(k, v, q))
     out_h = torch.empty(st.out.shape, dtype=st.out.dtype).pin_memory()
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
     for i in range(W + K):
@@ -343,10 +344,7 @@ def run_e2e(wl, pool, seq_lens, K, W, flush):
         j = i - W
         if j >= 0:
             ev[j][0].record(stream)
-        k, v, q = host[i]
-        gs.k.copy_(k, non_blocking=True)
-        gs.v.copy_(v, non_blocking=True)
-        gs.q.copy_(q, non_blocking=True)
+        gs.inputs.copy_(host[i], non_blocking=True)
         gs.replay()
         out_h.copy_(st.out, non_blocking=True)
         if j >= 0:
@@ -354,7 +352,7 @@ def run_e2e(wl, pool, seq_lens, K, W, flush):
     torch.cuda.synchronize()
     st.check()
     us = statistics.mean(a.elapsed_time(b) * 1e3 for a, b in ev)
-    h2d = sum(t.numel() * t.element_size() for t in host[0])
+    h2d = host[0].numel() * host[0].element_size()
     d2h = out_h.numel() * out_h.element_size()
     return us, h2d, d2h
 

@@ -316,6 +316,74 @@ EKV_DEV void fma2(uint64_t& acc, uint64_t x, uint64_t y)
     asm("fma.rn.f32x2 %0, %1, %2, %0;" : "+l"(acc) : "l"(x), "l"(y));
 }
 
+// Producer warp of the role-split scoring kernels: walks chunks k = 0..K-1
+// (chunk c0 + k = pages (c0 + k) * PPS ...), lane i < PPS resolving page i of
+// the chunk, and fills stage k % NST: header int4 {sequence or -1, page,
+// tokens, 0} per page slot, and both metadata vectors of each present page
+// (all kv heads, vecb bytes each) by bulk copies completing `full`.
+template <int NST>
+EKV_DEV void ws_produce(const ScoreArgs& a, uint8_t* data, int stageb, int slots, int4* info, uint64_t* full,
+                        uint64_t* empty, int PPS, long long c0, int K, size_t vecb)
+{
+    const int lane = threadIdx.x & 31;
+    const long long items = (long long)a.B * a.max_pages;
+    const long long j0 = c0 * PPS;                       // first item of the CTA
+    auto pt_load = [&](long long j) -> int {
+        return j < items && j < (c0 + K) * PPS ? __ldg(&a.page_table[j]) : -1;
+    };
+    int cur = pt_load(j0 + lane);                        // entries of items j0 + 32m + lane
+    int nxt = pt_load(j0 + 32 + lane);
+    int lb = -1, lL = 0, lP = 0;
+    const int per_batch = 32 / PPS;                      // chunks per batch of entries
+    // lane i < PPS walks items j = (c0 + k) * PPS + i as (sequence bb, page pp)
+    long long jl = c0 * PPS + lane;
+    int bb = (int)(jl / a.max_pages), pp = (int)(jl - (long long)bb * a.max_pages);
+    for (int k = 0; k < K; ++k) {
+        const int s = k % NST;
+        if (k >= NST && !mbar_wait(&empty[s], ((k / NST) - 1) & 1, kWaitLimitNs)) {
+            if (lane == 0) report(a.status, ENTMAXKV_TIMEOUT);
+            break;
+        }
+        const int kb = k % per_batch;
+        const int pt = __shfl_sync(0xffffffffu, cur, kb * PPS + (lane < PPS ? lane : 0));
+        if (kb == per_batch - 1) {
+            cur = nxt;
+            nxt = pt_load(j0 + (long long)(k + 1 + per_batch) * PPS + lane);
+        }
+        int n = 0;
+        if (lane < PPS) {
+            const bool in = jl < items;
+            if (in) {
+                if (bb != lb) {
+                    lb = bb;
+                    lL = __ldg(&a.seq_lens[bb]);
+                    lP = pages_of(lL, a.ps, a.max_pages, a.status);
+                }
+                if (pp < lP) {
+                    if (pt < 0 || pt >= a.num_phys) report(a.status, ENTMAXKV_DEVICE_BOUNDS);
+                    else n = min(a.ps, lL - pp * a.ps);
+                }
+            }
+            info[s * slots + lane] = make_int4(in ? bb : -1, pp, n, 0);
+        }
+        jl += PPS;
+        pp += PPS;
+        while (pp >= a.max_pages) {
+            pp -= a.max_pages;
+            ++bb;
+        }
+        const unsigned copies = __ballot_sync(0xffffffffu, lane < PPS && n > 0);
+        __syncwarp();                                    // header writes before the arrive
+        if (lane == 0) mbar_arrive_expect_tx(&full[s], (uint32_t)(__popc(copies) * 2 * vecb));
+        if (lane < PPS && n > 0) {
+            uint8_t* dst = data + (size_t)s * stageb + lane * 2 * vecb;
+            const size_t off = (size_t)pt * vecb;
+            bulk_load(dst, static_cast<const uint8_t*>(a.row_a) + off, (uint32_t)vecb, &full[s]);
+            bulk_load(dst + vecb, static_cast<const uint8_t*>(a.row_b) + off, (uint32_t)vecb, &full[s]);
+        }
+    }
+}
+
 template <int D, int G>
 __global__ void __launch_bounds__(BoxWsShape<D, G>::CTA, 2) score_box16_kernel(const ScoreArgs a)
 {
@@ -344,62 +412,7 @@ __global__ void __launch_bounds__(BoxWsShape<D, G>::CTA, 2) score_box16_kernel(c
     __syncthreads();
 
     if (warp == kWsConsumers) {
-        // ------------------------------------------------ producer
-        const long long j0 = c0 * PPS;                   // first item of the CTA
-        auto pt_load = [&](long long j) -> int {
-            return j < items && j < (c0 + K) * PPS ? __ldg(&a.page_table[j]) : -1;
-        };
-        int cur = pt_load(j0 + lane);                    // entries of items j0 + 32m + lane
-        int nxt = pt_load(j0 + 32 + lane);
-        int lb = -1, lL = 0, lP = 0;
-        const int per_batch = 32 / PPS;                  // chunks per batch of entries
-        // lane i < PPS walks items j = (c0 + k) * PPS + i as (sequence bb, page pp)
-        long long jl = c0 * PPS + lane;
-        int bb = (int)(jl / a.max_pages), pp = (int)(jl - (long long)bb * a.max_pages);
-        for (int k = 0; k < K; ++k) {
-            const int s = k % NST;
-            if (k >= NST && !mbar_wait(&empty[s], ((k / NST) - 1) & 1, kWaitLimitNs)) {
-                if (lane == 0) report(a.status, ENTMAXKV_TIMEOUT);
-                break;
-            }
-            const int kb = k % per_batch;
-            const int pt = __shfl_sync(0xffffffffu, cur, kb * PPS + (lane < PPS ? lane : 0));
-            if (kb == per_batch - 1) {
-                cur = nxt;
-                nxt = pt_load(j0 + (long long)(k + 1 + per_batch) * PPS + lane);
-            }
-            int n = 0;
-            if (lane < PPS) {
-                const bool in = jl < items;
-                if (in) {
-                    if (bb != lb) {
-                        lb = bb;
-                        lL = __ldg(&a.seq_lens[bb]);
-                        lP = pages_of(lL, a.ps, a.max_pages, a.status);
-                    }
-                    if (pp < lP) {
-                        if (pt < 0 || pt >= a.num_phys) report(a.status, ENTMAXKV_DEVICE_BOUNDS);
-                        else n = min(a.ps, lL - pp * a.ps);
-                    }
-                }
-                info[s * S::SLOTS + lane] = make_int4(in ? bb : -1, pp, n, 0);
-            }
-            jl += PPS;
-            pp += PPS;
-            while (pp >= a.max_pages) {
-                pp -= a.max_pages;
-                ++bb;
-            }
-            const unsigned copies = __ballot_sync(0xffffffffu, lane < PPS && n > 0);
-            __syncwarp();                                // header writes before the arrive
-            if (lane == 0) mbar_arrive_expect_tx(&full[s], (uint32_t)(__popc(copies) * 2 * vecb));
-            if (lane < PPS && n > 0) {
-                uint8_t* dst = box_smem + s * S::STAGEB + lane * 2 * vecb;
-                const size_t off = (size_t)pt * vecb;
-                bulk_load(dst, static_cast<const uint8_t*>(a.row_a) + off, (uint32_t)vecb, &full[s]);
-                bulk_load(dst + vecb, static_cast<const uint8_t*>(a.row_b) + off, (uint32_t)vecb, &full[s]);
-            }
-        }
+        ws_produce<NST>(a, box_smem, S::STAGEB, S::SLOTS, info, full, empty, PPS, c0, K, vecb);
         return;   // the consumers keep the CTA alive until every copy has been consumed
     }
 

@@ -162,9 +162,18 @@ class GraphedStep:
         self.step = step
         pool = step.pool
         dev = pool.k_pool.device
-        self.q = torch.zeros(step.B, step.H_q, pool.d, dtype=torch.float32, device=dev)
-        self.k = torch.zeros(step.B, step.H_kv, 1, pool.d, dtype=pool.k_pool.dtype, device=dev)
-        self.v = torch.zeros_like(self.k)
+        # q, k and v are views of one device buffer, so a step's inputs can
+        # arrive in a single host-to-device copy (pack_host / inputs)
+        elt = pool.k_pool.element_size()
+        nq = step.B * step.H_q * pool.d * 4
+        nk = step.B * step.H_kv * pool.d * elt
+        al = lambda x: (x + 255) // 256 * 256
+        self._off = (0, al(nq), al(nq) + al(nk))
+        self._len = (nq, nk, nk)
+        self.inputs = torch.zeros(al(nq) + 2 * al(nk), dtype=torch.uint8, device=dev)
+        self.q = self._view(self.inputs, 0).view(torch.float32).view(step.B, step.H_q, pool.d)
+        self.k = self._view(self.inputs, 1).view(pool.k_pool.dtype).view(step.B, step.H_kv, 1, pool.d)
+        self.v = self._view(self.inputs, 2).view(pool.k_pool.dtype).view(step.B, step.H_kv, 1, pool.d)
         self.append = append
         self.rt = _CudaRT() if stage_events else None
         self.ev = [self.rt.event() for _ in range(5)] if stage_events else None
@@ -189,6 +198,18 @@ class GraphedStep:
             self._mark(3, cs)
             step.attend(self.q)
             self._mark(4, cs)
+
+    def _view(self, buf, i):
+        return buf[self._off[i]:self._off[i] + self._len[i]]
+
+    def pack_host(self, k, v, q):
+        """Pinned host buffer laid out like `inputs` holding (k, v, q) of one
+        step: copy it into `inputs` with one copy, then replay()."""
+        h = torch.zeros(self.inputs.numel(), dtype=torch.uint8).pin_memory()
+        for i, t in ((0, q), (1, k), (2, v)):
+            src = t.detach().to("cpu").contiguous().reshape(-1).view(torch.uint8)
+            self._view(h, i).copy_(src)
+        return h
 
     def _mark(self, i, stream):
         if self.ev is not None:

@@ -490,12 +490,15 @@ def test_graphed_step_equals_eager_step():
     eager = DecodeStep(pool_a, wl.page_table, lens_a, cfg.H_q, "topk", budget_frac=1 / 16, alpha=cfg.alpha)
     graphed = GraphedStep(DecodeStep(pool_b, wl.page_table, lens_b, cfg.H_q, "topk", budget_frac=1 / 16,
                                      alpha=cfg.alpha))
-    for t in range(3):
+    for t in range(4):
         k, v, q = wl.decode_token(t)
         eager(q, k, v)
-        graphed.q.copy_(q)
-        graphed.k.copy_(k)
-        graphed.v.copy_(v)
+        if t % 2:   # one packed copy from pinned host memory
+            graphed.inputs.copy_(graphed.pack_host(k, v, q), non_blocking=True)
+        else:
+            graphed.q.copy_(q)
+            graphed.k.copy_(k)
+            graphed.v.copy_(v)
         graphed.replay()
         torch.cuda.synchronize()
         assert torch.equal(eager.out, graphed.step.out)
