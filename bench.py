@@ -261,6 +261,10 @@ def run_native(args, rank, world, local):
         extra["topk_speedup_vs_full_softmax"] = round(fs / mean_us_all, 2)
         extra["gauss_speedup_vs_full_entmax"] = round(fe / extra["gauss_us_per_step"], 2)
         extra["gauss_speedup_vs_full_softmax"] = round(fs / extra["gauss_us_per_step"], 2)
+        extra.update({k: round(max_over_ranks(v, world), 2)
+                      for k, v in run_attend_variants(wl, pool, seq_lens, flush).items()})
+        extra["attend_variants_note"] = ("eager calls between events on one top-k 1/64 selection; "
+                                         "include launch latency not hidden by a graph")
 
     cpu = None
     if rank == 0 and not args.no_cpu:
@@ -386,6 +390,47 @@ def run_full(wl, pool, seq_lens, flush, reps=5, warm=3):
         res.append(statistics.mean(a.elapsed_time(b) * 1e3 for a, b in times))
         del ws
     return res[0], res[1]
+
+
+def run_attend_variants(wl, pool, seq_lens, flush, reps=5, warm=3):
+    """On one top-k 1/64 selection: sparse entmax attention (alpha 1.5, the
+    step's), softmax over the same pages (the matched-budget baseline) and
+    entmax with alpha = 1.25 (no closed form: Newton threshold, powf weights)."""
+    from sparse_long_context_min_b200 import binding as BND
+    from sparse_long_context_min_b200.step import DecodeStep
+    cfg = wl.cfg
+    stream = torch.cuda.current_stream()
+    step = DecodeStep(pool, wl.page_table, seq_lens, cfg.H_q, "topk", budget_frac=1 / 64, alpha=cfg.alpha)
+    step.score(wl.q)
+    step.choose()
+    out = torch.empty_like(step.out)
+    ws_s = torch.empty(BND.workspace_size(BND.OP_SPARSE_SOFTMAX, cfg.B, cfg.H_q, cfg.H_kv, wl.max_pages,
+                                          step.k_max, cfg.ps, cfg.d), dtype=torch.uint8, device="cuda")
+    calls = {
+        "sparse_entmax_attend_us": lambda: BND.sparse_attend(pool, wl.q, wl.page_table, seq_lens, step.sel,
+                                                             step.sel_count, cfg.alpha, cfg.scale, out,
+                                                             step.workspace, step.status),
+        "matched_budget_sparse_softmax_attend_us": lambda: BND.sparse_softmax_attend(
+            pool, wl.q, wl.page_table, seq_lens, step.sel, step.sel_count, cfg.scale, out, ws_s, step.status),
+        "sparse_entmax_alpha_1.25_attend_us": lambda: BND.sparse_attend(pool, wl.q, wl.page_table, seq_lens,
+                                                                        step.sel, step.sel_count, 1.25, cfg.scale,
+                                                                        out, step.workspace, step.status),
+    }
+    res = {}
+    for name, fn in calls.items():
+        times = []
+        for i in range(warm + reps):
+            flush.fill_(i & 0xFF)
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            fn()
+            b.record(stream)
+            if i >= warm:
+                times.append((a, b))
+        torch.cuda.synchronize()
+        res[name] = round(statistics.mean(a.elapsed_time(b) * 1e3 for a, b in times), 2)
+    step.check()
+    return res
 
 
 # ---------------------------------------------------------------- oracle timing

@@ -30,7 +30,12 @@
  *   h / G), d head dim, ps page size, P_b = ceil(seq_lens[b] / ps) pages of
  *   sequence b, max_pages the row length of page_table.
  * - Supported: d in {64, 128}; ps in {16, 64}; dtype F32 or BF16; G in
- *   {1, 2, 4, 8}; alpha in {1.5, 2.0}.
+ *   {1, 2, 4, 8}.  alpha (German summary, section 2: alpha-entmax for any
+ *   alpha > 1): the attention entry points take any alpha in (1, 16]; alpha
+ *   = 1.5 and 2 have closed-form thresholds, any other alpha a threshold by
+ *   safeguarded Newton steps in float64 and weights by powf.  The Gaussian
+ *   selector takes alpha in {1.5, 2.0} only (its expectations have closed
+ *   forms there) and returns ENTMAXKV_UNSUPPORTED otherwise.
  * - page_table[b][p] (int32, [B][max_pages]) is the physical page holding
  *   logical page p of sequence b; entries p >= P_b are never read.  Physical
  *   ids out of [0, num_phys_pages) are reported as ENTMAXKV_DEVICE_BOUNDS.
@@ -69,7 +74,8 @@ typedef enum {
     ENTMAXKV_OP_SELECT = 0,
     ENTMAXKV_OP_SPARSE_ATTEND = 1,
     ENTMAXKV_OP_FULL_ENTMAX = 2,
-    ENTMAXKV_OP_FULL_SOFTMAX = 3
+    ENTMAXKV_OP_FULL_SOFTMAX = 3,
+    ENTMAXKV_OP_SPARSE_SOFTMAX = 4
 } entmaxkv_op;
 
 /*
@@ -246,6 +252,27 @@ ENTMAXKV_API int entmaxkv_full_softmax_decode(const entmaxkv_pool* pool, const f
                                  const int32_t* page_table, int32_t max_pages,
                                  const int32_t* seq_lens, int32_t B, float scale, float* out,
                                  void* workspace, size_t ws_bytes, int32_t* status, void* stream);
+
+/*
+ * Softmax attention over the caller's selected pages: the sparse softmax
+ * decoding the pages compare EntmaxKV against at the same kept set / budget
+ * (German summary, section 3 "Vergleich" and section 4
+ * "Approximationsqualitaet": softmax has a dense tail, so any dropped token
+ * loses mass delta > 0, and the output error is bounded by 2 B delta).
+ *   out[b][h] = sum_{i in kept} softmax_kept(scale * q_h . k_i)_i v_i, the
+ *   softmax renormalised over the valid tokens of the listed pages,
+ *   [B][H_q][d] fp32; a kv head with an empty list gives zeros.
+ * sel, sel_count, k_max as in entmaxkv_sparse_attend (any set of distinct
+ * pages, e.g. the output of entmaxkv_select).  Split over the list with the
+ * log-sum-exp merge of entmaxkv_full_softmax_decode.
+ * workspace: entmaxkv_workspace_size(ENTMAXKV_OP_SPARSE_SOFTMAX, ...) bytes.
+ * Errors: as entmaxkv_sparse_attend.
+ */
+ENTMAXKV_API int entmaxkv_sparse_softmax_attend(const entmaxkv_pool* pool, const float* q, int32_t H_q,
+                                   const int32_t* page_table, int32_t max_pages,
+                                   const int32_t* seq_lens, int32_t B, const int32_t* sel,
+                                   const int32_t* sel_count, int32_t k_max, float scale, float* out,
+                                   void* workspace, size_t ws_bytes, int32_t* status, void* stream);
 
 /*
  * Bytes of device workspace an entry point needs (host only; uses the SM

@@ -19,13 +19,14 @@ STATIC_SCRATCH_BYTES = 16 << 20
 F32, BF16 = 0, 1
 SCORE_BBOX, SCORE_GAUSS = 0, 1
 SELECT_TOPK, SELECT_GAUSS = 0, 1
-OP_SELECT, OP_SPARSE_ATTEND, OP_FULL_ENTMAX, OP_FULL_SOFTMAX = range(4)
+OP_SELECT, OP_SPARSE_ATTEND, OP_FULL_ENTMAX, OP_FULL_SOFTMAX, OP_SPARSE_SOFTMAX = range(5)
 
 # every symbol the header declares (checked by the tests)
 SYMBOLS = (
     "entmaxkv_append_metadata", "entmaxkv_score_pages", "entmaxkv_select", "entmaxkv_sparse_attend",
     "entmaxkv_full_entmax_decode", "entmaxkv_full_softmax_decode", "entmaxkv_workspace_size",
     "entmaxkv_status_string", "entmaxkv_selftest_timeout", "entmaxkv_sparse_attend_static",
+    "entmaxkv_sparse_softmax_attend",
 )
 
 
@@ -62,6 +63,7 @@ def lib():
         L.entmaxkv_sparse_attend.argtypes = [PP, P, I, P, I, P, I, P, P, I, F, F, P, P, P, P, S, P, P]
         L.entmaxkv_full_entmax_decode.argtypes = [PP, P, I, P, I, P, I, F, F, P, P, P, P, S, P, P]
         L.entmaxkv_full_softmax_decode.argtypes = [PP, P, I, P, I, P, I, F, P, P, S, P, P]
+        L.entmaxkv_sparse_softmax_attend.argtypes = [PP, P, I, P, I, P, I, P, P, I, F, P, P, S, P, P]
         L.entmaxkv_workspace_size.argtypes = [I, I, I, I, I, I, I, I]
         L.entmaxkv_workspace_size.restype = ctypes.c_size_t
         L.entmaxkv_status_string.argtypes = [I]
@@ -189,6 +191,16 @@ def full_softmax_decode(pool, q, page_table, seq_lens, scale, out, workspace, st
                                               _p(seq_lens), B, scale, _p(out), _p(workspace),
                                               workspace.numel() * workspace.element_size(), _p(status),
                                               _stream(stream)), "full_softmax_decode")
+
+
+def sparse_softmax_attend(pool, q, page_table, seq_lens, sel, sel_count, scale, out, workspace, status,
+                          stream=None):
+    """Softmax attention over the listed pages (workspace: OP_SPARSE_SOFTMAX)."""
+    B, H_q, _ = q.shape
+    _check(lib().entmaxkv_sparse_softmax_attend(pool.c, _p(q), H_q, _p(page_table), page_table.shape[1],
+                                                _p(seq_lens), B, _p(sel), _p(sel_count), sel.shape[2], scale,
+                                                _p(out), _p(workspace), workspace.numel() * workspace.element_size(),
+                                                _p(status), _stream(stream)), "sparse_softmax_attend")
 
 
 def selftest_timeout(limit_ns, status, stream=None):

@@ -103,7 +103,11 @@ static int check_heads(int H_q, int H_kv)
     return ENTMAXKV_OK;
 }
 
+// The Gaussian selector has closed forms for alpha = 1.5 and 2 only; exact
+// attention takes any alpha in (1, 16] (other values by a safeguarded Newton
+// solve of the threshold and powf weights).
 static bool alpha_ok(float alpha) { return alpha == 1.5f || alpha == 2.0f; }
+static bool alpha_attend_ok(float alpha) { return alpha > 1.0f && alpha <= 16.0f; }
 
 // ------------------------------------------------------------------ workspace
 static size_t round256(size_t x) { return (x + 255) & ~size_t(255); }
@@ -123,22 +127,27 @@ struct AttnLayout {
     size_t xbuf, cmax, opart, mlpart, lmax, tau, counters, total;
 };
 
+// attention ops over a caller's page list / with softmax weights
+static bool is_sparse(int op) { return op == ENTMAXKV_OP_SPARSE_ATTEND || op == ENTMAXKV_OP_SPARSE_SOFTMAX; }
+static bool is_softmax(int op) { return op == ENTMAXKV_OP_FULL_SOFTMAX || op == ENTMAXKV_OP_SPARSE_SOFTMAX; }
+
 static AttnLayout attn_layout(int op, int B, int H_q, int H_kv, int max_pages, int k_max, int ps, int d)
 {
     AttnLayout L{};
-    const int list = op == ENTMAXKV_OP_SPARSE_ATTEND ? k_max : max_pages;
+    const bool soft = is_softmax(op);
+    const int list = is_sparse(op) ? k_max : max_pages;
     L.S = num_splits(B, H_kv, list);
     size_t off = 0;
     L.xbuf = off;
-    if (op != ENTMAXKV_OP_FULL_SOFTMAX) off += round256((size_t)B * H_q * list * ps * sizeof(float));
+    if (!soft) off += round256((size_t)B * H_q * list * ps * sizeof(float));
     L.cmax = off;
-    if (op != ENTMAXKV_OP_FULL_SOFTMAX) off += round256((size_t)B * H_q * list * ((ps + 15) / 16) * sizeof(float));
+    if (!soft) off += round256((size_t)B * H_q * list * ((ps + 15) / 16) * sizeof(float));
     L.opart = off;
     off += round256((size_t)B * H_q * L.S * d * sizeof(float));
     L.mlpart = off;
-    if (op == ENTMAXKV_OP_FULL_SOFTMAX) off += round256((size_t)B * H_q * L.S * 2 * sizeof(float));
+    if (soft) off += round256((size_t)B * H_q * L.S * 2 * sizeof(float));
     L.lmax = off;
-    if (op != ENTMAXKV_OP_FULL_SOFTMAX) off += round256((size_t)B * H_q * L.S * sizeof(float));
+    if (!soft) off += round256((size_t)B * H_q * L.S * sizeof(float));
     L.tau = off;
     off += round256((size_t)B * H_q * sizeof(float));
     L.counters = off;
@@ -157,9 +166,9 @@ static int attend_common(int op, const entmaxkv_pool* pool, const float* q, int 
     if (rc) return rc;
     if ((rc = check_heads(H_q, pool->H_kv))) return rc;
     if (B < 0 || max_pages <= 0) return ENTMAXKV_INVALID_ARG;
-    if (op != ENTMAXKV_OP_FULL_SOFTMAX && !alpha_ok(alpha)) return ENTMAXKV_UNSUPPORTED;
+    if (!is_softmax(op) && !alpha_attend_ok(alpha)) return ENTMAXKV_UNSUPPORTED;
     if (!(scale > 0.f) || !std::isfinite(scale)) return ENTMAXKV_INVALID_ARG;
-    if (op == ENTMAXKV_OP_SPARSE_ATTEND && (!sel || !sel_count || k_max <= 0)) return ENTMAXKV_INVALID_ARG;
+    if (is_sparse(op) && (!sel || !sel_count || k_max <= 0)) return ENTMAXKV_INVALID_ARG;
     if (B == 0) return ENTMAXKV_OK;
     if (!q || !page_table || !seq_lens || !out || !status) return ENTMAXKV_INVALID_ARG;
     const AttnLayout lay = attn_layout(op, B, H_q, pool->H_kv, max_pages, k_max, pool->ps, pool->d);
@@ -173,13 +182,13 @@ static int attend_common(int op, const entmaxkv_pool* pool, const float* q, int 
     a.page_table = page_table;
     a.max_pages = max_pages;
     a.seq_lens = seq_lens;
-    a.sel = op == ENTMAXKV_OP_SPARSE_ATTEND ? sel : nullptr;
-    a.sel_count = op == ENTMAXKV_OP_SPARSE_ATTEND ? sel_count : nullptr;
-    a.k_max = op == ENTMAXKV_OP_SPARSE_ATTEND ? k_max : max_pages;
+    a.sel = is_sparse(op) ? sel : nullptr;
+    a.sel_count = is_sparse(op) ? sel_count : nullptr;
+    a.k_max = is_sparse(op) ? k_max : max_pages;
     a.num_phys = pool->num_phys_pages;
     a.S = lay.S;
     a.alpha = alpha;
-    a.xscale = op == ENTMAXKV_OP_FULL_SOFTMAX ? scale : (alpha - 1.0f) * scale;
+    a.xscale = is_softmax(op) ? scale : (alpha - 1.0f) * scale;
     char* ws = static_cast<char*>(workspace);
     a.xbuf = reinterpret_cast<float*>(ws + lay.xbuf);
     a.cmax = reinterpret_cast<float*>(ws + lay.cmax);
@@ -199,7 +208,7 @@ static int attend_common(int op, const entmaxkv_pool* pool, const float* q, int 
         if ((rc = make_pool_map(&vmap, *pool, pool->v_pool))) return rc;
     }
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    if (op == ENTMAXKV_OP_FULL_SOFTMAX) return launch_softmax_attend(*pool, a, B, &kmap, &vmap, st);
+    if (is_softmax(op)) return launch_softmax_attend(*pool, a, B, &kmap, &vmap, st);
     return launch_entmax_attend(*pool, a, B, &kmap, &vmap, st);
 }
 
@@ -305,14 +314,22 @@ int entmaxkv_full_softmax_decode(const entmaxkv_pool* pool, const float* q, int3
                          stream);
 }
 
+int entmaxkv_sparse_softmax_attend(const entmaxkv_pool* pool, const float* q, int32_t H_q,
+                                   const int32_t* page_table, int32_t max_pages, const int32_t* seq_lens, int32_t B,
+                                   const int32_t* sel, const int32_t* sel_count, int32_t k_max, float scale,
+                                   float* out, void* workspace, size_t ws_bytes, int32_t* status, void* stream)
+{
+    return attend_common(ENTMAXKV_OP_SPARSE_SOFTMAX, pool, q, H_q, page_table, max_pages, seq_lens, B, sel,
+                         sel_count, k_max, 1.5f, scale, out, nullptr, nullptr, workspace, ws_bytes, status, stream);
+}
+
 size_t entmaxkv_workspace_size(int32_t op, int32_t B, int32_t H_q, int32_t H_kv, int32_t max_pages, int32_t k_max,
                                int32_t ps, int32_t d)
 {
     if (B <= 0 || H_q <= 0 || H_kv <= 0 || max_pages <= 0 || ps <= 0 || d <= 0) return 0;
     if (op == ENTMAXKV_OP_SELECT) return 0;
-    if (op == ENTMAXKV_OP_SPARSE_ATTEND && k_max <= 0) return 0;
-    if (op != ENTMAXKV_OP_SPARSE_ATTEND && op != ENTMAXKV_OP_FULL_ENTMAX && op != ENTMAXKV_OP_FULL_SOFTMAX)
-        return 0;
+    if (is_sparse(op) && k_max <= 0) return 0;
+    if (!is_sparse(op) && op != ENTMAXKV_OP_FULL_ENTMAX && op != ENTMAXKV_OP_FULL_SOFTMAX) return 0;
     return attn_layout(op, B, H_q, H_kv, max_pages, k_max, ps, d).total;
 }
 

@@ -451,6 +451,7 @@ __global__ void __launch_bounds__(kTauBlock) tau_kernel(int ps, const AttnArgs a
     const size_t row = (size_t)b * a.H_q + h;
     const float* x = a.xbuf + row * (size_t)a.k_max * ps;
     const bool a2 = a.alpha == 2.0f;
+    const bool gen = !a2 && a.alpha != 1.5f;          // any other alpha: no closed form
 
     float M = -INFINITY;
     for (int s = tid; s < a.S; s += kTauBlock) M = fmaxf(M, a.lmax[row * a.S + s]);
@@ -550,7 +551,7 @@ __global__ void __launch_bounds__(kTauBlock) tau_kernel(int ps, const AttnArgs a
         suf[i] = suf[i] - loc[i] + above;                // bins of the threads above mine
     }
     double best_lo = thr;
-    {
+    if (!gen) {
         double S0 = suf[0], S1 = suf[1], S2 = suf[2];     // sums over bins > my last bin
         for (int k = BPT - 1; k >= 0; --k) {
             const int j = j0 + k;
@@ -573,8 +574,44 @@ __global__ void __launch_bounds__(kTauBlock) tau_kernel(int ps, const AttnArgs a
     const float* src = spill ? x : cand;
     const int len = spill ? n : ncand;
 
-    // --- Newton / closed form over {x > lo_t}
     double tau = lo_t;
+    if (gen) {
+        // --- any alpha: Newton steps on G(t) = F(t)^(1/r) - 1, F(t) = sum (x - t)_+^r,
+        // inside the bracket [M - 1, M] (F(M - 1) >= 1 > F(M) = 0), bisection
+        // where a step leaves it.  For r >= 1, F^(1/r) is the r-norm of (x - t)_+:
+        // convex, decreasing and close to linear, so steps from the left never
+        // pass the root and converge in a few iterations (exactly in one when a
+        // single value is above t).  Terms in float (powf), sums in float64.
+        const double r = 1.0 / ((double)a.alpha - 1.0);
+        const float rf = (float)r;
+        double lo = thr, hi = (double)M;
+        for (int it = 0; it < 100; ++it) {
+            double v[3] = {0.0, 0.0, 0.0};
+            float unused0 = INFINITY, unused1 = -INFINITY;
+            for (int i = tid; i < len; i += kTauBlock) {
+                const double vd = (double)src[i];
+                if (vd > tau) {
+                    const float u = (float)(vd - tau);
+                    const float pu = powf(u, rf);
+                    v[0] += (double)pu;
+                    v[1] += (double)pu / (double)u;
+                }
+            }
+            tau_reduce(R, it, v, unused0, unused1);
+            const double F = v[0], S1 = r * v[1];          // F and -dF/dt
+            if (F >= 1.0) lo = tau; else hi = tau;
+            if (F == 1.0 || hi - lo <= 1e-13 * fmax(1.0, fabs(tau))) break;
+            double nt = (F > 0.0 && S1 > 0.0) ? tau + r * F * (1.0 - pow(F, -1.0 / r)) / S1 : 0.5 * (lo + hi);
+            if (!(nt > lo && nt < hi)) nt = 0.5 * (lo + hi);
+            // the float terms fix F to about 1e-7 relative, tau to about 1e-8
+            if (fabs(nt - tau) <= 1e-8 * fmax(1.0, fabs(tau))) {
+                tau = nt;
+                break;
+            }
+            tau = nt;
+        }
+    } else
+    // --- Newton / closed form over {x > lo_t}
     for (int it = 0; it < 100; ++it) {
         double v[3] = {0.0, 0.0, 0.0};
         float minS = INFINITY, maxN = -INFINITY;
@@ -727,6 +764,8 @@ __global__ void __launch_bounds__(kThreads) pv_bf16_kernel(const __grid_constant
     const int cnt = list_count(a, b, g, P);
     const Range r = split_range(cnt, a.S, s);
     const bool a2 = a.alpha == 2.0f;
+    const bool a15 = a.alpha == 1.5f;
+    const float rexp = 1.0f / (a.alpha - 1.0f);   // weight exponent for any other alpha
     const size_t xstride = (size_t)a.k_max * PS;
     const size_t row0h = (size_t)b * a.H_q + (size_t)g * a.G;
 
@@ -841,7 +880,7 @@ __global__ void __launch_bounds__(kThreads) pv_bf16_kernel(const __grid_constant
                     if (head < a.G && valid) {
                         const float xv = a.xbuf[(row0h + head) * xstride + (size_t)idx * PS + prow];
                         const float u = fmaxf(xv - tau_s[head], 0.f);
-                        p = a2 ? u : u * u;
+                        p = a2 ? u : (a15 ? u * u : powf(u, rexp));
                     }
                     uint32_t hi, lo;
                     split_bf16(p, hi, lo);
@@ -940,6 +979,8 @@ __global__ void __launch_bounds__(kThreads) pv_f32_kernel(const float* __restric
     tab_fill(a, b, g, r, P);
     const size_t xstride = (size_t)a.k_max * ps;
     const bool a2 = a.alpha == 2.0f;
+    const bool a15 = a.alpha == 1.5f;
+    const double rexp = 1.0 / ((double)a.alpha - 1.0);
     for (int w = tid; w < a.G * D; w += kThreads) {
         const int head = w / D, dd = w % D;
         const size_t row = (size_t)b * a.H_q + (size_t)g * a.G + head;
@@ -953,7 +994,7 @@ __global__ void __launch_bounds__(kThreads) pv_f32_kernel(const float* __restric
                 const float xv = a.xbuf[row * xstride + (size_t)idx * ps + t];
                 const double u = fmax((double)xv - (double)tau, 0.0);
                 if (u > 0.0) {
-                    const double p = a2 ? u : u * u;
+                    const double p = a2 ? u : (a15 ? u * u : pow(u, rexp));
                     acc = fma(p, (double)v_pool[(((size_t)phys * a.H_kv + g) * ps + t) * D + dd], acc);
                 }
             }

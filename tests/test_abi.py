@@ -42,6 +42,10 @@ def test_workspace_sizes():
     assert B.workspace_size(B.OP_FULL_SOFTMAX, 1, 32, 8, 16385, 0, 64, 128) < small
     assert B.workspace_size(B.OP_SELECT, 1, 32, 8, 16385, 256, 64, 128) == 0
     assert B.workspace_size(B.OP_SPARSE_ATTEND, 0, 32, 8, 10, 1, 64, 128) == 0
+    # sparse softmax keeps no scores: partials and merge terms only
+    sm = B.workspace_size(B.OP_SPARSE_SOFTMAX, 1, 32, 8, 16385, 256, 64, 128)
+    assert 0 < sm < small
+    assert B.workspace_size(B.OP_SPARSE_SOFTMAX, 1, 32, 8, 16385, 0, 64, 128) == 0
 
 
 def test_host_validation_without_gpu():
@@ -62,6 +66,18 @@ def test_host_validation_without_gpu():
     rc = lib.entmaxkv_select(B.SELECT_TOPK, None, None, None, None, None, 64, 1, 32, 8, 100, 300, 0.0, 1.5,
                              0.0, 256, None, None, None, None, 0, st, None)
     assert rc == B.INVALID_ARG           # budget above k_max
+    pool = B.CPool(16, 16, 16, 16, 16, 16, 16, 10, 8, 64, 128, B.BF16)
+    rc = lib.entmaxkv_sparse_softmax_attend(ctypes.byref(pool), ctypes.c_void_p(16), 32, ctypes.c_void_p(16), 10,
+                                            ctypes.c_void_p(16), 1, None, None, 4, 0.1, ctypes.c_void_p(16),
+                                            ctypes.c_void_p(256), 1 << 20, st, None)
+    assert rc == B.INVALID_ARG           # no page list
+    rc = lib.entmaxkv_select(B.SELECT_GAUSS, None, None, None, None, None, 64, 1, 32, 8, 100, -1, 0.0, 1.7,
+                             0.5, 100, None, None, None, None, 0, st, None)
+    assert rc == B.UNSUPPORTED           # the Gaussian selector has closed forms for alpha 1.5 and 2 only
+    rc = lib.entmaxkv_full_entmax_decode(ctypes.byref(pool), ctypes.c_void_p(16), 32, ctypes.c_void_p(16), 10,
+                                         ctypes.c_void_p(16), 1, 1.0, 0.1, ctypes.c_void_p(16), None, None,
+                                         ctypes.c_void_p(256), 1 << 20, st, None)
+    assert rc == B.UNSUPPORTED           # alpha must exceed 1
 
 
 @pytest.mark.parametrize("B_", [0])

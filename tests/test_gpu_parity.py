@@ -360,6 +360,38 @@ def test_full_entmax_and_softmax(built):
             H.compare_out(out_s[b, g * G:(g + 1) * G], s_ref, cfg.dtype)
 
 
+@pytest.mark.parametrize("alpha", [1.25, 1.7, 3.0])
+def test_any_alpha_sparse_and_full(built, alpha):
+    """alpha outside {1.5, 2}: threshold by the safeguarded Newton solve,
+    weights by powf; against the oracle's bisection threshold."""
+    wl, pool, seq_lens, oseqs = built
+    cfg = wl.cfg
+    G = cfg.G
+    step = DecodeStep(pool, wl.page_table, seq_lens, cfg.H_q, "topk", budget_frac=1 / 16, alpha=alpha)
+    step.score(wl.q)
+    step.choose()
+    st = _status()
+    out = torch.empty_like(step.out)
+    tau = torch.empty_like(step.tau)
+    B.sparse_attend(pool, wl.q, wl.page_table, seq_lens, step.sel, step.sel_count, alpha, H.scale32(cfg), out,
+                    step.workspace, st, tau_out=tau)
+    full = torch.empty_like(out)
+    ws = torch.empty(B.workspace_size(B.OP_FULL_ENTMAX, cfg.B, cfg.H_q, cfg.H_kv, wl.max_pages, 0, cfg.ps,
+                                      cfg.d), dtype=torch.uint8, device="cuda")
+    B.full_entmax_decode(pool, wl.q, wl.page_table, seq_lens, alpha, H.scale32(cfg), full, ws, st)
+    _assert_ok(st)
+    sel, cnt = step.sel.cpu().numpy(), step.sel_count.cpu().numpy()
+    out, tau, full = out.cpu().numpy(), tau.cpu().numpy(), full.cpu().numpy()
+    for b, o in enumerate(oseqs):
+        for g in range(cfg.H_kv)[:3]:
+            pages = sel[b, g, :cnt[b, g]]
+            o_ref, t_ref = o.attention(g, pages, alpha)
+            H.compare_out(out[b, g * G:(g + 1) * G], o_ref, cfg.dtype)
+            assert np.all(np.abs(tau[b, g * G:(g + 1) * G] - t_ref) <= 1e-5 * np.maximum(1, np.abs(t_ref)))
+            f_ref, _ = o.attention(g, np.arange(cfg.pages(b)), alpha)
+            H.compare_out(full[b, g * G:(g + 1) * G], f_ref, cfg.dtype)
+
+
 def test_support_recovery_on_gpu():
     """If the kept pages hold the support, sparse == full (oracle: bitwise)."""
     wl = _wl(2, [8192 + 33])
@@ -434,9 +466,10 @@ def test_host_validation_rejects_bad_arguments():
     with pytest.raises(B.EntmaxKVError) as e:
         B.full_entmax_decode(pool, wl.q, wl.page_table, seq_lens, 1.5, 0.1, out, small, st)
     assert e.value.code == B.WORKSPACE
-    with pytest.raises(B.EntmaxKVError) as e:
-        B.full_entmax_decode(pool, wl.q, wl.page_table, seq_lens, 3.0, 0.1, out, small, st)
-    assert e.value.code == B.UNSUPPORTED
+    for alpha in (1.0, 0.5, 20.0):        # alpha-entmax needs alpha > 1; the library stops at 16
+        with pytest.raises(B.EntmaxKVError) as e:
+            B.full_entmax_decode(pool, wl.q, wl.page_table, seq_lens, alpha, 0.1, out, small, st)
+        assert e.value.code == B.UNSUPPORTED
 
 
 def test_bounded_wait_times_out_and_context_survives():

@@ -76,7 +76,7 @@ def _variational(x, alpha):
     return np.clip(best.x, 0.0, None)
 
 
-@pytest.mark.parametrize("alpha", [1.5, 2.0])
+@pytest.mark.parametrize("alpha", [1.5, 2.0, 1.25, 3.0])
 def test_variational_definition(alpha):
     rng = np.random.default_rng(3)
     for _ in range(6):
@@ -112,7 +112,7 @@ def _brute_force(x, alpha):
     return tau
 
 
-@pytest.mark.parametrize("alpha", [1.5, 2.0, 1.7])
+@pytest.mark.parametrize("alpha", [1.5, 2.0, 1.7, 1.25, 3.0])
 def test_brute_force_supports(alpha):
     rng = np.random.default_rng(4)
     for n in range(1, 9):
