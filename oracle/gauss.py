@@ -19,6 +19,7 @@ taken here (the plainest one consistent with the entmax definition):
   n_p the number of tokens in page p; with u = m' - tau and z = u / sigma':
       alpha = 2:   E[(X - tau)_+]   = u Phi(z) + sigma' phi(z)
       alpha = 1.5: E[(X - tau)_+^2] = (u^2 + sigma'^2) Phi(z) + u sigma' phi(z)
+      other alpha: numerical integration (adaptive quadrature)
       sigma' = 0:  max(u, 0)^(1/(alpha-1));
 * the estimated page maximum is the Gaussian expected-maximum approximation
   est_max_p = m_p + sqrt(v_p) * z_{n_p}, z_n = sqrt(2 ln n) (z_1 = 0), i.e. a
@@ -33,6 +34,7 @@ found by bisection on a bracket grown by doubling steps.
 import math
 
 import numpy as np
+from scipy.integrate import quad
 from scipy.special import ndtr
 
 
@@ -40,21 +42,46 @@ def _phi(z):
     return np.exp(-0.5 * z * z) / math.sqrt(2.0 * math.pi)
 
 
-def g(mp, sp, tau, alpha):
-    """E[(X - tau)_+^(1/(alpha-1))] for X ~ N(mp, sp^2), elementwise, float64."""
+def _g_quad(u, s, r):
+    """E[(Y)_+^r] for Y ~ N(u, s^2), s > 0, by adaptive quadrature.
+
+    With z = u / s the expectation is s^r * int_0^inf y^r phi(y - z) dy.  The
+    integrand is negligible (below exp(-72) of its peak) outside
+    |y - z| <= 12; on [0, ...] the factor y^r is handled by the quadrature's
+    algebraic endpoint weight."""
+    z = u / s
+    lo, hi = max(0.0, z - 12.0), z + 12.0
+    if hi <= 0.0:
+        return 0.0
+    if lo == 0.0:
+        val, _ = quad(lambda y: _phi(y - z), 0.0, hi, weight="alg", wvar=(r, 0.0),
+                      epsabs=0.0, epsrel=1e-12, limit=400)
+    else:
+        val, _ = quad(lambda y: y ** r * _phi(y - z), lo, hi, points=[z], epsabs=0.0, epsrel=1e-12,
+                      limit=400)
+    return s ** r * val
+
+
+def g(mp, sp, tau, alpha, method="closed"):
+    """E[(X - tau)_+^(1/(alpha-1))] for X ~ N(mp, sp^2), elementwise, float64.
+
+    alpha = 1.5 and 2 have closed forms; any other alpha (or method="quad")
+    integrates numerically."""
     mp = np.asarray(mp, dtype=np.float64)
     sp = np.asarray(sp, dtype=np.float64)
     u = mp - tau
+    r = 1.0 / (alpha - 1.0)
     with np.errstate(divide="ignore", invalid="ignore"):
         z = np.where(sp > 0, u / np.where(sp > 0, sp, 1.0), 0.0)
-    if alpha == 2.0:
+    if method == "closed" and alpha == 2.0:
         gauss = u * ndtr(z) + sp * _phi(z)
-        point = np.maximum(u, 0.0)
-    elif alpha == 1.5:
+    elif method == "closed" and alpha == 1.5:
         gauss = (u * u + sp * sp) * ndtr(z) + u * sp * _phi(z)
-        point = np.maximum(u, 0.0) ** 2
     else:
-        raise ValueError("closed forms only for alpha in {1.5, 2}")
+        uu, ss = np.broadcast_arrays(u, sp)
+        gauss = np.array([_g_quad(a, b, r) if b > 0 else 0.0 for a, b in zip(uu.ravel(), ss.ravel())])
+        gauss = gauss.reshape(uu.shape)
+    point = np.maximum(u, 0.0) ** r
     return np.where(sp > 0, gauss, point)
 
 

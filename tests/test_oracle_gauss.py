@@ -27,7 +27,7 @@ def test_g_worked_examples(ex):
     assert abs(float(val) - ex["g"]) < 1e-14
 
 
-@pytest.mark.parametrize("alpha", [1.5, 2.0])
+@pytest.mark.parametrize("alpha", [1.5, 2.0, 1.25, 3.0])
 def test_g_against_quadrature(alpha):
     r = 1.0 / (alpha - 1.0)
     for m, s, tau in [(0.3, 0.25, 0.9), (1.8, 0.15, 1.9), (-1.0, 2.0, 0.5), (0.0, 1e-3, -0.01),
@@ -38,7 +38,7 @@ def test_g_against_quadrature(alpha):
         assert abs(float(gauss.g(m, s, tau, alpha)) - val) < 1e-10 + 1e-9 * abs(val)
 
 
-@pytest.mark.parametrize("alpha", [1.5, 2.0])
+@pytest.mark.parametrize("alpha", [1.5, 2.0, 1.25, 1.8, 3.0])
 def test_g_against_monte_carlo(alpha):
     rng = np.random.default_rng(20)
     r = 1.0 / (alpha - 1.0)
@@ -49,14 +49,25 @@ def test_g_against_monte_carlo(alpha):
         assert abs(y.mean() - float(gauss.g(m, s, tau, alpha))) < 4 * se
 
 
-@pytest.mark.parametrize("alpha", [1.5, 2.0])
+@pytest.mark.parametrize("alpha", [1.5, 2.0, 1.25, 3.0])
 def test_point_pages_reduce_to_exact_entmax(alpha):
     rng = np.random.default_rng(21)
     for n in (1, 5, 64, 1000):
         s = rng.standard_normal(n)
         tau = gauss.tau_hat(s, np.zeros(n), np.ones(n), alpha)
-        exact = entmax.tau_sort((alpha - 1.0) * s, alpha)
+        exact = entmax.tau_bisect((alpha - 1.0) * s, alpha)
         assert abs(tau - exact) < 1e-10
+
+
+@pytest.mark.parametrize("alpha", [1.5, 2.0])
+def test_quadrature_path_matches_closed_forms(alpha):
+    """The numerical path used for alpha outside {1.5, 2}, forced at 1.5 and 2."""
+    m = np.array([0.3, 1.8, -1.0, 0.0, 2.0, 0.1, 5.0, -3.0])
+    s = np.array([0.25, 0.15, 2.0, 1e-3, 0.5, 0.3, 0.01, 0.2])
+    for tau in (-0.5, 0.0, 0.9, 1.9, 2.5):
+        a = gauss.g(m, s, tau, alpha, method="closed")
+        b = gauss.g(m, s, tau, alpha, method="quad")
+        np.testing.assert_allclose(b, a, rtol=1e-9, atol=1e-14)
 
 
 @pytest.mark.parametrize("alpha", [1.5, 2.0])
@@ -70,6 +81,19 @@ def test_F_decreasing_and_root(alpha):
     assert abs(gauss.F(t, m, v, n, alpha) - 1.0) < 1e-9
     grid = np.linspace(t - 2, t + 2, 81)
     vals = [gauss.F(x, m, v, n, alpha) for x in grid]
+    assert all(a > b for a, b in zip(vals, vals[1:]))
+
+
+@pytest.mark.parametrize("alpha", [1.25, 3.0])
+def test_F_decreasing_and_root_any_alpha(alpha):
+    rng = np.random.default_rng(23)
+    P = 24
+    m = rng.standard_normal(P)
+    v = (0.5 * rng.random(P)) ** 2
+    n = rng.integers(1, 65, P)
+    t = gauss.tau_hat(m, v, n, alpha, iters=60)
+    assert abs(gauss.F(t, m, v, n, alpha) - 1.0) < 1e-8
+    vals = [gauss.F(x, m, v, n, alpha) for x in np.linspace(t - 1, t + 1, 9)]
     assert all(a > b for a, b in zip(vals, vals[1:]))
 
 
