@@ -395,7 +395,8 @@ def run_full(wl, pool, seq_lens, flush, reps=5, warm=3):
 def run_attend_variants(wl, pool, seq_lens, flush, reps=5, warm=3):
     """On one top-k 1/64 selection: sparse entmax attention (alpha 1.5, the
     step's), softmax over the same pages (the matched-budget baseline) and
-    entmax with alpha = 1.25 (no closed form: Newton threshold, powf weights)."""
+    entmax with alpha = 1.25 (no closed form: Newton threshold, powf weights);
+    and the Gaussian selection with alpha = 3 (quadrature expectations)."""
     from sparse_long_context_min_b200 import binding as BND
     from sparse_long_context_min_b200.step import DecodeStep
     cfg = wl.cfg
@@ -416,6 +417,9 @@ def run_attend_variants(wl, pool, seq_lens, flush, reps=5, warm=3):
                                                                         step.sel, step.sel_count, 1.25, cfg.scale,
                                                                         out, step.workspace, step.status),
     }
+    gstep = DecodeStep(pool, wl.page_table, seq_lens, cfg.H_q, "gauss", alpha=3.0, delta=0.5)
+    gstep.score(wl.q)
+    calls["gauss_select_alpha_3_us"] = gstep.choose     # quadrature expectations (no closed form)
     res = {}
     for name, fn in calls.items():
         times = []
@@ -430,6 +434,7 @@ def run_attend_variants(wl, pool, seq_lens, flush, reps=5, warm=3):
         torch.cuda.synchronize()
         res[name] = round(statistics.mean(a.elapsed_time(b) * 1e3 for a, b in times), 2)
     step.check()
+    gstep.check()
     return res
 
 

@@ -34,8 +34,9 @@
  *   alpha > 1): the attention entry points take any alpha in (1, 16]; alpha
  *   = 1.5 and 2 have closed-form thresholds, any other alpha a threshold by
  *   safeguarded Newton steps in float64 and weights by powf.  The Gaussian
- *   selector takes alpha in {1.5, 2.0} only (its expectations have closed
- *   forms there) and returns ENTMAXKV_UNSUPPORTED otherwise.
+ *   selector takes alpha = 1.5 or 2 (closed-form expectations) and any alpha
+ *   in [1.25, 16] (expectations by a 32-node Gauss-Legendre rule); other
+ *   alpha return ENTMAXKV_UNSUPPORTED.
  * - page_table[b][p] (int32, [B][max_pages]) is the physical page holding
  *   logical page p of sequence b; entries p >= P_b are never read.  Physical
  *   ids out of [0, num_phys_pages) are reported as ENTMAXKV_DEVICE_BOUNDS.

@@ -103,10 +103,12 @@ static int check_heads(int H_q, int H_kv)
     return ENTMAXKV_OK;
 }
 
-// The Gaussian selector has closed forms for alpha = 1.5 and 2 only; exact
-// attention takes any alpha in (1, 16] (other values by a safeguarded Newton
-// solve of the threshold and powf weights).
-static bool alpha_ok(float alpha) { return alpha == 1.5f || alpha == 2.0f; }
+// Exact attention takes any alpha in (1, 16] (other than 1.5 and 2 by a
+// safeguarded Newton solve of the threshold and powf weights).  The Gaussian
+// selector has closed forms at 1.5 and 2 and integrates numerically for alpha
+// in [1.25, 16]; closer to 1 the power 1/(alpha-1) exceeds 4 and the fixed
+// quadrature rule loses accuracy.
+static bool alpha_gauss_ok(float alpha) { return alpha == 1.5f || alpha == 2.0f || (alpha >= 1.25f && alpha <= 16.0f); }
 static bool alpha_attend_ok(float alpha) { return alpha > 1.0f && alpha <= 16.0f; }
 
 // ------------------------------------------------------------------ workspace
@@ -271,7 +273,7 @@ int entmaxkv_select(int32_t mode, const float* ub, const float* m, const float* 
         if (B == 0) return ENTMAXKV_OK;
         if (!ub || !seq_lens || !sel || !sel_count || !status) return ENTMAXKV_INVALID_ARG;
     } else if (mode == ENTMAXKV_SELECT_GAUSS) {
-        if (!alpha_ok(alpha)) return ENTMAXKV_UNSUPPORTED;
+        if (!alpha_gauss_ok(alpha)) return ENTMAXKV_UNSUPPORTED;
         if (!std::isfinite(delta) || k_max < max_pages) return ENTMAXKV_INVALID_ARG;
         if (B == 0) return ENTMAXKV_OK;
         if (!m || !v || !est_max || !seq_lens || !sel || !sel_count || !tau_hat || !status)

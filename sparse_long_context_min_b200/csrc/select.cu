@@ -519,6 +519,7 @@ topk_cluster_kernel(const float* __restrict__ ub, const int32_t* __restrict__ se
 // it is replaced by bisection (or by doubling while no upper end is known).
 
 constexpr int kTauThreads = 512;
+constexpr int kGLNodes = 32;
 
 EKV_DEV void gauss_term(float mp, float sp, float tau, bool a2, float& g, float& dg)
 {
@@ -549,9 +550,63 @@ EKV_DEV void gauss_term(float mp, float sp, float tau, bool a2, float& g, float&
 // CTAs hold the same values and take the same steps.
 constexpr int kGaussTauCTAs = 4;
 
+// Any other alpha (r = 1/(alpha-1) not 1 or 2): E[(X - tau)_+^r] for
+// X ~ N(m', s'^2) by a 32-node Gauss-Legendre rule, with u = m' - tau and
+// z = u / s':
+//   z > 8:          int_{-8}^{8} (u + s' w)^r phi(w) dw   (the mass is away from 0);
+//   -10 < z <= 8:   int_0^T (s' t^2)^r phi(t^2 - z) 2t dt, T^2 = max(z + 8, 2)
+//                   (y = t^2 removes the y^r endpoint behaviour at 0);
+//   z <= -10:       0 (below exp(-50)).
+// g is the expectation and dg = -d/dtau of it (r times the same integrals of
+// the (r-1)-th power).
+struct GLTable {
+    float x[kGLNodes], w[kGLNodes];   // nodes and weights on [-1, 1]
+};
+
+EKV_DEV void gauss_term_any(float mp, float sp, float tau, float r, const GLTable& gl, float& g, float& dg)
+{
+    const float u = mp - tau;
+    if (!(sp > 0.f)) {
+        const float up = fmaxf(u, 0.f);
+        g = up > 0.f ? powf(up, r) : 0.f;
+        dg = up > 0.f ? r * powf(up, r - 1.f) : 0.f;
+        return;
+    }
+    const float z = u / sp;
+    g = dg = 0.f;
+    if (z <= -10.f) return;
+    const float c = 0.3989422804014327f;
+    float s0 = 0.f, s1 = 0.f;
+    if (z > 8.f) {
+#pragma unroll 8
+        for (int k = 0; k < kGLNodes; ++k) {
+            const float w = 8.f * gl.x[k];
+            const float y = fmaf(sp, w, u);
+            const float ph = c * expf(-0.5f * w * w) * 8.f * gl.w[k];
+            const float yr = powf(y, r);
+            s0 = fmaf(yr, ph, s0);
+            s1 = fmaf(yr / y, ph, s1);
+        }
+    } else {
+        const float T = sqrtf(fmaxf(z + 8.f, 2.f));
+#pragma unroll 8
+        for (int k = 0; k < kGLNodes; ++k) {
+            const float t = 0.5f * T * (gl.x[k] + 1.f);
+            const float y = sp * t * t;
+            const float e = t * t - z;
+            const float ph = c * expf(-0.5f * e * e) * t * T * gl.w[k];   // phi * 2t * (T/2) w
+            const float yr = powf(y, r);
+            s0 = fmaf(yr, ph, s0);
+            s1 = fmaf(yr / y, ph, s1);
+        }
+    }
+    g = s0;
+    dg = r * s1;
+}
+
 __global__ void __launch_bounds__(kTauThreads)
 gauss_tau_kernel(const float* __restrict__ m, const float* __restrict__ v, const int32_t* __restrict__ seq_lens,
-                 int ps, int H_q, int max_pages, float alpha, float* __restrict__ tau_hat)
+                 int ps, int H_q, int max_pages, float alpha, float* __restrict__ tau_hat, const GLTable gl)
 {
     pdl_enter();
     constexpr int C = kGaussTauCTAs, NW = kTauThreads / 32;
@@ -567,6 +622,8 @@ gauss_tau_kernel(const float* __restrict__ m, const float* __restrict__ v, const
     const int P = pages_of(L, ps, max_pages, nullptr);
     const float am1 = alpha - 1.0f;
     const bool a2 = alpha == 2.0f;
+    const bool any = !a2 && alpha != 1.5f;
+    const float rexp = 1.0f / am1;
     const float* mh = m + ((size_t)b * H_q + h) * max_pages;
     const float* vh = v + ((size_t)b * H_q + h) * max_pages;
     if (P == 0) {   // the same on every CTA of the cluster: no barrier is met
@@ -598,7 +655,8 @@ gauss_tau_kernel(const float* __restrict__ m, const float* __restrict__ v, const
             const float sp = am1 * sqrtf(fmaxf(vh[p], 0.f));
             const int n = min(ps, L - p * ps);
             float gv, dg;
-            gauss_term(mp, sp, tf, a2, gv, dg);
+            if (any) gauss_term_any(mp, sp, tf, rexp, gl, gv, dg);
+            else gauss_term(mp, sp, tf, a2, gv, dg);
             F += (double)n * gv;
             dF += (double)n * dg;
         }
@@ -744,6 +802,36 @@ gauss_keep_kernel(const float* __restrict__ est, const float* __restrict__ tau_h
     cluster_wait();     // no CTA leaves while another may still read its shared memory
 }
 
+// Gauss-Legendre nodes and weights on [-1, 1]: roots of P_n by Newton steps
+// from the Chebyshev-like guess cos(pi (i + 3/4) / (n + 1/2)), weights
+// 2 / ((1 - x^2) P_n'(x)^2); float64, computed once.
+static const GLTable& gl_table()
+{
+    static const GLTable t = [] {
+        GLTable r{};
+        const int n = kGLNodes;
+        for (int i = 0; i < n; ++i) {
+            double x = std::cos(M_PI * (i + 0.75) / (n + 0.5)), dp = 0.0;
+            for (int it = 0; it < 100; ++it) {
+                double p0 = 1.0, p1 = x;            // P_0, P_1
+                for (int k = 2; k <= n; ++k) {
+                    const double p2 = ((2.0 * k - 1.0) * x * p1 - (k - 1.0) * p0) / k;
+                    p0 = p1;
+                    p1 = p2;
+                }
+                dp = n * (x * p1 - p0) / (x * x - 1.0);   // P_n'(x)
+                const double dx = p1 / dp;
+                x -= dx;
+                if (std::fabs(dx) < 1e-16) break;
+            }
+            r.x[i] = (float)x;
+            r.w[i] = (float)(2.0 / ((1.0 - x * x) * dp * dp));
+        }
+        return r;
+    }();
+    return t;
+}
+
 int launch_select(int mode, const float* ub, const float* m, const float* v, const float* est,
                   const int32_t* seq_lens, int ps, int B, int H_q, int H_kv, int max_pages, int budget,
                   float budget_frac, float alpha, float delta, int k_max, int32_t* sel, int32_t* sel_count,
@@ -767,7 +855,7 @@ int launch_select(int mode, const float* ub, const float* m, const float* v, con
                        k_max, sel, sel_count, status);
     } else {
         launch_pdl_cluster(gauss_tau_kernel, dim3(H_q * kGaussTauCTAs, B), dim3(kTauThreads), kGaussTauCTAs, 0, stream,
-                           m, v, seq_lens, ps, H_q, max_pages, alpha, tau_hat);
+                           m, v, seq_lens, ps, H_q, max_pages, alpha, tau_hat, gl_table());
         if (cudaGetLastError() != cudaSuccess) return ENTMAXKV_CUDA_ERROR;
         const int G = H_q / H_kv;
 #define EKV_KEEP(GG)                                                                                            \

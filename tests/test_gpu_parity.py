@@ -12,7 +12,7 @@ import pytest
 import torch
 
 import helpers as H
-from oracle import attend, select
+from oracle import attend, gauss, select
 from sparse_long_context_min_b200 import binding as B
 from sparse_long_context_min_b200 import workloads
 from sparse_long_context_min_b200.step import DecodeStep, build_pool
@@ -273,6 +273,39 @@ def test_gauss_selection(alpha, delta):
             assert set(must_keep.tolist()) <= kept
             assert not (set(must_drop.tolist()) & kept)
             assert list(sel[b, g, :cnt[b, g]]) == sorted(kept)
+
+
+@pytest.mark.parametrize("alpha", [1.25, 3.0])
+def test_gauss_selection_any_alpha(alpha):
+    """alpha outside {1.5, 2}: tau_hat from the 32-node Gauss-Legendre
+    expectations against the oracle's adaptive quadrature, and the keep
+    decisions outside the threshold's uncertainty band."""
+    wl = _wl(3, [4096 + 33])
+    cfg = wl.cfg
+    pool, seq_lens = build_pool(wl)
+    delta = 0.5
+    step = DecodeStep(pool, wl.page_table, seq_lens, cfg.H_q, "gauss", alpha=alpha, delta=delta)
+    step.score(wl.q)
+    step.choose()
+    step.check()
+    tau_gpu = step.tau_hat.cpu().numpy()
+    sel, cnt = step.sel.cpu().numpy(), step.sel_count.cpu().numpy()
+    G = cfg.G
+    o = H.OracleSeq(wl, 0)
+    for g in (0, 6):
+        m, v, est = o.gauss(g)
+        n = o.meta(g)["count"]
+        ref = np.array([gauss.tau_hat(m[h].astype(np.float64), v[h].astype(np.float64), n, alpha, iters=60)
+                        for h in range(G)])
+        got = tau_gpu[0, g * G:(g + 1) * G].astype(np.float64)
+        assert np.all(np.abs(got - ref) <= H.TAU_HAT_TOL * np.maximum(1.0, np.abs(ref))), (got, ref)
+        band = np.abs(got - ref) + 1e-6 * np.maximum(1.0, np.abs(ref))
+        margin = (alpha - 1.0) * est.astype(np.float64) - (ref[:, None] - delta)
+        must_keep = np.nonzero(np.any(margin > band[:, None], axis=0))[0]
+        must_drop = np.nonzero(np.all(margin < -band[:, None], axis=0))[0]
+        kept = set(sel[0, g, :cnt[0, g]].tolist())
+        assert set(must_keep.tolist()) <= kept
+        assert not (set(must_drop.tolist()) & kept)
 
 
 def test_sparse_attend_against_oracle(built):
