@@ -10,8 +10,10 @@
  * Conventions shared by every entry point
  * ---------------------------------------
  * - Every pointer argument is CUDA device memory owned by the caller, unless
- *   the comment says "host".  The library never allocates or frees memory and
- *   keeps no state between calls.
+ *   the comment says "host".  The attention outputs (out, tau_out) may also be
+ *   pinned host memory mapped into the device's address space: the kernels
+ *   then store results straight to the host.  The library never allocates or
+ *   frees memory and keeps no state between calls.
  * - Every call is asynchronous on `stream` (a cudaStream_t passed as void*;
  *   NULL is the legacy default stream).  Inputs must stay valid and outputs
  *   untouched until the stream reaches the work.

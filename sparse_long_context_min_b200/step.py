@@ -40,10 +40,12 @@ class DecodeStep:
     """One decode step of a configuration: scores, selects and attends.
 
     mode "topk" (budget pages or budget_frac) or "gauss" (alpha, delta).
+    out: optional float32 [B][H_q][d] result buffer, on the device or in
+    pinned host memory.
     """
 
     def __init__(self, pool, page_table, seq_lens, H_q, mode="topk", budget=-1, budget_frac=0.0,
-                 alpha=1.5, delta=0.5, extra_pages=0):
+                 alpha=1.5, delta=0.5, extra_pages=0, out=None):
         self.pool, self.page_table, self.seq_lens = pool, page_table, seq_lens
         self.B = seq_lens.shape[0]
         self.H_q, self.H_kv = H_q, pool.H_kv
@@ -70,7 +72,9 @@ class DecodeStep:
             self.tau_hat = torch.empty(self.B, H_q, **f32)
         self.sel = torch.empty(self.B, self.H_kv, self.k_max, **i32)
         self.sel_count = torch.empty(self.B, self.H_kv, **i32)
-        self.out = torch.empty(self.B, H_q, pool.d, **f32)
+        # out may be pinned host memory (mapped into the device's address space):
+        # the attention kernels then store the result straight to the host
+        self.out = torch.empty(self.B, H_q, pool.d, **f32) if out is None else out
         self.tau = torch.empty(self.B, H_q, **f32)
         ws = B.workspace_size(B.OP_SPARSE_ATTEND, self.B, H_q, self.H_kv, self.max_pages, self.k_max,
                               pool.ps, pool.d)

@@ -571,5 +571,17 @@ def test_graphed_step_equals_eager_step():
         assert torch.equal(lens_a, lens_b)
     eager.check()
     graphed.step.check()
+    # the same step writing its result straight into pinned host memory
+    pool_c, lens_c = build_pool(wl)
+    out_h = torch.empty(1, cfg.H_q, cfg.d, dtype=torch.float32).pin_memory()
+    hosted = GraphedStep(DecodeStep(pool_c, wl.page_table, lens_c, cfg.H_q, "topk", budget_frac=1 / 16,
+                                    alpha=cfg.alpha, out=out_h), stage_events=False)
+    for t in range(4):
+        k, v, q = wl.decode_token(t)
+        hosted.inputs.copy_(hosted.pack_host(k, v, q), non_blocking=True)
+        hosted.replay()
+    torch.cuda.synchronize()
+    hosted.step.check()
+    assert torch.equal(out_h, graphed.step.out.cpu())
     stages = graphed.stage_us()
     assert set(stages) == set(GraphedStep.STAGES)
