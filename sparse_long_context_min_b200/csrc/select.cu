@@ -548,7 +548,8 @@ EKV_DEV void gauss_term(float mp, float sp, float tau, bool a2, float& g, float&
 // per-CTA sums are exchanged through distributed shared memory (double
 // buffered by iteration parity) and added in rank order by every CTA, so all
 // CTAs hold the same values and take the same steps.
-constexpr int kGaussTauCTAs = 4;
+constexpr int kGaussTauCTAs = 8;
+constexpr int kGaussTauReg = 4;      // pages per thread whose terms' inputs stay in registers
 
 // Any other alpha (r = 1/(alpha-1) not 1 or 2): E[(X - tau)_+^r] for
 // X ~ N(m', s'^2) by a 32-node Gauss-Legendre rule, with u = m' - tau and
@@ -605,17 +606,18 @@ EKV_DEV void gauss_term_any(float mp, float sp, float tau, float r, const GLTabl
 }
 
 __global__ void __launch_bounds__(kTauThreads)
-gauss_tau_kernel(const float* __restrict__ m, const float* __restrict__ v, const int32_t* __restrict__ seq_lens,
-                 int ps, int H_q, int max_pages, float alpha, float* __restrict__ tau_hat, const GLTable gl)
+gauss_tau_kernel(const float* __restrict__ m, const float* __restrict__ v, const float* __restrict__ est,
+                 const int32_t* __restrict__ seq_lens, int ps, int H_q, int max_pages, float alpha,
+                 float* __restrict__ tau_hat, const GLTable gl)
 {
     pdl_enter();
-    constexpr int C = kGaussTauCTAs, NW = kTauThreads / 32;
+    constexpr int C = kGaussTauCTAs, NW = kTauThreads / 32, KR = kGaussTauReg;
     __shared__ double red[2][NW];
-    __shared__ float redf[NW];
+    __shared__ float redf[2][NW];
     __shared__ double pub[2][2];          // this CTA's (F, F') of the iterations of each parity
-    __shared__ float pub_mx;
+    __shared__ float pub_mx[2];
     __shared__ double gsum[2];
-    __shared__ float gmx;
+    __shared__ float gmx[2];
     const int r = (int)cluster_rank();
     const int b = blockIdx.y, h = blockIdx.x / C, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int L = seq_lens[b];
@@ -626,31 +628,82 @@ gauss_tau_kernel(const float* __restrict__ m, const float* __restrict__ v, const
     const float rexp = 1.0f / am1;
     const float* mh = m + ((size_t)b * H_q + h) * max_pages;
     const float* vh = v + ((size_t)b * H_q + h) * max_pages;
+    const float* eh = est + ((size_t)b * H_q + h) * max_pages;
     if (P == 0) {   // the same on every CTA of the cluster: no barrier is met
         if (tid == 0 && r == 0) tau_hat[(size_t)b * H_q + h] = INFINITY;
         return;
     }
     const int chunk = (P + C - 1) / C;
     const int p0 = min(P, r * chunk), p1 = min(P, p0 + chunk);
-
-    float mx = -INFINITY;
-    for (int p = p0 + tid; p < p1; p += kTauThreads) mx = fmaxf(mx, am1 * mh[p]);
-    mx = block_max(mx, redf);
-    if (tid == 0) pub_mx = mx;
-    cluster_sync();
-    if (warp == 0) {
-        float x = lane < C ? ld_dsmem_f32(dsmem(&pub_mx, lane)) : -INFINITY;
-        x = warp_max(x);
-        if (lane == 0) gmx = x;
+    // inputs of this thread's first KR pages, kept for every iteration: m', s', tokens
+    float rm[KR], rs[KR];
+    int rn[KR];
+    float mx = -INFINITY, emx = -INFINITY;
+#pragma unroll
+    for (int k = 0; k < KR; ++k) {
+        const int p = p0 + tid + k * kTauThreads;
+        rn[k] = 0;
+        rm[k] = rs[k] = 0.f;
+        if (p < p1) {
+            rm[k] = am1 * mh[p];
+            rs[k] = am1 * sqrtf(fmaxf(vh[p], 0.f));
+            rn[k] = min(ps, L - p * ps);
+            mx = fmaxf(mx, rm[k]);
+            emx = fmaxf(emx, am1 * eh[p]);
+        }
+    }
+    for (int p = p0 + tid + KR * kTauThreads; p < p1; p += kTauThreads) {
+        mx = fmaxf(mx, am1 * mh[p]);
+        emx = fmaxf(emx, am1 * eh[p]);
+    }
+    mx = warp_max(mx);
+    emx = warp_max(emx);
+    if (lane == 0) {
+        redf[0][warp] = mx;
+        redf[1][warp] = emx;
     }
     __syncthreads();
-    double lo = (double)gmx - 1.0;   // F(lo) >= 1 (Jensen: the top page alone gives >= 1)
+    if (warp == 0) {
+        float a = lane < NW ? redf[0][lane] : -INFINITY;
+        float c = lane < NW ? redf[1][lane] : -INFINITY;
+        a = warp_max(a);
+        c = warp_max(c);
+        if (lane == 0) {
+            pub_mx[0] = a;
+            pub_mx[1] = c;
+        }
+    }
+    cluster_sync();
+    if (warp == 0) {
+        float a = lane < C ? ld_dsmem_f32(dsmem(&pub_mx[0], lane)) : -INFINITY;
+        float c = lane < C ? ld_dsmem_f32(dsmem(&pub_mx[1], lane)) : -INFINITY;
+        a = warp_max(a);
+        c = warp_max(c);
+        if (lane == 0) {
+            gmx[0] = a;
+            gmx[1] = c;
+        }
+    }
+    __syncthreads();
+    double lo = (double)gmx[0] - 1.0;   // F(lo) >= 1 (Jensen: the top page alone gives >= 1)
     double hi = INFINITY;
-    double tau = lo;
+    // first guess half a unit below the largest estimated page maximum: the
+    // threshold sits just under the top scores, so this usually starts a step
+    // or two from the root (the bracket keeps any start safe)
+    double tau = fmax(lo, (double)gmx[1] - 0.5);
     for (int it = 0; it < 60; ++it) {
         double F = 0.0, dF = 0.0;
         const float tf = (float)tau;
-        for (int p = p0 + tid; p < p1; p += kTauThreads) {
+#pragma unroll
+        for (int k = 0; k < KR; ++k) {
+            if (rn[k] == 0) continue;
+            float gv, dg;
+            if (any) gauss_term_any(rm[k], rs[k], tf, rexp, gl, gv, dg);
+            else gauss_term(rm[k], rs[k], tf, a2, gv, dg);
+            F += (double)rn[k] * gv;
+            dF += (double)rn[k] * dg;
+        }
+        for (int p = p0 + tid + KR * kTauThreads; p < p1; p += kTauThreads) {
             const float mp = am1 * mh[p];
             const float sp = am1 * sqrtf(fmaxf(vh[p], 0.f));
             const int n = min(ps, L - p * ps);
@@ -855,7 +908,7 @@ int launch_select(int mode, const float* ub, const float* m, const float* v, con
                        k_max, sel, sel_count, status);
     } else {
         launch_pdl_cluster(gauss_tau_kernel, dim3(H_q * kGaussTauCTAs, B), dim3(kTauThreads), kGaussTauCTAs, 0, stream,
-                           m, v, seq_lens, ps, H_q, max_pages, alpha, tau_hat, gl_table());
+                           m, v, est, seq_lens, ps, H_q, max_pages, alpha, tau_hat, gl_table());
         if (cudaGetLastError() != cudaSuccess) return ENTMAXKV_CUDA_ERROR;
         const int G = H_q / H_kv;
 #define EKV_KEEP(GG)                                                                                            \
