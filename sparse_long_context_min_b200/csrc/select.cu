@@ -237,7 +237,7 @@ topk_kernel(const float* __restrict__ ub, const int32_t* __restrict__ seq_lens, 
 // decisions and meet the same cluster barriers.
 //  round: [min, max] of the keys in play; if equal, the keys in play are
 //         tied and the `need` lowest indices among them are kept; otherwise
-//         a 2048-bin histogram over a linear map of [min, max] gives the
+//         a 512-bin histogram over a linear map of [min, max] gives the
 //         bucket T holding the need-th key; if T holds at most kCCap keys
 //         they are gathered and ranked exactly, else the next round
 //         narrows to T.
@@ -245,9 +245,9 @@ topk_kernel(const float* __restrict__ ub, const int32_t* __restrict__ seq_lens, 
 //         of lower rank.
 constexpr int kTopkCTAs = 8;
 constexpr int kCThreads = 512;
-constexpr int kCBins = 2048;     // 4 per thread
+constexpr int kCBins = kCThreads; // one bin per thread (each CTA reads every CTA's bins)
 constexpr int kCCap = 1024;
-constexpr int kCRounds = 32;     // each round shrinks the range >= 2048x: covers every float range
+constexpr int kCRounds = 40;     // each round shrinks the range >= 512x: 40 rounds cover every float range
 
 struct TopkClusterShared {
     __align__(16) int hist[kCBins];          // this CTA's histogram of the round
@@ -389,28 +389,17 @@ topk_cluster_kernel(const float* __restrict__ ub, const int32_t* __restrict__ se
         for (int e = 0; e < KPT; ++e)
             if (inplay(e)) atomicAdd(&sh.hist[bucket_of(kv[e], mn, w)], 1);
         cluster_sync();
-        // thread t sums bins jb..jb+3 over the cluster (thread 0 the top four)
-        const int jb = kCBins - 4 * (tid + 1);
-        int hs[4] = {0, 0, 0, 0};
+        // thread t sums bin jb = NB - 1 - t over the cluster (thread 0 the top bin)
+        const int jb = kCBins - 1 - tid;
+        int hsum = 0;
 #pragma unroll
-        for (int q = 0; q < C; ++q) {
-            const uint4 v = ld_dsmem_v4(dsmem(&sh.hist[jb], q));
-            hs[0] += (int)v.x;
-            hs[1] += (int)v.y;
-            hs[2] += (int)v.z;
-            hs[3] += (int)v.w;
-        }
-        const int s4 = hs[0] + hs[1] + hs[2] + hs[3];
-        const int incl = block_scan_incl(s4, sh.wsum);
-        int above = incl - s4;   // keys in bins above jb + 3
-#pragma unroll
-        for (int u = 3; u >= 0; --u) {
-            if (above < need && need <= above + hs[u]) {
-                sh.T = jb + u;
-                sh.need = need - above;
-                sh.cT = hs[u];
-            }
-            above += hs[u];
+        for (int q = 0; q < C; ++q) hsum += ld_dsmem_s32(dsmem(&sh.hist[jb], q));
+        const int incl = block_scan_incl(hsum, sh.wsum);
+        const int above = incl - hsum;   // keys in the bins above jb
+        if (above < need && need <= above + hsum) {
+            sh.T = jb;
+            sh.need = need - above;
+            sh.cT = hsum;
         }
         __syncthreads();
         const int T = sh.T;
