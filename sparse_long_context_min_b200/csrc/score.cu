@@ -606,10 +606,12 @@ int launch_score(const entmaxkv_pool& pool, const float* q, int H_q, const int32
         a.row_a = pool.kmin;
         a.row_b = pool.kmax;
         if (pool.dtype == ENTMAXKV_BF16) {
-            // the role-split kernel needs H_kv to divide the rows of a round and
-            // at most 32 pages per stage (one producer lane each)
+            // the role-split kernel needs H_kv to divide the rows of a round, and
+            // a number of pages per stage that divides 32 (one producer lane per
+            // page; page-table entries come in batches of 32)
             const int set = kWsConsumers * (32 / (8 * (G >= 2 ? G / 2 : 1)));
-            if (set % pool.H_kv == 0 && kWsRounds * set / pool.H_kv <= 32)
+            const int pps = set % pool.H_kv == 0 ? kWsRounds * set / pool.H_kv : 0;
+            if (pps > 0 && pps <= 32 && 32 % pps == 0)
                 return pool.d == 128 ? dispatch_box16<128>(G, a, stream) : dispatch_box16<64>(G, a, stream);
             return pool.d == 128 ? dispatch_g<uint16_t, 128, false>(G, a, zt, stream)
                                  : dispatch_g<uint16_t, 64, false>(G, a, zt, stream);
