@@ -98,7 +98,7 @@ __global__ void append_kernel(T* __restrict__ k_pool, T* __restrict__ v_pool, T*
 // seq_lens itself -- no other block reads that sequence's length, so no second
 // kernel is needed.
 template <typename T>
-__global__ void append_small_kernel(T* __restrict__ k_pool, T* __restrict__ v_pool, T* __restrict__ kmin,
+__global__ void __launch_bounds__(1024) append_small_kernel(T* __restrict__ k_pool, T* __restrict__ v_pool, T* __restrict__ kmin,
                                     T* __restrict__ kmax, float* __restrict__ mean, float* __restrict__ m2,
                                     int32_t* __restrict__ count, int num_phys, int H_kv, int ps, int d,
                                     const T* __restrict__ k_new, const T* __restrict__ v_new, int n_new,
@@ -107,6 +107,15 @@ __global__ void append_small_kernel(T* __restrict__ k_pool, T* __restrict__ v_po
 {
     pdl_enter();
     const int b = blockIdx.x;
+    // the first new token of this thread's first (kv head, coordinate) does not
+    // depend on the sequence length: load it before the length and page id
+    const int w0 = threadIdx.x;
+    T pk = T(0), pv = T(0);
+    if (n_new > 0 && w0 < H_kv * d) {
+        const size_t src = ((size_t)b * H_kv + w0 / d) * n_new * d + w0 % d;
+        pk = k_new[src];
+        pv = v_new[src];
+    }
     const int base = seq_lens[b];
     __syncthreads();                      // every thread has read the length
     if (base < 0) {
@@ -143,10 +152,11 @@ __global__ void append_small_kernel(T* __restrict__ k_pool, T* __restrict__ v_po
             for (int t = t0; t < t1; ++t) {
                 const int slot = t - lp * ps;
                 const size_t src = (src0 + (t - base)) * d + j;
-                const T kx = k_new[src];
+                const bool pre = w == w0 && t == base;
+                const T kx = pre ? pk : k_new[src];
                 const size_t dst = (row * ps + slot) * d + j;
                 k_pool[dst] = kx;
-                v_pool[dst] = v_new[src];
+                v_pool[dst] = pre ? pv : v_new[src];
                 const float x = kv_to_f32<T>(kx);
                 if (slot == 0) {
                     mu = x;

@@ -464,6 +464,8 @@ __global__ void __launch_bounds__(kTauBlock) tau_kernel(int ps, const AttnArgs a
         return;
     }
     const double thr = (double)M - 1.0;
+    // float prefilter at or below thr: most scores fail it without a float64 step
+    const float thr_f = nextafterf((float)thr, -INFINITY);
     if (tid == 0) ncand = 0;
     for (int i = tid; i < kTauBins; i += kTauBlock) hist[i] = 0;
     __syncthreads();
@@ -483,6 +485,7 @@ __global__ void __launch_bounds__(kTauBlock) tau_kernel(int ps, const AttnArgs a
         int c = 0;
 #pragma unroll
         for (int e = 0; e < 4 * U; ++e) {
+            if (!(v[e] > thr_f)) continue;
             const double d = (double)v[e] - thr;
             if (d > 0.0) {
                 ++c;
@@ -503,7 +506,7 @@ __global__ void __launch_bounds__(kTauBlock) tau_kernel(int ps, const AttnArgs a
         int pos = wbase + incl - c;
 #pragma unroll
         for (int e = 0; e < 4 * U; ++e)
-            if ((double)v[e] > thr) {
+            if (v[e] > thr_f && (double)v[e] > thr) {
                 if (pos < kTauCap) cand[pos] = v[e];
                 ++pos;
             }
