@@ -198,10 +198,12 @@ def _topk_cases():
     dense[5] = -1e30
     rng.shuffle(dense)                                   # 3000 distinct keys a few ulps apart
     wide = rng.standard_normal(60000).astype(np.float32) # several keys per thread
-    return {"big_tie": big_tie, "outlier": outlier, "dense": dense, "wide": wide}
+    huge = rng.standard_normal(70001).astype(np.float32) # past the cluster kernel: global-memory top-k
+    huge[rng.permutation(70001)[:3000]] = 0.5            # with a large tie
+    return {"big_tie": big_tie, "outlier": outlier, "dense": dense, "wide": wide, "huge": huge}
 
 
-@pytest.mark.parametrize("case", ["big_tie", "outlier", "dense", "wide"])
+@pytest.mark.parametrize("case", ["big_tie", "outlier", "dense", "wide", "huge"])
 def test_topk_narrowing_rounds(case):
     """Key sets whose threshold bucket holds more than the exact-rank capacity,
     so the selection narrows over several rounds (or ends in a tie round)."""
