@@ -270,7 +270,7 @@ def run_native(args, rank, world, local):
     if rank == 0 and not args.no_cpu:
         cpu = cpu_baseline(wl, pool, budget_frac=1 / 64, seconds=8.0)
 
-    n_launch = 7   # append + advance, score, select, qk + tau + pv (one graph replay)
+    n_launch = 6   # append (one token: no separate length kernel), score, top-k, qk + tau + pv per replay
     step_gbs = by["total"] / (mean_us_all * 1e-6) / 1e9
     score_gbs = by["score"] / (score_us * 1e-6) / 1e9
     clk = clocks.summary()
