@@ -480,7 +480,7 @@ def run_reference(args, rank, world):
         return
     if torch.cuda.is_available():
         torch.cuda.set_device(0)
-    wl = make_workload(args.context, 0)
+    wl = make_workload(args.context, 0, device="cuda" if torch.cuda.is_available() else "cpu")
     from oracle import replica
     cfg = wl.cfg
     keys, vals = wl.sequence(0, heads=[0])
