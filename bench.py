@@ -47,6 +47,9 @@ def parse():
     ap.add_argument("--context", type=int, default=1 << 20, help="tokens per sequence (default 2^20)")
     ap.add_argument("--no-baselines", action="store_true", help="skip the full-cache and Gaussian timings")
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline leg")
+    ap.add_argument("--replay-only", choices=["topk", "gauss"], default=None,
+                    help="build the workload, capture that step as a graph and replay it --steps times "
+                         "without timing (a short program for profiler launch lists)")
     return ap.parse_args()
 
 
@@ -507,8 +510,33 @@ def run_reference(args, rank, world):
     print(json.dumps(line), flush=True)
 
 
+def replay_only(args):
+    """Capture one decode step (top-k 1/64 or the Gaussian selector, Delta 0.5)
+    of the bench workload as a graph and replay it; prints nothing but "ok"."""
+    from sparse_long_context_min_b200.step import DecodeStep, GraphedStep, build_pool
+    wl = make_workload(args.context, 0)
+    cfg = wl.cfg
+    pool, seq_lens = build_pool(wl)
+    st = DecodeStep(pool, wl.page_table, seq_lens, cfg.H_q, args.replay_only, budget_frac=1 / 64,
+                    alpha=cfg.alpha, delta=0.5)
+    gs = GraphedStep(st, append=True, stage_events=False)
+    flush = torch.empty(256 * MiB, dtype=torch.uint8, device="cuda")
+    for i in range(args.steps):
+        k, v, q = wl.decode_token(i)
+        gs.inputs.copy_(gs.pack_host(k, v, q), non_blocking=True)
+        flush.fill_(i & 0xFF)
+        gs.replay()
+    torch.cuda.synchronize()
+    st.check()
+    print("ok", args.replay_only)
+
+
 def main():
     args = parse()
+    if args.replay_only:
+        torch.cuda.set_device(0)
+        replay_only(args)
+        return
     rank, world, local = dist_init(args.gpus)
     try:
         if args.impl == "reference":
