@@ -26,7 +26,7 @@
 namespace ekv {
 
 constexpr int kScoreCTA = 512;
-constexpr int kScoreStages = 4;
+constexpr int kScoreStages = 2;
 
 struct ZTable {
     float z[65];
