@@ -310,6 +310,38 @@ def test_gauss_selection_any_alpha(alpha):
         assert not (set(must_drop.tolist()) & kept)
 
 
+@pytest.mark.parametrize("alpha", [1.5, 2.0])
+def test_gauss_selection_many_pages(alpha):
+    """Synthetic page statistics for 40001 pages (more than a CTA's register
+    share in the tau_hat solve and several keep tiles per CTA): tau_hat
+    against the oracle, and the kept set equal to the fp32 keep rule
+    evaluated with the GPU's own tau_hat."""
+    rng = np.random.default_rng(31)
+    P, G, ps, delta = 40001, 4, 16, 0.5
+    m = (0.6 * rng.standard_normal((1, G, P))).astype(np.float32)
+    v = (0.3 * rng.random((1, G, P)) ** 2).astype(np.float32)
+    count = np.full(P, ps, dtype=np.int64)
+    count[-1] = 7                                          # ragged last page
+    z = gauss.z_table(ps).astype(np.float32)
+    est = (m + np.sqrt(v) * z[count][None, None, :]).astype(np.float32)
+    L = (P - 1) * ps + 7
+    seq_lens = torch.tensor([L], dtype=torch.int32, device="cuda")
+    sel = torch.full((1, 1, P), -7, dtype=torch.int32, device="cuda")
+    cnt = torch.empty(1, 1, dtype=torch.int32, device="cuda")
+    tau_hat = torch.empty(1, G, device="cuda")
+    st = _status()
+    B.select(B.SELECT_GAUSS, seq_lens, ps, G, 1, P, P, sel, cnt, st, m=torch.from_numpy(m).cuda(),
+             v=torch.from_numpy(v).cuda(), est_max=torch.from_numpy(est).cuda(), alpha=alpha, delta=delta,
+             tau_hat=tau_hat)
+    _assert_ok(st)
+    got = tau_hat.cpu().numpy()[0].astype(np.float64)
+    ref = np.array([gauss.tau_hat(m[0, h].astype(np.float64), v[0, h].astype(np.float64), count, alpha)
+                    for h in range(G)])
+    assert np.all(np.abs(got - ref) <= H.TAU_HAT_TOL * np.maximum(1.0, np.abs(ref))), (got, ref)
+    kept = sel[0, 0, :int(cnt[0, 0])].cpu().numpy()
+    assert np.array_equal(kept, select.gauss_keep(est[0], tau_hat.cpu().numpy()[0], alpha, delta))
+
+
 def test_sparse_attend_against_oracle(built):
     wl, pool, seq_lens, oseqs = built
     cfg = wl.cfg
