@@ -164,9 +164,19 @@ SHAPES = {
 }
 
 
-@pytest.mark.parametrize("shape", list(SHAPES))
+# fp32 caches take the streaming scoring kernel and the CUDA-core attention
+FP32_SHAPES = {
+    "f32_g8_d128_ps64": dict(H_q=64, H_kv=8, d=128, ps=64),
+    "f32_g2_d128_ps16": dict(H_q=8, H_kv=4, d=128, ps=16),
+}
+
+
+@pytest.mark.parametrize("shape", list(SHAPES) + list(FP32_SHAPES))
 def test_head_and_page_shapes(shape):
-    wl = _wl(2, [3001, 1234], **SHAPES[shape])
+    if shape in FP32_SHAPES:
+        wl = _wl(1, [3001, 1234], **FP32_SHAPES[shape])
+    else:
+        wl = _wl(2, [3001, 1234], **SHAPES[shape])
     cfg = wl.cfg
     pool, seq_lens = build_pool(wl)
     step = DecodeStep(pool, wl.page_table, seq_lens, cfg.H_q, "topk", budget_frac=1 / 8, alpha=cfg.alpha)
