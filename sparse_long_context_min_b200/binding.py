@@ -1,10 +1,12 @@
 """Thin ctypes binding over the EntmaxKV C ABI (include/entmaxkv.h).
 
-Argument marshalling only: every function below passes torch tensors' device
-pointers, sizes and the current CUDA stream to the entry point of the same
-name and raises on a non-zero host status.  All work runs in the CUDA library;
-there is no other implementation to fall back to -- if the shared library is
-missing the first call raises.
+Argument marshalling only: every function below checks that each tensor can
+be handed to the library as a plain pointer (dtype, dense layout, enough
+elements for the sizes the call passes, memory the current GPU can address),
+then passes the tensors' pointers, sizes and the current CUDA stream to the
+entry point of the same name and raises on a non-zero host status.  All work
+runs in the CUDA library; there is no other implementation to fall back to --
+if the shared library is missing the first call raises.
 """
 import ctypes
 import os
@@ -31,8 +33,8 @@ SYMBOLS = (
 
 
 class EntmaxKVError(RuntimeError):
-    def __init__(self, code, where):
-        super().__init__("%s: %s (status %d)" % (where, status_string(code), code))
+    def __init__(self, code, where, detail=None):
+        super().__init__("%s: %s (status %d)" % (where, detail or status_string(code), code))
         self.code = code
 
 
@@ -90,6 +92,51 @@ def _p(t):
     return None if t is None else ctypes.c_void_p(t.data_ptr())
 
 
+class _Args:
+    """Checks of one call's tensors before anything is launched.  The library
+    takes plain pointers, so a tensor of the wrong dtype or rank, a strided
+    view, fewer elements than the sizes passed address, or memory the current
+    GPU cannot reach would be read or written out of bounds; `need` checks the
+    layout of each tensor as it is named and `reachable` then checks that every
+    one is the current device's memory or pinned (mapped) host memory."""
+
+    def __init__(self, where):
+        self.where = where
+        self.seen = []
+
+    def fail(self, detail, code=INVALID_ARG):
+        raise EntmaxKVError(code, self.where, detail)
+
+    def need(self, t, name, dtype=None, numel=0, dims=None):
+        if t is None:
+            self.fail("%s is required" % name)
+        if dtype is not None and t.dtype != dtype:
+            self.fail("%s must be %s, not %s" % (name, dtype, t.dtype))
+        if dims is not None and t.dim() != dims:
+            self.fail("%s must have %d dimensions, not %d" % (name, dims, t.dim()))
+        if not t.is_contiguous():
+            self.fail("%s must be contiguous" % name)
+        if t.numel() < numel:
+            self.fail("%s holds %d elements; the call addresses %d" % (name, t.numel(), numel))
+        self.seen.append((name, t))
+        return t
+
+    def reachable(self):
+        dev = capturing = None
+        for name, t in self.seen:
+            if t.is_cuda:
+                dev = torch.cuda.current_device() if dev is None else dev
+                if t.get_device() != dev:
+                    self.fail("%s is on cuda:%d, the current device is cuda:%d" % (name, t.get_device(), dev))
+                continue
+            if capturing is None:
+                # the pinned-memory query is not issued while a CUDA graph is
+                # being captured; the eager call before a capture checks it
+                capturing = torch.cuda.is_available() and torch.cuda.is_current_stream_capturing()
+            if not capturing and not t.is_pinned():
+                self.fail("%s must be in device memory or pinned host memory" % name)
+
+
 def _stream(stream):
     s = torch.cuda.current_stream() if stream is None else stream
     return ctypes.c_void_p(s.cuda_stream)
@@ -104,9 +151,24 @@ class Pool:
     """
 
     def __init__(self, k_pool, v_pool, kmin, kmax, mean, m2, count):
+        a = _Args("Pool")
+        if k_pool.dtype not in (torch.float32, torch.bfloat16):
+            a.fail("k_pool must be float32 or bfloat16, not %s" % k_pool.dtype, UNSUPPORTED)
+        a.need(k_pool, "k_pool", dims=4)
+        num_phys, H_kv, ps, d = k_pool.shape
+        meta = num_phys * H_kv * d
+        a.need(v_pool, "v_pool", k_pool.dtype, k_pool.numel(), dims=4)
+        a.need(kmin, "kmin", k_pool.dtype, meta)
+        a.need(kmax, "kmax", k_pool.dtype, meta)
+        a.need(mean, "mean", torch.float32, meta)
+        a.need(m2, "m2", torch.float32, meta)
+        a.need(count, "count", torch.int32, num_phys)
+        if tuple(v_pool.shape) != tuple(k_pool.shape):
+            a.fail("v_pool must have k_pool's shape")
+        a.reachable()
         self.k_pool, self.v_pool = k_pool, v_pool
         self.kmin, self.kmax, self.mean, self.m2, self.count = kmin, kmax, mean, m2, count
-        self.num_phys, self.H_kv, self.ps, self.d = k_pool.shape
+        self.num_phys, self.H_kv, self.ps, self.d = num_phys, H_kv, ps, d
         self.dtype = BF16 if k_pool.dtype == torch.bfloat16 else F32
         self._c = CPool(k_pool.data_ptr(), v_pool.data_ptr(), kmin.data_ptr(), kmax.data_ptr(),
                         mean.data_ptr(), m2.data_ptr(), count.data_ptr(), self.num_phys, self.H_kv,
@@ -126,30 +188,100 @@ class Pool:
         return ctypes.byref(self._c)
 
 
+I32, F32T = torch.int32, torch.float32
+
+
+def _query(a, pool, q):
+    """q [B, H_q, d] float32 with the pool's d; returns (B, H_q)."""
+    a.need(q, "q", F32T, dims=3)
+    if q.shape[2] != pool.d:
+        a.fail("q has %d dims per head, the pool %d" % (q.shape[2], pool.d))
+    return q.shape[0], q.shape[1]
+
+
+def _table(a, page_table, seq_lens, B):
+    """page_table [>= B, max_pages] and seq_lens [>= B], both int32; returns max_pages."""
+    a.need(page_table, "page_table", I32, dims=2)
+    if page_table.shape[0] < B:
+        a.fail("page_table has %d rows for %d sequences" % (page_table.shape[0], B))
+    a.need(seq_lens, "seq_lens", I32, B)
+    return page_table.shape[1]
+
+
+def _page_list(a, pool, sel, sel_count, B):
+    """sel [>= B, H_kv, k_max] and sel_count [>= B * H_kv], int32; returns k_max."""
+    a.need(sel, "sel", I32, dims=3)
+    if sel.shape[0] < B or sel.shape[1] != pool.H_kv:
+        a.fail("sel must be [B, H_kv, k_max] with B = %d and H_kv = %d" % (B, pool.H_kv))
+    a.need(sel_count, "sel_count", I32, B * pool.H_kv)
+    return sel.shape[2]
+
+
+def _outputs(a, pool, out, tau_out, v_pages, status, B, H_q):
+    a.need(out, "out", F32T, B * H_q * pool.d)
+    if tau_out is not None:
+        a.need(tau_out, "tau_out", F32T, B * H_q)
+    if v_pages is not None:
+        a.need(v_pages, "v_pages", I32, B * pool.H_kv)
+    a.need(status, "status", I32, 1)
+
+
+def _bytes(t):
+    return t.numel() * t.element_size()
+
+
 def append_metadata(pool, k_new, v_new, page_table, seq_lens, status, stream=None):
     """k_new, v_new [B, H_kv, n_new, d]; seq_lens advanced in place on the device."""
-    B, _, n_new, _ = k_new.shape
+    a = _Args("append_metadata")
+    a.need(k_new, "k_new", pool.k_pool.dtype, dims=4)
+    B, H_kv, n_new, d = k_new.shape
+    if H_kv != pool.H_kv or d != pool.d:
+        a.fail("k_new must be [B, %d, n_new, %d]" % (pool.H_kv, pool.d))
+    a.need(v_new, "v_new", pool.k_pool.dtype, k_new.numel(), dims=4)
+    max_pages = _table(a, page_table, seq_lens, B)
+    a.need(status, "status", I32, 1)
+    a.reachable()
     _check(lib().entmaxkv_append_metadata(pool.c, _p(k_new), _p(v_new), n_new, _p(page_table),
-                                          page_table.shape[1], _p(seq_lens), B, _p(status),
-                                          _stream(stream)), "append_metadata")
+                                          max_pages, _p(seq_lens), B, _p(status),
+                                          _stream(stream)), a.where)
 
 
 def score_pages(pool, q, page_table, seq_lens, mode, scale, status, ub=None, m=None, v=None,
                 est_max=None, stream=None):
-    B, H_q, _ = q.shape
-    _check(lib().entmaxkv_score_pages(pool.c, _p(q), H_q, _p(page_table), page_table.shape[1],
+    a = _Args("score_pages")
+    B, H_q = _query(a, pool, q)
+    max_pages = _table(a, page_table, seq_lens, B)
+    a.need(status, "status", I32, 1)
+    if mode == SCORE_BBOX:
+        a.need(ub, "ub", F32T, B * pool.H_kv * max_pages)
+    elif mode == SCORE_GAUSS:
+        for t, name in ((m, "m"), (v, "v"), (est_max, "est_max")):
+            a.need(t, name, F32T, B * H_q * max_pages)
+    a.reachable()
+    _check(lib().entmaxkv_score_pages(pool.c, _p(q), H_q, _p(page_table), max_pages,
                                       _p(seq_lens), B, mode, scale, _p(ub), _p(m), _p(v), _p(est_max),
-                                      _p(status), _stream(stream)), "score_pages")
+                                      _p(status), _stream(stream)), a.where)
 
 
 def select(mode, seq_lens, ps, H_q, H_kv, max_pages, k_max, sel, sel_count, status, ub=None, m=None,
            v=None, est_max=None, budget=-1, budget_frac=0.0, alpha=1.5, delta=0.0, tau_hat=None,
            stream=None):
+    a = _Args("select")
+    a.need(seq_lens, "seq_lens", I32, dims=1)
     B = seq_lens.shape[0]
+    a.need(sel, "sel", I32, B * H_kv * k_max)
+    a.need(sel_count, "sel_count", I32, B * H_kv)
+    a.need(status, "status", I32, 1)
+    if mode == SELECT_TOPK:
+        a.need(ub, "ub", F32T, B * H_kv * max_pages)
+    elif mode == SELECT_GAUSS:
+        for t, name in ((m, "m"), (v, "v"), (est_max, "est_max")):
+            a.need(t, name, F32T, B * H_q * max_pages)
+        a.need(tau_hat, "tau_hat", F32T, B * H_q)
+    a.reachable()
     _check(lib().entmaxkv_select(mode, _p(ub), _p(m), _p(v), _p(est_max), _p(seq_lens), ps, B, H_q,
                                  H_kv, max_pages, budget, budget_frac, alpha, delta, k_max, _p(sel),
-                                 _p(sel_count), _p(tau_hat), None, 0, _p(status), _stream(stream)),
-           "select")
+                                 _p(sel_count), _p(tau_hat), None, 0, _p(status), _stream(stream)), a.where)
 
 
 def workspace_size(op, B, H_q, H_kv, max_pages, k_max, ps, d):
@@ -158,50 +290,78 @@ def workspace_size(op, B, H_q, H_kv, max_pages, k_max, ps, d):
 
 def sparse_attend(pool, q, page_table, seq_lens, sel, sel_count, alpha, scale, out, workspace, status,
                   tau_out=None, v_pages=None, stream=None):
-    B, H_q, _ = q.shape
-    _check(lib().entmaxkv_sparse_attend(pool.c, _p(q), H_q, _p(page_table), page_table.shape[1],
-                                        _p(seq_lens), B, _p(sel), _p(sel_count), sel.shape[2], alpha,
+    a = _Args("sparse_attend")
+    B, H_q = _query(a, pool, q)
+    max_pages = _table(a, page_table, seq_lens, B)
+    k_max = _page_list(a, pool, sel, sel_count, B)
+    _outputs(a, pool, out, tau_out, v_pages, status, B, H_q)
+    a.need(workspace, "workspace")
+    a.reachable()
+    _check(lib().entmaxkv_sparse_attend(pool.c, _p(q), H_q, _p(page_table), max_pages,
+                                        _p(seq_lens), B, _p(sel), _p(sel_count), k_max, alpha,
                                         scale, _p(out), _p(tau_out), _p(v_pages), _p(workspace),
-                                        workspace.numel() * workspace.element_size(), _p(status),
-                                        _stream(stream)), "sparse_attend")
+                                        _bytes(workspace), _p(status), _stream(stream)), a.where)
 
 
 def sparse_attend_static(pool, q, page_table, seq_lens, sel, sel_count, alpha, scale, out, status,
                          tau_out=None, v_pages=None, stream=None):
     """sparse_attend with the library's built-in scratch buffer (no workspace)."""
-    B, H_q, _ = q.shape
-    _check(lib().entmaxkv_sparse_attend_static(pool.c, _p(q), H_q, _p(page_table), page_table.shape[1],
-                                               _p(seq_lens), B, _p(sel), _p(sel_count), sel.shape[2], alpha,
+    a = _Args("sparse_attend_static")
+    B, H_q = _query(a, pool, q)
+    max_pages = _table(a, page_table, seq_lens, B)
+    k_max = _page_list(a, pool, sel, sel_count, B)
+    _outputs(a, pool, out, tau_out, v_pages, status, B, H_q)
+    a.reachable()
+    _check(lib().entmaxkv_sparse_attend_static(pool.c, _p(q), H_q, _p(page_table), max_pages,
+                                               _p(seq_lens), B, _p(sel), _p(sel_count), k_max, alpha,
                                                scale, _p(out), _p(tau_out), _p(v_pages), _p(status),
-                                               _stream(stream)), "sparse_attend_static")
+                                               _stream(stream)), a.where)
 
 
 def full_entmax_decode(pool, q, page_table, seq_lens, alpha, scale, out, workspace, status,
                        tau_out=None, v_pages=None, stream=None):
-    B, H_q, _ = q.shape
-    _check(lib().entmaxkv_full_entmax_decode(pool.c, _p(q), H_q, _p(page_table), page_table.shape[1],
+    a = _Args("full_entmax_decode")
+    B, H_q = _query(a, pool, q)
+    max_pages = _table(a, page_table, seq_lens, B)
+    _outputs(a, pool, out, tau_out, v_pages, status, B, H_q)
+    a.need(workspace, "workspace")
+    a.reachable()
+    _check(lib().entmaxkv_full_entmax_decode(pool.c, _p(q), H_q, _p(page_table), max_pages,
                                              _p(seq_lens), B, alpha, scale, _p(out), _p(tau_out), _p(v_pages),
-                                             _p(workspace), workspace.numel() * workspace.element_size(),
-                                             _p(status), _stream(stream)), "full_entmax_decode")
+                                             _p(workspace), _bytes(workspace), _p(status), _stream(stream)),
+           a.where)
 
 
 def full_softmax_decode(pool, q, page_table, seq_lens, scale, out, workspace, status, stream=None):
-    B, H_q, _ = q.shape
-    _check(lib().entmaxkv_full_softmax_decode(pool.c, _p(q), H_q, _p(page_table), page_table.shape[1],
+    a = _Args("full_softmax_decode")
+    B, H_q = _query(a, pool, q)
+    max_pages = _table(a, page_table, seq_lens, B)
+    _outputs(a, pool, out, None, None, status, B, H_q)
+    a.need(workspace, "workspace")
+    a.reachable()
+    _check(lib().entmaxkv_full_softmax_decode(pool.c, _p(q), H_q, _p(page_table), max_pages,
                                               _p(seq_lens), B, scale, _p(out), _p(workspace),
-                                              workspace.numel() * workspace.element_size(), _p(status),
-                                              _stream(stream)), "full_softmax_decode")
+                                              _bytes(workspace), _p(status), _stream(stream)), a.where)
 
 
 def sparse_softmax_attend(pool, q, page_table, seq_lens, sel, sel_count, scale, out, workspace, status,
                           stream=None):
     """Softmax attention over the listed pages (workspace: OP_SPARSE_SOFTMAX)."""
-    B, H_q, _ = q.shape
-    _check(lib().entmaxkv_sparse_softmax_attend(pool.c, _p(q), H_q, _p(page_table), page_table.shape[1],
-                                                _p(seq_lens), B, _p(sel), _p(sel_count), sel.shape[2], scale,
-                                                _p(out), _p(workspace), workspace.numel() * workspace.element_size(),
-                                                _p(status), _stream(stream)), "sparse_softmax_attend")
+    a = _Args("sparse_softmax_attend")
+    B, H_q = _query(a, pool, q)
+    max_pages = _table(a, page_table, seq_lens, B)
+    k_max = _page_list(a, pool, sel, sel_count, B)
+    _outputs(a, pool, out, None, None, status, B, H_q)
+    a.need(workspace, "workspace")
+    a.reachable()
+    _check(lib().entmaxkv_sparse_softmax_attend(pool.c, _p(q), H_q, _p(page_table), max_pages,
+                                                _p(seq_lens), B, _p(sel), _p(sel_count), k_max, scale,
+                                                _p(out), _p(workspace), _bytes(workspace),
+                                                _p(status), _stream(stream)), a.where)
 
 
 def selftest_timeout(limit_ns, status, stream=None):
-    _check(lib().entmaxkv_selftest_timeout(int(limit_ns), _p(status), _stream(stream)), "selftest_timeout")
+    a = _Args("selftest_timeout")
+    a.need(status, "status", I32, 1)
+    a.reachable()
+    _check(lib().entmaxkv_selftest_timeout(int(limit_ns), _p(status), _stream(stream)), a.where)
