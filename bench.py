@@ -62,15 +62,19 @@ def hbm_peak():
 
 
 # ---------------------------------------------------------------- distributed
-def dist_init(n):
+def dist_init(n, backend="nccl"):
+    """One process per GPU under torchrun.  The native arm reduces its timings
+    over NCCL; the reference arm (host cores only) needs no GPU and uses gloo."""
+    import datetime
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
-    if world > 1:
-        import datetime
+    timeout = datetime.timedelta(seconds=120)
+    if world > 1 and backend == "nccl":
         torch.cuda.set_device(local)
-        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                             device_id=torch.device("cuda", local))
+        torch.distributed.init_process_group("nccl", timeout=timeout, device_id=torch.device("cuda", local))
+    elif world > 1:
+        torch.distributed.init_process_group(backend, timeout=timeout)
     elif torch.cuda.is_available():
         torch.cuda.set_device(0)
     return rank, world, local
@@ -150,6 +154,13 @@ def make_workload(context, rank, device="cuda", appends=256):
     cfg = workloads.config(4)
     cfg = dataclasses.replace(cfg, lengths=[context], seed=cfg.seed + 100 * rank, decode_steps=appends)
     return workloads.Workload(cfg, device=device)
+
+
+def workload_name(context):
+    """The bench workload, named the same way by both arms."""
+    head = "million-token decode" if context == 1 << 20 else "decode at %d tokens" % context
+    return ("%s: B=1 x %d tokens per GPU, 32/8 heads, d=128, page 64, bf16 KV, alpha=1.5, top-k 1/64 of pages, "
+            "append 1 token per step" % (head, context))
 
 
 def algorithmic_bytes(cfg, k_pages, v_pages, mode):
@@ -291,8 +302,7 @@ def run_native(args, rank, world, local):
         "dtype": "bf16",
         "data": "synthetic (seeded clustered-page keys, planted tokens; no dataset)",
         "config": {
-            "workload": "million-token decode: B=1 x 2^20 tokens per GPU, 32/8 heads, d=128, page 64, bf16 KV, "
-                        "alpha=1.5, top-k 1/64 of pages (256), append 1 token per step",
+            "workload": workload_name(cfg.lengths[0]),
             "global_batch": world,
             "seq_len": cfg.lengths[0],
             "parallelism": "replicas: one independent sequence per GPU" if world > 1 else "single GPU",
@@ -497,12 +507,12 @@ def run_reference(args, rank, world):
         oracle_sample(wl, 0, 1 / 64, meta, keys, vals)
     per = (time.perf_counter() - t0) / args.steps * cfg.H_kv * 1e6
     sample = ("kv head 0 of 8 per step (replica bounds over all pages, top-k, float64 entmax attention over "
-              "the kept pages), scaled x8")
+              "the kept pages; page metadata built before timing, no token appended), scaled x8")
     line = {"metric": METRIC, "value": round(per, 1), "unit": "us/step", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": round(per / 1e3, 3), "higher_is_better": False,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": "million-token decode: B=1 x 2^20 tokens, 32/8 heads, d=128, page 64, "
-                                   "alpha=1.5, top-k 1/64", "seq_len": cfg.lengths[0]},
+            "config": {"workload": workload_name(cfg.lengths[0]),
+                       "seq_len": cfg.lengths[0]},
             "impl": "reference",
             "cpu_baseline": {"value": round(per, 1), "unit": "us/step", "cores": 1, "kind": "oracle",
                              "sample": sample},
@@ -537,7 +547,7 @@ def main():
         torch.cuda.set_device(0)
         replay_only(args)
         return
-    rank, world, local = dist_init(args.gpus)
+    rank, world, local = dist_init(args.gpus, "gloo" if args.impl == "reference" else "nccl")
     try:
         if args.impl == "reference":
             run_reference(args, rank, world)

@@ -1,0 +1,84 @@
+"""bench.py's host side on the CPU: the reference arm's JSON line (alone and
+under torchrun with two gloo ranks, where rank 0 alone prints), the workload
+name both arms share, and the algorithmic byte count of a step against a
+count by hand."""
+import json
+import os
+import socket
+import subprocess
+import sys
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+import bench  # noqa: E402
+
+KEYS = {"metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better", "scaling",
+        "vs_baseline", "dtype", "data", "config", "impl", "cpu_baseline", "e2e"}
+
+
+def _port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _check_reference_line(line, n):
+    d = json.loads(line)
+    assert KEYS <= set(d)
+    assert d["impl"] == "reference" and d["n_gpus"] == n and d["higher_is_better"] is False
+    assert d["metric"] == bench.METRIC and d["unit"] == "us/step" and d["value"] > 0
+    assert d["config"]["workload"] == bench.workload_name(65536)
+    cb = d["cpu_baseline"]
+    assert cb["kind"] == "oracle" and cb["cores"] == 1 and cb["value"] == d["value"] and cb["sample"]
+    assert d["e2e"] == {"value": d["value"], "unit": "us/step", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
+
+
+ARGS = ["bench.py", "--impl", "reference", "--steps", "1", "--warmup", "1", "--context", "65536"]
+
+
+def test_reference_arm_one_process():
+    env = dict(os.environ, CUDA_VISIBLE_DEVICES="")
+    r = subprocess.run([sys.executable] + ARGS, cwd=ROOT, env=env, capture_output=True, text=True, timeout=300)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [l for l in r.stdout.splitlines() if l.startswith("{")]
+    assert len(lines) == 1
+    _check_reference_line(lines[0], 1)
+
+
+def test_reference_arm_two_ranks_rank0_prints_once():
+    env = dict(os.environ, CUDA_VISIBLE_DEVICES="")
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", "--nproc-per-node", "2",
+           "--master-addr", "127.0.0.1", "--master-port", str(_port())] + ARGS + ["--gpus", "2"]
+    r = subprocess.run(cmd, cwd=ROOT, env=env, capture_output=True, text=True, timeout=300)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [l for l in r.stdout.splitlines() if l.startswith("{")]
+    assert len(lines) == 1
+    _check_reference_line(lines[0], 2)
+
+
+def test_workload_names():
+    assert bench.workload_name(1 << 20).startswith("million-token decode: B=1 x 1048576 tokens per GPU")
+    assert bench.workload_name(65536).startswith("decode at 65536 tokens: B=1 x 65536 tokens")
+
+
+def test_algorithmic_bytes_by_hand():
+    """The million-token step after one appended token: 16385 pages per kv head,
+    257 pages kept per kv head (2056 page-heads), 278 of them holding weight."""
+    import dataclasses
+    from sparse_long_context_min_b200 import workloads
+    cfg = dataclasses.replace(workloads.config(4), lengths=[(1 << 20) + 1])
+    by = bench.algorithmic_bytes(cfg, 2056, 278, "topk")
+    P = 16385
+    kmin_kmax = P * 8 * 128 * 2 * 2              # bf16 k_min and k_max of every (page, kv head)
+    bounds = 8 * P * 4                           # fp32 bound per (kv head, page), written
+    table = P * 4
+    keys = 2056 * 64 * 128 * 2                   # K of the kept page-heads
+    values = 278 * 64 * 128 * 2                  # V of the page-heads holding weight
+    append = 8 * 128 * 2 * 2 + 8 * 128 * 2 * (2 * 2 + 2 * 4)   # token K, V; metadata row read + write
+    out = 32 * 128 * 4
+    assert by["score"] == kmin_kmax + bounds + table
+    assert by["attend"] == keys + values
+    assert by["total"] == kmin_kmax + bounds + table + keys + values + append + out
+    assert abs(by["total"] / 1e6 - 105.99) < 0.01
+    g = bench.algorithmic_bytes(cfg, 0, 0, "gauss")
+    assert g["score"] == P * 8 * 128 * 2 * 4 + 3 * 32 * P * 4 + table    # mean, m2 read; m, v, est written
