@@ -189,6 +189,11 @@ ENTMAXKV_API int entmaxkv_select(int32_t mode, const float* ub, const float* m, 
  *   For every query head h of kv head g: x_i = (alpha-1) * scale * q_h . k_i
  *   over the valid tokens of pages sel[b][g][0 .. sel_count[b][g]), tau solved
  *   so that sum_i [x_i - tau]_+^(1/(alpha-1)) = 1, out[b][h] = sum_i p_i v_i.
+ *   sel [B][H_kv][k_max] int32 holds distinct logical page ids in [0, pages
+ *   of sequence b), in any order (entmaxkv_select emits them ascending); a
+ *   page listed twice counts twice.  sel_count [B][H_kv] int32 in
+ *   [0, k_max].  An entry or count out of range is skipped (count clamped)
+ *   and reported as ENTMAXKV_DEVICE_BOUNDS.
  *   out [B][H_q][d] fp32; tau_out [B][H_q] fp32 (may be NULL).  A head with
  *   no valid token gets out = 0 and tau = +INFINITY.
  *   Value rows are loaded only for pages holding a token with p > 0 for some
