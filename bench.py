@@ -96,53 +96,102 @@ def max_over_ranks(x, world, device="cuda"):
 
 # ---------------------------------------------------------------- clocks
 class Clocks:
-    """nvidia-smi samples of SM clock and throttle reasons while running."""
+    """nvidia-smi samples of SM clock and throttle reasons during a timed region.
 
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+    The sampler starts `lead_s` before the region (nvidia-smi takes a moment to
+    come up) and each sample carries nvidia-smi's own timestamp, so the summary
+    keeps the samples taken between entering and leaving the region (all of
+    them if the clocks of the two cannot be compared).  The GPU is named by its
+    PCI address, which nvidia-smi and CUDA agree on whatever device indices a
+    process sees; the CUDA index is the fallback."""
+
+    FIELDS = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    REASONS = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+    TS_FORMAT = "%Y/%m/%d %H:%M:%S.%f"
 
-    def __init__(self, device_index):
+    def __init__(self, device_index, interval_ms=50, lead_s=0.5, smi="nvidia-smi"):
         self.dev = device_index
+        self.interval_ms = interval_ms
+        self.lead_s = lead_s
+        self.smi = smi
         self.proc = None
+        self.lines = []
+        self.t0 = self.t1 = None
+
+    def target(self):
+        """nvidia-smi's -i argument for CUDA device `dev`."""
+        try:
+            p = torch.cuda.get_device_properties(self.dev)
+            pci = "%08X:%02X:%02X.0" % (p.pci_domain_id, p.pci_bus_id, p.pci_device_id)
+            r = subprocess.run([self.smi, "-i", pci, "--query-gpu=index", "--format=csv,noheader"],
+                               capture_output=True, text=True, timeout=20)
+            if r.returncode == 0 and r.stdout.strip():
+                return pci
+        except Exception:
+            pass
+        return str(self.dev)
 
     def __enter__(self):
+        import datetime
         try:
             self.proc = subprocess.Popen(
-                ["nvidia-smi", "-i", str(self.dev), "--query-gpu=" + self.FIELDS, "--format=csv,noheader,nounits",
-                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+                [self.smi, "-i", self.target(), "--query-gpu=" + self.FIELDS, "--format=csv,noheader,nounits",
+                 "-lms", str(self.interval_ms)], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            time.sleep(self.lead_s)
         except Exception:
             self.proc = None
+        self.t0 = datetime.datetime.now()
         return self
 
     def __exit__(self, *a):
+        import datetime
+        import signal
+        self.t1 = datetime.datetime.now()
         self.lines = []
         if self.proc is not None:
-            self.proc.terminate()
+            time.sleep(self.interval_ms / 1000.0)          # one more sample after the region
+            out = ""
             try:
+                self.proc.send_signal(signal.SIGINT)       # nvidia-smi's own way to end a loop
                 out, _ = self.proc.communicate(timeout=5)
             except Exception:
                 self.proc.kill()
-                out = ""
-            self.lines = [l for l in out.splitlines() if l.strip()]
+                try:
+                    out, _ = self.proc.communicate(timeout=5)
+                except Exception:
+                    out = ""
+            self.lines = [l for l in (out or "").splitlines() if l.strip()]
 
     def summary(self):
-        sm, mx, reasons = [], None, set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for l in getattr(self, "lines", []):
+        import datetime
+        rows = []
+        for l in self.lines:
             f = [x.strip() for x in l.split(",")]
-            if len(f) < 9:
+            if len(f) < 10:
                 continue
             try:
-                sm.append(float(f[1]))
-                mx = float(f[2])
+                sm, mx = float(f[2]), float(f[3])
             except ValueError:
                 continue
-            for name, val in zip(names, f[5:9]):
-                if val.lower() == "active":
-                    reasons.add(name)
-        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx,
-                "reasons": sorted(reasons), "samples": len(sm)}
+            try:
+                ts = datetime.datetime.strptime(f[0], self.TS_FORMAT)
+            except ValueError:
+                ts = None
+            rows.append((ts, sm, mx, [n for n, v in zip(self.REASONS, f[6:10]) if v.lower() == "active"]))
+        window = "timed region"
+        stamped = [r for r in rows if r[0] is not None and self.t0 is not None]
+        inside = [r for r in stamped if self.t0 <= r[0] <= self.t1]
+        if not inside and stamped:
+            gap = lambda r: (self.t0 - r[0]) if r[0] < self.t0 else (r[0] - self.t1)
+            inside, window = [min(stamped, key=gap)], "nearest sample (the region was shorter than the interval)"
+        elif not inside:
+            inside, window = rows, ("all samples (timestamps not readable)" if rows else "no samples")
+        reasons = sorted({n for r in inside for n in r[3]})
+        return {"sm_mhz": statistics.median(r[1] for r in inside) if inside else None,
+                "sm_max_mhz": inside[-1][2] if inside else None, "reasons": reasons,
+                "samples": len(inside), "window": window}
 
 
 # ---------------------------------------------------------------- workload

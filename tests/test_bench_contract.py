@@ -82,3 +82,73 @@ def test_algorithmic_bytes_by_hand():
     assert abs(by["total"] / 1e6 - 105.99) < 0.01
     g = bench.algorithmic_bytes(cfg, 0, 0, "gauss")
     assert g["score"] == P * 8 * 128 * 2 * 4 + 3 * 32 * P * 4 + table    # mean, m2 read; m, v, est written
+
+
+FAKE_SMI = r'''#!{python}
+"""Stand-in for nvidia-smi: answers the one-shot index query, and in loop
+mode prints one CSV sample per interval until SIGINT."""
+import datetime, signal, sys, time
+args = sys.argv[1:]
+target = args[args.index("-i") + 1]
+if target not in ("0", "0000ABCD:3B:00.0"):
+    sys.exit(6)
+if "--query-gpu=index" in args:
+    print("0")
+    sys.exit(0)
+ms = int(args[args.index("-lms") + 1])
+stop = []
+signal.signal(signal.SIGINT, lambda *a: stop.append(1))
+i = 0
+while not stop:
+    ts = datetime.datetime.now().strftime("%Y/%m/%d %H:%M:%S.%f")[:-3]
+    slow = "Active" if {slow_from} <= i else "Not Active"
+    print("%s, 0, %d, 1965, 700.0, 0x0, %s, Not Active, Not Active, Not Active" % (ts, 1965 - i, slow), flush=True)
+    i += 1
+    time.sleep(ms / 1000.0)
+'''
+
+
+def _fake_smi(tmp_path, slow_from=10 ** 9):
+    p = tmp_path / "nvidia-smi"
+    p.write_text(FAKE_SMI.replace("{python}", sys.executable).replace("{slow_from}", str(slow_from)))
+    p.chmod(0o755)
+    return str(p)
+
+
+def test_clock_sampler_keeps_the_timed_region(tmp_path):
+    import time
+    c = bench.Clocks(0, interval_ms=20, lead_s=0.3, smi=_fake_smi(tmp_path))
+    with c:
+        time.sleep(0.3)
+    s = c.summary()
+    assert s["window"] == "timed region"
+    assert 5 <= s["samples"] <= 25          # ~15 samples inside, none of the lead-in
+    assert s["sm_max_mhz"] == 1965 and s["reasons"] == []
+    assert s["sm_mhz"] < 1965 - 10          # the lead-in samples (highest clocks) were dropped
+    assert len(c.lines) > s["samples"]
+
+
+def test_clock_sampler_reports_slowdown_and_short_regions(tmp_path):
+    c = bench.Clocks(0, interval_ms=20, lead_s=0.3, smi=_fake_smi(tmp_path, slow_from=0))
+    with c:
+        pass                                 # shorter than one interval
+    s = c.summary()
+    assert s["samples"] == 1 and s["window"].startswith("nearest sample")
+    assert s["reasons"] == ["hw_slowdown"]
+
+
+def test_clock_sampler_targets_the_pci_address(tmp_path, monkeypatch):
+    import types
+    props = types.SimpleNamespace(pci_domain_id=0xABCD, pci_bus_id=0x3B, pci_device_id=0)
+    monkeypatch.setattr(bench.torch.cuda, "get_device_properties", lambda i: props)
+    assert bench.Clocks(0, smi=_fake_smi(tmp_path)).target() == "0000ABCD:3B:00.0"
+    props.pci_bus_id = 0x3C                   # unknown to nvidia-smi: fall back to the index
+    assert bench.Clocks(0, smi=_fake_smi(tmp_path)).target() == "0"
+
+
+def test_clock_sampler_without_nvidia_smi():
+    c = bench.Clocks(0, smi="/nonexistent/nvidia-smi")
+    with c:
+        pass
+    s = c.summary()
+    assert s["samples"] == 0 and s["sm_mhz"] is None and s["window"] == "no samples"
