@@ -301,6 +301,8 @@ def run_native(args, rank, world, local):
     barrier(world)
     mean_us = statistics.mean(step_us)
     mean_us_all = max_over_ranks(mean_us, world)
+    best_us_all = max_over_ranks(min(step_us), world)
+    median_us_all = max_over_ranks(statistics.median(step_us), world)
     score_us = max_over_ranks(stage["score"], world)
     by = algorithmic_bytes(cfg, sel_total, v_total, "topk")
     peak, peak_kind = hbm_peak()
@@ -362,6 +364,8 @@ def run_native(args, rank, world, local):
             "achieved_gbs_step": round(step_gbs, 1),
             "frac_of_8tbs": round(step_gbs / HBM_NOMINAL_GBS, 4),
             "frac_of_measured_hbm": round(step_gbs / peak, 4),
+            "step_us_best": round(best_us_all, 2),
+            "step_us_median": round(median_us_all, 2),
             "stage_us": {k: round(v, 2) for k, v in stage.items()},
             "stage_note": "stage_us from a graph with event nodes between stages (no overlap across them)",
             **extra,
