@@ -4,7 +4,10 @@
   and against Monte-Carlo (10^6 draws, 4-sigma bound), and against the worked
   examples in tests/golden;
 * with one token per page and zero spread, F is the exact entmax mass, so
-  tau_hat must equal the exact entmax threshold of c1;
+  tau_hat must equal the exact entmax threshold of c1; with n equal tokens
+  per page it is the threshold of the multiset repeating each page n times;
+* F against a Monte-Carlo over the token scores in score space, which fixes
+  the map (m, v) -> ((alpha-1) m, (alpha-1) sqrt(v)) of the entmax input;
 * F is strictly decreasing and F(tau_hat) = 1;
 * the z table against sqrt(2 ln n).
 """
@@ -106,3 +109,41 @@ def test_est_max_single_token_equals_mean():
     m = np.array([[0.3, -1.2]])
     v = np.array([[0.0, 0.0]])
     np.testing.assert_array_equal(gauss.est_max(m, v, np.array([[1, 1]]), 64), m)
+
+
+@pytest.mark.parametrize("alpha", [1.5, 2.0, 3.0])
+def test_pages_of_equal_tokens_reduce_to_exact_entmax_of_the_multiset(alpha):
+    """A page whose n tokens share one score (zero spread) weighs that score n
+    times: tau_hat equals the exact entmax threshold of the multiset in which
+    every page's score is repeated n_p times (pins the n_p weighting)."""
+    rng = np.random.default_rng(24)
+    s = rng.standard_normal(40)
+    n = rng.integers(1, 65, 40)
+    tau = gauss.tau_hat(s, np.zeros(40), n, alpha)
+    exact = entmax.tau_bisect((alpha - 1.0) * np.repeat(s, n), alpha)
+    assert abs(tau - exact) < 1e-10
+    # and it differs from the one-token-per-page threshold whenever n is not all ones
+    assert abs(tau - entmax.tau_bisect((alpha - 1.0) * s, alpha)) > 1e-3
+
+
+@pytest.mark.parametrize("alpha", [1.5, 2.0, 3.0])
+def test_F_is_the_expected_mass_of_the_page_draws(alpha):
+    """F(tau) = sum_p n_p E[((alpha-1) s - tau)_+^(1/(alpha-1))] with s ~ N(m_p, v_p)
+    in score space: Monte-Carlo over the token scores themselves (pins the map
+    from a page's score mean and variance to the entmax input's, (alpha-1) m and
+    (alpha-1) sqrt(v))."""
+    rng = np.random.default_rng(25)
+    P = 6
+    m = rng.uniform(-0.5, 2.0, P)
+    v = rng.uniform(0.05, 0.8, P)
+    n = rng.integers(1, 65, P)
+    r = 1.0 / (alpha - 1.0)
+    draws = 400_000
+    for tau in (0.2, 0.6):
+        est, var = 0.0, 0.0
+        for p in range(P):
+            x = (alpha - 1.0) * (m[p] + math.sqrt(v[p]) * rng.standard_normal(draws))
+            y = n[p] * np.maximum(x - tau, 0.0) ** r
+            est += y.mean()
+            var += y.var() / draws
+        assert abs(gauss.F(tau, m, v, n, alpha) - est) < 4.5 * math.sqrt(var)
