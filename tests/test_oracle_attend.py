@@ -7,7 +7,8 @@
 * o equals P @ V computed by a matrix product (a different summation order);
 * softmax baseline: equal scores give the mean value vector; a dominating
   score gives that token's value;
-* two tokens at alpha = 2 follow the textbook sparsemax closed form;
+* two tokens at alpha = 2 follow the textbook sparsemax closed form, and at
+  alpha = 1.5 the quadratic solved by hand on x = (alpha - 1) scale q.k;
 * softmax over a kept subset equals the full softmax weights restricted to
   the subset and renormalised, and obeys the same 2 B delta bound with a
   positive delta whenever a token is dropped (section 3);
@@ -113,3 +114,21 @@ def test_subset_softmax_is_the_renormalised_restriction():
         assert np.all(delta > 0)
         err = np.linalg.norm(o_sub - o_full, axis=1)
         assert np.all(err <= 2 * B * delta + 1e-12)
+
+
+def test_two_token_entmax_15_closed_form():
+    """alpha = 1.5 over two tokens, solved by hand on x = (alpha - 1) * scale * q.k:
+    both tokens carry weight iff |x1 - x2| < 1, and then (x1 - tau)^2 + (x2 - tau)^2 = 1
+    gives tau = ((x1 + x2) - sqrt(2 - (x1 - x2)^2)) / 2 and p_i = (x_i - tau)^2.
+    Pins the (alpha - 1) factor of the entmax input (alpha = 2 cannot)."""
+    V = np.array([[1.0, 0.0], [0.0, 1.0]])
+    q = np.array([[1.0]])
+    for s1, s2, scale in [(1.0, 0.0, 1.0), (0.3, 1.1, 1.0), (2.5, 0.0, 1.0), (4.0, 1.0, 0.5), (0.0, 0.0, 1.0)]:
+        x1, x2 = 0.5 * scale * s1, 0.5 * scale * s2
+        if abs(x1 - x2) < 1.0:
+            tau = ((x1 + x2) - np.sqrt(2.0 - (x1 - x2) ** 2)) / 2.0
+            p = [(x1 - tau) ** 2, (x2 - tau) ** 2]
+        else:
+            p = [1.0, 0.0] if x1 > x2 else [0.0, 1.0]
+        o, _, _ = attend.entmax_attention(q, np.array([[s1], [s2]]), V, 1.5, scale)
+        np.testing.assert_allclose(o[0], p, atol=1e-13)
