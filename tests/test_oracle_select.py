@@ -80,3 +80,18 @@ def test_gauss_keep_bands():
     keep, drop = select.gauss_keep_bands(est, np.array([1.0]), 1.5, 0.0, 0.1)
     # margins 0.5*est - 1 = -0.5, 0, 0.5
     assert list(keep) == [2] and list(drop) == [0]
+
+
+def test_gauss_keep_threshold_is_inclusive_and_a_union_over_the_group():
+    """A page is kept when (alpha-1) est reaches tau_hat - Delta (equality
+    included, decided in fp32), and for a kv head when any query head of its
+    group keeps it."""
+    f = np.float32
+    at = f(0.75)
+    est = np.array([[at, np.nextafter(at, f(-1)), np.nextafter(at, f(2))]], dtype=np.float32)
+    assert list(select.gauss_keep(est, np.array([f(1.0)]), 2.0, 0.25)) == [0, 2]
+    est2 = np.array([[1.0, -3.0, -3.0, -3.0],
+                     [-3.0, -3.0, 1.0, -3.0]], dtype=np.float32)
+    tau = np.array([f(0.2), f(0.2)])
+    assert list(select.gauss_keep(est2, tau, 1.5, 0.0)) == [0, 2]
+    assert list(select.gauss_keep(est2[:1], tau[:1], 1.5, 0.0)) == [0]
