@@ -15,7 +15,7 @@ import os
 import numpy as np
 import pytest
 
-from oracle import pages, replica
+from oracle import gauss, pages, replica
 
 GOLD = json.load(open(os.path.join(os.path.dirname(__file__), "golden", "worked_examples.json")))
 
@@ -176,3 +176,37 @@ def test_replica_gauss_against_f64(ps, d):
     # pages with one token have zero spread: the estimate is the mean score
     one = np.nonzero(r["count"] == 1)[0]
     assert one.size == 0 or np.array_equal(est[:, one], m[:, one])
+
+
+def test_gauss_scores_are_the_score_moments_when_keys_vary_in_one_coordinate():
+    """With keys that differ in a single coordinate the diagonal model is
+    exact: m and v must equal the mean and population variance of the true
+    scores scale * q.k over the page (pins scale^2 and q^2 in v)."""
+    rng = np.random.default_rng(17)
+    d, n, scale = 16, 23, 0.37
+    for j in (0, 5, 15):
+        c = rng.standard_normal(d)
+        keys = np.tile(c, (n, 1))
+        keys[:, j] += 2.0 * rng.standard_normal(n)
+        q = rng.standard_normal((3, d))
+        meta = pages.page_metadata(keys, n)
+        m, v = pages.gauss_scores(q, meta["mean"], meta["var"], scale)
+        s = scale * (keys @ q.T)                       # [n, heads]
+        np.testing.assert_allclose(m[:, 0], s.mean(axis=0), rtol=1e-12, atol=1e-12)
+        np.testing.assert_allclose(v[:, 0], s.var(axis=0), rtol=1e-10, atol=1e-12)
+
+
+def test_estimated_page_maximum_scales_with_the_spread():
+    """est_max - m is proportional to the standard deviation sqrt(v) (scaling
+    the scores by c scales it by c), zero for one token, and positive and
+    increasing in the page's token count from two tokens on."""
+    m = np.array([0.4, -1.0, 2.0])
+    v = np.array([0.09, 0.25, 1.0])
+    for n in (2, 3, 17, 64):
+        nn = np.full(3, n)
+        e1 = gauss.est_max(m, v, nn, 64) - m
+        e4 = gauss.est_max(3.0 * m, 9.0 * v, nn, 64) - 3.0 * m
+        np.testing.assert_allclose(e4, 3.0 * e1, rtol=1e-12)
+        assert np.all(e1 > 0)
+    grow = [float(gauss.est_max(m[:1], v[:1], np.array([n]), 64)[0]) for n in range(1, 65)]
+    assert grow[0] == m[0] and all(a < b for a, b in zip(grow, grow[1:]))
