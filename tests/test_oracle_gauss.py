@@ -147,3 +147,16 @@ def test_F_is_the_expected_mass_of_the_page_draws(alpha):
             est += y.mean()
             var += y.var() / draws
         assert abs(gauss.F(tau, m, v, n, alpha) - est) < 4.5 * math.sqrt(var)
+
+
+def test_z_bounds_the_expected_maximum_of_n_normals():
+    """z_n = sqrt(2 ln n) is the textbook upper bound on E[max of n independent
+    standard normals] (from E[max] <= ln(n E[exp(t X)]) / t at t = z_n), and
+    not far above it at page sizes: the estimate adds a spread-proportional
+    margin of the right size to the page mean."""
+    rng = np.random.default_rng(26)
+    z = gauss.z_table(64)
+    for n in (4, 16, 64):
+        mx = rng.standard_normal((100_000, n)).max(axis=1)
+        mean, se = mx.mean(), mx.std() / math.sqrt(mx.size)
+        assert mean - 4 * se <= z[n] <= 1.7 * (mean + 4 * se)

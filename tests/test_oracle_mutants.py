@@ -154,6 +154,10 @@ def z_without_root(ps):
     return np.array([0.0, 0.0] + [2.0 * math.log(n) for n in range(2, ps + 1)])
 
 
+def z_half_log(ps):
+    return np.array([0.0, 0.0] + [math.sqrt(math.log(n)) for n in range(2, ps + 1)])
+
+
 def est_with_variance(m, v, n, ps):
     return np.asarray(m, dtype=np.float64) + np.maximum(v, 0.0) * gauss.z_table(ps)[np.asarray(n)]
 
@@ -232,7 +236,10 @@ CASES = [
     ("partial last page dropped", attend, "token_indices", drops_partial_page, TA.test_token_indices_ragged),
     ("delta counts the kept mass", attend, "dropped_mass", kept_mass,
      lambda: TA.test_support_recovery_is_bitwise_exact(1.5)),
-    ("z_n without the square root", gauss, "z_table", z_without_root, TG.test_z_table),
+    ("z_n without the square root", gauss, "z_table", z_without_root,
+     TG.test_z_bounds_the_expected_maximum_of_n_normals),
+    ("z_n = sqrt(ln n)", gauss, "z_table", z_half_log,
+     TG.test_z_bounds_the_expected_maximum_of_n_normals),
     ("page maximum from the variance", gauss, "est_max", est_with_variance,
      TP.test_estimated_page_maximum_scales_with_the_spread),
     ("page maximum with z of n - 1", gauss, "est_max", est_z_off_by_one,
