@@ -13,7 +13,9 @@
  *   the comment says "host".  The attention outputs (out, tau_out) may also be
  *   pinned host memory mapped into the device's address space: the kernels
  *   then store results straight to the host.  The library never allocates or
- *   frees memory and keeps no state between calls.
+ *   frees memory and keeps no state between calls (the built-in scratch of
+ *   entmaxkv_sparse_attend_static and per-device caches of the SM count and
+ *   kernel attributes aside).
  * - Every call is asynchronous on `stream` (a cudaStream_t passed as void*;
  *   NULL is the legacy default stream).  Inputs must stay valid and outputs
  *   untouched until the stream reaches the work.
