@@ -169,7 +169,10 @@ ENTMAXKV_API int entmaxkv_score_pages(const entmaxkv_pool* pool, const float* q,
  *     alpha and delta are ignored.
  *   mode ENTMAXKV_SELECT_GAUSS (policy 2): per query head solve
  *     sum_p n_p E[((alpha-1) s - tau)_+^(1/(alpha-1))] = 1 for tau_hat, s ~
- *     N(m_p, v_p), by bisection in fp32; keep page p for kv head g when
+ *     N(m_p, v_p), by Newton steps on log F kept inside a bracket (bisection
+ *     where a step leaves it; page terms in fp32, sums in float64; it stops
+ *     when |F - 1| < 1e-7, the bracket or the step falls below the terms'
+ *     accuracy, or after 60 steps); keep page p for kv head g when
  *     (alpha-1) * est_max[h][p] >= tau_hat[h] - delta for some h in g.
  *     tau_hat [B][H_q] fp32 is written.  Needs k_max >= max_pages.  ub,
  *     budget and budget_frac are ignored.
