@@ -51,3 +51,51 @@ def test_walk_centres_and_short_sequences():
     k0, _ = wl.sequence(0)
     k1, _ = wl.sequence(1)
     assert k0.shape == (8, 0, 128) and k1.shape == (8, 300, 128)
+
+
+def _page_stats(keys, ps, planted_pos):
+    """Page means and within-page deviations of one kv head's keys, planted tokens left out."""
+    k = keys.float()
+    L = k.shape[0]
+    P = L // ps
+    mask = torch.ones(L, dtype=torch.bool)
+    mask[list(planted_pos)] = False
+    means, dev = [], []
+    for p in range(P):
+        blk = k[p * ps:(p + 1) * ps][mask[p * ps:(p + 1) * ps]]
+        mu = blk.mean(0)
+        means.append(mu)
+        dev.append(blk - mu)
+    return torch.stack(means), torch.cat(dev)
+
+
+def test_clustered_keys_follow_the_recipe():
+    """Centres N(0, I) per (page, kv head), tokens centre + 0.3 N(0, I)."""
+    import dataclasses
+    cfg = dataclasses.replace(workloads.config(2), lengths=[64 * 200])
+    wl = workloads.Workload(cfg)
+    keys, vals = wl.sequence(0, heads=[0])
+    planted = [p for h in range(cfg.G) for p in wl.planted(0).get(h, [])]
+    means, dev = _page_stats(keys[0], cfg.ps, planted)
+    assert 0.93 < float(means.std()) < 1.07
+    assert 0.29 < float(dev.std()) < 0.31
+    assert abs(float(vals.float().mean())) < 0.01 and 0.98 < float(vals.float().std()) < 1.02
+    assert 0.97 < float(wl.q.std()) < 1.03
+
+
+def test_walk_centres_follow_the_recipe():
+    """c_{p+1} = 0.9 c_p + 0.44 N(0, I): lag-one correlation 0.9 and variance
+    near the stationary 0.44^2 / (1 - 0.81) = 1.02; tokens spread 0.5."""
+    import dataclasses
+    cfg = dataclasses.replace(workloads.config(3), B=1, lengths=[64 * 600])
+    wl = workloads.Workload(cfg)
+    keys, _ = wl.sequence(0, heads=[2])
+    planted = [p for h in range(2 * cfg.G, 3 * cfg.G) for p in wl.planted(0).get(h, [])]
+    means, dev = _page_stats(keys[0], cfg.ps, planted)
+    a, b = means[:-1], means[1:]
+    corr = float(((a - a.mean(0)) * (b - b.mean(0))).mean() / (a.std() * b.std()))
+    assert 0.85 < corr < 0.94
+    assert 0.8 < float(means.var()) < 1.25
+    assert 0.48 < float(dev.std()) < 0.52
+    counts = [len(v) for v in wl.planted(0).values()]
+    assert len(counts) == cfg.H_q and all(16 <= c <= 512 for c in counts)
