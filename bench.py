@@ -234,6 +234,72 @@ def score_bytes(cfg, mode):
     return algorithmic_bytes(cfg, 0, 0, mode)["score"]
 
 
+N_LAUNCH = 6   # per step: append (one token, no separate length kernel), score, top-k, qk, tau, pv
+
+
+def native_line(cfg, world, K, W, mean_us, best_us, median_us, score_us, stage, sel_total, v_total, extra, e2e,
+                clk, cpu, peak):
+    """The native arm's JSON line from the measured numbers (times are the
+    max over ranks; e2e = (us per step, H2D bytes, D2H bytes); peak = (GB/s,
+    "measured" or "fallback"))."""
+    by = algorithmic_bytes(cfg, sel_total, v_total, "topk")
+    peak_gbs, peak_kind = peak
+    e2e_us, h2d, d2h = e2e
+    step_gbs = by["total"] / (mean_us * 1e-6) / 1e9
+    score_gbs = by["score"] / (score_us * 1e-6) / 1e9
+    line = {
+        "metric": METRIC,
+        "value": round(mean_us, 2),
+        "unit": "us/step",
+        "n_gpus": world,
+        "steps": K,
+        "warmup": W,
+        "ms_per_step": round(mean_us / 1e3, 5),
+        "higher_is_better": False,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic (seeded clustered-page keys, planted tokens; no dataset)",
+        "config": {
+            "workload": workload_name(cfg.lengths[0]),
+            "global_batch": world,
+            "seq_len": cfg.lengths[0],
+            "parallelism": "replicas: one independent sequence per GPU" if world > 1 else "single GPU",
+            "l2": "flushed between steps (256 MiB write outside the step events)",
+            "selected_pages_per_step": round(sel_total, 1),
+            "value_pages_loaded_per_step": round(v_total, 1),
+            "algorithmic_bytes_per_step": by["total"],
+            "achieved_gbs_step": round(step_gbs, 1),
+            "frac_of_8tbs": round(step_gbs / HBM_NOMINAL_GBS, 4),
+            "frac_of_measured_hbm": round(step_gbs / peak_gbs, 4),
+            "step_us_best": round(best_us, 2),
+            "step_us_median": round(median_us, 2),
+            "stage_us": {k: round(v, 2) for k, v in stage.items()},
+            "stage_note": "stage_us from a graph with event nodes between stages (no overlap across them)",
+            **extra,
+        },
+        "roofline": {
+            "kernel": "score_box16_kernel (entmaxkv_score_pages, bbox, bf16)",
+            "bound": "hbm",
+            "achieved": round(score_gbs, 1),
+            "peak": peak_gbs,
+            "peak_kind": peak_kind,
+            "unit": "GB/s",
+            "frac": round(score_gbs / peak_gbs, 4),
+            "traffic": round(SCORE_DRAM_BYTES_PER_ROW * sum(cfg.pages(b) for b in range(cfg.B)) * cfg.H_kv),
+            "traffic_note": "ncu dram__bytes_read+write of the 2^18-token case scaled by rows",
+            "bytes_per_launch": by["score"],
+        },
+        "e2e": {"value": round(e2e_us, 2), "unit": "us/step", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h},
+        "gpu_launches": N_LAUNCH * K,
+        "clocks": clk,
+    }
+    if cpu is not None:
+        line["cpu_baseline"] = cpu
+    return line
+
+
 # ---------------------------------------------------------------- native arm
 def run_native(args, rank, world, local):
     import numpy as np
@@ -304,8 +370,6 @@ def run_native(args, rank, world, local):
     best_us_all = max_over_ranks(min(step_us), world)
     median_us_all = max_over_ranks(statistics.median(step_us), world)
     score_us = max_over_ranks(stage["score"], world)
-    by = algorithmic_bytes(cfg, sel_total, v_total, "topk")
-    peak, peak_kind = hbm_peak()
 
     # ---- e2e through the C ABI with host buffers (copies inside the timed region)
     e2e_us, h2d, d2h = run_e2e(wl, pool, seq_lens, K, W, flush)
@@ -335,60 +399,8 @@ def run_native(args, rank, world, local):
     if rank == 0 and not args.no_cpu:
         cpu = cpu_baseline(wl, pool, budget_frac=1 / 64, seconds=8.0)
 
-    n_launch = 6   # append (one token: no separate length kernel), score, top-k, qk + tau + pv per replay
-    step_gbs = by["total"] / (mean_us_all * 1e-6) / 1e9
-    score_gbs = by["score"] / (score_us * 1e-6) / 1e9
-    clk = clocks.summary()
-    line = {
-        "metric": METRIC,
-        "value": round(mean_us_all, 2),
-        "unit": "us/step",
-        "n_gpus": world,
-        "steps": K,
-        "warmup": W,
-        "ms_per_step": round(mean_us_all / 1e3, 5),
-        "higher_is_better": False,
-        "scaling": "weak",
-        "vs_baseline": None,
-        "dtype": "bf16",
-        "data": "synthetic (seeded clustered-page keys, planted tokens; no dataset)",
-        "config": {
-            "workload": workload_name(cfg.lengths[0]),
-            "global_batch": world,
-            "seq_len": cfg.lengths[0],
-            "parallelism": "replicas: one independent sequence per GPU" if world > 1 else "single GPU",
-            "l2": "flushed between steps (256 MiB write outside the step events)",
-            "selected_pages_per_step": round(sel_total, 1),
-            "value_pages_loaded_per_step": round(v_total, 1),
-            "algorithmic_bytes_per_step": by["total"],
-            "achieved_gbs_step": round(step_gbs, 1),
-            "frac_of_8tbs": round(step_gbs / HBM_NOMINAL_GBS, 4),
-            "frac_of_measured_hbm": round(step_gbs / peak, 4),
-            "step_us_best": round(best_us_all, 2),
-            "step_us_median": round(median_us_all, 2),
-            "stage_us": {k: round(v, 2) for k, v in stage.items()},
-            "stage_note": "stage_us from a graph with event nodes between stages (no overlap across them)",
-            **extra,
-        },
-        "roofline": {
-            "kernel": "score_box16_kernel (entmaxkv_score_pages, bbox, bf16)",
-            "bound": "hbm",
-            "achieved": round(score_gbs, 1),
-            "peak": peak,
-            "peak_kind": peak_kind,
-            "unit": "GB/s",
-            "frac": round(score_gbs / peak, 4),
-            "traffic": round(SCORE_DRAM_BYTES_PER_ROW * sum(cfg.pages(b) for b in range(cfg.B)) * cfg.H_kv),
-            "traffic_note": "ncu dram__bytes_read+write of the 2^18-token case scaled by rows",
-            "bytes_per_launch": by["score"],
-        },
-        "e2e": {"value": round(e2e_us, 2), "unit": "us/step", "h2d_bytes_per_step": h2d,
-                "d2h_bytes_per_step": d2h},
-        "gpu_launches": n_launch * K,
-        "clocks": clk,
-    }
-    if cpu is not None:
-        line["cpu_baseline"] = cpu
+    line = native_line(cfg, world, K, W, mean_us_all, best_us_all, median_us_all, score_us, stage, sel_total,
+                       v_total, extra, (e2e_us, h2d, d2h), clocks.summary(), cpu, hbm_peak())
     if rank == 0:
         print(json.dumps(line), flush=True)
 

@@ -152,3 +152,34 @@ def test_clock_sampler_without_nvidia_smi():
         pass
     s = c.summary()
     assert s["samples"] == 0 and s["sm_mhz"] is None and s["window"] == "no samples"
+
+
+def test_native_line_carries_the_contract():
+    """The native arm's JSON line from measured numbers (those of a B200 run):
+    every key of the contract, the roofline fraction from the algorithmic bytes
+    and the kernel time, and the cpu_baseline when rank 0 timed the oracle."""
+    import dataclasses
+    from sparse_long_context_min_b200 import workloads
+    cfg = dataclasses.replace(workloads.config(4), lengths=[1 << 20])
+    stage = {"append": 9.6, "score": 28.8, "select": 16.4, "attend": 47.3}
+    clk = {"sm_mhz": 1965.0, "sm_max_mhz": 1965.0, "reasons": [], "samples": 12, "window": "timed region"}
+    cpu = {"value": 378791.7, "unit": "us/step", "cores": 1, "kind": "oracle", "sample": "kv head 0"}
+    line = bench.native_line(cfg, 1, 20, 5, 88.19, 86.0, 88.0, 28.78, stage, 2056, 278.2, {"x": 1},
+                             (100.91, 20480, 16384), clk, cpu, (6528.7, "measured"))
+    json.loads(json.dumps(line))
+    assert {"metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better",
+            "scaling", "vs_baseline", "dtype", "data", "config", "roofline", "e2e", "gpu_launches", "clocks",
+            "cpu_baseline"} <= set(line)
+    assert line["value"] == 88.19 and line["higher_is_better"] is False and line["scaling"] == "weak"
+    assert line["gpu_launches"] == 6 * 20 and line["config"]["x"] == 1
+    r = line["roofline"]
+    assert {"bound", "achieved", "peak", "unit", "frac", "traffic"} <= set(r)
+    by = bench.algorithmic_bytes(cfg, 2056, 278.2, "topk")
+    assert abs(r["achieved"] - by["score"] / 28.78e-6 / 1e9) < 0.1
+    assert abs(r["frac"] - r["achieved"] / 6528.7) < 1e-3
+    assert r["traffic"] == round(bench.SCORE_DRAM_BYTES_PER_ROW * 16384 * 8)
+    assert line["e2e"] == {"value": 100.91, "unit": "us/step", "h2d_bytes_per_step": 20480,
+                           "d2h_bytes_per_step": 16384}
+    assert line["config"]["step_us_best"] == 86.0 and line["config"]["workload"] == bench.workload_name(1 << 20)
+    assert "cpu_baseline" not in bench.native_line(cfg, 2, 20, 5, 88.19, 86.0, 88.0, 28.78, stage, 2056, 278.2,
+                                                   {}, (100.91, 20480, 16384), clk, None, (6650.0, "fallback"))
