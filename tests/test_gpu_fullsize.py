@@ -44,18 +44,27 @@ def _oracle_seq(wl, b, toks):
     return keys, vals, toks[-1][2][b].float().cpu().numpy()
 
 
-def _check_topk(wl, st, toks, samples, frac=None, budget=-1):
+def _check_topk(wl, st, toks, samples, frac=None, budget=-1, select_all=False):
+    """Top-k sets against the replica bounds (every kv head of every sequence
+    when select_all, else the sampled ones) and the entmax attention of the
+    sampled (sequence, kv head) pairs against the oracle."""
     cfg = wl.cfg
     G = cfg.G
     sel, cnt, out = st.sel.cpu().numpy(), st.sel_count.cpu().numpy(), st.out.cpu().numpy()
-    for b, g in samples:
-        keys, vals, q = _oracle_seq(wl, b, toks)
+    heads = [(b, g) for b in range(cfg.B) for g in range(cfg.H_kv)] if select_all else list(samples)
+    seqs = {}
+    for b, g in heads:
+        if b not in seqs:
+            seqs[b] = _oracle_seq(wl, b, toks)
+        keys, vals, q = seqs[b]
         L = keys.shape[1]
         meta = replica.page_meta(keys[g], cfg.ps)
         qg = q[g * G:(g + 1) * G]
         _, ubg = replica.bound(qg, meta["kmin"], meta["kmax"], H.scale32(cfg))
         pages = select.topk(ubg, select.budget_pages(len(ubg), budget, frac if frac is not None else 0.0))
         assert np.array_equal(sel[b, g, :cnt[b, g]], pages), (b, g)
+        if (b, g) not in samples:
+            continue
         tok = attend.token_indices(pages, L, cfg.ps)
         o_ref, _, _ = attend.entmax_attention(qg, keys[g][tok], vals[g][tok], cfg.alpha, 1 / math.sqrt(cfg.d))
         H.compare_out(out[b, g * G:(g + 1) * G], o_ref, cfg.dtype)
@@ -73,17 +82,22 @@ def test_config2_llama_budgets(budget):
     wl = workloads.Workload(workloads.config(2), device="cuda")
     pool, seq_lens = build_pool(wl)
     st, toks = _graphed_steps(wl, pool, seq_lens, "topk", 2, budget=budget)
-    _check_topk(wl, st, toks, [(0, 1), (0, 6)], budget=budget)
+    _check_topk(wl, st, toks, [(0, 1), (0, 6)], budget=budget, select_all=True)
 
 
 def test_config4_million_topk():
     wl = workloads.Workload(workloads.config(4), device="cuda")
     pool, seq_lens = build_pool(wl)
     st, toks = _graphed_steps(wl, pool, seq_lens, "topk", 3, budget_frac=1 / 64)
-    _check_topk(wl, st, toks, [(0, 0), (0, 5)], frac=1 / 64)
+    _check_topk(wl, st, toks, [(0, 0), (0, 5)], frac=1 / 64, select_all=True)
 
 
 def _check_gauss(wl, st, toks, samples, alpha, delta):
+    """Gaussian selection of the sampled (sequence, kv head) pairs: tau_hat
+    within its tolerance of the oracle's float64 root, the kept set equal bit
+    for bit to the fp32 keep rule at the GPU's own threshold (decisions against
+    the oracle's threshold may differ only inside the band its error spans),
+    and the attention output against the oracle fed the GPU's kept set."""
     cfg = wl.cfg
     G = cfg.G
     sel, cnt, out = st.sel.cpu().numpy(), st.sel_count.cpu().numpy(), st.out.cpu().numpy()
@@ -96,24 +110,19 @@ def _check_gauss(wl, st, toks, samples, alpha, delta):
         m, v, est = replica.gauss(qg, meta["mean"], meta["m2"], meta["count"], H.scale32(cfg), cfg.ps)
         ref = np.array([gauss.tau_hat(m[h].astype(np.float64), v[h].astype(np.float64), meta["count"], alpha)
                         for h in range(G)])
-        got = tau_gpu[b, g * G:(g + 1) * G].astype(np.float64)
-        assert np.all(np.abs(got - ref) <= H.TAU_HAT_TOL * np.maximum(1.0, np.abs(ref))), (got, ref)
-        band = np.abs(got - ref) + 1e-6 * np.maximum(1.0, np.abs(ref))
-        margin = (alpha - 1.0) * est.astype(np.float64) - (ref[:, None] - delta)
-        must_keep = set(np.nonzero(np.any(margin > band[:, None], axis=0))[0].tolist())
-        must_drop = set(np.nonzero(np.all(margin < -band[:, None], axis=0))[0].tolist())
+        got = tau_gpu[b, g * G:(g + 1) * G]
+        g64 = got.astype(np.float64)
+        assert np.all(np.abs(g64 - ref) <= H.TAU_HAT_TOL * np.maximum(1.0, np.abs(ref))), (got, ref)
         kept = sel[b, g, :cnt[b, g]]
-        assert must_keep <= set(kept.tolist()) and not (must_drop & set(kept.tolist()))
-        # the oracle's own set: the fp32 rule with its float64 threshold
+        assert np.array_equal(kept, select.gauss_keep(est, got, alpha, delta)), (b, g)
+        band = np.abs(g64 - ref) + 1e-6 * np.maximum(1.0, np.abs(ref))
+        must_keep, must_drop = select.gauss_keep_bands(est, ref, alpha, delta, band[:, None])
         own = select.gauss_keep(est, ref.astype(np.float32), alpha, delta)
-        if np.array_equal(own, kept):
-            tok = attend.token_indices(own, L, cfg.ps)
-            o_ref, _, _ = attend.entmax_attention(qg, keys[g][tok], vals[g][tok], alpha, 1 / math.sqrt(cfg.d))
-            H.compare_out(out[b, g * G:(g + 1) * G], o_ref, cfg.dtype)
-        else:
-            # only pages inside the threshold's uncertainty band can differ
-            diff = set(own.tolist()) ^ set(kept.tolist())
-            assert not (diff & (must_keep | must_drop))
+        diff = set(own.tolist()) ^ set(kept.tolist())
+        assert not (diff & (set(must_keep.tolist()) | set(must_drop.tolist())))
+        tok = attend.token_indices(kept, L, cfg.ps)
+        o_ref, _, _ = attend.entmax_attention(qg, keys[g][tok], vals[g][tok], alpha, 1 / math.sqrt(cfg.d))
+        H.compare_out(out[b, g * G:(g + 1) * G], o_ref, cfg.dtype)
 
 
 @pytest.mark.parametrize("alpha", [1.5, 2.0])

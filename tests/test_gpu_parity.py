@@ -255,69 +255,78 @@ def test_score_gauss_bitexact(built):
             assert np.all(e[b, sl, P:] == -np.inf)
 
 
+def _check_gauss_head(o, g, got, alpha, delta, kept, iters=100):
+    """Gaussian selection of one kv head against the oracle.
+
+    got: the GPU's tau_hat of the group's query heads.  tau_hat must lie within
+    its tolerance of the oracle's float64 root; the kept set must equal, bit for
+    bit, the fp32 keep rule evaluated with the GPU's own threshold (the page
+    estimates are bit-equal to the replica's, so only the threshold can differ);
+    against the oracle's threshold, decisions may differ only inside the band the
+    threshold's error spans.  Returns the number of such in-band differences."""
+    G = o.cfg.G
+    m, v, est = o.gauss(g)
+    n = o.meta(g)["count"]
+    ref = np.array([gauss.tau_hat(m[h].astype(np.float64), v[h].astype(np.float64), n, alpha, iters=iters)
+                    for h in range(G)])
+    got = np.asarray(got, dtype=np.float32)
+    g64 = got.astype(np.float64)
+    assert np.all(np.abs(g64 - ref) <= H.TAU_HAT_TOL * np.maximum(1.0, np.abs(ref))), (got, ref)
+    assert np.array_equal(kept, select.gauss_keep(est, got, alpha, delta))
+    band = np.abs(g64 - ref) + 1e-6 * np.maximum(1.0, np.abs(ref))
+    must_keep, must_drop = select.gauss_keep_bands(est, ref, alpha, delta, band[:, None])
+    own = select.gauss_keep(est, ref.astype(np.float32), alpha, delta)
+    diff = set(own.tolist()) ^ set(kept.tolist())
+    assert not (diff & (set(must_keep.tolist()) | set(must_drop.tolist())))
+    return len(diff)
+
+
 @pytest.mark.parametrize("alpha", [1.5, 2.0])
 @pytest.mark.parametrize("delta", [0.0, 0.5])
 def test_gauss_selection(alpha, delta):
+    """Config-3 keys (random-walk pages, planted support), two ragged
+    sequences: tau_hat, the exact kept sets of every kv head, and the entmax
+    attention over the GPU's kept pages against the oracle."""
     wl = _wl(3, [8192 + 20, 4096 + 1])
     cfg = wl.cfg
     pool, seq_lens = build_pool(wl)
     step = DecodeStep(pool, wl.page_table, seq_lens, cfg.H_q, "gauss", alpha=alpha, delta=delta)
-    step.score(wl.q)
-    step.choose()
+    step(wl.q)
     step.check()
     tau_gpu = step.tau_hat.cpu().numpy()
-    sel, cnt = step.sel.cpu().numpy(), step.sel_count.cpu().numpy()
+    sel, cnt, out = step.sel.cpu().numpy(), step.sel_count.cpu().numpy(), step.out.cpu().numpy()
     G = cfg.G
     for b in range(cfg.B):
         o = H.OracleSeq(wl, b)
         for g in range(cfg.H_kv):
-            ref = o.tau_hat(g, alpha)
-            got = tau_gpu[b, g * G:(g + 1) * G].astype(np.float64)
-            assert np.all(np.abs(got - ref) <= H.TAU_HAT_TOL * np.maximum(1.0, np.abs(ref))), (got, ref)
-            # the replica's keep rule with the oracle threshold: every decision
-            # outside the threshold's uncertainty band must match
-            _, _, est = o.gauss(g)
-            band = np.abs(got - ref) + 1e-6 * np.maximum(1.0, np.abs(ref))
-            margin = (alpha - 1.0) * est.astype(np.float64) - (ref[:, None] - delta)
-            must_keep = np.nonzero(np.any(margin > band[:, None], axis=0))[0]
-            must_drop = np.nonzero(np.all(margin < -band[:, None], axis=0))[0]
-            kept = set(sel[b, g, :cnt[b, g]].tolist())
-            assert set(must_keep.tolist()) <= kept
-            assert not (set(must_drop.tolist()) & kept)
-            assert list(sel[b, g, :cnt[b, g]]) == sorted(kept)
+            kept = sel[b, g, :cnt[b, g]]
+            _check_gauss_head(o, g, tau_gpu[b, g * G:(g + 1) * G], alpha, delta, kept)
+            o_ref, _ = o.attention(g, kept, alpha)
+            H.compare_out(out[b, g * G:(g + 1) * G], o_ref, cfg.dtype)
 
 
-@pytest.mark.parametrize("alpha", [1.25, 3.0])
+@pytest.mark.parametrize("alpha", [1.05, 1.1, 1.25, 3.0])
 def test_gauss_selection_any_alpha(alpha):
     """alpha outside {1.5, 2}: tau_hat from the 32-node Gauss-Legendre
-    expectations against the oracle's adaptive quadrature, and the keep
-    decisions outside the threshold's uncertainty band."""
+    expectations (placed on the integrand's peak, so powers up to 1/(alpha-1)
+    = 20 keep their mass) against the oracle's adaptive quadrature, the exact
+    kept sets, and the attention over the GPU's kept pages."""
     wl = _wl(3, [4096 + 33])
     cfg = wl.cfg
     pool, seq_lens = build_pool(wl)
     delta = 0.5
     step = DecodeStep(pool, wl.page_table, seq_lens, cfg.H_q, "gauss", alpha=alpha, delta=delta)
-    step.score(wl.q)
-    step.choose()
+    step(wl.q)
     step.check()
     tau_gpu = step.tau_hat.cpu().numpy()
-    sel, cnt = step.sel.cpu().numpy(), step.sel_count.cpu().numpy()
+    sel, cnt, out = step.sel.cpu().numpy(), step.sel_count.cpu().numpy(), step.out.cpu().numpy()
     G = cfg.G
     o = H.OracleSeq(wl, 0)
     for g in (0, 6):
-        m, v, est = o.gauss(g)
-        n = o.meta(g)["count"]
-        ref = np.array([gauss.tau_hat(m[h].astype(np.float64), v[h].astype(np.float64), n, alpha, iters=60)
-                        for h in range(G)])
-        got = tau_gpu[0, g * G:(g + 1) * G].astype(np.float64)
-        assert np.all(np.abs(got - ref) <= H.TAU_HAT_TOL * np.maximum(1.0, np.abs(ref))), (got, ref)
-        band = np.abs(got - ref) + 1e-6 * np.maximum(1.0, np.abs(ref))
-        margin = (alpha - 1.0) * est.astype(np.float64) - (ref[:, None] - delta)
-        must_keep = np.nonzero(np.any(margin > band[:, None], axis=0))[0]
-        must_drop = np.nonzero(np.all(margin < -band[:, None], axis=0))[0]
-        kept = set(sel[0, g, :cnt[0, g]].tolist())
-        assert set(must_keep.tolist()) <= kept
-        assert not (set(must_drop.tolist()) & kept)
+        kept = sel[0, g, :cnt[0, g]]
+        _check_gauss_head(o, g, tau_gpu[0, g * G:(g + 1) * G], alpha, delta, kept, iters=60)
+        o_ref, _ = o.attention(g, kept, alpha)
+        H.compare_out(out[0, g * G:(g + 1) * G], o_ref, cfg.dtype)
 
 
 @pytest.mark.parametrize("alpha", [1.5, 2.0])
