@@ -46,18 +46,18 @@ def _g_quad(u, s, r):
     """E[(Y)_+^r] for Y ~ N(u, s^2), s > 0, by adaptive quadrature.
 
     With z = u / s the expectation is s^r * int_0^inf y^r phi(y - z) dy.  The
-    integrand is negligible (below exp(-72) of its peak) outside
-    |y - z| <= 12; on [0, ...] the factor y^r is handled by the quadrature's
-    algebraic endpoint weight."""
+    log of the integrand, r ln y - (y - z)^2 / 2, is concave (second derivative
+    -(1 + r / y^2) <= -1) with its peak at y* = (z + sqrt(z^2 + 4 r)) / 2, so the
+    integrand is below exp(-72) of its peak outside |y - y*| <= 12; [0, ...] is
+    integrated with the quadrature's algebraic endpoint weight for y^r."""
     z = u / s
-    lo, hi = max(0.0, z - 12.0), z + 12.0
-    if hi <= 0.0:
-        return 0.0
+    ys = 0.5 * (z + math.sqrt(z * z + 4.0 * r))
+    lo, hi = max(0.0, ys - 12.0), ys + 12.0
     if lo == 0.0:
         val, _ = quad(lambda y: _phi(y - z), 0.0, hi, weight="alg", wvar=(r, 0.0),
                       epsabs=0.0, epsrel=1e-12, limit=400)
     else:
-        val, _ = quad(lambda y: y ** r * _phi(y - z), lo, hi, points=[z], epsabs=0.0, epsrel=1e-12,
+        val, _ = quad(lambda y: y ** r * _phi(y - z), lo, hi, points=[ys], epsabs=0.0, epsrel=1e-12,
                       limit=400)
     return s ** r * val
 

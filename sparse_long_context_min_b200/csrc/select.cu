@@ -541,13 +541,17 @@ constexpr int kGaussTauCTAs = 8;
 constexpr int kGaussTauReg = 4;      // pages per thread whose terms' inputs stay in registers
 
 // Any other alpha (r = 1/(alpha-1) not 1 or 2): E[(X - tau)_+^r] for
-// X ~ N(m', s'^2) by a 32-node Gauss-Legendre rule, with u = m' - tau and
-// z = u / s':
-//   z > 8:          int_{-8}^{8} (u + s' w)^r phi(w) dw   (the mass is away from 0);
-//   -10 < z <= 8:   int_0^T (s' t^2)^r phi(t^2 - z) 2t dt, T^2 = max(z + 8, 2)
-//                   (y = t^2 removes the y^r endpoint behaviour at 0);
-//   z <= -10:       0 (below exp(-50)).
-// g is the expectation and dg = -d/dtau of it (r times the same integrals of
+// X ~ N(m', s'^2), with u = m' - tau and z = u / s', is s'^r times
+// I(z) = int_0^inf y^r phi(y - z) dy.  The log of the integrand,
+// r ln y - (y - z)^2 / 2, is concave with its peak at y* = (z + sqrt(z^2 + 4r)) / 2
+// and second derivative -(1 + r / y^2): below y* it falls at least as fast as
+// a Gaussian of width w = 1 / sqrt(1 + r / y*^2), above y* at least as fast as
+// one of width w' = 1 / sqrt(1 + r / (y* + 10)^2), so [y* - 10 w, y* + 10 w']
+// holds all but about exp(-50) of it.  A 32-node Gauss-Legendre rule covers
+// that interval in y when it starts above 0, else [0, y* + 10 w'] in t with
+// y = t^2 (which removes the y^r endpoint behaviour at 0).  Terms are formed
+// as powf(s' y, r), so s'^r y^r never overflows where the product is small.
+// g is the expectation and dg = -d/dtau of it (r times the same integral of
 // the (r-1)-th power).
 struct GLTable {
     float x[kGLNodes], w[kGLNodes];   // nodes and weights on [-1, 1]
@@ -564,30 +568,36 @@ EKV_DEV void gauss_term_any(float mp, float sp, float tau, float r, const GLTabl
     }
     const float z = u / sp;
     g = dg = 0.f;
-    if (z <= -10.f) return;
+    const float ys = 0.5f * (z + sqrtf(fmaf(z, z, 4.f * r)));
+    const float w = rsqrtf(1.f + r / (ys * ys));
+    const float yh = ys + 10.f;
+    const float hi = ys + 10.f * rsqrtf(1.f + r / (yh * yh));
+    if (hi <= 0.f) return;
+    const float lo = ys - 10.f * w;
     const float c = 0.3989422804014327f;
     float s0 = 0.f, s1 = 0.f;
-    if (z > 8.f) {
+    if (lo > 0.f) {
+        const float half = 0.5f * (hi - lo), mid = 0.5f * (hi + lo);
 #pragma unroll 8
         for (int k = 0; k < kGLNodes; ++k) {
-            const float w = 8.f * gl.x[k];
-            const float y = fmaf(sp, w, u);
-            const float ph = c * expf(-0.5f * w * w) * 8.f * gl.w[k];
-            const float yr = powf(y, r);
+            const float y = fmaf(half, gl.x[k], mid);
+            const float e = y - z;
+            const float ph = c * expf(-0.5f * e * e) * half * gl.w[k];
+            const float yr = powf(sp * y, r);
             s0 = fmaf(yr, ph, s0);
-            s1 = fmaf(yr / y, ph, s1);
+            s1 = fmaf(yr / (sp * y), ph, s1);
         }
     } else {
-        const float T = sqrtf(fmaxf(z + 8.f, 2.f));
+        const float T = sqrtf(hi);
 #pragma unroll 8
         for (int k = 0; k < kGLNodes; ++k) {
             const float t = 0.5f * T * (gl.x[k] + 1.f);
-            const float y = sp * t * t;
-            const float e = t * t - z;
+            const float y = t * t;
+            const float e = y - z;
             const float ph = c * expf(-0.5f * e * e) * t * T * gl.w[k];   // phi * 2t * (T/2) w
-            const float yr = powf(y, r);
+            const float yr = powf(sp * y, r);
             s0 = fmaf(yr, ph, s0);
-            s1 = fmaf(yr / y, ph, s1);
+            s1 = fmaf(y > 0.f ? yr / (sp * y) : 0.f, ph, s1);
         }
     }
     g = s0;

@@ -30,7 +30,7 @@ def test_g_worked_examples(ex):
     assert abs(float(val) - ex["g"]) < 1e-14
 
 
-@pytest.mark.parametrize("alpha", [1.5, 2.0, 1.25, 3.0])
+@pytest.mark.parametrize("alpha", [1.5, 2.0, 1.25, 3.0, 1.1, 1.05])
 def test_g_against_quadrature(alpha):
     r = 1.0 / (alpha - 1.0)
     for m, s, tau in [(0.3, 0.25, 0.9), (1.8, 0.15, 1.9), (-1.0, 2.0, 0.5), (0.0, 1e-3, -0.01),
@@ -41,7 +41,7 @@ def test_g_against_quadrature(alpha):
         assert abs(float(gauss.g(m, s, tau, alpha)) - val) < 1e-10 + 1e-9 * abs(val)
 
 
-@pytest.mark.parametrize("alpha", [1.5, 2.0, 1.25, 1.8, 3.0])
+@pytest.mark.parametrize("alpha", [1.5, 2.0, 1.25, 1.8, 3.0, 1.1])
 def test_g_against_monte_carlo(alpha):
     rng = np.random.default_rng(20)
     r = 1.0 / (alpha - 1.0)
@@ -52,7 +52,7 @@ def test_g_against_monte_carlo(alpha):
         assert abs(y.mean() - float(gauss.g(m, s, tau, alpha))) < 4 * se
 
 
-@pytest.mark.parametrize("alpha", [1.5, 2.0, 1.25, 3.0])
+@pytest.mark.parametrize("alpha", [1.5, 2.0, 1.25, 3.0, 1.1])
 def test_point_pages_reduce_to_exact_entmax(alpha):
     rng = np.random.default_rng(21)
     for n in (1, 5, 64, 1000):
@@ -87,7 +87,7 @@ def test_F_decreasing_and_root(alpha):
     assert all(a > b for a, b in zip(vals, vals[1:]))
 
 
-@pytest.mark.parametrize("alpha", [1.25, 3.0])
+@pytest.mark.parametrize("alpha", [1.25, 3.0, 1.1, 1.05])
 def test_F_decreasing_and_root_any_alpha(alpha):
     rng = np.random.default_rng(23)
     P = 24
@@ -160,3 +160,22 @@ def test_z_bounds_the_expected_maximum_of_n_normals():
         mx = rng.standard_normal((100_000, n)).max(axis=1)
         mean, se = mx.mean(), mx.std() / math.sqrt(mx.size)
         assert mean - 4 * se <= z[n] <= 1.7 * (mean + 4 * se)
+
+
+@pytest.mark.parametrize("alpha", [1.1, 1.05])
+def test_quadrature_follows_the_peak_of_large_powers(alpha):
+    """For r = 1/(alpha-1) large, the integrand y^r phi(y - z) peaks at
+    y* = (z + sqrt(z^2 + 4r)) / 2, well above z: the expectation must keep the
+    mass there.  Against the same integral over the whole half line, with the
+    peak given to the integrator, and against the closed form of the raw
+    moments for z = 0 (E[Y_+^r] = 2^(r/2 - 1) Gamma((r + 1)/2) / sqrt(pi))."""
+    r = 1.0 / (alpha - 1.0)
+    for z in (-3.0, 0.0, 2.0):
+        ys = 0.5 * (z + math.sqrt(z * z + 4.0 * r))
+        f = lambda y: y ** r * math.exp(-0.5 * (y - z) ** 2) / math.sqrt(2 * math.pi)  # noqa: E731
+        val = quad(f, 0.0, ys, epsabs=0.0, epsrel=1e-13, limit=400)[0] + \
+            quad(f, ys, ys + 60.0, epsabs=0.0, epsrel=1e-13, limit=400)[0]
+        got = float(gauss.g(z, 1.0, 0.0, alpha))
+        assert abs(got - val) <= 1e-9 * val
+    moment = 2 ** (r / 2 - 1) * math.gamma((r + 1) / 2) / math.sqrt(math.pi)
+    assert abs(float(gauss.g(0.0, 1.0, 0.0, alpha)) - moment) <= 1e-9 * moment
