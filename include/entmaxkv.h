@@ -39,8 +39,8 @@
  *   = 1.5 and 2 have closed-form thresholds, any other alpha a threshold by
  *   safeguarded Newton steps in float64 and weights by powf.  The Gaussian
  *   selector takes alpha = 1.5 or 2 (closed-form expectations) and any alpha
- *   in [1.25, 16] (expectations by a 32-node Gauss-Legendre rule); other
- *   alpha return ENTMAXKV_UNSUPPORTED.
+ *   in [1.05, 16] (expectations by a 32-node Gauss-Legendre rule placed on
+ *   the integrand's peak); other alpha return ENTMAXKV_UNSUPPORTED.
  * - page_table[b][p] (int32, [B][max_pages]) is the physical page holding
  *   logical page p of sequence b; entries p >= P_b are never read.  Physical
  *   ids out of [0, num_phys_pages) are reported as ENTMAXKV_DEVICE_BOUNDS.
@@ -223,8 +223,10 @@ ENTMAXKV_API int entmaxkv_sparse_attend(const entmaxkv_pool* pool, const float* 
  * synchronise the device.  This call takes its scratch memory from a buffer
  * built into the library (ENTMAXKV_STATIC_SCRATCH_BYTES, 16 MiB, held on every
  * GPU that loads the library until the process exits) instead of a workspace.
- *   Arguments, layouts and results are those of entmaxkv_sparse_attend.
- *   Returns ENTMAXKV_STATIC_LIMIT, launching nothing, when
+ *   Arguments, layouts and results are those of entmaxkv_sparse_attend, and
+ *   its argument checks run first (a bad call returns the same code from
+ *   both entry points, whatever its size).  Then it returns
+ *   ENTMAXKV_STATIC_LIMIT, launching nothing, when
  *   entmaxkv_workspace_size(ENTMAXKV_OP_SPARSE_ATTEND, ...) exceeds the buffer
  *   (e.g. about 5 sequences of 2^20 tokens at a 1/64 budget with 32 query
  *   heads of 128 dims).

@@ -43,6 +43,63 @@ int ensure_smem(const void* func, int bytes)
     return 0;
 }
 
+int ensure_cluster_kernel(const void* func, int smem)
+{
+    static std::mutex mu;
+    static const void* seen_f[256];
+    static int seen_d[256];
+    static int nseen = 0;
+    if (ensure_smem(func, smem)) return 1;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return 1;
+    std::lock_guard<std::mutex> lock(mu);
+    for (int i = 0; i < nseen; ++i)
+        if (seen_f[i] == func && seen_d[i] == dev) return 0;
+    if (cudaFuncSetAttribute(func, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) != cudaSuccess) return 1;
+    if (nseen < 256) {
+        seen_f[nseen] = func;
+        seen_d[nseen] = dev;
+        ++nseen;
+    }
+    return 0;
+}
+
+int max_active_clusters(const void* func, int cluster, int threads, int smem)
+{
+    struct Entry {
+        const void* f;
+        int dev, cluster, threads, smem, n;
+    };
+    static std::mutex mu;
+    static Entry seen[256];
+    static int nseen = 0;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+    std::lock_guard<std::mutex> lock(mu);
+    for (int i = 0; i < nseen; ++i)
+        if (seen[i].f == func && seen[i].dev == dev && seen[i].cluster == cluster && seen[i].threads == threads &&
+            seen[i].smem == smem)
+            return seen[i].n;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(cluster, 1, 1);
+    cfg.blockDim = dim3(threads, 1, 1);
+    cfg.dynamicSmemBytes = smem;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = cluster;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, func, &cfg) != cudaSuccess) {
+        cudaGetLastError();   // clear the error: the caller tries a smaller cluster
+        n = 0;
+    }
+    if (nseen < 256) seen[nseen++] = Entry{func, dev, cluster, threads, smem, n};
+    return n;
+}
+
 // ------------------------------------------------------------------ TMA descriptors
 static PFN_cuTensorMapEncodeTiled_v12000 encode_fn()
 {
@@ -105,10 +162,10 @@ static int check_heads(int H_q, int H_kv)
 
 // Exact attention takes any alpha in (1, 16] (other than 1.5 and 2 by a
 // safeguarded Newton solve of the threshold and powf weights).  The Gaussian
-// selector has closed forms at 1.5 and 2 and integrates numerically for alpha
-// in [1.25, 16]; closer to 1 the power 1/(alpha-1) exceeds 4 and the fixed
-// quadrature rule loses accuracy.
-static bool alpha_gauss_ok(float alpha) { return alpha == 1.5f || alpha == 2.0f || (alpha >= 1.25f && alpha <= 16.0f); }
+// selector has closed forms at 1.5 and 2 and integrates numerically for any
+// other alpha in [1.05, 16] (r = 1/(alpha-1) up to 20: the rule follows the
+// integrand's peak, and float32 powers stay finite).
+static bool alpha_gauss_ok(float alpha) { return alpha == 1.5f || alpha == 2.0f || (alpha >= 1.05f && alpha <= 16.0f); }
 static bool alpha_attend_ok(float alpha) { return alpha > 1.0f && alpha <= 16.0f; }
 
 // ------------------------------------------------------------------ workspace
@@ -126,7 +183,7 @@ static int num_splits(int B, int H_kv, int list_pages)
 
 struct AttnLayout {
     int S;
-    size_t xbuf, cmax, opart, mlpart, lmax, tau, counters, total;
+    size_t xbuf, cmax, opart, mlpart, lmax, tau, counters, lbound, ccnt, cval, cidx, total;
 };
 
 // attention ops over a caller's page list / with softmax weights
@@ -154,15 +211,23 @@ static AttnLayout attn_layout(int op, int B, int H_q, int H_kv, int max_pages, i
     off += round256((size_t)B * H_q * sizeof(float));
     L.counters = off;
     off += round256((size_t)B * H_kv * sizeof(int32_t));
+    // threshold bounds and candidates of the fused bf16 entmax kernel
+    const size_t rows = soft ? 0 : (size_t)B * H_q * kFusedMaxSplits;
+    L.lbound = off;
+    off += round256(rows * sizeof(float));
+    L.ccnt = off;
+    off += round256(rows * sizeof(int32_t));
+    L.cval = off;
+    off += round256(rows * kFusedCandCap * sizeof(float));
+    L.cidx = off;
+    off += round256(rows * kFusedCandCap * sizeof(int32_t));
     L.total = off;
     return L;
 }
 
-static int attend_common(int op, const entmaxkv_pool* pool, const float* q, int H_q, const int32_t* page_table,
-                         int max_pages, const int32_t* seq_lens, int B, const int32_t* sel,
-                         const int32_t* sel_count, int k_max, float alpha, float scale, float* out,
-                         float* tau_out, int32_t* v_pages, void* workspace, size_t ws_bytes, int32_t* status,
-                         void* stream)
+int attend_check(int op, const entmaxkv_pool* pool, const float* q, int H_q, const int32_t* page_table,
+                 int max_pages, const int32_t* seq_lens, int B, const int32_t* sel, const int32_t* sel_count,
+                 int k_max, float alpha, float scale, const float* out, const int32_t* status)
 {
     int rc = check_pool(pool, true, false);
     if (rc) return rc;
@@ -173,6 +238,18 @@ static int attend_common(int op, const entmaxkv_pool* pool, const float* q, int 
     if (is_sparse(op) && (!sel || !sel_count || k_max <= 0)) return ENTMAXKV_INVALID_ARG;
     if (B == 0) return ENTMAXKV_OK;
     if (!q || !page_table || !seq_lens || !out || !status) return ENTMAXKV_INVALID_ARG;
+    return ENTMAXKV_OK;
+}
+
+static int attend_common(int op, const entmaxkv_pool* pool, const float* q, int H_q, const int32_t* page_table,
+                         int max_pages, const int32_t* seq_lens, int B, const int32_t* sel,
+                         const int32_t* sel_count, int k_max, float alpha, float scale, float* out,
+                         float* tau_out, int32_t* v_pages, void* workspace, size_t ws_bytes, int32_t* status,
+                         void* stream)
+{
+    int rc = attend_check(op, pool, q, H_q, page_table, max_pages, seq_lens, B, sel, sel_count, k_max, alpha,
+                          scale, out, status);
+    if (rc || B == 0) return rc;
     const AttnLayout lay = attn_layout(op, B, H_q, pool->H_kv, max_pages, k_max, pool->ps, pool->d);
     if (!workspace || ws_bytes < lay.total || !aligned16(workspace)) return ENTMAXKV_WORKSPACE;
 
@@ -200,6 +277,10 @@ static int attend_common(int op, const entmaxkv_pool* pool, const float* q, int 
     a.vpages = v_pages;
     a.tau = reinterpret_cast<float*>(ws + lay.tau);
     a.counters = reinterpret_cast<int32_t*>(ws + lay.counters);
+    a.lbound = reinterpret_cast<float*>(ws + lay.lbound);
+    a.ccnt = reinterpret_cast<int32_t*>(ws + lay.ccnt);
+    a.cval = reinterpret_cast<float*>(ws + lay.cval);
+    a.cidx = reinterpret_cast<int32_t*>(ws + lay.cidx);
     a.out = out;
     a.tau_out = tau_out;
     a.status = status;

@@ -7,36 +7,31 @@
 // Section 4 compares against full-cache entmax and full-cache softmax
 // (FlashDecoding) decoding.
 //
-// The threshold tau needs every candidate score before any weight is known,
-// so entmax attention runs as three kernels on the caller's stream:
-//   K pass   (qk_*):  split-KV CTAs gather key pages through the page table
-//                     (TMA tile loads into 128-byte-swizzled shared memory,
-//                     4-stage mbarrier pipeline), score the GQA head group
-//                     with mma.sync (keys bf16, query split into a bf16 high
-//                     and low part so the product keeps ~16 mantissa bits),
-//                     and write x = (alpha-1) * scale * q.k per listed token;
-//   tau solve (tau_): one CTA per (sequence, query head) keeps the scores
-//                     above max x - 1 (no other score can be in the support)
-//                     and runs Newton steps from the left on the restricted
-//                     normalisation equation until the support is stable,
-//                     then takes the closed form on that support in float64;
-//   V pass   (pv_*):  the same splits gather value pages, turn x into
-//                     p = [x - tau]_+^(1/(alpha-1)) (split bf16 high + low) and
-//                     accumulate P.V with mma.sync in fp32; the last CTA of a
-//                     (sequence, kv head) adds the split partials in split
-//                     order (deterministic).
+// The threshold tau needs every candidate score before any weight is known.
+// With a bf16 cache one launch does everything (entmax_bf16_kernel): the
+// split-KV CTAs of a (sequence, kv head) form a thread-block cluster and
+// cluster barriers separate
+//   K pass:    gather key pages through the page table (TMA tile loads into
+//              128-byte-swizzled shared memory, mbarrier pipeline), score the
+//              GQA head group with mma.sync (keys bf16, query split into a
+//              bf16 high and low part so the product keeps ~16 mantissa bits),
+//              write x = (alpha-1) * scale * q.k per listed token;
+//   threshold: a lower bound of tau from the chunk maxima, the scores above it
+//              as candidates, Newton steps from the left and the closed form
+//              on the final support in float64;
+//   V pass:    gather the value pages holding weight, turn x into
+//              p = [x - tau]_+^(1/(alpha-1)) (split bf16 high + low) and
+//              accumulate P.V with mma.sync in fp32; the partials are added
+//              in a fixed order (deterministic).
+// fp32 caches (small configurations) take three plain CUDA-core kernels with
+// the same split structure (qk_f32_kernel, tau_kernel, pv_f32_kernel).
 // The softmax baseline does K and V in one pass with an online softmax and a
 // log-sum-exp merge of the splits.
-//
-// fp32 caches (small configurations) take plain CUDA-core kernels that follow
-// the same split structure and workspace.
 #include "common.cuh"
 #include "kernels.cuh"
 
 namespace ekv {
 
-constexpr int kStagesQK = 4;
-constexpr int kStagesPV = 4;
 constexpr int kStagesSM = 3;
 constexpr int kPsPad = 8;   // padding (bf16 elements) of a row of the P tile
 
@@ -204,137 +199,6 @@ EKV_DEV float group_lane_max(float v)
     v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 8));
     v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 16));
     return v;
-}
-
-// Write this split's maximum score of every head of the group (all threads
-// call; `wm` is shared [4][8]).
-EKV_DEV void write_split_max(const AttnArgs& a, int b, int g, int s, const float* run, int NT, float (*wm)[8])
-{
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, c = lane & 3;
-    for (int nt = 0; nt < NT; ++nt) {
-        const float m = group_lane_max(run[nt]);
-        if (lane < 4) wm[warp][4 * nt + c] = m;
-    }
-    __syncthreads();
-    if (threadIdx.x < a.G) {
-        const int h = threadIdx.x;
-        const float m = fmaxf(fmaxf(wm[0][h], wm[1][h]), fmaxf(wm[2][h], wm[3][h]));
-        a.lmax[((size_t)b * a.H_q + (size_t)g * a.G + h) * a.S + s] = m;
-    }
-}
-
-template <int D, int PS, int NT>
-__global__ void __launch_bounds__(kThreads) qk_bf16_kernel(const __grid_constant__ CUtensorMap kmap, const AttnArgs a)
-{
-    pdl_enter();
-    constexpr int STAGE = kStageTok * D * 2;
-    constexpr int PPS = kStageTok / PS;
-    constexpr int KS = D / 16;
-    extern __shared__ uint8_t smem_raw[];
-    uint8_t* smem = smem_align<1024>(smem_raw);
-    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kStagesQK * STAGE);
-    __shared__ int abort_flag;
-    __shared__ float wm[4][8];
-
-    const int b = blockIdx.z, g = blockIdx.y, s = blockIdx.x;
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int L = a.seq_lens[b];
-    const int P = pages_of(L, PS, a.max_pages, a.status);
-    const int cnt = list_count(a, b, g, P);
-    if (s == 0 && tid == 0) a.counters[(size_t)b * a.H_kv + g] = 0;
-    const Range r = split_range(cnt, a.S, s);
-    const int nst = r.end > r.start ? (r.end - r.start + PPS - 1) / PPS : 0;
-    tab_fill(a, b, g, r, P);
-
-    // start the key loads first; the query fragments are prepared meanwhile
-    if (tid == 0) {
-        abort_flag = 0;
-        if (nst > 0) {
-            prefetch_tmap(&kmap);
-            for (int i = 0; i < kStagesQK; ++i) mbar_init(&bars[i], 1);
-            fence_mbar_init();
-            for (int st = 0; st < min(kStagesQK, nst); ++st)
-                issue_stage<D, PS>(a, &kmap, smem + st * STAGE, &bars[st], b, g, r, st, P);
-        }
-    }
-    float run[NT];
-#pragma unroll
-    for (int nt = 0; nt < NT; ++nt) run[nt] = -INFINITY;
-    if (nst == 0) {
-        write_split_max(a, b, g, s, run, NT, wm);
-        return;
-    }
-    uint32_t bq[NT][KS][2];
-    load_q_frags<D, NT>(a, b, g, a.xscale, bq);
-    __syncthreads();
-
-    const uint32_t sbase = smem_addr(smem);
-    const size_t xstride = (size_t)a.k_max * PS;
-    const size_t cstride = (size_t)a.k_max * (PS / 16);
-    for (int st = 0; st < nst; ++st) {
-        const int slot = st % kStagesQK;
-        if (!mbar_wait(&bars[slot], (st / kStagesQK) & 1, kWaitLimitNs)) {
-            abort_flag = 1;
-            report(a.status, ENTMAXKV_TIMEOUT);
-        }
-        __syncthreads();
-        if (abort_flag) {
-            if (tid == 0)
-                for (int k = st; k < min(st + kStagesQK, nst); ++k)
-                    mbar_wait(&bars[k % kStagesQK], (k / kStagesQK) & 1, kWaitLimitNs);
-            return;
-        }
-        const uint32_t base = sbase + slot * STAGE;
-        const int row0 = warp * 16;
-        float acc[NT][4];
-#pragma unroll
-        for (int nt = 0; nt < NT; ++nt) acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0.f;
-        const int arow = row0 + (lane & 7) + ((lane >> 3) & 1) * 8;
-#pragma unroll
-        for (int j = 0; j < KS; ++j) {
-            uint32_t af[4];
-            ldsm_x4(swz_addr(base, arow, 2 * j + (lane >> 4)), af);
-#pragma unroll
-            for (int nt = 0; nt < NT; ++nt) mma_bf16(acc[nt], af, bq[nt][j][0], bq[nt][j][1]);
-        }
-        // the warp's 16 rows lie in one page (16 divides PS): one list entry
-        const int gi = lane >> 2, c = lane & 3;
-        const int idx = r.start + st * PPS + row0 / PS;
-        if (idx < r.end) {
-            int lp;
-            const int phys = resolve(a, b, g, idx, P, lp, false);
-            float cm[NT];
-#pragma unroll
-            for (int nt = 0; nt < NT; ++nt) cm[nt] = -INFINITY;
-#pragma unroll
-            for (int rr = 0; rr < 2; ++rr) {
-                const int prow = (row0 + gi + 8 * rr) % PS;
-                const bool valid = phys >= 0 && lp * PS + prow < L;
-#pragma unroll
-                for (int nt = 0; nt < NT; ++nt) {
-                    const int head = 4 * nt + c;
-                    const float x = valid ? acc[nt][2 * rr] + acc[nt][2 * rr + 1] : -INFINITY;
-                    cm[nt] = fmaxf(cm[nt], x);
-                    if (head < a.G)
-                        a.xbuf[((size_t)b * a.H_q + (size_t)g * a.G + head) * xstride + (size_t)idx * PS + prow] = x;
-                }
-            }
-            // chunk maxima: the V pass decides from these which pages hold weight
-#pragma unroll
-            for (int nt = 0; nt < NT; ++nt) {
-                const float m = group_lane_max(cm[nt]);
-                run[nt] = fmaxf(run[nt], m);
-                const int head = 4 * nt + c;
-                if (gi == 0 && head < a.G)
-                    a.cmax[((size_t)b * a.H_q + (size_t)g * a.G + head) * cstride + (size_t)idx * (PS / 16) +
-                           (row0 % PS) / 16] = m;
-            }
-        }
-        __syncthreads();
-        if (tid == 0 && st + kStagesQK < nst)
-            issue_stage<D, PS>(a, &kmap, smem + slot * STAGE, &bars[slot], b, g, r, st + kStagesQK, P);
-    }
-    write_split_max(a, b, g, s, run, NT, wm);
 }
 
 // fp32 cache: each thread scores (token, head) pairs of a page with a float64
@@ -742,234 +606,6 @@ EKV_DEV void reduce_splits(const AttnArgs& a, int b, int g)
 // that feeds the TMA pipeline.
 constexpr int kActWin = 512;
 
-template <int D, int PS, int NT>
-__global__ void __launch_bounds__(kThreads) pv_bf16_kernel(const __grid_constant__ CUtensorMap vmap, const AttnArgs a)
-{
-    pdl_enter();
-    constexpr int STAGE = kStageTok * D * 2;
-    constexpr int PPS = kStageTok / PS;
-    constexpr int MTW = D / 64;           // 16-row m-tiles (head-dim rows) per warp
-    constexpr int PROW = kStageTok + kPsPad;
-    extern __shared__ uint8_t smem_raw[];
-    uint8_t* smem = smem_align<1024>(smem_raw);
-    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kStagesPV * STAGE);
-    uint16_t* ps_tile = reinterpret_cast<uint16_t*>(smem + kStagesPV * STAGE + 64);   // [8*NT][PROW]
-    __shared__ int abort_flag;
-    __shared__ int act[kActWin];
-    __shared__ unsigned char flag[kActWin];
-    __shared__ int nact;
-    __shared__ float tau_s[8];
-
-    const int b = blockIdx.z, g = blockIdx.y, s = blockIdx.x;
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int L = a.seq_lens[b];
-    const int P = pages_of(L, PS, a.max_pages, a.status);
-    const int cnt = list_count(a, b, g, P);
-    const Range r = split_range(cnt, a.S, s);
-    const bool a2 = a.alpha == 2.0f;
-    const bool a15 = a.alpha == 1.5f;
-    const float rexp = 1.0f / (a.alpha - 1.0f);   // weight exponent for any other alpha
-    const size_t xstride = (size_t)a.k_max * PS;
-    const size_t row0h = (size_t)b * a.H_q + (size_t)g * a.G;
-
-    float acc[NT][MTW][4];
-#pragma unroll
-    for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-        for (int m = 0; m < MTW; ++m) acc[nt][m][0] = acc[nt][m][1] = acc[nt][m][2] = acc[nt][m][3] = 0.f;
-
-    tab_fill(a, b, g, r, P);
-    if (tid < 8) tau_s[tid] = tid < a.G ? a.tau[row0h + tid] : INFINITY;
-    if (tid == 0) {
-        abort_flag = 0;
-        prefetch_tmap(&vmap);
-        for (int i = 0; i < kStagesPV; ++i) mbar_init(&bars[i], 1);
-        fence_mbar_init();
-    }
-    for (int i = tid; i < 8 * NT * PROW; i += kThreads) ps_tile[i] = 0;
-    __syncthreads();
-    const uint32_t sbase = smem_addr(smem);
-    const uint32_t pbase = smem_addr(ps_tile);
-    int gst = 0;          // stages issued so far (barrier phase bookkeeping)
-    int loaded = 0;
-
-    for (int w0 = r.start; w0 < r.end; w0 += kActWin) {
-        const int wn = min(kActWin, r.end - w0);
-        // --- which pages of the window hold weight
-        for (int i = tid; i < wn; i += kThreads) flag[i] = 0;
-        __syncthreads();
-        {
-            constexpr int C = PS / 16;          // 16-token chunk maxima per page
-            const size_t cstride = (size_t)a.k_max * C;
-            const int items = wn * a.G;
-            for (int it = tid; it < items; it += kThreads) {
-                const int j = it / a.G, h = it % a.G;
-                const float* cp = a.cmax + (row0h + h) * cstride + (size_t)(w0 + j) * C;
-                float m = -INFINITY;
-                if constexpr (C % 4 == 0) {
-#pragma unroll
-                    for (int k = 0; k < C; k += 4) {
-                        const float4 v = *reinterpret_cast<const float4*>(cp + k);
-                        m = fmaxf(m, fmaxf(fmaxf(v.x, v.y), fmaxf(v.z, v.w)));
-                    }
-                } else {
-#pragma unroll
-                    for (int k = 0; k < C; ++k) m = fmaxf(m, cp[k]);
-                }
-                if (m > tau_s[h]) flag[j] = 1;
-            }
-        }
-        __syncthreads();
-        if (warp == 0) {   // ordered compaction of the flags
-            int base = 0;
-            for (int i0 = 0; i0 < wn; i0 += 32) {
-                const bool f = (i0 + lane < wn) && flag[i0 + lane];
-                const unsigned m = __ballot_sync(0xffffffffu, f);
-                if (f) act[base + __popc(m & ((1u << lane) - 1u))] = w0 + i0 + lane;
-                base += __popc(m);
-            }
-            if (lane == 0) nact = base;
-        }
-        __syncthreads();
-        const int na = nact;
-        loaded += na;
-        const int nst = (na + PPS - 1) / PPS;
-        if (nst == 0) continue;
-        // --- pipeline over the active pages
-        auto issue = [&](int st, int slot_) {
-            uint8_t* dst = smem + slot_ * STAGE;
-            int phys[PPS];
-            uint32_t bytes = 0;
-#pragma unroll
-            for (int i = 0; i < PPS; ++i) {
-                const int ai = st * PPS + i;
-                int lp;
-                phys[i] = ai < na ? resolve(a, b, g, act[ai], P, lp, true) : -1;
-                if (phys[i] >= 0) bytes += PS * D * 2;
-            }
-            mbar_arrive_expect_tx(&bars[slot_], bytes);
-#pragma unroll
-            for (int i = 0; i < PPS; ++i) {
-                if (phys[i] < 0) continue;
-                const int y = (phys[i] * a.H_kv + g) * PS;
-#pragma unroll
-                for (int hh = 0; hh < D / 64; ++hh)
-                    tma_load_2d(dst + hh * (kStageTok * 128) + i * PS * 128, &vmap, &bars[slot_], hh * 64, y);
-            }
-        };
-        if (tid == 0)
-            for (int st = 0; st < min(kStagesPV, nst); ++st) issue(st, (gst + st) % kStagesPV);
-        for (int st = 0; st < nst; ++st) {
-            const int gs = gst + st;
-            const int slot = gs % kStagesPV;
-            // weights of this stage: token tid % 64, heads (tid / 64) * 2 * NT ...
-            {
-                const int t = tid & (kStageTok - 1);
-                const int ai = st * PPS + t / PS;
-                const int prow = t % PS;
-                int idx = -1;
-                bool valid = false;
-                if (ai < na) {
-                    idx = act[ai];
-                    int lp;
-                    const int phys = resolve(a, b, g, idx, P, lp, false);
-                    valid = phys >= 0 && lp * PS + prow < L;
-                }
-                const int hbase = (tid >> 6) * 2 * NT;
-#pragma unroll
-                for (int k = 0; k < 2 * NT; ++k) {
-                    const int head = hbase + k;
-                    float p = 0.f;
-                    if (head < a.G && valid) {
-                        const float xv = a.xbuf[(row0h + head) * xstride + (size_t)idx * PS + prow];
-                        const float u = fmaxf(xv - tau_s[head], 0.f);
-                        p = a2 ? u : (a15 ? u * u : powf(u, rexp));
-                    }
-                    uint32_t hi, lo;
-                    split_bf16(p, hi, lo);
-                    ps_tile[(2 * head) * PROW + t] = (uint16_t)hi;
-                    ps_tile[(2 * head + 1) * PROW + t] = (uint16_t)lo;
-                }
-            }
-            if (!mbar_wait(&bars[slot], (gs / kStagesPV) & 1, kWaitLimitNs)) {
-                abort_flag = 1;
-                report(a.status, ENTMAXKV_TIMEOUT);
-            }
-            __syncthreads();
-            if (abort_flag) {
-                if (tid == 0)
-                    for (int k = st; k < min(st + kStagesPV, nst); ++k)
-                        mbar_wait(&bars[(gst + k) % kStagesPV], ((gst + k) / kStagesPV) & 1, kWaitLimitNs);
-                return;
-            }
-            // rows without a valid token are zeroed so zero weights never meet garbage
-            {
-                const int t = tid & (kStageTok - 1);
-                const int half = tid >> 6;
-                if (half < D / 64) {
-                    const int ai = st * PPS + t / PS;
-                    bool valid = false;
-                    if (ai < na) {
-                        int lp;
-                        const int phys = resolve(a, b, g, act[ai], P, lp, false);
-                        valid = phys >= 0 && lp * PS + (t % PS) < L;
-                    }
-                    if (!valid) {
-                        uint4* rowp = reinterpret_cast<uint4*>(smem + slot * STAGE + half * (kStageTok * 128) + t * 128);
-#pragma unroll
-                        for (int k = 0; k < 8; ++k) rowp[k] = make_uint4(0, 0, 0, 0);
-                        fence_proxy_async();
-                    }
-                }
-            }
-            __syncthreads();
-            const uint32_t base = sbase + slot * STAGE;
-            const int n = lane >> 2, c = lane & 3;
-#pragma unroll
-            for (int kk = 0; kk < kStageTok / 16; ++kk) {
-                uint32_t b0[NT], b1[NT];
-#pragma unroll
-                for (int nt = 0; nt < NT; ++nt) {
-                    const uint32_t pr = pbase + ((8 * nt + n) * PROW + 16 * kk + 2 * c) * 2;
-                    asm volatile("ld.shared.b32 %0, [%1];" : "=r"(b0[nt]) : "r"(pr));
-                    asm volatile("ld.shared.b32 %0, [%1];" : "=r"(b1[nt]) : "r"(pr + 16));
-                }
-                const int mi = lane >> 3;
-                const int trow = 16 * kk + (lane & 7) + 8 * (mi >> 1);
-#pragma unroll
-                for (int m = 0; m < MTW; ++m) {
-                    const int d0 = 16 * (warp * MTW + m);
-                    uint32_t af[4];
-                    ldsm_x4_t(swz_addr(base, trow, d0 / 8 + (mi & 1)), af);
-#pragma unroll
-                    for (int nt = 0; nt < NT; ++nt) mma_bf16(acc[nt][m], af, b0[nt], b1[nt]);
-                }
-            }
-            __syncthreads();
-            if (tid == 0 && st + kStagesPV < nst) issue(st + kStagesPV, (gs + kStagesPV) % kStagesPV);
-        }
-        gst += nst;
-    }
-    if (tid == 0 && a.vpages) atomicAdd(&a.vpages[(size_t)b * a.H_kv + g], loaded);
-    // partial output of this split: o[head 4nt + c][d]
-    {
-        const int c = lane & 3, gi = lane >> 2;
-#pragma unroll
-        for (int nt = 0; nt < NT; ++nt) {
-            const int head = 4 * nt + c;
-            if (head >= a.G) continue;
-            const size_t row = (row0h + head) * a.S + s;
-#pragma unroll
-            for (int m = 0; m < MTW; ++m) {
-                const int d = 16 * (warp * MTW + m) + gi;
-                a.opart[row * D + d] = acc[nt][m][0] + acc[nt][m][1];
-                a.opart[row * D + d + 8] = acc[nt][m][2] + acc[nt][m][3];
-            }
-        }
-    }
-    reduce_splits<D, false>(a, b, g);
-}
-
 template <int D>
 __global__ void __launch_bounds__(kThreads) pv_f32_kernel(const float* __restrict__ v_pool, int ps, const AttnArgs a)
 {
@@ -1021,6 +657,827 @@ __global__ void __launch_bounds__(kThreads) pv_f32_kernel(const float* __restric
         atomicAdd(&a.vpages[(size_t)b * a.H_kv + g], n);
     }
     reduce_splits<D, false>(a, b, g);
+}
+
+// ====================================================================== fused entmax (bf16 cache)
+// One launch runs the K pass, the threshold and the V pass.  The S splits of
+// a (sequence, kv head) form one thread-block cluster, whose CTAs are
+// scheduled together, so cluster barriers can separate the phases and the
+// CTAs can read each other's shared memory (distributed shared memory):
+//   K pass      each split scores its pages and writes x and the 16-token
+//               chunk maxima to the workspace;
+//   local       each split, one warp per query head, finds a lower bound t_s
+//               of tau from its own chunk maxima (split_bound) and keeps its
+//               scores above t_s, with their list positions, in its shared
+//               memory (local_candidates);
+//   barrier 1
+//   threshold   every CTA reads every split's bound and candidates; the
+//               largest bound is a lower bound of tau for the whole group, so
+//               the candidates above it hold every score that can carry
+//               weight (gather_candidates); tau of every query head is solved
+//               from them, one warp per head, with the same operations in the
+//               same order in every CTA, so all splits hold the same tau; the
+//               candidates above tau mark the value pages that hold weight,
+//               and CTA s takes every S-th of them in list order, their page
+//               ids read from the owning split's table;
+//   V pass      each CTA accumulates P.V over its value pages and keeps its
+//               partial output in shared memory;
+//   barrier 2
+//   merge       CTA r adds the partials of the output elements
+//               [r E / S, (r + 1) E / S) in CTA order (deterministic);
+//   barrier 3   no CTA leaves while another may still read its memory.
+// Where a split has more candidates than its slots hold, every CTA instead
+// solves over all the group's scores (global memory, written before barrier 1
+// with a fence) and loads the value pages of its own split.  No CTA leaves
+// before the last barrier, whatever happens (a timed-out copy only skips
+// work).
+constexpr int kFusedStages = 4;
+constexpr int kPubCap = 256;         // candidates a split keeps per query head for the others
+constexpr int kBitWords = 1024;      // weighted-page bitmap: lists of up to 32768 pages
+
+// Warp-wide sum of three doubles and min / max of two floats (xor butterfly:
+// every lane ends with the same values).
+EKV_DEV void warp_red5(double (&v)[3], float& mn, float& mx)
+{
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+#pragma unroll
+        for (int i = 0; i < 3; ++i) v[i] += __shfl_xor_sync(0xffffffffu, v[i], o);
+        mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    }
+}
+
+// Where the candidates of a head's threshold are read from.
+struct TauSrc {
+    const float* x;     // the head's scores over the listed tokens (global), mode 1
+    int n;              // listed tokens
+    const float* cand;  // the candidate scores (shared), mode 0
+    int ncand;
+    int mode;           // 0: cand, 1: every score above lo
+    double lo;          // every candidate is > lo; every other score is <= lo <= tau
+};
+
+// f(x) for every candidate x of the head; lane l takes every 32nd one.
+template <typename Fn>
+EKV_DEV void for_candidates(const TauSrc& s, Fn&& f)
+{
+    const int lane = threadIdx.x & 31;
+    if (s.mode == 0) {
+        for (int i = lane; i < s.ncand; i += 32) f(s.cand[i]);
+    } else {
+        for (int k = lane; k < s.n; k += 32) {
+            const float v = __ldcg(s.x + k);
+            if ((double)v > s.lo) f(v);
+        }
+    }
+}
+
+// Newton steps from the left on F_c(t) = sum_j (v_j - t)_+^r over the n
+// values in `vals` (shared, read lane-strided), from t0 with F_c(t0) >= 1.
+// For r >= 1, F_c is convex and decreasing, so every iterate stays at or below
+// its root; the result keeps a rounding margin below the last iterate.  For
+// r < 1 the start is returned.
+EKV_DEV double newton_bound(const float* vals, int n, double t0, double r, bool a2, bool a15)
+{
+    if (r < 1.0) return t0;
+    const int lane = threadIdx.x & 31;
+    double t = t0;
+    for (int it = 0; it < 8; ++it) {
+        double F = 0.0, dF = 0.0;
+        for (int j = lane; j < n; j += 32) {
+            const double u = (double)vals[j] - t;
+            if (u > 0.0) {
+                const double p1 = a2 ? 1.0 : (a15 ? u : pow(u, r - 1.0));
+                F += p1 * u;
+                dF += r * p1;
+            }
+        }
+        F = warp_sum(F);
+        dF = warp_sum(dF);
+        if (!(F > 1.0) || !(dF > 0.0)) break;          // at (or by rounding past) the root
+        const double nt = t + (F - 1.0) / dF;
+        if (!(nt > t)) break;
+        const bool small = nt - t <= 1e-3 * fmax(1.0, fabs(t));
+        t = nt;
+        if (small) break;                              // close enough: the bound only prunes
+    }
+    return t - 1e-9 * fmax(1.0, fabs(t));
+}
+
+// Lower bound of tau from one split's chunk maxima, by one warp.  cm: the
+// head's chunk-maximum row, own chunks [c0, c1); m_s the split's largest
+// score.  Every chunk maximum is the score of a distinct token, so for any
+// subset of the head's tokens sum_i (x_i - t)_+^r >= sum over the subset's
+// chunk maxima, and the root of the latter is at or below tau.  The chunks
+// above m_s - 1 (the only ones that can matter) are kept in (lc, lcv); *nlc
+// is their number (more than cap: the list is unusable).
+EKV_DEV float split_bound(const float* cm, int c0, int c1, float m_s, double r, bool a2, bool a15, int* lc,
+                          float* lcv, int cap, int* nlc)
+{
+    const int lane = threadIdx.x & 31;
+    const unsigned below = (1u << lane) - 1u;
+    if (!(m_s > -INFINITY)) {
+        *nlc = 0;
+        return -INFINITY;
+    }
+    const double thr = (double)m_s - 1.0;
+    int n = 0;
+    constexpr int U = 8;
+    for (int i0 = c0; i0 < c1; i0 += 32 * U) {
+        float v[U];
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const int i = i0 + u * 32 + lane;
+            v[u] = i < c1 ? cm[i] : -INFINITY;
+        }
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const bool keep = (double)v[u] > thr;
+            const unsigned m = __ballot_sync(0xffffffffu, keep);
+            const int pos = n + __popc(m & below);
+            if (keep && pos < cap) {
+                lc[pos] = i0 + u * 32 + lane;
+                lcv[pos] = v[u];
+            }
+            n += __popc(m);
+        }
+    }
+    __syncwarp();
+    *nlc = n;
+    const double t = n <= cap ? newton_bound(lcv, n, thr, r, a2, a15) : thr;
+    return __double2float_rd(t);
+}
+
+// One split's candidates of one head, by one warp: its scores above t with
+// their list positions, into (pval, ppos) (shared, at most kPubCap kept);
+// returns how many there are.  The chunks to read come from the list of
+// split_bound when it is usable (t is at least m_s - 1), else from all the
+// split's chunks [c0, c1).
+EKV_DEV int local_candidates(const float* x, int c0, int c1, int* lc, const float* lcv, int nlc, int cap, float t,
+                             float* pval, int* ppos)
+{
+    const int lane = threadIdx.x & 31;
+    const unsigned below = (1u << lane) - 1u;
+    constexpr int U = 8;
+    int nf = 0;
+    const bool listed = nlc <= cap;
+    if (listed) {                                      // chunks above t, compacted in place (order kept)
+        for (int j0 = 0; j0 < nlc; j0 += 32) {
+            const int j = j0 + lane;
+            const bool keep = j < nlc && lcv[j] > t;
+            const int c = keep ? lc[j] : 0;
+            const unsigned m = __ballot_sync(0xffffffffu, keep);
+            __syncwarp();
+            if (keep) lc[nf + __popc(m & below)] = c;
+            nf += __popc(m);
+            __syncwarp();
+        }
+    }
+    const int nk = listed ? nf * 16 : (c1 - c0) * 16;
+    int nc = 0;
+    for (int k0 = 0; k0 < nk; k0 += 32 * U) {
+        float v[U];
+        int pos[U];
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const int k = k0 + u * 32 + lane;
+            pos[u] = k < nk ? (listed ? lc[k >> 4] * 16 + (k & 15) : c0 * 16 + k) : 0;
+            v[u] = k < nk ? x[pos[u]] : -INFINITY;
+        }
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const bool keep = v[u] > t;
+            const unsigned m = __ballot_sync(0xffffffffu, keep);
+            const int q = nc + __popc(m & below);
+            if (keep && q < kPubCap) {
+                pval[q] = v[u];
+                ppos[q] = pos[u];
+            }
+            nc += __popc(m);
+        }
+    }
+    __syncwarp();
+    return nc;
+}
+
+// The group's candidates of one head above tlb, gathered by one warp from the
+// S splits' lists (distributed shared memory: pval / ppos / n of split q live
+// in CTA q of the cluster) into (cv, ci), in split order; returns how many
+// (-1 when more than cap).  pre: per-warp shared scratch of S + 1 ints.
+EKV_DEV int gather_candidates(const float* pval, const int* ppos, int nq, int S, float tlb, float* cv, int* ci,
+                              int cap, int* pre)
+{
+    const int lane = threadIdx.x & 31;
+    const unsigned below = (1u << lane) - 1u;
+    // nq: split lane's count (lanes >= S hold 0); prefix sums into pre[0..S]
+    int incl = nq;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int t = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += t;
+    }
+    if (lane < S) pre[lane + 1] = incl;
+    if (lane == 0) pre[0] = 0;
+    const int total = __shfl_sync(0xffffffffu, incl, 31);
+    __syncwarp();
+    constexpr int U = 8;
+    int n = 0;
+    for (int k0 = 0; k0 < total; k0 += 32 * U) {
+        float v[U];
+        int p[U];
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const int k = k0 + u * 32 + lane;
+            v[u] = -INFINITY;
+            p[u] = 0;
+            if (k < total) {
+                int lo = 0, hi = S;                    // the split q with pre[q] <= k < pre[q + 1]
+                while (hi - lo > 1) {
+                    const int mid = (lo + hi) >> 1;
+                    if (pre[mid] <= k) lo = mid; else hi = mid;
+                }
+                const int i = k - pre[lo];
+                v[u] = ld_dsmem_f32(dsmem(pval + i, lo));
+                p[u] = ld_dsmem_s32(dsmem(ppos + i, lo));
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const bool keep = v[u] > tlb;
+            const unsigned m = __ballot_sync(0xffffffffu, keep);
+            const int q = n + __popc(m & below);
+            if (keep && q < cap) {
+                cv[q] = v[u];
+                ci[q] = p[u];
+            }
+            n += __popc(m);
+        }
+    }
+    __syncwarp();
+    return n <= cap ? n : -1;
+}
+
+// tau from the candidates of src: alpha = 2 and 1.5 by Newton steps from the
+// bound src.lo until the support is consistent, then the closed form on that
+// support in float64; any other alpha by safeguarded Newton steps on
+// F^(1/r) inside [src.lo, M].  One warp; every lane returns tau.
+EKV_DEV double solve_tau(const TauSrc& src, float M, float alpha)
+{
+    const bool a2 = alpha == 2.0f;
+    const bool a15 = alpha == 1.5f;
+    double tau = src.lo;
+    if (!a2 && !a15) {
+        // Newton on G(t) = F(t)^(1/r) - 1 inside [lo, hi] (F(lo) >= 1 > F(M) = 0),
+        // bisection where a step leaves it; terms in float (powf), sums in float64
+        const double r = 1.0 / ((double)alpha - 1.0);
+        const float rf = (float)r;
+        double lo = src.lo, hi = (double)M;
+        for (int it = 0; it < 100; ++it) {
+            double v[3] = {0.0, 0.0, 0.0};
+            float u0 = INFINITY, u1 = -INFINITY;
+            for_candidates(src, [&](float f) {
+                const double vd = (double)f;
+                if (vd > tau) {
+                    const float u = (float)(vd - tau);
+                    const float pu = powf(u, rf);
+                    v[0] += (double)pu;
+                    v[1] += (double)pu / (double)u;
+                }
+            });
+            warp_red5(v, u0, u1);
+            const double F = v[0], S1 = r * v[1];
+            if (F >= 1.0) lo = tau; else hi = tau;
+            if (F == 1.0 || hi - lo <= 1e-13 * fmax(1.0, fabs(tau))) break;
+            double nt = (F > 0.0 && S1 > 0.0) ? tau + r * F * (1.0 - pow(F, -1.0 / r)) / S1 : 0.5 * (lo + hi);
+            if (!(nt > lo && nt < hi)) nt = 0.5 * (lo + hi);
+            if (fabs(nt - tau) <= 1e-8 * fmax(1.0, fabs(tau))) {
+                tau = nt;
+                break;
+            }
+            tau = nt;
+        }
+        return tau;
+    }
+    double kprev = -1.0;
+    for (int it = 0; it < 100; ++it) {
+        double v[3] = {0.0, 0.0, 0.0};
+        float minS = INFINITY, maxN = -INFINITY;
+        for_candidates(src, [&](float f) {
+            const double vd = (double)f;
+            if (vd > tau) {
+                v[0] += 1.0;
+                v[1] += vd;
+                v[2] = fma(vd, vd, v[2]);
+                minS = fminf(minS, f);
+            } else {
+                maxN = fmaxf(maxN, f);
+            }
+        });
+        warp_red5(v, minS, maxN);
+        const double k = v[0], sx = v[1], sxx = v[2];
+        if (a2 || k == kprev) {
+            // the support held still for a step: the closed form on it
+            double tcf;
+            bool ok;
+            if (a2) {
+                tcf = (sx - 1.0) / k;
+                ok = true;
+            } else {
+                const double mean = sx / k, msq = sxx / k;
+                const double disc = mean * mean - msq + 1.0 / k;
+                ok = disc >= 0.0;
+                tcf = ok ? mean - sqrt(disc) : 0.0;
+            }
+            // consistent support: every kept value above tcf, every dropped one at or
+            // below it (the values at or below the bound are below tau as well)
+            if (ok && tcf < (double)minS && (double)maxN <= tcf && tcf >= src.lo) return tcf;
+            if (a2) {
+                if (!(tcf != tau) || !isfinite(tcf)) break;
+                tau = tcf;
+                continue;
+            }
+        }
+        kprev = k;
+        // Newton step on sum (x - t)^2 = 1 over the current support (from the left)
+        const double s1 = sx - k * tau;
+        const double s2 = sxx - 2.0 * tau * sx + k * tau * tau;
+        const double nt = tau + (s2 - 1.0) / (2.0 * s1);
+        if (!(nt != tau) || !isfinite(nt)) {
+            kprev = k;                                 // closed form next time round
+            continue;
+        }
+        tau = nt;
+    }
+    return tau;
+}
+
+// Exclusive prefix sum of one int per thread over a 128-thread block (two
+// block barriers inside); *total gets the block's sum.
+EKV_DEV int block_excl_scan128(int v, int* wsum, int* total)
+{
+    const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+    int incl = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int t = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += t;
+    }
+    __syncthreads();
+    if (lane == 31) wsum[w] = incl;
+    __syncthreads();
+    int before = 0;
+    for (int i = 0; i < w; ++i) before += wsum[i];
+    *total = wsum[0] + wsum[1] + wsum[2] + wsum[3];
+    return before + incl - v;
+}
+
+// List position j of (b, g) -> physical page (and logical page in lp), read
+// from the page table of the split that owns j (distributed shared memory;
+// splits of `per` positions), or from global memory when that split resolved
+// none.
+EKV_DEV int resolve_peer(const AttnArgs& a, int b, int g, int j, int P, int per, int& lp)
+{
+    const int q = j / per;
+    const int li = j - q * per;
+    if (li < ld_dsmem_s32(dsmem(&tab_n, q))) {
+        lp = ld_dsmem_s32(dsmem(&tab_lp[li], q));
+        return ld_dsmem_s32(dsmem(&tab_phys[li], q));
+    }
+    return resolve_g(a, b, g, j, P, lp, true);
+}
+
+template <int D, int PS, int NT>
+__global__ void __launch_bounds__(kThreads) entmax_bf16_kernel(const __grid_constant__ CUtensorMap kmap,
+                                                               const __grid_constant__ CUtensorMap vmap,
+                                                               const AttnArgs a)
+{
+    pdl_enter();
+    constexpr int NSTG = kFusedStages;
+    constexpr int STAGE = kStageTok * D * 2;
+    constexpr int PPS = kStageTok / PS;
+    constexpr int KS = D / 16;
+    constexpr int MTW = D / 64;            // 16-row m-tiles (head-dim rows) per warp in the V pass
+    constexpr int PROW = kStageTok + kPsPad;
+    constexpr int C = PS / 16;             // 16-token chunks per page
+    constexpr int WSCR = NSTG * STAGE / 4; // per-warp scratch (in the stage buffers) between the passes
+    constexpr int LC_CAP = WSCR / (8 * NT);// chunk-list entries per head (index + value)
+    constexpr int CAND_CAP = WSCR / 8;     // gathered candidates of the head being solved (value + position)
+    static_assert(kFusedMaxSplits <= 31, "split counts are held one per lane");
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = smem_align<1024>(smem_raw);
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + NSTG * STAGE);
+    uint16_t* ps_tile = reinterpret_cast<uint16_t*>(smem + NSTG * STAGE + 64);   // [8*NT][PROW]
+    float* part = reinterpret_cast<float*>(smem);                                // [G][D] after the V pass
+    __shared__ int abort_flag;
+    __shared__ float wm[4][8];
+    __shared__ float smax[8];
+    __shared__ float tau_s[8];
+    __shared__ int fallback;
+    __shared__ int wsum[4];
+    __shared__ int pre[4][kFusedMaxSplits + 1];
+    __shared__ int act[kActWin];
+    __shared__ int act_phys[kActWin];
+    __shared__ int act_lp[kActWin];
+    __shared__ unsigned char flag[kActWin];
+    __shared__ int nact;
+    __shared__ unsigned int bits[kBitWords];
+    // what this split publishes to the others (read through distributed shared memory)
+    __shared__ float pub_t[8], pub_m[8];
+    __shared__ int pub_n[8];
+    __shared__ float pub_val[8][kPubCap];
+    __shared__ int pub_pos[8][kPubCap];
+
+    const int b = blockIdx.z, g = blockIdx.y, s = blockIdx.x;   // s = rank in the cluster
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int L = a.seq_lens[b];
+    const int P = pages_of(L, PS, a.max_pages, a.status);
+    const int cnt = list_count(a, b, g, P);
+    const Range r = split_range(cnt, a.S, s);
+    const int per_split = (cnt + a.S - 1) / a.S;
+    const int nst = r.end > r.start ? (r.end - r.start + PPS - 1) / PPS : 0;
+    const size_t row0h = (size_t)b * a.H_q + (size_t)g * a.G;
+    const size_t xstride = (size_t)a.k_max * PS;
+    const size_t cstride = (size_t)a.k_max * C;
+    const uint32_t sbase = smem_addr(smem);
+    const bool a2 = a.alpha == 2.0f;
+    const bool a15 = a.alpha == 1.5f;
+    const double rpow = a2 ? 1.0 : (a15 ? 2.0 : 1.0 / ((double)a.alpha - 1.0));
+    tab_fill(a, b, g, r, P);
+
+    // ------------------------------------------------------------ K pass
+    if (tid == 0) {
+        abort_flag = 0;
+        fallback = 0;
+        prefetch_tmap(&kmap);
+        prefetch_tmap(&vmap);
+        for (int i = 0; i < NSTG; ++i) mbar_init(&bars[i], 1);
+        fence_mbar_init();
+        for (int st = 0; st < min(NSTG, nst); ++st)
+            issue_stage<D, PS>(a, &kmap, smem + st * STAGE, &bars[st], b, g, r, st, P);
+    }
+    for (int i = tid; i < kBitWords; i += kThreads) bits[i] = 0;
+    if (tid < 8) {
+        pub_t[tid] = -INFINITY;
+        pub_m[tid] = -INFINITY;
+        pub_n[tid] = 0;
+    }
+    float run[NT];
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) run[nt] = -INFINITY;
+    uint32_t bq[NT][KS][2];
+    load_q_frags<D, NT>(a, b, g, a.xscale, bq);
+    __syncthreads();
+    int kst = 0;
+    for (; kst < nst; ++kst) {
+        const int st = kst;
+        const int slot = st % NSTG;
+        if (!mbar_wait(&bars[slot], (st / NSTG) & 1, kWaitLimitNs)) {
+            abort_flag = 1;
+            report(a.status, ENTMAXKV_TIMEOUT);
+        }
+        __syncthreads();
+        if (abort_flag) break;
+        const uint32_t base = sbase + slot * STAGE;
+        const int row0 = warp * 16;
+        float acc[NT][4];
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0.f;
+        const int arow = row0 + (lane & 7) + ((lane >> 3) & 1) * 8;
+#pragma unroll
+        for (int j = 0; j < KS; ++j) {
+            uint32_t af[4];
+            ldsm_x4(swz_addr(base, arow, 2 * j + (lane >> 4)), af);
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) mma_bf16(acc[nt], af, bq[nt][j][0], bq[nt][j][1]);
+        }
+        // the warp's 16 rows lie in one page (16 divides PS): one list entry, one chunk
+        const int gi = lane >> 2, c = lane & 3;
+        const int idx = r.start + st * PPS + row0 / PS;
+        if (idx < r.end) {
+            int lp;
+            const int phys = resolve(a, b, g, idx, P, lp, false);
+            float cmx[NT];
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) cmx[nt] = -INFINITY;
+#pragma unroll
+            for (int rr = 0; rr < 2; ++rr) {
+                const int prow = (row0 + gi + 8 * rr) % PS;
+                const bool valid = phys >= 0 && lp * PS + prow < L;
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt) {
+                    const int head = 4 * nt + c;
+                    const float xv = valid ? acc[nt][2 * rr] + acc[nt][2 * rr + 1] : -INFINITY;
+                    cmx[nt] = fmaxf(cmx[nt], xv);
+                    if (head < a.G) a.xbuf[(row0h + head) * xstride + (size_t)idx * PS + prow] = xv;
+                }
+            }
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) {
+                const float m = group_lane_max(cmx[nt]);
+                run[nt] = fmaxf(run[nt], m);
+                const int head = 4 * nt + c;
+                if (gi == 0 && head < a.G)
+                    a.cmax[(row0h + head) * cstride + (size_t)idx * C + (row0 % PS) / 16] = m;
+            }
+        }
+        __syncthreads();
+        if (tid == 0 && st + NSTG < nst)
+            issue_stage<D, PS>(a, &kmap, smem + slot * STAGE, &bars[slot], b, g, r, st + NSTG, P);
+    }
+    if (abort_flag && tid == 0)   // copies still in flight must land before the buffers are reused
+        for (int k = kst; k < min(kst + NSTG, nst); ++k) mbar_wait(&bars[k % NSTG], (k / NSTG) & 1, kWaitLimitNs);
+    // this split's largest score per head
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+        const float m = group_lane_max(run[nt]);
+        if (lane < 4) wm[warp][4 * nt + (lane & 3)] = m;
+    }
+    __syncthreads();
+    if (tid < 8) smax[tid] = tid < a.G ? fmaxf(fmaxf(wm[0][tid], wm[1][tid]), fmaxf(wm[2][tid], wm[3][tid])) : -INFINITY;
+    __syncthreads();
+
+    // ------------------------------------------------------------ local bound and candidates
+    const int c0 = r.start * C, c1 = r.end * C;
+    if (!abort_flag) {
+        for (int h = warp, k = 0; h < a.G; h += 4, ++k) {
+            const size_t row = row0h + h;
+            int* lc = reinterpret_cast<int*>(smem + warp * WSCR + k * LC_CAP * 8);
+            float* lcv = reinterpret_cast<float*>(smem + warp * WSCR + k * LC_CAP * 8 + LC_CAP * 4);
+            int nlc;
+            const float t = split_bound(a.cmax + row * cstride, c0, c1, smax[h], rpow, a2, a15, lc, lcv, LC_CAP, &nlc);
+            const int n = local_candidates(a.xbuf + row * xstride, c0, c1, lc, lcv, nlc, LC_CAP, t, pub_val[h],
+                                           pub_pos[h]);
+            if (lane == 0) {
+                pub_t[h] = t;
+                pub_m[h] = smax[h];
+                pub_n[h] = n;
+            }
+        }
+    }
+    __threadfence();   // the scores in global memory are read by the other splits in the fallback
+    __syncthreads();
+    cluster_sync();
+
+    // ------------------------------------------------------------ threshold (every CTA, whole group)
+    const bool bitmap_ok = cnt <= kBitWords * 32;
+    if (!abort_flag) {
+        float* cv = reinterpret_cast<float*>(smem + warp * WSCR);
+        int* ci = reinterpret_cast<int*>(smem + warp * WSCR + CAND_CAP * 4);
+        for (int h = warp; h < a.G; h += 4) {
+            const size_t row = row0h + h;
+            float M = -INFINITY, tlb = -INFINITY;
+            int nq = 0;
+            if (lane < a.S) {
+                M = ld_dsmem_f32(dsmem(&pub_m[h], lane));
+                tlb = ld_dsmem_f32(dsmem(&pub_t[h], lane));
+                nq = ld_dsmem_s32(dsmem(&pub_n[h], lane));
+            }
+            M = warp_max(M);
+            tlb = warp_max(tlb);
+            const bool over = __any_sync(0xffffffffu, nq > kPubCap);
+            double tau;
+            int nc = -1;
+            if (!(M > -INFINITY)) {
+                tau = INFINITY;
+                nc = 0;
+            } else {
+                if (!over) nc = gather_candidates(pub_val[h], pub_pos[h], nq, a.S, tlb, cv, ci, CAND_CAP, pre[warp]);
+                if (nc >= 0) {
+                    TauSrc src{nullptr, 0, cv, nc, 0, (double)tlb};
+                    tau = solve_tau(src, M, a.alpha);
+                    // value pages holding weight: the pages of the candidates above tau
+                    if (bitmap_ok)
+                        for (int k = lane; k < nc; k += 32)
+                            if ((double)cv[k] > tau) {
+                                const int pg = ci[k] / PS;
+                                atomicOr(&bits[pg >> 5], 1u << (pg & 31));
+                            }
+                } else {
+                    // more candidates than the slots hold: every score of the head above the bound
+                    TauSrc src{a.xbuf + row * xstride, cnt * PS, nullptr, 0, 1, (double)tlb};
+                    tau = solve_tau(src, M, a.alpha);
+                    if (lane == 0) fallback = 1;
+                }
+            }
+            if (lane == 0) {
+                tau_s[h] = (float)tau;
+                if (s == 0 && a.tau_out) a.tau_out[row] = (float)tau;
+            }
+            __syncwarp();
+        }
+    }
+    if (tid < 8 && tid >= a.G) tau_s[tid] = INFINITY;
+    fence_proxy_async();   // the scratch writes above come before the V copies into the same buffers
+    __syncthreads();
+    const bool balanced = !fallback && bitmap_ok;
+
+    // ------------------------------------------------------------ V pass
+    const float rexp = 1.0f / (a.alpha - 1.0f);
+    float acc[NT][MTW][4];
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+        for (int m = 0; m < MTW; ++m) acc[nt][m][0] = acc[nt][m][1] = acc[nt][m][2] = acc[nt][m][3] = 0.f;
+    for (int i = tid; i < 8 * NT * PROW; i += kThreads) ps_tile[i] = 0;
+    int gst = nst;        // stages through the barriers so far (phase bookkeeping)
+    int loaded = 0;
+    const uint32_t pbase = smem_addr(ps_tile);
+    // balanced: the weighted pages in list order, CTA s taking ranks s, s + S, ...
+    // (windows of kActWin of them); otherwise the weighted pages of its own split
+    const int words = (cnt + 31) / 32;
+    const int wpt = (words + kThreads - 1) / kThreads;
+    int rank0 = 0, nw = 0, share = 0;
+    if (balanced) {
+        int mine = 0;
+        for (int w = tid * wpt; w < min(words, (tid + 1) * wpt); ++w) mine += __popc(bits[w]);
+        int tot;
+        rank0 = block_excl_scan128(mine, wsum, &tot);
+        share = tot > s ? (tot - s + a.S - 1) / a.S : 0;
+        nw = (share + kActWin - 1) / kActWin;
+    } else {
+        nw = (r.end - r.start + kActWin - 1) / kActWin;
+    }
+    for (int win = 0; win < nw && !abort_flag; ++win) {
+        if (balanced) {
+            // this CTA's entries [win * kActWin, ...) of its share: list positions of
+            // the weighted pages of rank s + j S
+            if (tid == 0) nact = min(kActWin, share - win * kActWin);
+            int rk = rank0;
+            for (int w = tid * wpt; w < min(words, (tid + 1) * wpt); ++w) {
+                unsigned m = bits[w];
+                while (m) {
+                    const int bit = __ffs(m) - 1;
+                    m &= m - 1;
+                    if (rk >= s && (rk - s) % a.S == 0) {
+                        const int j = (rk - s) / a.S - win * kActWin;
+                        if (j >= 0 && j < kActWin) act[j] = w * 32 + bit;
+                    }
+                    ++rk;
+                }
+            }
+            __syncthreads();
+            for (int i = tid; i < nact; i += kThreads) {
+                int lp;
+                act_phys[i] = resolve_peer(a, b, g, act[i], P, per_split, lp);
+                act_lp[i] = lp;
+            }
+        } else {
+            const int w0 = r.start + win * kActWin;
+            const int wn = min(kActWin, r.end - w0);
+            for (int i = tid; i < wn; i += kThreads) flag[i] = 0;
+            __syncthreads();
+            for (int it = tid; it < wn * a.G; it += kThreads) {
+                const int j = it / a.G, h = it % a.G;
+                const float* cp = a.cmax + (row0h + h) * cstride + (size_t)(w0 + j) * C;
+                float m = -INFINITY;
+#pragma unroll
+                for (int k = 0; k < C; ++k) m = fmaxf(m, cp[k]);
+                if (m > tau_s[h]) flag[j] = 1;
+            }
+            __syncthreads();
+            if (warp == 0) {   // ordered compaction of the flags
+                int base = 0;
+                for (int i0 = 0; i0 < wn; i0 += 32) {
+                    const bool f = (i0 + lane < wn) && flag[i0 + lane];
+                    const unsigned m = __ballot_sync(0xffffffffu, f);
+                    if (f) act[base + __popc(m & ((1u << lane) - 1u))] = w0 + i0 + lane;
+                    base += __popc(m);
+                }
+                if (lane == 0) nact = base;
+            }
+            __syncthreads();
+            for (int i = tid; i < nact; i += kThreads) {
+                int lp;
+                act_phys[i] = resolve(a, b, g, act[i], P, lp, true);
+                act_lp[i] = lp;
+            }
+        }
+        __syncthreads();
+        const int na = nact;
+        loaded += na;
+        const int nsv = (na + PPS - 1) / PPS;
+        auto issue = [&](int st, int slot_) {
+            uint8_t* dst = smem + slot_ * STAGE;
+            uint32_t bytes = 0;
+#pragma unroll
+            for (int i = 0; i < PPS; ++i) {
+                const int ai = st * PPS + i;
+                if (ai < na && act_phys[ai] >= 0) bytes += PS * D * 2;
+            }
+            mbar_arrive_expect_tx(&bars[slot_], bytes);
+#pragma unroll
+            for (int i = 0; i < PPS; ++i) {
+                const int ai = st * PPS + i;
+                if (ai >= na || act_phys[ai] < 0) continue;
+                const int y = (act_phys[ai] * a.H_kv + g) * PS;
+#pragma unroll
+                for (int hh = 0; hh < D / 64; ++hh)
+                    tma_load_2d(dst + hh * (kStageTok * 128) + i * PS * 128, &vmap, &bars[slot_], hh * 64, y);
+            }
+        };
+        if (tid == 0)
+            for (int st = 0; st < min(NSTG, nsv); ++st) issue(st, (gst + st) % NSTG);
+        int st = 0;
+        for (; st < nsv; ++st) {
+            const int gs = gst + st;
+            const int slot = gs % NSTG;
+            const int t = tid & (kStageTok - 1);
+            const int ai = st * PPS + t / PS;
+            const bool valid = ai < na && act_phys[ai] >= 0 && act_lp[ai] * PS + (t % PS) < L;
+            {   // weights of this stage: token tid % 64, heads (tid / 64) * 2 * NT ...
+                const int hbase = (tid >> 6) * 2 * NT;
+#pragma unroll
+                for (int k = 0; k < 2 * NT; ++k) {
+                    const int head = hbase + k;
+                    float p = 0.f;
+                    if (head < a.G && valid) {
+                        const float xv = __ldcg(a.xbuf + (row0h + head) * xstride + (size_t)act[ai] * PS + t % PS);
+                        const float u = fmaxf(xv - tau_s[head], 0.f);
+                        p = a2 ? u : (a15 ? u * u : powf(u, rexp));
+                    }
+                    uint32_t hi, lo;
+                    split_bf16(p, hi, lo);
+                    ps_tile[(2 * head) * PROW + t] = (uint16_t)hi;
+                    ps_tile[(2 * head + 1) * PROW + t] = (uint16_t)lo;
+                }
+            }
+            if (!mbar_wait(&bars[slot], (gs / NSTG) & 1, kWaitLimitNs)) {
+                abort_flag = 1;
+                report(a.status, ENTMAXKV_TIMEOUT);
+            }
+            __syncthreads();
+            if (abort_flag) break;
+            // rows without a valid token are zeroed so zero weights never meet garbage
+            if ((tid >> 6) < D / 64 && !valid) {
+                uint4* rowp = reinterpret_cast<uint4*>(smem + slot * STAGE + (tid >> 6) * (kStageTok * 128) + t * 128);
+#pragma unroll
+                for (int k = 0; k < 8; ++k) rowp[k] = make_uint4(0, 0, 0, 0);
+                fence_proxy_async();
+            }
+            __syncthreads();
+            const uint32_t base = sbase + slot * STAGE;
+            const int n = lane >> 2, c = lane & 3;
+#pragma unroll
+            for (int kk = 0; kk < kStageTok / 16; ++kk) {
+                uint32_t b0[NT], b1[NT];
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt) {
+                    const uint32_t pr = pbase + ((8 * nt + n) * PROW + 16 * kk + 2 * c) * 2;
+                    asm volatile("ld.shared.b32 %0, [%1];" : "=r"(b0[nt]) : "r"(pr));
+                    asm volatile("ld.shared.b32 %0, [%1];" : "=r"(b1[nt]) : "r"(pr + 16));
+                }
+                const int mi = lane >> 3;
+                const int trow = 16 * kk + (lane & 7) + 8 * (mi >> 1);
+#pragma unroll
+                for (int m = 0; m < MTW; ++m) {
+                    const int d0 = 16 * (warp * MTW + m);
+                    uint32_t af[4];
+                    ldsm_x4_t(swz_addr(base, trow, d0 / 8 + (mi & 1)), af);
+#pragma unroll
+                    for (int nt = 0; nt < NT; ++nt) mma_bf16(acc[nt][m], af, b0[nt], b1[nt]);
+                }
+            }
+            __syncthreads();
+            if (tid == 0 && st + NSTG < nsv) issue(st + NSTG, (gs + NSTG) % NSTG);
+        }
+        if (abort_flag && tid == 0)   // copies still in flight must land before the CTA moves on
+            for (int k = st; k < min(st + NSTG, nsv); ++k)
+                mbar_wait(&bars[(gst + k) % NSTG], ((gst + k) / NSTG) & 1, kWaitLimitNs);
+        gst += nsv;
+        __syncthreads();   // act and nact are rebuilt by the next window
+    }
+    if (tid == 0 && a.vpages) atomicAdd(&a.vpages[(size_t)b * a.H_kv + g], loaded);
+    // partial output of this CTA into shared memory (every copy has landed or
+    // been waited out above): part[head 4nt + c][d]
+    __syncthreads();
+    {
+        const int c = lane & 3, gi = lane >> 2;
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+            const int head = 4 * nt + c;
+            if (head >= a.G) continue;
+#pragma unroll
+            for (int m = 0; m < MTW; ++m) {
+                const int d = 16 * (warp * MTW + m) + gi;
+                part[head * D + d] = acc[nt][m][0] + acc[nt][m][1];
+                part[head * D + d + 8] = acc[nt][m][2] + acc[nt][m][3];
+            }
+        }
+    }
+    __syncthreads();
+    cluster_sync();
+
+    // ------------------------------------------------------------ merge
+    const int E = a.G * D;
+    const int per = (E + a.S - 1) / a.S;
+    for (int e = s * per + tid; e < min(E, (s + 1) * per); e += kThreads) {
+        const int head = e / D, dd = e % D;
+        float sum = 0.f;
+        for (int q = 0; q < a.S; ++q) sum += ld_dsmem_f32(dsmem(part + e, q));
+        a.out[(row0h + head) * D + dd] = sum;
+    }
+    cluster_sync();       // no CTA leaves while another may still read its shared memory
 }
 
 // ====================================================================== softmax
@@ -1321,21 +1778,28 @@ __global__ void selftest_timeout_kernel(uint64_t limit_ns, int32_t* status)
 }
 
 // ====================================================================== launch
+// Splits of the fused kernel: the largest power of two up to 16 that the list
+// length and two CTAs per SM allow, and that the device can place as one
+// cluster with the kernel's resources.
+static int fused_splits(const void* kern, int smem, int units, int list)
+{
+    int S = kFusedMaxSplits;
+    while (S > 1 && (S > list || (long long)units * S > 2ll * num_sms())) S >>= 1;
+    while (S > 1 && max_active_clusters(kern, S, kThreads, smem) < 1) S >>= 1;
+    return S;
+}
+
 template <int D, int PS, int NT>
-static int launch_entmax_bf16(const AttnArgs& a, int B, const CUtensorMap* kmap, const CUtensorMap* vmap,
+static int launch_entmax_bf16(const AttnArgs& a0, int B, const CUtensorMap* kmap, const CUtensorMap* vmap,
                               cudaStream_t stream)
 {
-    dim3 grid(a.S, a.H_kv, B);
-    const int qk_smem = kStagesQK * kStageTok * D * 2 + 1024 + 64;
-    const int pv_smem = kStagesPV * kStageTok * D * 2 + 1024 + 64 + 8 * NT * (kStageTok + kPsPad) * 2;
-    if (ensure_smem((const void*)qk_bf16_kernel<D, PS, NT>, qk_smem)) return ENTMAXKV_CUDA_ERROR;
-    if (ensure_smem((const void*)pv_bf16_kernel<D, PS, NT>, pv_smem)) return ENTMAXKV_CUDA_ERROR;
-    launch_pdl(qk_bf16_kernel<D, PS, NT>, dim3(grid), dim3(kThreads), qk_smem, stream, *kmap, a);
-    if (cudaGetLastError() != cudaSuccess) return ENTMAXKV_CUDA_ERROR;
-    if (ensure_smem((const void*)tau_kernel, kTauSmem)) return ENTMAXKV_CUDA_ERROR;
-    launch_pdl(tau_kernel, dim3(dim3(a.H_q, B)), dim3(kTauBlock), kTauSmem, stream, PS, a);
-    if (cudaGetLastError() != cudaSuccess) return ENTMAXKV_CUDA_ERROR;
-    launch_pdl(pv_bf16_kernel<D, PS, NT>, dim3(grid), dim3(kThreads), pv_smem, stream, *vmap, a);
+    const void* kern = (const void*)entmax_bf16_kernel<D, PS, NT>;
+    const int smem = kFusedStages * kStageTok * D * 2 + 1024 + 64 + 8 * NT * (kStageTok + kPsPad) * 2;
+    if (ensure_cluster_kernel(kern, smem)) return ENTMAXKV_CUDA_ERROR;
+    AttnArgs a = a0;
+    a.S = fused_splits(kern, smem, B * a.H_kv, a.k_max);   // <= the workspace layout's split count
+    launch_pdl_cluster(entmax_bf16_kernel<D, PS, NT>, dim3(a.S, a.H_kv, B), dim3(kThreads), a.S, smem, stream,
+                       *kmap, *vmap, a);
     return cudaGetLastError() == cudaSuccess ? ENTMAXKV_OK : ENTMAXKV_CUDA_ERROR;
 }
 

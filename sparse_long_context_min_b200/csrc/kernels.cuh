@@ -12,6 +12,11 @@
 
 namespace ekv {
 
+// The fused bf16 entmax kernel runs at most kFusedMaxSplits splits per (sequence,
+// kv head), each publishing up to kFusedCandCap threshold candidates per query head.
+constexpr int kFusedMaxSplits = 16;
+constexpr int kFusedCandCap = 256;
+
 // Arguments shared by the attention kernels (passed by value).
 struct AttnArgs {
     const float* q;                // [B][H_q][d]
@@ -34,6 +39,10 @@ struct AttnArgs {
     float* lmax;                   // [B][H_q][S] largest score of each split (K pass)
     int32_t* vpages;               // [B][H_kv] value pages loaded (V pass adds), or NULL
     int32_t* counters;             // [B][H_kv] arrival counters of the split reduction
+    float* lbound;                 // [B][H_q][S] each split's lower bound of tau (fused bf16 kernel)
+    int32_t* ccnt;                 // [B][H_q][S] each split's candidate count (fused bf16 kernel)
+    float* cval;                   // [B][H_q][S][kFusedCandCap] candidate scores (fused bf16 kernel)
+    int32_t* cidx;                 // [B][H_q][S][kFusedCandCap] their list positions (fused bf16 kernel)
     float* out;                    // [B][H_q][d]
     float* tau_out;                // [B][H_q] or NULL
     int32_t* status;
@@ -59,6 +68,12 @@ int launch_entmax_attend(const entmaxkv_pool& pool, const AttnArgs& a, int B, co
 int launch_softmax_attend(const entmaxkv_pool& pool, const AttnArgs& a, int B, const CUtensorMap* kmap,
                           const CUtensorMap* vmap, cudaStream_t stream);
 
+// Host-side argument checks of the attention entry points (op: entmaxkv_op),
+// everything but the workspace; ENTMAXKV_OK when the call may proceed.
+int attend_check(int op, const entmaxkv_pool* pool, const float* q, int H_q, const int32_t* page_table,
+                 int max_pages, const int32_t* seq_lens, int B, const int32_t* sel, const int32_t* sel_count,
+                 int k_max, float alpha, float scale, const float* out, const int32_t* status);
+
 int launch_selftest_timeout(int64_t limit_ns, int32_t* status, cudaStream_t stream);
 
 // set the dynamic shared memory limit of a kernel once per device
@@ -66,6 +81,14 @@ int ensure_smem(const void* func, int bytes);
 
 // SM count of the current device
 int num_sms();
+
+// Dynamic shared memory limit and permission for clusters above 8 CTAs of a
+// cluster kernel, once per device.
+int ensure_cluster_kernel(const void* func, int smem);
+
+// Clusters of `cluster` CTAs (threads, smem each) the current device can run
+// at once (0 when none fits); cached per (kernel, size, device).
+int max_active_clusters(const void* func, int cluster, int threads, int smem);
 
 // Launch with programmatic stream serialization (the kernel calls pdl_enter()).
 template <typename... KArgs, typename... Args>

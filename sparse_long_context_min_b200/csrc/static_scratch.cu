@@ -53,8 +53,11 @@ int entmaxkv_sparse_attend_static(const entmaxkv_pool* pool, const float* q, int
                                   float alpha, float scale, float* out, float* tau_out, int32_t* v_pages,
                                   int32_t* status, void* stream)
 {
-    if (!pool || B < 0 || k_max <= 0 || max_pages <= 0) return ENTMAXKV_INVALID_ARG;
-    if (B == 0) return ENTMAXKV_OK;
+    // the argument checks of entmaxkv_sparse_attend come first, so a bad call
+    // gets the same code from both entry points whatever its size
+    const int rc = ekv::attend_check(ENTMAXKV_OP_SPARSE_ATTEND, pool, q, H_q, page_table, max_pages, seq_lens, B,
+                                     sel, sel_count, k_max, alpha, scale, out, status);
+    if (rc || B == 0) return rc;
     const size_t need = entmaxkv_workspace_size(ENTMAXKV_OP_SPARSE_ATTEND, B, H_q, pool->H_kv, max_pages, k_max,
                                                 pool->ps, pool->d);
     if (need == 0) return ENTMAXKV_INVALID_ARG;

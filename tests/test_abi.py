@@ -71,9 +71,9 @@ def test_host_validation_without_gpu():
                                             ctypes.c_void_p(16), 1, None, None, 4, 0.1, ctypes.c_void_p(16),
                                             ctypes.c_void_p(256), 1 << 20, st, None)
     assert rc == B.INVALID_ARG           # no page list
-    rc = lib.entmaxkv_select(B.SELECT_GAUSS, None, None, None, None, None, 64, 1, 32, 8, 100, -1, 0.0, 1.1,
+    rc = lib.entmaxkv_select(B.SELECT_GAUSS, None, None, None, None, None, 64, 1, 32, 8, 100, -1, 0.0, 1.02,
                              0.5, 100, None, None, None, None, 0, st, None)
-    assert rc == B.UNSUPPORTED           # the Gaussian selector's quadrature covers alpha >= 1.25
+    assert rc == B.UNSUPPORTED           # the Gaussian selector's quadrature covers alpha >= 1.05
     rc = lib.entmaxkv_full_entmax_decode(ctypes.byref(pool), ctypes.c_void_p(16), 32, ctypes.c_void_p(16), 10,
                                          ctypes.c_void_p(16), 1, 1.0, 0.1, ctypes.c_void_p(16), None, None,
                                          ctypes.c_void_p(256), 1 << 20, st, None)
@@ -86,3 +86,30 @@ def test_empty_batch_is_a_noop(B_):
     pool = B.CPool(16, 16, 16, 16, 16, 16, 16, 10, 8, 64, 128, B.BF16)
     rc = lib.entmaxkv_append_metadata(ctypes.byref(pool), None, None, 1, None, 10, None, B_, None, None)
     assert rc == B.OK
+
+
+def test_static_entry_checks_arguments_before_its_size():
+    """entmaxkv_sparse_attend_static runs entmaxkv_sparse_attend's argument
+    checks before comparing the problem with its built-in buffer, so a bad
+    call gets the same code from both entry points; a valid oversized call is
+    refused with ENTMAXKV_STATIC_LIMIT.  Nothing here reaches the GPU."""
+    lib = B.lib()
+    st = ctypes.c_void_p(16)
+    pool = B.CPool(16, 16, 16, 16, 16, 16, 16, 10, 8, 64, 128, B.BF16)
+    Bn, H_q, max_pages, k_max = 64, 32, 20000, 20000       # far beyond the buffer
+    assert B.workspace_size(B.OP_SPARSE_ATTEND, Bn, H_q, 8, max_pages, k_max, 64, 128) > B.STATIC_SCRATCH_BYTES
+
+    def call(alpha=1.5, scale=0.088, H=H_q, sel=ctypes.c_void_p(16), out=ctypes.c_void_p(16)):
+        return lib.entmaxkv_sparse_attend_static(ctypes.byref(pool), ctypes.c_void_p(16), H, ctypes.c_void_p(16),
+                                                 max_pages, ctypes.c_void_p(16), Bn, sel, ctypes.c_void_p(16),
+                                                 k_max, ctypes.c_float(alpha), ctypes.c_float(scale), out, None,
+                                                 None, st, None)
+
+    assert call(alpha=1.0) == B.UNSUPPORTED                 # alpha-entmax needs alpha > 1
+    assert call(alpha=20.0) == B.UNSUPPORTED
+    assert call(scale=-1.0) == B.INVALID_ARG
+    assert call(H=30) == B.INVALID_ARG                       # 30 query heads over 8 kv heads
+    assert call(H=24) == B.UNSUPPORTED                       # group of 3
+    assert call(sel=None) == B.INVALID_ARG                   # no page list
+    assert call(out=None) == B.INVALID_ARG
+    assert call() == B.STATIC_LIMIT
