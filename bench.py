@@ -41,15 +41,21 @@ MiB = 1 << 20
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
-    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--steps", type=int, default=1000)
+    ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--context", type=int, default=1 << 20, help="tokens per sequence (default 2^20)")
     ap.add_argument("--no-baselines", action="store_true", help="skip the full-cache and Gaussian timings")
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline leg")
+    ap.add_argument("--no-configs", action="store_true",
+                    help="skip the per-configuration legs (configurations 2, 3 and 5 at their sizes)")
     ap.add_argument("--replay-only", choices=["topk", "gauss"], default=None,
                     help="build the workload, capture that step as a graph and replay it --steps times "
                          "without timing (a short program for profiler launch lists)")
+    ap.add_argument("--oracle-leg", action="store_true",
+                    help="time the CPU oracle on this host's cores and print one JSON line (no GPU)")
+    ap.add_argument("--leg-seconds", type=float, default=8.0,
+                    help="time budget of each part of the oracle leg (seconds)")
     return ap.parse_args()
 
 
@@ -234,11 +240,24 @@ def score_bytes(cfg, mode):
     return algorithmic_bytes(cfg, 0, 0, mode)["score"]
 
 
-N_LAUNCH = 6   # per step: append (one token, no separate length kernel), score, top-k, qk, tau, pv
+N_LAUNCH = 4   # per step: append (one token, advances the length itself), score, top-k, fused attention
+
+
+def roofline_entry(kernel, nbytes, us, peak, traffic=None, note=None):
+    """{bound, achieved, peak, unit, frac, traffic} of a kernel moving `nbytes`
+    algorithmic bytes in `us` microseconds, against the copy peak (GB/s)."""
+    peak_gbs, peak_kind = peak
+    achieved = nbytes / (us * 1e-6) / 1e9
+    e = {"kernel": kernel, "bound": "hbm", "achieved": round(achieved, 1), "peak": peak_gbs, "peak_kind": peak_kind,
+         "unit": "GB/s", "frac": round(achieved / peak_gbs, 4), "frac_of_8tbs": round(achieved / HBM_NOMINAL_GBS, 4),
+         "traffic": traffic, "bytes_per_launch": nbytes}
+    if note:
+        e["traffic_note"] = note
+    return e
 
 
 def native_line(cfg, world, K, W, mean_us, best_us, median_us, score_us, stage, sel_total, v_total, extra, e2e,
-                clk, cpu, peak):
+                clk, cpu, peak, attend_us=None):
     """The native arm's JSON line from the measured numbers (times are the
     max over ranks; e2e = (us per step, H2D bytes, D2H bytes); peak = (GB/s,
     "measured" or "fallback"))."""
@@ -246,7 +265,6 @@ def native_line(cfg, world, K, W, mean_us, best_us, median_us, score_us, stage, 
     peak_gbs, peak_kind = peak
     e2e_us, h2d, d2h = e2e
     step_gbs = by["total"] / (mean_us * 1e-6) / 1e9
-    score_gbs = by["score"] / (score_us * 1e-6) / 1e9
     line = {
         "metric": METRIC,
         "value": round(mean_us, 2),
@@ -278,98 +296,105 @@ def native_line(cfg, world, K, W, mean_us, best_us, median_us, score_us, stage, 
             "stage_note": "stage_us from a graph with event nodes between stages (no overlap across them)",
             **extra,
         },
-        "roofline": {
-            "kernel": "score_box16_kernel (entmaxkv_score_pages, bbox, bf16)",
-            "bound": "hbm",
-            "achieved": round(score_gbs, 1),
-            "peak": peak_gbs,
-            "peak_kind": peak_kind,
-            "unit": "GB/s",
-            "frac": round(score_gbs / peak_gbs, 4),
-            "traffic": round(SCORE_DRAM_BYTES_PER_ROW * sum(cfg.pages(b) for b in range(cfg.B)) * cfg.H_kv),
-            "traffic_note": "ncu dram__bytes_read+write of the 2^18-token case scaled by rows",
-            "bytes_per_launch": by["score"],
-        },
+        "roofline": roofline_entry("score_box16_kernel (entmaxkv_score_pages, bbox, bf16)", by["score"], score_us,
+                                   peak, round(SCORE_DRAM_BYTES_PER_ROW * sum(cfg.pages(b) for b in range(cfg.B))
+                                               * cfg.H_kv),
+                                   "ncu dram__bytes_read+write of the 2^18-token case scaled by rows"),
         "e2e": {"value": round(e2e_us, 2), "unit": "us/step", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h},
         "gpu_launches": N_LAUNCH * K,
         "clocks": clk,
     }
+    if attend_us:
+        line["roofline_attend"] = roofline_entry(
+            "entmax_bf16_kernel (entmaxkv_sparse_attend: K pass, threshold, V pass)", by["attend"], attend_us, peak,
+            None, "keys of the selected page-heads plus values of those holding weight")
     if cpu is not None:
         line["cpu_baseline"] = cpu
     return line
 
 
 # ---------------------------------------------------------------- native arm
+def timed_replays(gs, step, toks, warm, steps, flush, stream, stages=False):
+    """`warm` + `steps` replays of a graphed step, issued back to back with no
+    host synchronisation: per step the step's inputs are copied in (device to
+    device), the L2 is flushed (256 MiB write) and the replay is bracketed by
+    CUDA events on the stream; the selected and loaded-value page counts add up
+    on the device.  Returns (per-step us, mean selected page-heads, mean value
+    page-heads, mean stage us or None)."""
+    sel_acc = torch.zeros((), dtype=torch.int64, device="cuda")
+    vp_acc = torch.zeros((), dtype=torch.int64, device="cuda")
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    stage_sum = None
+    for i in range(warm + steps):
+        k, v, q = toks[i]
+        gs.q.copy_(q)
+        gs.k.copy_(k)
+        gs.v.copy_(v)
+        step.v_pages.zero_()
+        flush.fill_(i & 0xFF)
+        j = i - warm
+        if j >= 0:
+            ev[j][0].record(stream)
+        gs.replay()
+        if j >= 0:
+            ev[j][1].record(stream)
+            sel_acc += step.sel_count.sum()
+            vp_acc += step.v_pages.sum()
+            if stages:   # event nodes of the instrumented graph: read after each replay
+                torch.cuda.synchronize()
+                st = gs.stage_us()
+                stage_sum = dict(st) if stage_sum is None else {n: stage_sum[n] + st[n] for n in st}
+    torch.cuda.synchronize()
+    step.check()
+    us = [a.elapsed_time(b) * 1e3 for a, b in ev]
+    stage = {n: x / steps for n, x in stage_sum.items()} if stage_sum else None
+    return us, sel_acc.item() / steps, vp_acc.item() / steps, stage
+
+
+def decode_tokens(wl, first, n):
+    return [wl.decode_token(first + i) for i in range(n)]
+
+
 def run_native(args, rank, world, local):
-    import numpy as np
-    from sparse_long_context_min_b200 import binding as BND
     from sparse_long_context_min_b200.step import DecodeStep, GraphedStep, build_pool
 
     torch.manual_seed(0)
-    # tokens appended during the run: top-k (two graphs) + e2e + Gaussian (two graphs)
-    appends = 3 * (args.steps + args.warmup) + 2 * (max(3, args.steps // 4) + 3) + 64
+    K, W = args.steps, args.warmup
+    Ks = min(K, 200)                         # replays of the instrumented graph (stage breakdown)
+    Kg = min(K, 200)                         # Gaussian-selector replays
+    # tokens appended during the run: the top-k graphs, the e2e leg, the Gaussian graph
+    appends = (W + K) + (W + Ks) + (W + K) + (W + Kg) + 64
     wl = make_workload(args.context, rank, appends=appends)
     cfg = wl.cfg
     pool, seq_lens = build_pool(wl)
     torch.cuda.synchronize()
     stream = torch.cuda.current_stream()
     flush = torch.empty(256 * MiB, dtype=torch.uint8, device="cuda")
-    K, W = args.steps, args.warmup
-    total_steps = W + K
 
-    def one_mode(mode, budget_frac=1 / 64, delta=0.5, steps=None, warm=None):
-        """K graphed steps timed with events around each replay (plain graph, so
-        kernels overlap across stage boundaries), then K replays of a graph with
-        event nodes between stages for the per-stage breakdown.  Returns per-step
-        us, mean stage us, mean selected and loaded-value page-heads per step."""
-        steps = K if steps is None else steps
-        warm = W if warm is None else warm
-        st = DecodeStep(pool, wl.page_table, seq_lens, cfg.H_q, mode, budget_frac=budget_frac, alpha=cfg.alpha,
-                        delta=delta)
-        plain = GraphedStep(st, append=True, stage_events=False)
-        inst = GraphedStep(st, append=True, stage_events=True)
-        toks = [wl.decode_token(i) for i in range(2 * (warm + steps))]
-        e0 = torch.cuda.Event(enable_timing=True)
-        e1 = torch.cuda.Event(enable_timing=True)
-        step_us, stages, sel, vp = [], [], [], []
-        for phase, gs in (("step", plain), ("stages", inst)):
-            for i in range(warm + steps):
-                k, v, q = toks[(0 if phase == "step" else warm + steps) + i]
-                gs.q.copy_(q)
-                gs.k.copy_(k)
-                gs.v.copy_(v)
-                st.v_pages.zero_()
-                flush.fill_(i & 0xFF)
-                e0.record(stream)
-                gs.replay()
-                e1.record(stream)
-                torch.cuda.synchronize()
-                if i < warm:
-                    continue
-                if phase == "step":
-                    step_us.append(e0.elapsed_time(e1) * 1e3)
-                    sel.append(int(st.sel_count.sum().item()))
-                    vp.append(int(st.v_pages.sum().item()))
-                else:
-                    stages.append(gs.stage_us())
-        st.check()
-        stage = {n: statistics.mean(x[n] for x in stages) for n in GraphedStep.STAGES} if stages[0] else {}
-        return step_us, stage, statistics.mean(sel), statistics.mean(vp)
-
-    # ---- headline: top-k 1/64, timed K steps bracketed by barrier + sync
-    clocks = Clocks(local)
+    # ---- headline: top-k 1/64, K graphed steps bracketed by barrier + sync
+    step = DecodeStep(pool, wl.page_table, seq_lens, cfg.H_q, "topk", budget_frac=1 / 64, alpha=cfg.alpha)
+    plain = GraphedStep(step, append=True, stage_events=False)
+    inst = GraphedStep(step, append=True, stage_events=True)
+    toks = decode_tokens(wl, 0, W + K)
+    clocks = Clocks(local, interval_ms=10)
     barrier(world)
     torch.cuda.synchronize()
     with clocks:
-        step_us, stage, sel_total, v_total = one_mode("topk")
+        step_us, sel_total, v_total, _ = timed_replays(plain, step, toks, W, K, flush, stream)
     torch.cuda.synchronize()
     barrier(world)
     mean_us = statistics.mean(step_us)
     mean_us_all = max_over_ranks(mean_us, world)
     best_us_all = max_over_ranks(min(step_us), world)
     median_us_all = max_over_ranks(statistics.median(step_us), world)
+    del toks
+    # stage breakdown from the instrumented graph (outside the timed region)
+    toks = decode_tokens(wl, W + K, W + Ks)
+    _, _, _, stage = timed_replays(inst, step, toks, W, Ks, flush, stream, stages=True)
+    del toks
     score_us = max_over_ranks(stage["score"], world)
+    attend_us = max_over_ranks(stage["attend"], world)
 
     # ---- e2e through the C ABI with host buffers (copies inside the timed region)
     e2e_us, h2d, d2h = run_e2e(wl, pool, seq_lens, K, W, flush)
@@ -377,11 +402,14 @@ def run_native(args, rank, world, local):
 
     extra = {}
     if not args.no_baselines:
-        g_us, g_stage, g_sel, g_v = one_mode("gauss", steps=max(3, K // 4), warm=3)
+        gstep = DecodeStep(pool, wl.page_table, seq_lens, cfg.H_q, "gauss", alpha=cfg.alpha, delta=0.5)
+        ggraph = GraphedStep(gstep, append=True, stage_events=False)
+        toks = decode_tokens(wl, 3 * (W + K), W + Kg)
+        g_us, g_sel, g_v, _ = timed_replays(ggraph, gstep, toks, W, Kg, flush, stream)
+        del toks, ggraph
         extra["gauss_value_pages"] = round(g_v, 1)
         extra["gauss_us_per_step"] = round(max_over_ranks(statistics.mean(g_us), world), 2)
         extra["gauss_selected_pages"] = round(g_sel, 1)
-        extra["gauss_stage_us"] = {k: round(v, 2) for k, v in g_stage.items()}
         fe, fs = run_full(wl, pool, seq_lens, flush)
         fe, fs = max_over_ranks(fe, world), max_over_ranks(fs, world)
         extra["full_entmax_us"] = round(fe, 1)
@@ -394,13 +422,17 @@ def run_native(args, rank, world, local):
                       for k, v in run_attend_variants(wl, pool, seq_lens, flush).items()})
         extra["attend_variants_note"] = ("eager calls between events on one top-k 1/64 selection; "
                                          "include launch latency not hidden by a graph")
+    del pool
+    torch.cuda.empty_cache()
+    if world == 1 and not args.no_configs:
+        extra["per_config"] = config_legs(flush, W, min(K, 200), hbm_peak())
 
     cpu = None
     if rank == 0 and not args.no_cpu:
-        cpu = cpu_baseline(wl, pool, budget_frac=1 / 64, seconds=8.0)
+        cpu = cpu_baseline_subprocess(args.context, args.leg_seconds)
 
     line = native_line(cfg, world, K, W, mean_us_all, best_us_all, median_us_all, score_us, stage, sel_total,
-                       v_total, extra, (e2e_us, h2d, d2h), clocks.summary(), cpu, hbm_peak())
+                       v_total, extra, (e2e_us, h2d, d2h), clocks.summary(), cpu, hbm_peak(), attend_us)
     if rank == 0:
         print(json.dumps(line), flush=True)
 
@@ -408,7 +440,7 @@ def run_native(args, rank, world, local):
 def run_e2e(wl, pool, seq_lens, K, W, flush):
     """Same step through the public API (the graphed step) with the step's
     inputs in pinned host memory: one H2D copy of q and the new token (packed
-    by GraphedStep.pack_host); the result is written by the attention kernels
+    by GraphedStep.pack_host); the result is written by the attention kernel
     straight into pinned host memory (the D2H transfer of the output) inside
     the events."""
     from sparse_long_context_min_b200.step import DecodeStep, GraphedStep
@@ -420,7 +452,7 @@ def run_e2e(wl, pool, seq_lens, K, W, flush):
     gs = GraphedStep(st, append=True, stage_events=False)
     host = []
     for i in range(W + K):
-        k, v, q = wl.decode_token(10_000 + i)
+        k, v, q = wl.decode_token(1_000_000 + i)
         host.append(gs.pack_host(k, v, q))
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
     for i in range(W + K):
@@ -517,69 +549,208 @@ def run_attend_variants(wl, pool, seq_lens, flush, reps=5, warm=3):
     return res
 
 
+def config_legs(flush, W, steps, peak):
+    """One-GPU timings of the other benchmark configurations at their stated
+    sizes, each step graphed with its token append and the L2 flushed between
+    steps: configuration 2 (131072 tokens, top-k budgets of 64, 128 and 256
+    pages), 3 (B = 4 x 262144 tokens, Gaussian selector, alpha in {1.5, 2},
+    Delta in {0, 0.5, 1}) and 5 (ragged B = 1, 8, 32, top-k 1/16).  Per leg:
+    us per step, algorithmic bytes, GB/s and the fraction of the copy peak."""
+    import dataclasses
+    from sparse_long_context_min_b200 import workloads
+    from sparse_long_context_min_b200.step import DecodeStep, GraphedStep, build_pool
+    stream = torch.cuda.current_stream()
+    peak_gbs = peak[0]
+    out = {}
+
+    def leg(wl, pool, seq_lens, name, mode, first, **kw):
+        cfg = wl.cfg
+        st = DecodeStep(pool, wl.page_table, seq_lens, cfg.H_q, mode, alpha=kw.pop("alpha", cfg.alpha), **kw)
+        gs = GraphedStep(st, append=True, stage_events=False)
+        toks = decode_tokens(wl, first, W + steps)
+        us, sel, vp, _ = timed_replays(gs, st, toks, W, steps, flush, stream)
+        mean = statistics.mean(us)
+        by = algorithmic_bytes(cfg, sel, vp, mode)["total"]
+        gbs = by / (mean * 1e-6) / 1e9
+        out[name] = {"us_per_step": round(mean, 2), "selected_page_heads": round(sel, 1),
+                     "value_page_heads": round(vp, 1), "algorithmic_bytes": int(by), "gbs": round(gbs, 1),
+                     "frac_of_measured_hbm": round(gbs / peak_gbs, 4), "frac_of_8tbs": round(gbs / HBM_NOMINAL_GBS, 4)}
+        del gs, st, toks
+
+    per = W + steps
+    c2 = workloads.config(2)
+    wl = workloads.Workload(dataclasses.replace(c2, decode_steps=3 * per + 64), device="cuda")
+    pool, lens = build_pool(wl)
+    for i, budget in enumerate(c2.budgets):
+        leg(wl, pool, lens, "config2_topk_%d_pages" % budget, "topk", i * per, budget=budget)
+    del wl, pool, lens
+    torch.cuda.empty_cache()
+    c3 = workloads.config(3)
+    wl = workloads.Workload(dataclasses.replace(c3, decode_steps=6 * per + 64), device="cuda")
+    pool, lens = build_pool(wl)
+    i = 0
+    for alpha in c3.alphas:
+        for delta in c3.deltas:
+            leg(wl, pool, lens, "config3_gauss_alpha%g_delta%g" % (alpha, delta), "gauss", i * per, alpha=alpha,
+                delta=delta)
+            i += 1
+    del wl, pool, lens
+    torch.cuda.empty_cache()
+    for B in (1, 8, 32):
+        c5 = workloads.config(5, B=B)
+        wl = workloads.Workload(dataclasses.replace(c5, decode_steps=per + 64), device="cuda")
+        pool, lens = build_pool(wl)
+        leg(wl, pool, lens, "config5_ragged_B%d_topk_1_16" % B, "topk", 0, budget_frac=c5.budget_frac)
+        del wl, pool, lens
+        torch.cuda.empty_cache()
+    out["note"] = ("graphed steps with the token append, L2 flushed between steps, %d timed after %d warm-up; "
+                   "bytes counted as for the headline (metadata of every page, keys of the kept page-heads, values "
+                   "of those holding weight, append, page table, output)" % (steps, W))
+    return out
+
+
 # ---------------------------------------------------------------- oracle timing
-def oracle_sample(wl, g, budget_frac, meta, keys, vals):
-    """The oracle's sparse step for kv head g: replica bounds, top-k, entmax attention."""
-    from oracle import attend, replica, select
-    cfg = wl.cfg
-    qg = wl.q[0, g * cfg.G:(g + 1) * cfg.G].cpu().numpy()
-    _, ubg = replica.bound(qg, meta["kmin"], meta["kmax"], float(torch.tensor(cfg.scale, dtype=torch.float32)))
-    pages = select.topk(ubg, select.budget_pages(len(ubg), -1, budget_frac))
-    tok = attend.token_indices(pages, cfg.lengths[0], cfg.ps)
-    o, tau, _ = attend.entmax_attention(qg, keys[tok], vals[tok], cfg.alpha, 1.0 / math.sqrt(cfg.d))
-    return o
+# The oracle runs in a process that never touches the GPU: its data are
+# generated on the host, then a pool of worker processes forked from it shares
+# them (copy on write) to time the all-core leg.
+_LEG = {}
 
 
-def cpu_baseline(wl, pool, budget_frac, seconds):
-    """Time the oracle (as it stands) on the host cores: one kv head's share of
-    the sparse step, repeated for about `seconds`, scaled to the 8 heads."""
+def _widen(u16):
+    """bf16 bit patterns (uint16 / int16 numpy) -> float32, exactly."""
+    import numpy as np
+    return (u16.astype(np.uint32) << 16).view(np.float32)
+
+
+def _leg_setup(context):
+    import numpy as np
     from oracle import replica
+    wl = make_workload(context, 0, device="cpu")
     cfg = wl.cfg
-    keys, vals = wl.sequence(0, heads=[0])
-    keys = keys[0].float().cpu().numpy()
-    vals = vals[0].float().cpu().numpy()
-    meta = replica.page_meta(keys, cfg.ps)          # metadata exists before a decode step
+    keys, vals = wl.sequence(0)
+    kb = keys.view(torch.int16).numpy().view(np.uint16)
+    vb = vals.view(torch.int16).numpy().view(np.uint16)
+    # the page metadata exists before a decode step: built once, outside the timing
+    metas = [replica.page_meta(_widen(kb[g]), cfg.ps) for g in range(cfg.H_kv)]
+    _LEG.update(cfg=cfg, q=wl.q[0].numpy(), k=kb, v=vb, metas=metas,
+                scale32=float(np.float32(1.0 / math.sqrt(cfg.d))))
+
+
+def _leg_sparse_head(g):
+    """The oracle's sparse step for kv head g: replica bounds over every page,
+    top-k 1/64, float64 entmax attention over the kept pages."""
+    from oracle import attend, replica, select
+    cfg = _LEG["cfg"]
+    G = cfg.G
+    qg = _LEG["q"][g * G:(g + 1) * G]
+    m = _LEG["metas"][g]
+    _, ubg = replica.bound(qg, m["kmin"], m["kmax"], _LEG["scale32"])
+    pages = select.topk(ubg, select.budget_pages(len(ubg), -1, 1 / 64))
+    tok = attend.token_indices(pages, cfg.lengths[0], cfg.ps)
+    o, _, _ = attend.entmax_attention(qg, _widen(_LEG["k"][g][tok]), _widen(_LEG["v"][g][tok]), cfg.alpha,
+                                      1.0 / math.sqrt(cfg.d))
+    return float(o[0, 0])
+
+
+def _leg_full_head(g):
+    """The oracle's full-cache entmax decode for kv head g (every token)."""
+    from oracle import attend
+    cfg = _LEG["cfg"]
+    G = cfg.G
+    o, _, _ = attend.entmax_attention(_LEG["q"][g * G:(g + 1) * G], _widen(_LEG["k"][g]), _widen(_LEG["v"][g]),
+                                      cfg.alpha, 1.0 / math.sqrt(cfg.d))
+    return float(o[0, 0])
+
+
+def _leg_cores():
+    return len(os.sched_getaffinity(0))
+
+
+def _leg_pool(n):
+    import multiprocessing as mp
+    return mp.get_context("fork").Pool(n)
+
+
+def oracle_leg(context, seconds):
+    """The oracle, as it stands, timed on this host's cores (this process must
+    not have touched the GPU): a sparse decode step over the 8 kv heads on one
+    core and on min(cores, 8) worker processes (one kv head each), and the
+    full-cache entmax decode of one kv head on one core, scaled to the 8."""
+    _leg_setup(context)
+    cfg = _LEG["cfg"]
+    H = cfg.H_kv
     t0 = time.perf_counter()
-    n = 0
+    n1 = 0
     while True:
-        oracle_sample(wl, 0, budget_frac, meta, keys, vals)
-        n += 1
+        for g in range(H):
+            _leg_sparse_head(g)
+        n1 += 1
         if time.perf_counter() - t0 > seconds:
             break
-    per_head = (time.perf_counter() - t0) / n
-    us = per_head * cfg.H_kv * 1e6
-    return {"value": round(us, 1), "unit": "us/step", "cores": 1, "kind": "oracle",
-            "sample": "kv head 0 of 8 (4 query heads): replica bounds over all 16384 pages, top-k, float64 "
-                      "entmax attention over the 256 kept pages; %d repetitions, scaled x8 to a full step" % n}
+    single = (time.perf_counter() - t0) / n1
+    cores = _leg_cores()
+    workers = max(1, min(cores, H))
+    with _leg_pool(workers) as pool:
+        pool.map(_leg_sparse_head, range(H))                   # start-up and warm
+        t0 = time.perf_counter()
+        nm = 0
+        while True:
+            pool.map(_leg_sparse_head, range(H))
+            nm += 1
+            if time.perf_counter() - t0 > seconds:
+                break
+        multi = (time.perf_counter() - t0) / nm
+    t0 = time.perf_counter()
+    _leg_full_head(0)
+    full = (time.perf_counter() - t0) * H
+    return {"value": round(multi * 1e6, 1), "unit": "us/step", "cores": workers, "kind": "oracle",
+            "host_cores": cores, "single_core_us_per_step": round(single * 1e6, 1),
+            "full_cache_us_per_step_single_core": round(full * 1e6, 1),
+            "sample": ("the sparse decode step of the bench workload (%d tokens): replica bounds over every page, "
+                       "top-k 1/64, float64 entmax attention over the kept pages, for each of the 8 kv heads; "
+                       "value = %d worker processes, one kv head each, %d steps; single core %d steps; full-cache "
+                       "entmax decode of kv head 0 on one core, scaled x8" % (context, workers, nm, n1))}
+
+
+def cpu_baseline_subprocess(context, seconds):
+    """oracle_leg in a fresh process (this one holds a CUDA context, and the
+    oracle's worker pool is forked)."""
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--oracle-leg", "--context", str(context),
+                        "--leg-seconds", str(seconds)], capture_output=True, text=True, timeout=1800,
+                       env=dict(os.environ, CUDA_VISIBLE_DEVICES=""))
+    lines = [l for l in r.stdout.splitlines() if l.startswith("{")]
+    if r.returncode != 0 or not lines:
+        raise RuntimeError("oracle leg failed: " + r.stderr[-2000:])
+    return json.loads(lines[-1])
 
 
 def run_reference(args, rank, world):
+    """The reference arm: the oracle, as it stands, on this host's cores (no
+    GPU); each step is the sparse decode step over the 8 kv heads on
+    min(cores, 8) worker processes, one kv head each."""
     if rank != 0:
         return
-    if torch.cuda.is_available():
-        torch.cuda.set_device(0)
-    wl = make_workload(args.context, 0, device="cuda" if torch.cuda.is_available() else "cpu")
-    from oracle import replica
-    cfg = wl.cfg
-    keys, vals = wl.sequence(0, heads=[0])
-    keys = keys[0].float().cpu().numpy()
-    vals = vals[0].float().cpu().numpy()
-    meta = replica.page_meta(keys, cfg.ps)
-    for _ in range(args.warmup):
-        oracle_sample(wl, 0, 1 / 64, meta, keys, vals)
-    t0 = time.perf_counter()
-    for _ in range(args.steps):
-        oracle_sample(wl, 0, 1 / 64, meta, keys, vals)
-    per = (time.perf_counter() - t0) / args.steps * cfg.H_kv * 1e6
-    sample = ("kv head 0 of 8 per step (replica bounds over all pages, top-k, float64 entmax attention over "
-              "the kept pages; page metadata built before timing, no token appended), scaled x8")
+    _leg_setup(args.context)
+    cfg = _LEG["cfg"]
+    H = cfg.H_kv
+    workers = max(1, min(_leg_cores(), H))
+    with _leg_pool(workers) as pool:
+        for _ in range(args.warmup):
+            pool.map(_leg_sparse_head, range(H))
+        t0 = time.perf_counter()
+        for _ in range(args.steps):
+            pool.map(_leg_sparse_head, range(H))
+        per = (time.perf_counter() - t0) / args.steps * 1e6
+    sample = ("sparse decode step over the 8 kv heads (replica bounds over every page, top-k 1/64, float64 entmax "
+              "attention over the kept pages; page metadata built before timing, no token appended), %d worker "
+              "processes, one kv head each" % workers)
     line = {"metric": METRIC, "value": round(per, 1), "unit": "us/step", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": round(per / 1e3, 3), "higher_is_better": False,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": {"workload": workload_name(cfg.lengths[0]),
                        "seq_len": cfg.lengths[0]},
             "impl": "reference",
-            "cpu_baseline": {"value": round(per, 1), "unit": "us/step", "cores": 1, "kind": "oracle",
+            "cpu_baseline": {"value": round(per, 1), "unit": "us/step", "cores": workers, "kind": "oracle",
                              "sample": sample},
             "e2e": {"value": round(per, 1), "unit": "us/step", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
@@ -608,6 +779,9 @@ def replay_only(args):
 
 def main():
     args = parse()
+    if args.oracle_leg:
+        print(json.dumps(oracle_leg(args.context, args.leg_seconds)), flush=True)
+        return
     if args.replay_only:
         torch.cuda.set_device(0)
         replay_only(args)

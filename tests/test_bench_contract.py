@@ -29,7 +29,7 @@ def _check_reference_line(line, n):
     assert d["metric"] == bench.METRIC and d["unit"] == "us/step" and d["value"] > 0
     assert d["config"]["workload"] == bench.workload_name(65536)
     cb = d["cpu_baseline"]
-    assert cb["kind"] == "oracle" and cb["cores"] == 1 and cb["value"] == d["value"] and cb["sample"]
+    assert cb["kind"] == "oracle" and 1 <= cb["cores"] <= 8 and cb["value"] == d["value"] and cb["sample"]
     assert d["e2e"] == {"value": d["value"], "unit": "us/step", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
 
 
@@ -168,21 +168,39 @@ def test_native_line_carries_the_contract():
     clk = {"sm_mhz": 1965.0, "sm_max_mhz": 1965.0, "reasons": [], "samples": 12, "window": "timed region"}
     cpu = {"value": 378791.7, "unit": "us/step", "cores": 1, "kind": "oracle", "sample": "kv head 0"}
     line = bench.native_line(cfg, 1, 20, 5, 88.19, 86.0, 88.0, 28.78, stage, 2056, 278.2, {"x": 1},
-                             (100.91, 20480, 16384), clk, cpu, (6528.7, "measured"))
+                             (100.91, 20480, 16384), clk, cpu, (6528.7, "measured"), attend_us=21.5)
     json.loads(json.dumps(line))
     assert {"metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better",
             "scaling", "vs_baseline", "dtype", "data", "config", "roofline", "e2e", "gpu_launches", "clocks",
             "cpu_baseline"} <= set(line)
     assert line["value"] == 88.19 and line["higher_is_better"] is False and line["scaling"] == "weak"
-    assert line["gpu_launches"] == 6 * 20 and line["config"]["x"] == 1
+    assert line["gpu_launches"] == 4 * 20 and line["config"]["x"] == 1
     r = line["roofline"]
     assert {"bound", "achieved", "peak", "unit", "frac", "traffic"} <= set(r)
     by = bench.algorithmic_bytes(cfg, 2056, 278.2, "topk")
     assert abs(r["achieved"] - by["score"] / 28.78e-6 / 1e9) < 0.1
     assert abs(r["frac"] - r["achieved"] / 6528.7) < 1e-3
     assert r["traffic"] == round(bench.SCORE_DRAM_BYTES_PER_ROW * 16384 * 8)
+    ra = line["roofline_attend"]                 # the fused attention kernel on the bytes it must read
+    assert abs(ra["achieved"] - by["attend"] / 21.5e-6 / 1e9) < 0.1
+    assert abs(ra["frac_of_8tbs"] - ra["achieved"] / 8000.0) < 1e-3 and ra["traffic"] is None
     assert line["e2e"] == {"value": 100.91, "unit": "us/step", "h2d_bytes_per_step": 20480,
                            "d2h_bytes_per_step": 16384}
     assert line["config"]["step_us_best"] == 86.0 and line["config"]["workload"] == bench.workload_name(1 << 20)
     assert "cpu_baseline" not in bench.native_line(cfg, 2, 20, 5, 88.19, 86.0, 88.0, 28.78, stage, 2056, 278.2,
                                                    {}, (100.91, 20480, 16384), clk, None, (6650.0, "fallback"))
+
+
+def test_oracle_leg_on_the_host_cores():
+    """The cpu_baseline leg runs the oracle in a process without a GPU: one
+    core, then one worker process per kv head (up to the host's cores), and
+    the full-cache decode of one kv head; a small context keeps it short."""
+    env = dict(os.environ, CUDA_VISIBLE_DEVICES="")
+    r = subprocess.run([sys.executable, "bench.py", "--oracle-leg", "--context", "65536", "--leg-seconds", "0.2"],
+                       cwd=ROOT, env=env, capture_output=True, text=True, timeout=600)
+    assert r.returncode == 0, r.stderr[-2000:]
+    d = json.loads([l for l in r.stdout.splitlines() if l.startswith("{")][-1])
+    assert d["kind"] == "oracle" and d["unit"] == "us/step" and d["value"] > 0
+    assert d["cores"] == min(8, len(os.sched_getaffinity(0))) and d["host_cores"] == len(os.sched_getaffinity(0))
+    assert d["single_core_us_per_step"] > 0 and d["full_cache_us_per_step_single_core"] > 0
+    assert "65536 tokens" in d["sample"]
