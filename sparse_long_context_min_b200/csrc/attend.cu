@@ -32,6 +32,8 @@
 
 namespace ekv {
 
+constexpr int kStagesQK = 4;
+constexpr int kStagesPV = 4;
 constexpr int kStagesSM = 3;
 constexpr int kPsPad = 8;   // padding (bf16 elements) of a row of the P tile
 
@@ -199,6 +201,137 @@ EKV_DEV float group_lane_max(float v)
     v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 8));
     v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 16));
     return v;
+}
+
+// Write this split's maximum score of every head of the group (all threads
+// call; `wm` is shared [4][8]).
+EKV_DEV void write_split_max(const AttnArgs& a, int b, int g, int s, const float* run, int NT, float (*wm)[8])
+{
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, c = lane & 3;
+    for (int nt = 0; nt < NT; ++nt) {
+        const float m = group_lane_max(run[nt]);
+        if (lane < 4) wm[warp][4 * nt + c] = m;
+    }
+    __syncthreads();
+    if (threadIdx.x < a.G) {
+        const int h = threadIdx.x;
+        const float m = fmaxf(fmaxf(wm[0][h], wm[1][h]), fmaxf(wm[2][h], wm[3][h]));
+        a.lmax[((size_t)b * a.H_q + (size_t)g * a.G + h) * a.S + s] = m;
+    }
+}
+
+template <int D, int PS, int NT>
+__global__ void __launch_bounds__(kThreads) qk_bf16_kernel(const __grid_constant__ CUtensorMap kmap, const AttnArgs a)
+{
+    pdl_enter();
+    constexpr int STAGE = kStageTok * D * 2;
+    constexpr int PPS = kStageTok / PS;
+    constexpr int KS = D / 16;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = smem_align<1024>(smem_raw);
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kStagesQK * STAGE);
+    __shared__ int abort_flag;
+    __shared__ float wm[4][8];
+
+    const int b = blockIdx.z, g = blockIdx.y, s = blockIdx.x;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int L = a.seq_lens[b];
+    const int P = pages_of(L, PS, a.max_pages, a.status);
+    const int cnt = list_count(a, b, g, P);
+    if (s == 0 && tid == 0) a.counters[(size_t)b * a.H_kv + g] = 0;
+    const Range r = split_range(cnt, a.S, s);
+    const int nst = r.end > r.start ? (r.end - r.start + PPS - 1) / PPS : 0;
+    tab_fill(a, b, g, r, P);
+
+    // start the key loads first; the query fragments are prepared meanwhile
+    if (tid == 0) {
+        abort_flag = 0;
+        if (nst > 0) {
+            prefetch_tmap(&kmap);
+            for (int i = 0; i < kStagesQK; ++i) mbar_init(&bars[i], 1);
+            fence_mbar_init();
+            for (int st = 0; st < min(kStagesQK, nst); ++st)
+                issue_stage<D, PS>(a, &kmap, smem + st * STAGE, &bars[st], b, g, r, st, P);
+        }
+    }
+    float run[NT];
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) run[nt] = -INFINITY;
+    if (nst == 0) {
+        write_split_max(a, b, g, s, run, NT, wm);
+        return;
+    }
+    uint32_t bq[NT][KS][2];
+    load_q_frags<D, NT>(a, b, g, a.xscale, bq);
+    __syncthreads();
+
+    const uint32_t sbase = smem_addr(smem);
+    const size_t xstride = (size_t)a.k_max * PS;
+    const size_t cstride = (size_t)a.k_max * (PS / 16);
+    for (int st = 0; st < nst; ++st) {
+        const int slot = st % kStagesQK;
+        if (!mbar_wait(&bars[slot], (st / kStagesQK) & 1, kWaitLimitNs)) {
+            abort_flag = 1;
+            report(a.status, ENTMAXKV_TIMEOUT);
+        }
+        __syncthreads();
+        if (abort_flag) {
+            if (tid == 0)
+                for (int k = st; k < min(st + kStagesQK, nst); ++k)
+                    mbar_wait(&bars[k % kStagesQK], (k / kStagesQK) & 1, kWaitLimitNs);
+            return;
+        }
+        const uint32_t base = sbase + slot * STAGE;
+        const int row0 = warp * 16;
+        float acc[NT][4];
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0.f;
+        const int arow = row0 + (lane & 7) + ((lane >> 3) & 1) * 8;
+#pragma unroll
+        for (int j = 0; j < KS; ++j) {
+            uint32_t af[4];
+            ldsm_x4(swz_addr(base, arow, 2 * j + (lane >> 4)), af);
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) mma_bf16(acc[nt], af, bq[nt][j][0], bq[nt][j][1]);
+        }
+        // the warp's 16 rows lie in one page (16 divides PS): one list entry
+        const int gi = lane >> 2, c = lane & 3;
+        const int idx = r.start + st * PPS + row0 / PS;
+        if (idx < r.end) {
+            int lp;
+            const int phys = resolve(a, b, g, idx, P, lp, false);
+            float cm[NT];
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) cm[nt] = -INFINITY;
+#pragma unroll
+            for (int rr = 0; rr < 2; ++rr) {
+                const int prow = (row0 + gi + 8 * rr) % PS;
+                const bool valid = phys >= 0 && lp * PS + prow < L;
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt) {
+                    const int head = 4 * nt + c;
+                    const float x = valid ? acc[nt][2 * rr] + acc[nt][2 * rr + 1] : -INFINITY;
+                    cm[nt] = fmaxf(cm[nt], x);
+                    if (head < a.G)
+                        a.xbuf[((size_t)b * a.H_q + (size_t)g * a.G + head) * xstride + (size_t)idx * PS + prow] = x;
+                }
+            }
+            // chunk maxima: the V pass decides from these which pages hold weight
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) {
+                const float m = group_lane_max(cm[nt]);
+                run[nt] = fmaxf(run[nt], m);
+                const int head = 4 * nt + c;
+                if (gi == 0 && head < a.G)
+                    a.cmax[((size_t)b * a.H_q + (size_t)g * a.G + head) * cstride + (size_t)idx * (PS / 16) +
+                           (row0 % PS) / 16] = m;
+            }
+        }
+        __syncthreads();
+        if (tid == 0 && st + kStagesQK < nst)
+            issue_stage<D, PS>(a, &kmap, smem + slot * STAGE, &bars[slot], b, g, r, st + kStagesQK, P);
+    }
+    write_split_max(a, b, g, s, run, NT, wm);
 }
 
 // fp32 cache: each thread scores (token, head) pairs of a page with a float64
@@ -606,6 +739,234 @@ EKV_DEV void reduce_splits(const AttnArgs& a, int b, int g)
 // that feeds the TMA pipeline.
 constexpr int kActWin = 512;
 
+template <int D, int PS, int NT>
+__global__ void __launch_bounds__(kThreads) pv_bf16_kernel(const __grid_constant__ CUtensorMap vmap, const AttnArgs a)
+{
+    pdl_enter();
+    constexpr int STAGE = kStageTok * D * 2;
+    constexpr int PPS = kStageTok / PS;
+    constexpr int MTW = D / 64;           // 16-row m-tiles (head-dim rows) per warp
+    constexpr int PROW = kStageTok + kPsPad;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = smem_align<1024>(smem_raw);
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kStagesPV * STAGE);
+    uint16_t* ps_tile = reinterpret_cast<uint16_t*>(smem + kStagesPV * STAGE + 64);   // [8*NT][PROW]
+    __shared__ int abort_flag;
+    __shared__ int act[kActWin];
+    __shared__ unsigned char flag[kActWin];
+    __shared__ int nact;
+    __shared__ float tau_s[8];
+
+    const int b = blockIdx.z, g = blockIdx.y, s = blockIdx.x;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int L = a.seq_lens[b];
+    const int P = pages_of(L, PS, a.max_pages, a.status);
+    const int cnt = list_count(a, b, g, P);
+    const Range r = split_range(cnt, a.S, s);
+    const bool a2 = a.alpha == 2.0f;
+    const bool a15 = a.alpha == 1.5f;
+    const float rexp = 1.0f / (a.alpha - 1.0f);   // weight exponent for any other alpha
+    const size_t xstride = (size_t)a.k_max * PS;
+    const size_t row0h = (size_t)b * a.H_q + (size_t)g * a.G;
+
+    float acc[NT][MTW][4];
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+        for (int m = 0; m < MTW; ++m) acc[nt][m][0] = acc[nt][m][1] = acc[nt][m][2] = acc[nt][m][3] = 0.f;
+
+    tab_fill(a, b, g, r, P);
+    if (tid < 8) tau_s[tid] = tid < a.G ? a.tau[row0h + tid] : INFINITY;
+    if (tid == 0) {
+        abort_flag = 0;
+        prefetch_tmap(&vmap);
+        for (int i = 0; i < kStagesPV; ++i) mbar_init(&bars[i], 1);
+        fence_mbar_init();
+    }
+    for (int i = tid; i < 8 * NT * PROW; i += kThreads) ps_tile[i] = 0;
+    __syncthreads();
+    const uint32_t sbase = smem_addr(smem);
+    const uint32_t pbase = smem_addr(ps_tile);
+    int gst = 0;          // stages issued so far (barrier phase bookkeeping)
+    int loaded = 0;
+
+    for (int w0 = r.start; w0 < r.end; w0 += kActWin) {
+        const int wn = min(kActWin, r.end - w0);
+        // --- which pages of the window hold weight
+        for (int i = tid; i < wn; i += kThreads) flag[i] = 0;
+        __syncthreads();
+        {
+            constexpr int C = PS / 16;          // 16-token chunk maxima per page
+            const size_t cstride = (size_t)a.k_max * C;
+            const int items = wn * a.G;
+            for (int it = tid; it < items; it += kThreads) {
+                const int j = it / a.G, h = it % a.G;
+                const float* cp = a.cmax + (row0h + h) * cstride + (size_t)(w0 + j) * C;
+                float m = -INFINITY;
+                if constexpr (C % 4 == 0) {
+#pragma unroll
+                    for (int k = 0; k < C; k += 4) {
+                        const float4 v = *reinterpret_cast<const float4*>(cp + k);
+                        m = fmaxf(m, fmaxf(fmaxf(v.x, v.y), fmaxf(v.z, v.w)));
+                    }
+                } else {
+#pragma unroll
+                    for (int k = 0; k < C; ++k) m = fmaxf(m, cp[k]);
+                }
+                if (m > tau_s[h]) flag[j] = 1;
+            }
+        }
+        __syncthreads();
+        if (warp == 0) {   // ordered compaction of the flags
+            int base = 0;
+            for (int i0 = 0; i0 < wn; i0 += 32) {
+                const bool f = (i0 + lane < wn) && flag[i0 + lane];
+                const unsigned m = __ballot_sync(0xffffffffu, f);
+                if (f) act[base + __popc(m & ((1u << lane) - 1u))] = w0 + i0 + lane;
+                base += __popc(m);
+            }
+            if (lane == 0) nact = base;
+        }
+        __syncthreads();
+        const int na = nact;
+        loaded += na;
+        const int nst = (na + PPS - 1) / PPS;
+        if (nst == 0) continue;
+        // --- pipeline over the active pages
+        auto issue = [&](int st, int slot_) {
+            uint8_t* dst = smem + slot_ * STAGE;
+            int phys[PPS];
+            uint32_t bytes = 0;
+#pragma unroll
+            for (int i = 0; i < PPS; ++i) {
+                const int ai = st * PPS + i;
+                int lp;
+                phys[i] = ai < na ? resolve(a, b, g, act[ai], P, lp, true) : -1;
+                if (phys[i] >= 0) bytes += PS * D * 2;
+            }
+            mbar_arrive_expect_tx(&bars[slot_], bytes);
+#pragma unroll
+            for (int i = 0; i < PPS; ++i) {
+                if (phys[i] < 0) continue;
+                const int y = (phys[i] * a.H_kv + g) * PS;
+#pragma unroll
+                for (int hh = 0; hh < D / 64; ++hh)
+                    tma_load_2d(dst + hh * (kStageTok * 128) + i * PS * 128, &vmap, &bars[slot_], hh * 64, y);
+            }
+        };
+        if (tid == 0)
+            for (int st = 0; st < min(kStagesPV, nst); ++st) issue(st, (gst + st) % kStagesPV);
+        for (int st = 0; st < nst; ++st) {
+            const int gs = gst + st;
+            const int slot = gs % kStagesPV;
+            // weights of this stage: token tid % 64, heads (tid / 64) * 2 * NT ...
+            {
+                const int t = tid & (kStageTok - 1);
+                const int ai = st * PPS + t / PS;
+                const int prow = t % PS;
+                int idx = -1;
+                bool valid = false;
+                if (ai < na) {
+                    idx = act[ai];
+                    int lp;
+                    const int phys = resolve(a, b, g, idx, P, lp, false);
+                    valid = phys >= 0 && lp * PS + prow < L;
+                }
+                const int hbase = (tid >> 6) * 2 * NT;
+#pragma unroll
+                for (int k = 0; k < 2 * NT; ++k) {
+                    const int head = hbase + k;
+                    float p = 0.f;
+                    if (head < a.G && valid) {
+                        const float xv = a.xbuf[(row0h + head) * xstride + (size_t)idx * PS + prow];
+                        const float u = fmaxf(xv - tau_s[head], 0.f);
+                        p = a2 ? u : (a15 ? u * u : powf(u, rexp));
+                    }
+                    uint32_t hi, lo;
+                    split_bf16(p, hi, lo);
+                    ps_tile[(2 * head) * PROW + t] = (uint16_t)hi;
+                    ps_tile[(2 * head + 1) * PROW + t] = (uint16_t)lo;
+                }
+            }
+            if (!mbar_wait(&bars[slot], (gs / kStagesPV) & 1, kWaitLimitNs)) {
+                abort_flag = 1;
+                report(a.status, ENTMAXKV_TIMEOUT);
+            }
+            __syncthreads();
+            if (abort_flag) {
+                if (tid == 0)
+                    for (int k = st; k < min(st + kStagesPV, nst); ++k)
+                        mbar_wait(&bars[(gst + k) % kStagesPV], ((gst + k) / kStagesPV) & 1, kWaitLimitNs);
+                return;
+            }
+            // rows without a valid token are zeroed so zero weights never meet garbage
+            {
+                const int t = tid & (kStageTok - 1);
+                const int half = tid >> 6;
+                if (half < D / 64) {
+                    const int ai = st * PPS + t / PS;
+                    bool valid = false;
+                    if (ai < na) {
+                        int lp;
+                        const int phys = resolve(a, b, g, act[ai], P, lp, false);
+                        valid = phys >= 0 && lp * PS + (t % PS) < L;
+                    }
+                    if (!valid) {
+                        uint4* rowp = reinterpret_cast<uint4*>(smem + slot * STAGE + half * (kStageTok * 128) + t * 128);
+#pragma unroll
+                        for (int k = 0; k < 8; ++k) rowp[k] = make_uint4(0, 0, 0, 0);
+                        fence_proxy_async();
+                    }
+                }
+            }
+            __syncthreads();
+            const uint32_t base = sbase + slot * STAGE;
+            const int n = lane >> 2, c = lane & 3;
+#pragma unroll
+            for (int kk = 0; kk < kStageTok / 16; ++kk) {
+                uint32_t b0[NT], b1[NT];
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt) {
+                    const uint32_t pr = pbase + ((8 * nt + n) * PROW + 16 * kk + 2 * c) * 2;
+                    asm volatile("ld.shared.b32 %0, [%1];" : "=r"(b0[nt]) : "r"(pr));
+                    asm volatile("ld.shared.b32 %0, [%1];" : "=r"(b1[nt]) : "r"(pr + 16));
+                }
+                const int mi = lane >> 3;
+                const int trow = 16 * kk + (lane & 7) + 8 * (mi >> 1);
+#pragma unroll
+                for (int m = 0; m < MTW; ++m) {
+                    const int d0 = 16 * (warp * MTW + m);
+                    uint32_t af[4];
+                    ldsm_x4_t(swz_addr(base, trow, d0 / 8 + (mi & 1)), af);
+#pragma unroll
+                    for (int nt = 0; nt < NT; ++nt) mma_bf16(acc[nt][m], af, b0[nt], b1[nt]);
+                }
+            }
+            __syncthreads();
+            if (tid == 0 && st + kStagesPV < nst) issue(st + kStagesPV, (gs + kStagesPV) % kStagesPV);
+        }
+        gst += nst;
+    }
+    if (tid == 0 && a.vpages) atomicAdd(&a.vpages[(size_t)b * a.H_kv + g], loaded);
+    // partial output of this split: o[head 4nt + c][d]
+    {
+        const int c = lane & 3, gi = lane >> 2;
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+            const int head = 4 * nt + c;
+            if (head >= a.G) continue;
+            const size_t row = (row0h + head) * a.S + s;
+#pragma unroll
+            for (int m = 0; m < MTW; ++m) {
+                const int d = 16 * (warp * MTW + m) + gi;
+                a.opart[row * D + d] = acc[nt][m][0] + acc[nt][m][1];
+                a.opart[row * D + d + 8] = acc[nt][m][2] + acc[nt][m][3];
+            }
+        }
+    }
+    reduce_splits<D, false>(a, b, g);
+}
+
 template <int D>
 __global__ void __launch_bounds__(kThreads) pv_f32_kernel(const float* __restrict__ v_pool, int ps, const AttnArgs a)
 {
@@ -662,16 +1023,18 @@ __global__ void __launch_bounds__(kThreads) pv_f32_kernel(const float* __restric
 // ====================================================================== fused entmax (bf16 cache)
 // One launch runs the K pass, the threshold and the V pass.  The S splits of
 // a (sequence, kv head) form one thread-block cluster, whose CTAs are
-// scheduled together, so cluster barriers can separate the phases and the
-// CTAs can read each other's shared memory (distributed shared memory):
+// scheduled together, so cluster barriers (about 0.2 us on B200) separate the
+// phases:
 //   K pass      each split scores its pages and writes x and the 16-token
 //               chunk maxima to the workspace;
 //   local       each split, one warp per query head, finds a lower bound t_s
-//               of tau from its own chunk maxima (split_bound) and keeps its
-//               scores above t_s, with their list positions, in its shared
-//               memory (local_candidates);
+//               of tau from its own chunk maxima (split_bound) and writes its
+//               scores above t_s, with their list positions, to its slots in
+//               the workspace (local_candidates); t_s, its largest score and
+//               its candidate count stay in shared memory;
 //   barrier 1
-//   threshold   every CTA reads every split's bound and candidates; the
+//   threshold   every CTA reads the splits' bounds and counts (distributed
+//               shared memory) and their candidates (global memory); the
 //               largest bound is a lower bound of tau for the whole group, so
 //               the candidates above it hold every score that can carry
 //               weight (gather_candidates); tau of every query head is solved
@@ -686,14 +1049,16 @@ __global__ void __launch_bounds__(kThreads) pv_f32_kernel(const float* __restric
 //   merge       CTA r adds the partials of the output elements
 //               [r E / S, (r + 1) E / S) in CTA order (deterministic);
 //   barrier 3   no CTA leaves while another may still read its memory.
-// Where a split has more candidates than its slots hold, every CTA instead
-// solves over all the group's scores (global memory, written before barrier 1
-// with a fence) and loads the value pages of its own split.  No CTA leaves
-// before the last barrier, whatever happens (a timed-out copy only skips
-// work).
+// Bulk data crosses CTAs through global memory (written before the barrier
+// behind a fence, read through L2 with ld.global.cg), a few words per CTA
+// through distributed shared memory.  Where a split has more candidates than
+// its slots hold, every CTA instead solves over all the group's scores and
+// loads the value pages of its own split.  No CTA leaves before the last
+// barrier, whatever happens (a timed-out copy only skips work).
 constexpr int kFusedStages = 4;
-constexpr int kPubCap = 256;         // candidates a split keeps per query head for the others
-constexpr int kBitWords = 1024;      // weighted-page bitmap: lists of up to 32768 pages
+constexpr int kCandCap = kFusedCandCap;   // candidate slots per (split, query head) in the workspace
+constexpr int kBitWords = 1024;           // weighted-page bitmap: lists of up to 32768 pages
+constexpr int kFusedMaxSplitTokens = 4096; // listed tokens per split (per query head) the fused kernel takes
 
 // Warp-wide sum of three doubles and min / max of two floats (xor butterfly:
 // every lane ends with the same values).
@@ -705,6 +1070,17 @@ EKV_DEV void warp_red5(double (&v)[3], float& mn, float& mx)
         for (int i = 0; i < 3; ++i) v[i] += __shfl_xor_sync(0xffffffffu, v[i], o);
         mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
         mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    }
+}
+
+// Warp-wide sums of three floats (xor butterfly, every lane the same values).
+EKV_DEV void warp_sum3(float& a, float& b, float& c)
+{
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        a += __shfl_xor_sync(0xffffffffu, a, o);
+        b += __shfl_xor_sync(0xffffffffu, b, o);
+        c += __shfl_xor_sync(0xffffffffu, c, o);
     }
 }
 
@@ -733,46 +1109,16 @@ EKV_DEV void for_candidates(const TauSrc& s, Fn&& f)
     }
 }
 
-// Newton steps from the left on F_c(t) = sum_j (v_j - t)_+^r over the n
-// values in `vals` (shared, read lane-strided), from t0 with F_c(t0) >= 1.
-// For r >= 1, F_c is convex and decreasing, so every iterate stays at or below
-// its root; the result keeps a rounding margin below the last iterate.  For
-// r < 1 the start is returned.
-EKV_DEV double newton_bound(const float* vals, int n, double t0, double r, bool a2, bool a15)
-{
-    if (r < 1.0) return t0;
-    const int lane = threadIdx.x & 31;
-    double t = t0;
-    for (int it = 0; it < 8; ++it) {
-        double F = 0.0, dF = 0.0;
-        for (int j = lane; j < n; j += 32) {
-            const double u = (double)vals[j] - t;
-            if (u > 0.0) {
-                const double p1 = a2 ? 1.0 : (a15 ? u : pow(u, r - 1.0));
-                F += p1 * u;
-                dF += r * p1;
-            }
-        }
-        F = warp_sum(F);
-        dF = warp_sum(dF);
-        if (!(F > 1.0) || !(dF > 0.0)) break;          // at (or by rounding past) the root
-        const double nt = t + (F - 1.0) / dF;
-        if (!(nt > t)) break;
-        const bool small = nt - t <= 1e-3 * fmax(1.0, fabs(t));
-        t = nt;
-        if (small) break;                              // close enough: the bound only prunes
-    }
-    return t - 1e-9 * fmax(1.0, fabs(t));
-}
-
 // Lower bound of tau from one split's chunk maxima, by one warp.  cm: the
 // head's chunk-maximum row, own chunks [c0, c1); m_s the split's largest
 // score.  Every chunk maximum is the score of a distinct token, so for any
 // subset of the head's tokens sum_i (x_i - t)_+^r >= sum over the subset's
-// chunk maxima, and the root of the latter is at or below tau.  The chunks
+// chunk maxima, and the root of the latter is at or below tau.  Up to three
+// Newton steps from m_s - 1 on that sum (convex and decreasing for r >= 1, so
+// the steps stay at or below its root; r < 1 keeps m_s - 1).  The chunks
 // above m_s - 1 (the only ones that can matter) are kept in (lc, lcv); *nlc
 // is their number (more than cap: the list is unusable).
-EKV_DEV float split_bound(const float* cm, int c0, int c1, float m_s, double r, bool a2, bool a15, int* lc,
+EKV_DEV float split_bound(const float* cm, int c0, int c1, float m_s, float r, bool a2, bool a15, int* lc,
                           float* lcv, int cap, int* nlc)
 {
     const int lane = threadIdx.x & 31;
@@ -781,7 +1127,7 @@ EKV_DEV float split_bound(const float* cm, int c0, int c1, float m_s, double r, 
         *nlc = 0;
         return -INFINITY;
     }
-    const double thr = (double)m_s - 1.0;
+    const float thr = __fsub_rd(m_s, 1.0f);
     int n = 0;
     constexpr int U = 8;
     for (int i0 = c0; i0 < c1; i0 += 32 * U) {
@@ -793,7 +1139,7 @@ EKV_DEV float split_bound(const float* cm, int c0, int c1, float m_s, double r, 
         }
 #pragma unroll
         for (int u = 0; u < U; ++u) {
-            const bool keep = (double)v[u] > thr;
+            const bool keep = v[u] > thr;
             const unsigned m = __ballot_sync(0xffffffffu, keep);
             const int pos = n + __popc(m & below);
             if (keep && pos < cap) {
@@ -805,17 +1151,34 @@ EKV_DEV float split_bound(const float* cm, int c0, int c1, float m_s, double r, 
     }
     __syncwarp();
     *nlc = n;
-    const double t = n <= cap ? newton_bound(lcv, n, thr, r, a2, a15) : thr;
-    return __double2float_rd(t);
+    float t = thr;
+    if (n <= cap && r >= 1.0f) {
+        for (int it = 0; it < 3; ++it) {
+            float F = 0.f, dF = 0.f, unused = 0.f;
+            for (int j = lane; j < n; j += 32) {
+                const float u = lcv[j] - t;
+                if (u > 0.f) {
+                    const float p1 = a2 ? 1.f : (a15 ? u : powf(u, r - 1.f));
+                    F = fmaf(p1, u, F);
+                    dF = fmaf(r, p1, dF);
+                }
+            }
+            warp_sum3(F, dF, unused);
+            if (!(F > 1.f) || !(dF > 0.f)) break;      // at (or by rounding past) the root
+            t += (F - 1.f) / dF;
+        }
+        t -= 1e-5f * fmaxf(1.f, fabsf(t));             // the float steps may have rounded past the root
+    }
+    return fmaxf(t, thr);                              // at least m_s - 1 (rounded down), itself a bound
 }
 
 // One split's candidates of one head, by one warp: its scores above t with
-// their list positions, into (pval, ppos) (shared, at most kPubCap kept);
-// returns how many there are.  The chunks to read come from the list of
-// split_bound when it is usable (t is at least m_s - 1), else from all the
-// split's chunks [c0, c1).
-EKV_DEV int local_candidates(const float* x, int c0, int c1, int* lc, const float* lcv, int nlc, int cap, float t,
-                             float* pval, int* ppos)
+// their list positions, to oval / oidx (global, at most kCandCap kept);
+// returns how many there are.  The chunks to read: those of split_bound's
+// list above t (the list holds every chunk above m_s - 1 <= t), or all the
+// split's chunks [c0, c1) when the list overflowed.
+EKV_DEV int local_candidates(const float* x, const float* cm, int c0, int c1, int* lc, const float* lcv, int nlc,
+                             int cap, float t, float* oval, int* oidx)
 {
     const int lane = threadIdx.x & 31;
     const unsigned below = (1u << lane) - 1u;
@@ -850,27 +1213,25 @@ EKV_DEV int local_candidates(const float* x, int c0, int c1, int* lc, const floa
             const bool keep = v[u] > t;
             const unsigned m = __ballot_sync(0xffffffffu, keep);
             const int q = nc + __popc(m & below);
-            if (keep && q < kPubCap) {
-                pval[q] = v[u];
-                ppos[q] = pos[u];
+            if (keep && q < kCandCap) {
+                oval[q] = v[u];
+                oidx[q] = pos[u];
             }
             nc += __popc(m);
         }
     }
-    __syncwarp();
     return nc;
 }
 
 // The group's candidates of one head above tlb, gathered by one warp from the
-// S splits' lists (distributed shared memory: pval / ppos / n of split q live
-// in CTA q of the cluster) into (cv, ci), in split order; returns how many
-// (-1 when more than cap).  pre: per-warp shared scratch of S + 1 ints.
-EKV_DEV int gather_candidates(const float* pval, const int* ppos, int nq, int S, float tlb, float* cv, int* ci,
+// S splits' slots (global: split q's at cval + q * kCandCap, n_q of them,
+// lane q holding n_q) into (cv, ci), in split order; returns how many (-1 when
+// more than cap).  pre: per-warp shared scratch of S + 1 ints.
+EKV_DEV int gather_candidates(const float* cval, const int* cidx, int nq, int S, float tlb, float* cv, int* ci,
                               int cap, int* pre)
 {
     const int lane = threadIdx.x & 31;
     const unsigned below = (1u << lane) - 1u;
-    // nq: split lane's count (lanes >= S hold 0); prefix sums into pre[0..S]
     int incl = nq;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
@@ -881,6 +1242,9 @@ EKV_DEV int gather_candidates(const float* pval, const int* ppos, int nq, int S,
     if (lane == 0) pre[0] = 0;
     const int total = __shfl_sync(0xffffffffu, incl, 31);
     __syncwarp();
+    int bounds[kFusedMaxSplits + 1];                   // prefix sums, in registers
+#pragma unroll
+    for (int q = 0; q <= kFusedMaxSplits; ++q) bounds[q] = q <= S ? pre[q] : total;
     constexpr int U = 8;
     int n = 0;
     for (int k0 = 0; k0 < total; k0 += 32 * U) {
@@ -889,18 +1253,16 @@ EKV_DEV int gather_candidates(const float* pval, const int* ppos, int nq, int S,
 #pragma unroll
         for (int u = 0; u < U; ++u) {
             const int k = k0 + u * 32 + lane;
-            v[u] = -INFINITY;
-            p[u] = 0;
-            if (k < total) {
-                int lo = 0, hi = S;                    // the split q with pre[q] <= k < pre[q + 1]
-                while (hi - lo > 1) {
-                    const int mid = (lo + hi) >> 1;
-                    if (pre[mid] <= k) lo = mid; else hi = mid;
+            int q = 0, before = 0;                     // split q holds candidates [pre[q], pre[q + 1])
+#pragma unroll
+            for (int j = 1; j <= kFusedMaxSplits; ++j)
+                if (k >= bounds[j]) {
+                    q = j;
+                    before = bounds[j];
                 }
-                const int i = k - pre[lo];
-                v[u] = ld_dsmem_f32(dsmem(pval + i, lo));
-                p[u] = ld_dsmem_s32(dsmem(ppos + i, lo));
-            }
+            const size_t off = (size_t)q * kCandCap + (k - before);
+            v[u] = k < total ? __ldcg(cval + off) : -INFINITY;
+            p[u] = k < total ? __ldcg(cidx + off) : 0;
         }
 #pragma unroll
         for (int u = 0; u < U; ++u) {
@@ -918,18 +1280,23 @@ EKV_DEV int gather_candidates(const float* pval, const int* ppos, int nq, int S,
     return n <= cap ? n : -1;
 }
 
-// tau from the candidates of src: alpha = 2 and 1.5 by Newton steps from the
-// bound src.lo until the support is consistent, then the closed form on that
-// support in float64; any other alpha by safeguarded Newton steps on
-// F^(1/r) inside [src.lo, M].  One warp; every lane returns tau.
+// tau from the candidates of src, one warp, every lane returns it.
+//  alpha = 2 and 1.5: steps in float from the bound src.lo -- Newton on
+//  sum (x - t)^2 = 1 for 1.5, the fixed point t = (sum x - 1) / k for 2, both
+//  from the left over the current support {x > t} -- until the support holds
+//  for a step; then the closed form on that support in float64, accepted when
+//  the support is consistent with it (every kept value above, every dropped
+//  one at or below).  Should rounding in float leave the support
+//  inconsistent, the same iteration runs in float64.
+//  Any other alpha: safeguarded Newton steps on F^(1/r) inside [src.lo, M].
 EKV_DEV double solve_tau(const TauSrc& src, float M, float alpha)
 {
     const bool a2 = alpha == 2.0f;
     const bool a15 = alpha == 1.5f;
-    double tau = src.lo;
     if (!a2 && !a15) {
         // Newton on G(t) = F(t)^(1/r) - 1 inside [lo, hi] (F(lo) >= 1 > F(M) = 0),
         // bisection where a step leaves it; terms in float (powf), sums in float64
+        double tau = src.lo;
         const double r = 1.0 / ((double)alpha - 1.0);
         const float rf = (float)r;
         double lo = src.lo, hi = (double)M;
@@ -959,13 +1326,13 @@ EKV_DEV double solve_tau(const TauSrc& src, float M, float alpha)
         }
         return tau;
     }
-    double kprev = -1.0;
-    for (int it = 0; it < 100; ++it) {
+    // exact closed form on the support {x > t}, float64; NaN when inconsistent
+    auto closed = [&](double t, double* next) -> double {
         double v[3] = {0.0, 0.0, 0.0};
         float minS = INFINITY, maxN = -INFINITY;
         for_candidates(src, [&](float f) {
             const double vd = (double)f;
-            if (vd > tau) {
+            if (vd > t) {
                 v[0] += 1.0;
                 v[1] += vd;
                 v[2] = fma(vd, vd, v[2]);
@@ -976,60 +1343,55 @@ EKV_DEV double solve_tau(const TauSrc& src, float M, float alpha)
         });
         warp_red5(v, minS, maxN);
         const double k = v[0], sx = v[1], sxx = v[2];
-        if (a2 || k == kprev) {
-            // the support held still for a step: the closed form on it
-            double tcf;
-            bool ok;
-            if (a2) {
-                tcf = (sx - 1.0) / k;
-                ok = true;
-            } else {
-                const double mean = sx / k, msq = sxx / k;
-                const double disc = mean * mean - msq + 1.0 / k;
-                ok = disc >= 0.0;
-                tcf = ok ? mean - sqrt(disc) : 0.0;
-            }
-            // consistent support: every kept value above tcf, every dropped one at or
-            // below it (the values at or below the bound are below tau as well)
-            if (ok && tcf < (double)minS && (double)maxN <= tcf && tcf >= src.lo) return tcf;
-            if (a2) {
-                if (!(tcf != tau) || !isfinite(tcf)) break;
-                tau = tcf;
-                continue;
-            }
+        double tcf;
+        bool ok;
+        if (a2) {
+            tcf = (sx - 1.0) / k;
+            ok = true;
+            *next = tcf;
+        } else {
+            const double mean = sx / k, msq = sxx / k;
+            const double disc = mean * mean - msq + 1.0 / k;
+            ok = disc >= 0.0;
+            tcf = ok ? mean - sqrt(disc) : 0.0;
+            const double s1 = sx - k * t;
+            const double s2 = sxx - 2.0 * t * sx + k * t * t;
+            *next = t + (s2 - 1.0) / (2.0 * s1);
         }
+        return (ok && tcf < (double)minS && (double)maxN <= tcf && tcf >= src.lo) ? tcf : NAN;
+    };
+    // float iteration to the support
+    float t = (float)src.lo;
+    float kprev = -1.f;
+    for (int it = 0; it < 64; ++it) {
+        float k = 0.f, s1 = 0.f, s2 = 0.f;
+        for_candidates(src, [&](float f) {
+            const float u = f - t;
+            if (u > 0.f) {
+                k += 1.f;
+                s1 += a2 ? f : u;
+                s2 = fmaf(u, u, s2);
+            }
+        });
+        warp_sum3(k, s1, s2);
+        if (k == kprev) break;
         kprev = k;
-        // Newton step on sum (x - t)^2 = 1 over the current support (from the left)
-        const double s1 = sx - k * tau;
-        const double s2 = sxx - 2.0 * tau * sx + k * tau * tau;
-        const double nt = tau + (s2 - 1.0) / (2.0 * s1);
-        if (!(nt != tau) || !isfinite(nt)) {
-            kprev = k;                                 // closed form next time round
-            continue;
-        }
-        tau = nt;
+        const float nt = a2 ? (s1 - 1.f) / k : t + (s2 - 1.f) / (2.f * s1);
+        if (!(nt > t)) break;
+        t = nt;
+    }
+    double next = 0.0;
+    const double tc = closed((double)t, &next);
+    if (tc == tc) return tc;
+    // float64 iteration from the bound (rounding left the float support off)
+    double tau = src.lo;
+    for (int it = 0; it < 100; ++it) {
+        const double c = closed(tau, &next);
+        if (c == c) return c;
+        if (!(next != tau) || !isfinite(next)) break;
+        tau = next;
     }
     return tau;
-}
-
-// Exclusive prefix sum of one int per thread over a 128-thread block (two
-// block barriers inside); *total gets the block's sum.
-EKV_DEV int block_excl_scan128(int v, int* wsum, int* total)
-{
-    const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
-    int incl = v;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-        const int t = __shfl_up_sync(0xffffffffu, incl, o);
-        if (lane >= o) incl += t;
-    }
-    __syncthreads();
-    if (lane == 31) wsum[w] = incl;
-    __syncthreads();
-    int before = 0;
-    for (int i = 0; i < w; ++i) before += wsum[i];
-    *total = wsum[0] + wsum[1] + wsum[2] + wsum[3];
-    return before + incl - v;
 }
 
 // List position j of (b, g) -> physical page (and logical page in lp), read
@@ -1048,7 +1410,7 @@ EKV_DEV int resolve_peer(const AttnArgs& a, int b, int g, int j, int P, int per,
 }
 
 template <int D, int PS, int NT>
-__global__ void __launch_bounds__(kThreads) entmax_bf16_kernel(const __grid_constant__ CUtensorMap kmap,
+__global__ void __launch_bounds__(kThreads, 2) entmax_bf16_kernel(const __grid_constant__ CUtensorMap kmap,
                                                                const __grid_constant__ CUtensorMap vmap,
                                                                const AttnArgs a)
 {
@@ -1081,12 +1443,15 @@ __global__ void __launch_bounds__(kThreads) entmax_bf16_kernel(const __grid_cons
     __shared__ int act_lp[kActWin];
     __shared__ unsigned char flag[kActWin];
     __shared__ int nact;
-    __shared__ unsigned int bits[kBitWords];
-    // what this split publishes to the others (read through distributed shared memory)
+    __shared__ unsigned int bits[kBitWords];      // weighted pages of the heads this CTA solved
+    __shared__ unsigned int vbits[kBitWords];     // weighted pages of every head
+    __shared__ float tau_pub[8];                  // tau of the heads this CTA solved
+    __shared__ int fb_all;
+    __shared__ int wbase[kBitWords];
+    // this split's bound, largest score and candidate count per head (read by
+    // the other CTAs through distributed shared memory)
     __shared__ float pub_t[8], pub_m[8];
     __shared__ int pub_n[8];
-    __shared__ float pub_val[8][kPubCap];
-    __shared__ int pub_pos[8][kPubCap];
 
     const int b = blockIdx.z, g = blockIdx.y, s = blockIdx.x;   // s = rank in the cluster
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -1102,13 +1467,15 @@ __global__ void __launch_bounds__(kThreads) entmax_bf16_kernel(const __grid_cons
     const uint32_t sbase = smem_addr(smem);
     const bool a2 = a.alpha == 2.0f;
     const bool a15 = a.alpha == 1.5f;
-    const double rpow = a2 ? 1.0 : (a15 ? 2.0 : 1.0 / ((double)a.alpha - 1.0));
+    const float rpow = a2 ? 1.0f : (a15 ? 2.0f : 1.0f / (a.alpha - 1.0f));
+    const size_t seg = (size_t)kFusedMaxSplits * kCandCap;   // candidate slots of one head row
     tab_fill(a, b, g, r, P);
 
     // ------------------------------------------------------------ K pass
     if (tid == 0) {
         abort_flag = 0;
         fallback = 0;
+        fb_all = 0;
         prefetch_tmap(&kmap);
         prefetch_tmap(&vmap);
         for (int i = 0; i < NSTG; ++i) mbar_init(&bars[i], 1);
@@ -1206,8 +1573,9 @@ __global__ void __launch_bounds__(kThreads) entmax_bf16_kernel(const __grid_cons
             float* lcv = reinterpret_cast<float*>(smem + warp * WSCR + k * LC_CAP * 8 + LC_CAP * 4);
             int nlc;
             const float t = split_bound(a.cmax + row * cstride, c0, c1, smax[h], rpow, a2, a15, lc, lcv, LC_CAP, &nlc);
-            const int n = local_candidates(a.xbuf + row * xstride, c0, c1, lc, lcv, nlc, LC_CAP, t, pub_val[h],
-                                           pub_pos[h]);
+            const int n = local_candidates(a.xbuf + row * xstride, a.cmax + row * cstride, c0, c1, lc, lcv, nlc,
+                                           LC_CAP, t, a.cval + row * seg + (size_t)s * kCandCap,
+                                           a.cidx + row * seg + (size_t)s * kCandCap);
             if (lane == 0) {
                 pub_t[h] = t;
                 pub_m[h] = smax[h];
@@ -1215,16 +1583,18 @@ __global__ void __launch_bounds__(kThreads) entmax_bf16_kernel(const __grid_cons
             }
         }
     }
-    __threadfence();   // the scores in global memory are read by the other splits in the fallback
+    __threadfence();   // candidates and scores in global memory are read by the other splits
     __syncthreads();
     cluster_sync();
 
-    // ------------------------------------------------------------ threshold (every CTA, whole group)
+    // ------------------------------------------------------------ threshold (one CTA per head)
+    // query head h is solved by CTA h % S, on its warp (h / S) % 4; the owner
+    // keeps tau, its fallback flag and the head's weighted pages for the others
     const bool bitmap_ok = cnt <= kBitWords * 32;
     if (!abort_flag) {
         float* cv = reinterpret_cast<float*>(smem + warp * WSCR);
         int* ci = reinterpret_cast<int*>(smem + warp * WSCR + CAND_CAP * 4);
-        for (int h = warp; h < a.G; h += 4) {
+        for (int h = s + warp * a.S; h < a.G; h += 4 * a.S) {
             const size_t row = row0h + h;
             float M = -INFINITY, tlb = -INFINITY;
             int nq = 0;
@@ -1235,14 +1605,16 @@ __global__ void __launch_bounds__(kThreads) entmax_bf16_kernel(const __grid_cons
             }
             M = warp_max(M);
             tlb = warp_max(tlb);
-            const bool over = __any_sync(0xffffffffu, nq > kPubCap);
+            const bool over = __any_sync(0xffffffffu, nq > kCandCap);
             double tau;
             int nc = -1;
             if (!(M > -INFINITY)) {
                 tau = INFINITY;
                 nc = 0;
             } else {
-                if (!over) nc = gather_candidates(pub_val[h], pub_pos[h], nq, a.S, tlb, cv, ci, CAND_CAP, pre[warp]);
+                if (!over)
+                    nc = gather_candidates(a.cval + row * seg, a.cidx + row * seg, nq, a.S, tlb, cv, ci, CAND_CAP,
+                                           pre[warp]);
                 if (nc >= 0) {
                     TauSrc src{nullptr, 0, cv, nc, 0, (double)tlb};
                     tau = solve_tau(src, M, a.alpha);
@@ -1261,16 +1633,33 @@ __global__ void __launch_bounds__(kThreads) entmax_bf16_kernel(const __grid_cons
                 }
             }
             if (lane == 0) {
-                tau_s[h] = (float)tau;
-                if (s == 0 && a.tau_out) a.tau_out[row] = (float)tau;
+                tau_pub[h] = (float)tau;
+                if (a.tau_out) a.tau_out[row] = (float)tau;
             }
             __syncwarp();
         }
     }
-    if (tid < 8 && tid >= a.G) tau_s[tid] = INFINITY;
     fence_proxy_async();   // the scratch writes above come before the V copies into the same buffers
     __syncthreads();
-    const bool balanced = !fallback && bitmap_ok;
+    cluster_sync();        // every owner's tau, flag and page bits are complete
+    const int owners = min(a.S, a.G);
+    const int words = (cnt + 31) / 32;
+    if (!abort_flag) {
+        if (tid < 8) tau_s[tid] = tid < a.G ? ld_dsmem_f32(dsmem(&tau_pub[tid], tid % a.S)) : INFINITY;
+        if (tid < 32) {
+            const int f = tid < owners ? ld_dsmem_s32(dsmem(&fallback, tid)) : 0;
+            const bool any = __any_sync(0xffffffffu, f != 0);
+            if (tid == 0) fb_all = any;
+        }
+        if (bitmap_ok)
+            for (int w = tid; w < words; w += kThreads) {
+                unsigned u = 0;
+                for (int q = 0; q < owners; ++q) u |= (unsigned)ld_dsmem_s32(dsmem(&bits[w], q));
+                vbits[w] = u;
+            }
+    }
+    __syncthreads();
+    const bool balanced = !fb_all && bitmap_ok;
 
     // ------------------------------------------------------------ V pass
     const float rexp = 1.0f / (a.alpha - 1.0f);
@@ -1285,14 +1674,26 @@ __global__ void __launch_bounds__(kThreads) entmax_bf16_kernel(const __grid_cons
     const uint32_t pbase = smem_addr(ps_tile);
     // balanced: the weighted pages in list order, CTA s taking ranks s, s + S, ...
     // (windows of kActWin of them); otherwise the weighted pages of its own split
-    const int words = (cnt + 31) / 32;
-    const int wpt = (words + kThreads - 1) / kThreads;
-    int rank0 = 0, nw = 0, share = 0;
+    int nw = 0, share = 0;
     if (balanced) {
-        int mine = 0;
-        for (int w = tid * wpt; w < min(words, (tid + 1) * wpt); ++w) mine += __popc(bits[w]);
-        int tot;
-        rank0 = block_excl_scan128(mine, wsum, &tot);
+        // rank of the first weighted page of every bitmap word (warp 0, 32 words a step)
+        if (warp == 0) {
+            int base = 0;
+            for (int w0 = 0; w0 < words; w0 += 32) {
+                const int c = w0 + lane < words ? __popc(vbits[w0 + lane]) : 0;
+                int incl = c;
+#pragma unroll
+                for (int o = 1; o < 32; o <<= 1) {
+                    const int t = __shfl_up_sync(0xffffffffu, incl, o);
+                    if (lane >= o) incl += t;
+                }
+                if (w0 + lane < words) wbase[w0 + lane] = base + incl - c;
+                base += __shfl_sync(0xffffffffu, incl, 31);
+            }
+            if (lane == 0) wsum[0] = base;
+        }
+        __syncthreads();
+        const int tot = wsum[0];
         share = tot > s ? (tot - s + a.S - 1) / a.S : 0;
         nw = (share + kActWin - 1) / kActWin;
     } else {
@@ -1303,9 +1704,9 @@ __global__ void __launch_bounds__(kThreads) entmax_bf16_kernel(const __grid_cons
             // this CTA's entries [win * kActWin, ...) of its share: list positions of
             // the weighted pages of rank s + j S
             if (tid == 0) nact = min(kActWin, share - win * kActWin);
-            int rk = rank0;
-            for (int w = tid * wpt; w < min(words, (tid + 1) * wpt); ++w) {
-                unsigned m = bits[w];
+            for (int w = tid; w < words; w += kThreads) {
+                unsigned m = vbits[w];
+                int rk = wbase[w];
                 while (m) {
                     const int bit = __ffs(m) - 1;
                     m &= m - 1;
@@ -1778,6 +2179,26 @@ __global__ void selftest_timeout_kernel(uint64_t limit_ns, int32_t* status)
 }
 
 // ====================================================================== launch
+// Long page lists: K pass, threshold and V pass as three kernels (the
+// threshold kernel gives each query head a 512-thread CTA).
+template <int D, int PS, int NT>
+static int launch_entmax_bf16_split(const AttnArgs& a, int B, const CUtensorMap* kmap, const CUtensorMap* vmap,
+                              cudaStream_t stream)
+{
+    dim3 grid(a.S, a.H_kv, B);
+    const int qk_smem = kStagesQK * kStageTok * D * 2 + 1024 + 64;
+    const int pv_smem = kStagesPV * kStageTok * D * 2 + 1024 + 64 + 8 * NT * (kStageTok + kPsPad) * 2;
+    if (ensure_smem((const void*)qk_bf16_kernel<D, PS, NT>, qk_smem)) return ENTMAXKV_CUDA_ERROR;
+    if (ensure_smem((const void*)pv_bf16_kernel<D, PS, NT>, pv_smem)) return ENTMAXKV_CUDA_ERROR;
+    launch_pdl(qk_bf16_kernel<D, PS, NT>, dim3(grid), dim3(kThreads), qk_smem, stream, *kmap, a);
+    if (cudaGetLastError() != cudaSuccess) return ENTMAXKV_CUDA_ERROR;
+    if (ensure_smem((const void*)tau_kernel, kTauSmem)) return ENTMAXKV_CUDA_ERROR;
+    launch_pdl(tau_kernel, dim3(dim3(a.H_q, B)), dim3(kTauBlock), kTauSmem, stream, PS, a);
+    if (cudaGetLastError() != cudaSuccess) return ENTMAXKV_CUDA_ERROR;
+    launch_pdl(pv_bf16_kernel<D, PS, NT>, dim3(grid), dim3(kThreads), pv_smem, stream, *vmap, a);
+    return cudaGetLastError() == cudaSuccess ? ENTMAXKV_OK : ENTMAXKV_CUDA_ERROR;
+}
+
 // Splits of the fused kernel: the largest power of two up to 16 that the list
 // length and two CTAs per SM allow, and that the device can place as one
 // cluster with the kernel's resources.
@@ -1798,6 +2219,10 @@ static int launch_entmax_bf16(const AttnArgs& a0, int B, const CUtensorMap* kmap
     if (ensure_cluster_kernel(kern, smem)) return ENTMAXKV_CUDA_ERROR;
     AttnArgs a = a0;
     a.S = fused_splits(kern, smem, B * a.H_kv, a.k_max);   // <= the workspace layout's split count
+    // long lists (the full cache, the Gaussian selector's worst case): each
+    // split's candidates would outgrow their slots, so the three-kernel path
+    if ((long long)((a.k_max + a.S - 1) / a.S) * PS > kFusedMaxSplitTokens)
+        return launch_entmax_bf16_split<D, PS, NT>(a0, B, kmap, vmap, stream);
     launch_pdl_cluster(entmax_bf16_kernel<D, PS, NT>, dim3(a.S, a.H_kv, B), dim3(kThreads), a.S, smem, stream,
                        *kmap, *vmap, a);
     return cudaGetLastError() == cudaSuccess ? ENTMAXKV_OK : ENTMAXKV_CUDA_ERROR;
