@@ -159,6 +159,24 @@ ENTMAXKV_API int entmaxkv_score_pages(const entmaxkv_pool* pool, const float* q,
                          float* est_max, int32_t* status, void* stream);
 
 /*
+ * entmaxkv_append_metadata followed by entmaxkv_score_pages(ENTMAXKV_SCORE_BBOX)
+ * over the new lengths, as one call (German summary, section 2.A: the
+ * metadata is kept current as tokens are appended, and every page is scored
+ * from it).  The results -- pool rows, metadata, count, the advanced seq_lens
+ * and ub -- equal those of the two calls made in turn, bit for bit.  With a
+ * bf16 cache, n_new <= ps and a head layout the role-split scoring kernel
+ * covers, the append runs inside the scoring launch: extra CTAs write the new
+ * tokens, update the touched pages' metadata and score those pages (same
+ * operation order) while the other CTAs score every untouched page; a small
+ * trailing kernel then advances seq_lens.  Otherwise the two calls run in
+ * turn.  Arguments as in those two calls; n_new = 0 only scores.
+ */
+ENTMAXKV_API int entmaxkv_append_score_pages(const entmaxkv_pool* pool, const void* k_new, const void* v_new,
+                                int32_t n_new, const float* q, int32_t H_q, const int32_t* page_table,
+                                int32_t max_pages, int32_t* seq_lens, int32_t B, float scale, float* ub,
+                                int32_t* status, void* stream);
+
+/*
  * Select candidate pages per (sequence, kv head) (German summary, section 2.B).
  *   Output sel [B][H_kv][k_max] int32 logical page ids sorted ascending, the
  *   first sel_count[b][g] entries valid; sel_count [B][H_kv] int32.

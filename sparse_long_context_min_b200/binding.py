@@ -28,7 +28,7 @@ SYMBOLS = (
     "entmaxkv_append_metadata", "entmaxkv_score_pages", "entmaxkv_select", "entmaxkv_sparse_attend",
     "entmaxkv_full_entmax_decode", "entmaxkv_full_softmax_decode", "entmaxkv_workspace_size",
     "entmaxkv_status_string", "entmaxkv_selftest_timeout", "entmaxkv_sparse_attend_static",
-    "entmaxkv_sparse_softmax_attend",
+    "entmaxkv_sparse_softmax_attend", "entmaxkv_append_score_pages",
 )
 
 
@@ -72,6 +72,7 @@ def lib():
         L.entmaxkv_status_string.restype = ctypes.c_char_p
         L.entmaxkv_selftest_timeout.argtypes = [ctypes.c_int64, P, P]
         L.entmaxkv_sparse_attend_static.argtypes = [PP, P, I, P, I, P, I, P, P, I, F, F, P, P, P, P, P]
+        L.entmaxkv_append_score_pages.argtypes = [PP, P, P, I, P, I, P, I, P, I, F, P, P, P]
         for name in SYMBOLS:
             if name not in ("entmaxkv_workspace_size", "entmaxkv_status_string"):
                 getattr(L, name).restype = ctypes.c_int
@@ -244,6 +245,27 @@ def append_metadata(pool, k_new, v_new, page_table, seq_lens, status, stream=Non
     _check(lib().entmaxkv_append_metadata(pool.c, _p(k_new), _p(v_new), n_new, _p(page_table),
                                           max_pages, _p(seq_lens), B, _p(status),
                                           _stream(stream)), a.where)
+
+
+def append_score_pages(pool, k_new, v_new, q, page_table, seq_lens, scale, status, ub, stream=None):
+    """append_metadata then score_pages(SCORE_BBOX) over the new lengths, in one
+    call (one scoring launch where the library can fold the append into it)."""
+    a = _Args("append_score_pages")
+    a.need(k_new, "k_new", pool.k_pool.dtype, dims=4)
+    B, H_kv, n_new, d = k_new.shape
+    if H_kv != pool.H_kv or d != pool.d:
+        a.fail("k_new must be [B, %d, n_new, %d]" % (pool.H_kv, pool.d))
+    a.need(v_new, "v_new", pool.k_pool.dtype, k_new.numel(), dims=4)
+    Bq, H_q = _query(a, pool, q)
+    if Bq != B:
+        a.fail("q holds %d sequences; k_new %d" % (Bq, B))
+    max_pages = _table(a, page_table, seq_lens, B)
+    a.need(ub, "ub", F32T, B * pool.H_kv * max_pages)
+    a.need(status, "status", I32, 1)
+    a.reachable()
+    _check(lib().entmaxkv_append_score_pages(pool.c, _p(k_new), _p(v_new), n_new, _p(q), H_q, _p(page_table),
+                                             max_pages, _p(seq_lens), B, scale, _p(ub), _p(status),
+                                             _stream(stream)), a.where)
 
 
 def score_pages(pool, q, page_table, seq_lens, mode, scale, status, ub=None, m=None, v=None,

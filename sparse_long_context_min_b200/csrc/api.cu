@@ -333,6 +333,27 @@ int entmaxkv_score_pages(const entmaxkv_pool* pool, const float* q, int32_t H_q,
                         status, static_cast<cudaStream_t>(stream));
 }
 
+int entmaxkv_append_score_pages(const entmaxkv_pool* pool, const void* k_new, const void* v_new, int32_t n_new,
+                                const float* q, int32_t H_q, const int32_t* page_table, int32_t max_pages,
+                                int32_t* seq_lens, int32_t B, float scale, float* ub, int32_t* status, void* stream)
+{
+    int rc = check_pool(pool, true, true);
+    if (rc) return rc;
+    if ((rc = check_heads(H_q, pool->H_kv))) return rc;
+    if (n_new < 0 || B < 0 || max_pages <= 0) return ENTMAXKV_INVALID_ARG;
+    if (!std::isfinite(scale)) return ENTMAXKV_INVALID_ARG;
+    if ((long long)n_new > (long long)max_pages * pool->ps) return ENTMAXKV_INVALID_ARG;
+    if (B == 0) return ENTMAXKV_OK;
+    if (!q || !page_table || !seq_lens || !ub || !status) return ENTMAXKV_INVALID_ARG;
+    if (n_new > 0 && (!k_new || !v_new)) return ENTMAXKV_INVALID_ARG;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (n_new == 0)
+        return launch_score(*pool, q, H_q, page_table, max_pages, seq_lens, B, ENTMAXKV_SCORE_BBOX, scale, ub,
+                            nullptr, nullptr, nullptr, status, st);
+    return launch_append_score(*pool, k_new, v_new, n_new, q, H_q, page_table, max_pages, seq_lens, B, scale, ub,
+                               status, st);
+}
+
 int entmaxkv_select(int32_t mode, const float* ub, const float* m, const float* v, const float* est_max,
                     const int32_t* seq_lens, int32_t ps, int32_t B, int32_t H_q, int32_t H_kv, int32_t max_pages,
                     int32_t budget, float budget_frac, float alpha, float delta, int32_t k_max, int32_t* sel,

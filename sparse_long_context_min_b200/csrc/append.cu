@@ -190,6 +190,12 @@ __global__ void advance_kernel(int32_t* seq_lens, int B, int n_new)
     if (b < B) seq_lens[b] += n_new;
 }
 
+int launch_advance(int32_t* seq_lens, int B, int n_new, cudaStream_t stream)
+{
+    launch_pdl(advance_kernel, dim3((B + 127) / 128), dim3(128), 0, stream, seq_lens, B, n_new);
+    return cudaGetLastError() == cudaSuccess ? ENTMAXKV_OK : ENTMAXKV_CUDA_ERROR;
+}
+
 int launch_append(const entmaxkv_pool& pool, const void* k_new, const void* v_new, int n_new,
                   const int32_t* page_table, int max_pages, int32_t* seq_lens, int B, int32_t* status,
                   cudaStream_t stream)

@@ -52,6 +52,16 @@ int launch_append(const entmaxkv_pool& pool, const void* k_new, const void* v_ne
                   const int32_t* page_table, int max_pages, int32_t* seq_lens, int B, int32_t* status,
                   cudaStream_t stream);
 
+// seq_lens[b] += n_new for b < B (after the previous grid has completed)
+int launch_advance(int32_t* seq_lens, int B, int n_new, cudaStream_t stream);
+
+// append (n_new tokens per sequence) and bounding-box scoring over the new
+// lengths in one launch where the layout allows, else the two in turn; the
+// results equal launch_append followed by launch_score(BBOX)
+int launch_append_score(const entmaxkv_pool& pool, const void* k_new, const void* v_new, int n_new, const float* q,
+                        int H_q, const int32_t* page_table, int max_pages, int32_t* seq_lens, int B, float scale,
+                        float* ub, int32_t* status, cudaStream_t stream);
+
 int launch_score(const entmaxkv_pool& pool, const float* q, int H_q, const int32_t* page_table,
                  int max_pages, const int32_t* seq_lens, int B, int mode, float scale, float* ub, float* m,
                  float* v, float* est, int32_t* status, cudaStream_t stream);

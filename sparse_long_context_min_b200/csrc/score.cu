@@ -88,6 +88,19 @@ struct ScoreArgs {
     float* v_out;
     float* e_out;
     int32_t* status;
+    // appended tokens scored in the same launch (bf16 bounding boxes): n_new
+    // tokens per sequence, written by the CTAs [nscore, nscore + B) while the
+    // others score every untouched page (n_new = 0: no append)
+    int n_new, nscore;
+    const uint16_t* k_new;  // [B][H_kv][n_new][d]
+    const uint16_t* v_new;
+    uint16_t* k_pool;       // [num_phys][H_kv][ps][d]
+    uint16_t* v_pool;
+    uint16_t* kmin_w;       // the metadata the appending CTAs update
+    uint16_t* kmax_w;
+    float* mean_w;
+    float* m2_w;
+    int32_t* count_w;
 };
 
 // sum over the 8 slice lanes of a row: ((S0+S1)+(S2+S3))+((S4+S5)+(S6+S7))
@@ -333,7 +346,7 @@ EKV_DEV void ws_produce(const ScoreArgs& a, uint8_t* data, int stageb, int slots
     };
     int cur = pt_load(j0 + lane);                        // entries of items j0 + 32m + lane
     int nxt = pt_load(j0 + 32 + lane);
-    int lb = -1, lL = 0, lP = 0;
+    int lb = -1, lL = 0, lP = 0, lT = 0;
     const int per_batch = 32 / PPS;                      // chunks per batch of entries
     // lane i < PPS walks items j = (c0 + k) * PPS + i as (sequence bb, page pp)
     long long jl = c0 * PPS + lane;
@@ -356,10 +369,14 @@ EKV_DEV void ws_produce(const ScoreArgs& a, uint8_t* data, int stageb, int slots
             if (in) {
                 if (bb != lb) {
                     lb = bb;
-                    lL = __ldg(&a.seq_lens[bb]);
+                    const int L0 = __ldg(&a.seq_lens[bb]);
+                    lL = L0 + a.n_new;                           // the length after this launch's append
                     lP = pages_of(lL, a.ps, a.max_pages, a.status);
+                    lT = a.n_new > 0 ? L0 / a.ps : lP;           // first page the append touches
                 }
-                if (pp < lP) {
+                if (pp >= lT && pp < lP) {
+                    n = -1;                                      // scored by the appending CTA
+                } else if (pp < lP) {
                     if (pt < 0 || pt >= a.num_phys) report(a.status, ENTMAXKV_DEVICE_BOUNDS);
                     else n = min(a.ps, lL - pp * a.ps);
                 }
@@ -384,6 +401,117 @@ EKV_DEV void ws_produce(const ScoreArgs& a, uint8_t* data, int stageb, int slots
     }
 }
 
+// An appending CTA of score_box16_kernel: appends the n_new tokens of
+// sequence b exactly as append_small_kernel does (pool rows, then per page
+// and coordinate the metadata in token order), and scores every page the
+// append touched from the metadata it has just written, in the canonical
+// order of entmaxkv.h (8 slices of D/8 coordinates, each a chain of fmaf in
+// ascending d from 0, combined as ((S0+S1)+(S2+S3))+((S4+S5)+(S6+S7)), times
+// scale, largest over the group's heads, -0 -> +0).  sm: shared scratch.
+template <int D, int G>
+EKV_DEV void append_and_score(const ScoreArgs& a, int b, uint8_t* sm)
+{
+    constexpr int SW = D / 8;
+    const int Hk = a.H_kv, ps = a.ps, n_new = a.n_new;
+    uint16_t* lo_s = reinterpret_cast<uint16_t*>(sm);                 // [H_kv][D] new k_min
+    uint16_t* hi_s = lo_s + Hk * D;                                   // [H_kv][D] new k_max
+    float* part = reinterpret_cast<float*>(sm + 4 * Hk * D);         // [H_kv][G][8] slice sums
+    const int base = a.seq_lens[b];
+    if (base < 0) {
+        if (threadIdx.x == 0) report(a.status, ENTMAXKV_DEVICE_BOUNDS);
+        return;
+    }
+    for (int lp = base / ps; lp * ps < base + n_new; ++lp) {
+        const int t0 = max(base, lp * ps);
+        const int t1 = min(base + n_new, (lp + 1) * ps);
+        if (lp >= a.max_pages) {
+            if (threadIdx.x == 0) report(a.status, ENTMAXKV_DEVICE_BOUNDS);
+            break;
+        }
+        const int phys = a.page_table[(size_t)b * a.max_pages + lp];
+        if (phys < 0 || phys >= a.num_phys) {
+            if (threadIdx.x == 0) report(a.status, ENTMAXKV_DEVICE_BOUNDS);
+            continue;
+        }
+        for (int w = threadIdx.x; w < Hk * D; w += blockDim.x) {
+            const int g = w / D, j = w % D;
+            const size_t row = (size_t)phys * Hk + g;
+            const size_t meta = row * D + j;
+            float mu = 0.f, s2 = 0.f, lof = 0.f, hif = 0.f;
+            uint16_t lo = 0, hi = 0;
+            if (t0 - lp * ps > 0) {                  // resume a partially filled page
+                mu = a.mean_w[meta];
+                s2 = a.m2_w[meta];
+                lo = a.kmin_w[meta];
+                hi = a.kmax_w[meta];
+                lof = bf16_bits_to_f32(lo);
+                hif = bf16_bits_to_f32(hi);
+            }
+            const size_t src0 = ((size_t)b * Hk + g) * n_new;
+            for (int t = t0; t < t1; ++t) {
+                const int slot = t - lp * ps;
+                const size_t src = (src0 + (t - base)) * D + j;
+                const uint16_t kx = a.k_new[src];
+                const size_t dst = (row * ps + slot) * D + j;
+                a.k_pool[dst] = kx;
+                a.v_pool[dst] = a.v_new[src];
+                const float x = bf16_bits_to_f32(kx);
+                if (slot == 0) {
+                    mu = x;
+                    s2 = 0.f;
+                    lo = hi = kx;
+                    lof = hif = x;
+                } else {
+                    const float n = (float)(slot + 1);
+                    const float d1 = __fsub_rn(x, mu);
+                    mu = __fadd_rn(mu, __fdiv_rn(d1, n));
+                    const float d2 = __fsub_rn(x, mu);
+                    s2 = __fmaf_rn(d1, d2, s2);
+                    if (x < lof) { lo = kx; lof = x; }
+                    if (x > hif) { hi = kx; hif = x; }
+                }
+            }
+            a.mean_w[meta] = mu;
+            a.m2_w[meta] = s2;
+            a.kmin_w[meta] = lo;
+            a.kmax_w[meta] = hi;
+            lo_s[w] = lo;
+            hi_s[w] = hi;
+        }
+        if (threadIdx.x == 0) a.count_w[phys] = t1 - lp * ps;
+        __syncthreads();
+        // slice sums of every (kv head, query head, slice)
+        for (int it = threadIdx.x; it < Hk * G * 8; it += blockDim.x) {
+            const int g = it / (G * 8), h = (it / 8) % G, k = it % 8;
+            const float* qh = a.q + ((size_t)b * a.H_q + (size_t)g * G + h) * D + k * SW;
+            const uint16_t* lo_r = lo_s + g * D + k * SW;
+            const uint16_t* hi_r = hi_s + g * D + k * SW;
+            float acc = 0.f;
+#pragma unroll
+            for (int e = 0; e < SW; ++e) {
+                const float qv = __ldg(qh + e);
+                acc = __fmaf_rn(qv, bf16_bits_to_f32(qv >= 0.f ? hi_r[e] : lo_r[e]), acc);
+            }
+            part[it] = acc;
+        }
+        __syncthreads();
+        for (int g = threadIdx.x; g < Hk; g += blockDim.x) {
+            float best = -INFINITY;
+#pragma unroll
+            for (int h = 0; h < G; ++h) {
+                const float* S = part + (g * G + h) * 8;
+                const float t = __fadd_rn(__fadd_rn(__fadd_rn(S[0], S[1]), __fadd_rn(S[2], S[3])),
+                                          __fadd_rn(__fadd_rn(S[4], S[5]), __fadd_rn(S[6], S[7])));
+                const float u = __fmul_rn(t, a.scale);
+                if (h == 0 || u > best) best = u;
+            }
+            if (best == 0.f) best = 0.f;   // -0 -> +0
+            a.ub[((size_t)b * Hk + g) * a.max_pages + lp] = best;
+        }
+        __syncthreads();
+    }
+}
+
 template <int D, int G>
 __global__ void __launch_bounds__(BoxWsShape<D, G>::CTA, 2) score_box16_kernel(const ScoreArgs a)
 {
@@ -391,6 +519,10 @@ __global__ void __launch_bounds__(BoxWsShape<D, G>::CTA, 2) score_box16_kernel(c
     using S = BoxWsShape<D, G>;
     constexpr int NST = kWsStages;
     extern __shared__ __align__(128) uint8_t box_smem[];
+    if ((int)blockIdx.x >= a.nscore) {                   // an appending CTA: no barriers below
+        append_and_score<D, G>(a, blockIdx.x - a.nscore, box_smem);
+        return;
+    }
     int4* info = reinterpret_cast<int4*>(box_smem + S::DATA);                     // [NST][SLOTS]
     uint64_t* full = reinterpret_cast<uint64_t*>(box_smem + S::DATA + NST * S::SLOTS * 16);
     uint64_t* empty = full + NST;
@@ -398,7 +530,7 @@ __global__ void __launch_bounds__(BoxWsShape<D, G>::CTA, 2) score_box16_kernel(c
     const int PPS = S::SLOTS / a.H_kv;                   // pages per stage (host checks H_kv | SLOTS)
     const long long items = (long long)a.B * a.max_pages;
     const long long nchunks = (items + PPS - 1) / PPS;
-    const long long per = (nchunks + gridDim.x - 1) / gridDim.x;
+    const long long per = (nchunks + a.nscore - 1) / a.nscore;
     const long long c0 = blockIdx.x * per;
     const int K = (int)max(0ll, min(nchunks, c0 + per) - c0);   // chunks of this CTA
     const size_t vecb = (size_t)a.H_kv * S::ROWB;        // one page's block of one vector
@@ -501,7 +633,7 @@ __global__ void __launch_bounds__(BoxWsShape<D, G>::CTA, 2) score_box16_kernel(c
             if (S::HS > 1) best = fmaxf(best, __shfl_xor_sync(0xffffffffu, best, 8));
             if (S::HS > 2) best = fmaxf(best, __shfl_xor_sync(0xffffffffu, best, 16));
             if (best == 0.f) best = 0.f;   // -0 -> +0
-            if (b >= 0 && w == 0) a.ub[((size_t)b * a.H_kv + g) * a.max_pages + p] = n > 0 ? best : -INFINITY;
+            if (b >= 0 && n >= 0 && w == 0) a.ub[((size_t)b * a.H_kv + g) * a.max_pages + p] = n > 0 ? best : -INFINITY;
         }
         __syncwarp();                                    // every lane is done with stage s
         if (lane == 0) mbar_arrive(&empty[s]);
@@ -527,7 +659,10 @@ static int launch_box16(const ScoreArgs& a, cudaStream_t stream)
     const int pps = S::SLOTS / a.H_kv;
     const long long chunks = ((long long)a.B * a.max_pages + pps - 1) / pps;
     const int grid = (int)std::max<long long>(1, std::min<long long>(chunks, (long long)occ[dev] * num_sms()));
-    launch_pdl(score_box16_kernel<D, G>, dim3(grid), dim3(S::CTA), S::SMEM, stream, a);
+    ScoreArgs b = a;
+    b.nscore = grid;
+    const int appenders = a.n_new > 0 ? a.B : 0;
+    launch_pdl(score_box16_kernel<D, G>, dim3(grid + appenders), dim3(S::CTA), S::SMEM, stream, b);
     return cudaGetLastError() == cudaSuccess ? ENTMAXKV_OK : ENTMAXKV_CUDA_ERROR;
 }
 
@@ -577,6 +712,59 @@ static int dispatch_g(int G, const ScoreArgs& a, const ZTable& zt, cudaStream_t 
     }
 }
 
+// The bf16 bounding-box scoring kernel with the role split covers this head
+// layout: H_kv divides the rows of a round, and the pages per stage divide
+// 32 (one producer lane per page; page-table entries come in batches of 32).
+static bool box16_layout(int G, int H_kv)
+{
+    const int set = kWsConsumers * (32 / (8 * (G >= 2 ? G / 2 : 1)));
+    const int pps = set % H_kv == 0 ? kWsRounds * set / H_kv : 0;
+    return pps > 0 && pps <= 32 && 32 % pps == 0;
+}
+
+int launch_append_score(const entmaxkv_pool& pool, const void* k_new, const void* v_new, int n_new, const float* q,
+                        int H_q, const int32_t* page_table, int max_pages, int32_t* seq_lens, int B, float scale,
+                        float* ub, int32_t* status, cudaStream_t stream)
+{
+    const int G = H_q / pool.H_kv;
+    if (pool.dtype != ENTMAXKV_BF16 || n_new > pool.ps || !box16_layout(G, pool.H_kv)) {
+        // the two calls in turn
+        int rc = launch_append(pool, k_new, v_new, n_new, page_table, max_pages, seq_lens, B, status, stream);
+        if (rc) return rc;
+        return launch_score(pool, q, H_q, page_table, max_pages, seq_lens, B, ENTMAXKV_SCORE_BBOX, scale, ub,
+                            nullptr, nullptr, nullptr, status, stream);
+    }
+    ScoreArgs a{};
+    a.row_a = pool.kmin;
+    a.row_b = pool.kmax;
+    a.q = q;
+    a.H_q = H_q;
+    a.H_kv = pool.H_kv;
+    a.ps = pool.ps;
+    a.num_phys = pool.num_phys_pages;
+    a.page_table = page_table;
+    a.max_pages = max_pages;
+    a.seq_lens = seq_lens;
+    a.B = B;
+    a.scale = scale;
+    a.ub = ub;
+    a.status = status;
+    a.n_new = n_new;
+    a.k_new = static_cast<const uint16_t*>(k_new);
+    a.v_new = static_cast<const uint16_t*>(v_new);
+    a.k_pool = static_cast<uint16_t*>(pool.k_pool);
+    a.v_pool = static_cast<uint16_t*>(pool.v_pool);
+    a.kmin_w = static_cast<uint16_t*>(pool.kmin);
+    a.kmax_w = static_cast<uint16_t*>(pool.kmax);
+    a.mean_w = pool.mean;
+    a.m2_w = pool.m2;
+    a.count_w = pool.count;
+    const int rc = pool.d == 128 ? dispatch_box16<128>(G, a, stream) : dispatch_box16<64>(G, a, stream);
+    if (rc) return rc;
+    // the lengths advance once every CTA of the scoring launch has read them
+    return launch_advance(seq_lens, B, n_new, stream);
+}
+
 int launch_score(const entmaxkv_pool& pool, const float* q, int H_q, const int32_t* page_table,
                  int max_pages, const int32_t* seq_lens, int B, int mode, float scale, float* ub, float* m,
                  float* v, float* est, int32_t* status, cudaStream_t stream)
@@ -606,12 +794,7 @@ int launch_score(const entmaxkv_pool& pool, const float* q, int H_q, const int32
         a.row_a = pool.kmin;
         a.row_b = pool.kmax;
         if (pool.dtype == ENTMAXKV_BF16) {
-            // the role-split kernel needs H_kv to divide the rows of a round, and
-            // a number of pages per stage that divides 32 (one producer lane per
-            // page; page-table entries come in batches of 32)
-            const int set = kWsConsumers * (32 / (8 * (G >= 2 ? G / 2 : 1)));
-            const int pps = set % pool.H_kv == 0 ? kWsRounds * set / pool.H_kv : 0;
-            if (pps > 0 && pps <= 32 && 32 % pps == 0)
+            if (box16_layout(G, pool.H_kv))
                 return pool.d == 128 ? dispatch_box16<128>(G, a, stream) : dispatch_box16<64>(G, a, stream);
             return pool.d == 128 ? dispatch_g<uint16_t, 128, false>(G, a, zt, stream)
                                  : dispatch_g<uint16_t, 64, false>(G, a, zt, stream);

@@ -105,11 +105,23 @@ class DecodeStep:
                         self.scale, self.out, self.workspace, self.status, tau_out=self.tau,
                         v_pages=self.v_pages, stream=stream)
 
+    def append_score(self, q, k_new, v_new, stream=None):
+        """Append (k_new, v_new) [B, H_kv, n, d], then score over the new lengths
+        (top-k mode: one library call, which can fold the append into the
+        scoring launch)."""
+        if self.mode == "topk":
+            B.append_score_pages(self.pool, k_new, v_new, q, self.page_table, self.seq_lens, self.scale,
+                                 self.status, self.ub, stream=stream)
+        else:
+            B.append_metadata(self.pool, k_new, v_new, self.page_table, self.seq_lens, self.status, stream=stream)
+            self.score(q, stream)
+
     def __call__(self, q, k_new=None, v_new=None, stream=None):
         """One step; appends (k_new, v_new) [B, H_kv, 1, d] first when given."""
         if k_new is not None:
-            B.append_metadata(self.pool, k_new, v_new, self.page_table, self.seq_lens, self.status, stream=stream)
-        self.score(q, stream)
+            self.append_score(q, k_new, v_new, stream)
+        else:
+            self.score(q, stream)
         self.choose(stream)
         self.attend(q, stream)
         return self.out
@@ -158,6 +170,8 @@ class GraphedStep:
     query and token into them, then replay().  With stage_events=True the
     graph also records an event node between stages; stage_us() returns the
     last replay's per-stage durations (append, score, select, attend) in us.
+    In top-k mode the append is part of the scoring call (append_score), so
+    the append stage is empty and the score stage holds both.
     """
 
     STAGES = ("append", "score", "select", "attend")
@@ -193,10 +207,13 @@ class GraphedStep:
         with torch.cuda.graph(self.graph):
             cs = torch.cuda.current_stream()
             self._mark(0, cs)
-            if append:
+            if append and step.mode != "topk":
                 B.append_metadata(pool, self.k, self.v, step.page_table, step.seq_lens, step.status)
             self._mark(1, cs)
-            step.score(self.q)
+            if append and step.mode == "topk":
+                step.append_score(self.q, self.k, self.v)
+            else:
+                step.score(self.q)
             self._mark(2, cs)
             step.choose()
             self._mark(3, cs)

@@ -95,6 +95,39 @@ def test_append_one_token_at_a_time_matches_whole_pages():
         assert torch.equal(a, b_), name
 
 
+@pytest.mark.parametrize("n_new", [1, 5, 64])
+def test_append_score_equals_append_then_score(n_new):
+    """entmaxkv_append_score_pages (the append folded into the scoring launch)
+    leaves exactly what entmaxkv_append_metadata followed by
+    entmaxkv_score_pages(BBOX) leaves: pool rows, metadata, counts, lengths and
+    bounds, bit for bit, over appends that fill, cross and start pages of a
+    ragged batch with permuted physical pages."""
+    wl = _wl(5, [5000, 12345 - 12, 777, 64 * 9], decode_steps=8 * 64)
+    cfg = wl.cfg
+    pool_a, lens_a = build_pool(wl)
+    pool_b, lens_b = build_pool(wl)
+    st = _status()
+    ub_a = torch.empty(cfg.B, cfg.H_kv, wl.max_pages, device="cuda")
+    ub_b = torch.empty_like(ub_a)
+    scale = H.scale32(cfg)
+    for t in range(4):
+        g = torch.Generator(device="cuda").manual_seed(100 + t)
+        k = torch.randn(cfg.B, cfg.H_kv, n_new, cfg.d, generator=g, device="cuda").to(cfg.dtype)
+        v = torch.randn(cfg.B, cfg.H_kv, n_new, cfg.d, generator=g, device="cuda").to(cfg.dtype)
+        q = torch.randn(cfg.B, cfg.H_q, cfg.d, generator=g, device="cuda")
+        B.append_metadata(pool_a, k, v, wl.page_table, lens_a, st)
+        B.score_pages(pool_a, q, wl.page_table, lens_a, B.SCORE_BBOX, scale, st, ub=ub_a)
+        B.append_score_pages(pool_b, k, v, q, wl.page_table, lens_b, scale, st, ub_b)
+        _assert_ok(st)
+        assert torch.equal(lens_a, lens_b)
+        for name in ("kmin", "kmax", "mean", "m2", "count", "k_pool", "v_pool"):
+            assert torch.equal(getattr(pool_a, name), getattr(pool_b, name)), (t, name)
+        for b in range(cfg.B):
+            P = (int(lens_a[b]) + cfg.ps - 1) // cfg.ps
+            assert torch.equal(ub_a[b, :, :P], ub_b[b, :, :P]), (t, b)
+            assert bool(torch.all(ub_b[b, :, P:] == -float("inf")))
+
+
 def test_score_bbox_bitexact(built):
     wl, pool, seq_lens, oseqs = built
     cfg = wl.cfg

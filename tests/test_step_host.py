@@ -24,7 +24,7 @@ def calls(monkeypatch):
             log.append((name, args, kw))
         return f
 
-    for name in ("append_metadata", "score_pages", "select", "sparse_attend"):
+    for name in ("append_metadata", "append_score_pages", "score_pages", "select", "sparse_attend"):
         monkeypatch.setattr(B, name, rec(name))
     monkeypatch.setattr(B, "workspace_size", lambda *a: 4096)
     return log
@@ -45,16 +45,22 @@ def test_topk_step_calls_and_buffers(calls, frac):
     q = torch.zeros(Bn, H_q, 128)
     k = torch.zeros(Bn, 8, 1, 128, dtype=torch.bfloat16)
     st(q, k, k)
-    assert [c[0] for c in calls] == ["append_metadata", "score_pages", "select", "sparse_attend"]
-    _, score_args, score_kw = calls[1]
+    # top-k: the token append and the bounding-box scoring are one library call
+    assert [c[0] for c in calls] == ["append_score_pages", "select", "sparse_attend"]
+    _, as_args, _ = calls[0]
+    assert as_args[1] is k and as_args[3] is q and tuple(as_args[8].shape) == (Bn, 8, max_pages)
+    calls.clear()
+    st(q)                                            # no token: scoring alone
+    assert [c[0] for c in calls] == ["score_pages", "select", "sparse_attend"]
+    _, score_args, score_kw = calls[0]
     assert score_args[4] == B.SCORE_BBOX and tuple(score_kw["ub"].shape) == (Bn, 8, max_pages)
-    _, sel_args, sel_kw = calls[2]
+    _, sel_args, sel_kw = calls[1]
     assert sel_args[0] == B.SELECT_TOPK and sel_kw["budget_frac"] == frac and sel_kw["budget"] == -1
     assert tuple(st.sel.shape) == (Bn, 8, st.k_max) and st.sel.dtype == torch.int32
     assert tuple(st.sel_count.shape) == (Bn, 8) and st.sel_count.dtype == torch.int32
     assert tuple(st.out.shape) == (Bn, H_q, 128) and st.out.dtype == torch.float32
     assert tuple(st.tau.shape) == (Bn, H_q) and st.workspace.numel() >= 4096
-    _, att_args, att_kw = calls[3]
+    _, att_args, att_kw = calls[2]
     assert att_args[4] is st.sel and att_args[5] is st.sel_count and att_kw["tau_out"] is st.tau
 
 
@@ -80,3 +86,10 @@ def test_fixed_budget_and_caller_output(calls):
     assert st.k_max == 7 and st.out is out
     st.attend(torch.zeros(1, 32, 128))
     assert calls[-1][1][8] is out
+
+
+def test_gauss_step_appends_then_scores(calls):
+    st = S.DecodeStep(_pool(), torch.zeros(1, 30, dtype=torch.int32), torch.tensor([64 * 20]), 32, "gauss")
+    k = torch.zeros(1, 8, 1, 128, dtype=torch.bfloat16)
+    st(torch.zeros(1, 32, 128), k, k)
+    assert [c[0] for c in calls] == ["append_metadata", "score_pages", "select", "sparse_attend"]
