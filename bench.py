@@ -56,6 +56,9 @@ def parse():
                     help="time the CPU oracle on this host's cores and print one JSON line (no GPU)")
     ap.add_argument("--leg-seconds", type=float, default=8.0,
                     help="time budget of each part of the oracle leg (seconds)")
+    ap.add_argument("--selector-sweep", action="store_true",
+                    help="time the top-k 1/64 and the Gaussian (Delta 0.5) steps at 2^18, 2^19 and 2^20 tokens "
+                         "and print one JSON line per (length, selector)")
     return ap.parse_args()
 
 
@@ -756,6 +759,37 @@ def run_reference(args, rank, world):
     print(json.dumps(line), flush=True)
 
 
+def selector_sweep(args):
+    """The two selectors against context length on configuration 4's generator
+    (B = 1, 32/8 heads, d = 128, pages of 64, bf16): us per graphed step with
+    its token append, selected and loaded-value page-heads, algorithmic bytes
+    and GB/s, for top-k 1/64 and the Gaussian selector with Delta = 0.5."""
+    from sparse_long_context_min_b200.step import DecodeStep, GraphedStep, build_pool
+    torch.cuda.set_device(0)
+    W, K = args.warmup, min(args.steps, 200)
+    stream = torch.cuda.current_stream()
+    flush = torch.empty(256 * MiB, dtype=torch.uint8, device="cuda")
+    for ctx in (1 << 18, 1 << 19, 1 << 20):
+        wl = make_workload(ctx, 0, appends=2 * (W + K) + 64)
+        cfg = wl.cfg
+        pool, lens = build_pool(wl)
+        for i, mode in enumerate(("topk", "gauss")):
+            st = DecodeStep(pool, wl.page_table, lens, cfg.H_q, mode, budget_frac=1 / 64, alpha=cfg.alpha,
+                            delta=0.5)
+            gs = GraphedStep(st, append=True, stage_events=False)
+            toks = decode_tokens(wl, i * (W + K), W + K)
+            us, sel, vp, _ = timed_replays(gs, st, toks, W, K, flush, stream)
+            mean = statistics.mean(us)
+            by = algorithmic_bytes(cfg, sel, vp, mode)["total"]
+            print(json.dumps({"context": ctx, "selector": "top-k 1/64" if mode == "topk" else "gaussian delta 0.5",
+                              "us_per_step": round(mean, 2), "selected_page_heads": round(sel, 1),
+                              "value_page_heads": round(vp, 1), "pages_per_kv_head": cfg.pages(0),
+                              "algorithmic_bytes": int(by), "gbs": round(by / (mean * 1e-6) / 1e9, 1)}), flush=True)
+            del gs, st, toks
+        del pool, lens, wl
+        torch.cuda.empty_cache()
+
+
 def replay_only(args):
     """Capture one decode step (top-k 1/64 or the Gaussian selector, Delta 0.5)
     of the bench workload as a graph and replay it; prints nothing but "ok"."""
@@ -785,6 +819,9 @@ def main():
     if args.replay_only:
         torch.cuda.set_device(0)
         replay_only(args)
+        return
+    if args.selector_sweep:
+        selector_sweep(args)
         return
     rank, world, local = dist_init(args.gpus, "gloo" if args.impl == "reference" else "nccl")
     try:
