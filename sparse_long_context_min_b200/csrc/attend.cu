@@ -1055,7 +1055,7 @@ __global__ void __launch_bounds__(kThreads) pv_f32_kernel(const float* __restric
 // its slots hold, every CTA instead solves over all the group's scores and
 // loads the value pages of its own split.  No CTA leaves before the last
 // barrier, whatever happens (a timed-out copy only skips work).
-constexpr int kFusedStages = 4;
+constexpr int kFusedStages = 5;
 constexpr int kCandCap = kFusedCandCap;   // candidate slots per (split, query head) in the workspace
 constexpr int kBitWords = 1024;           // weighted-page bitmap: lists of up to 32768 pages
 constexpr int kFusedMaxSplitTokens = 4096; // listed tokens per split (per query head) the fused kernel takes
@@ -1086,11 +1086,8 @@ EKV_DEV void warp_sum3(float& a, float& b, float& c)
 
 // Where the candidates of a head's threshold are read from.
 struct TauSrc {
-    const float* x;     // the head's scores over the listed tokens (global), mode 1
-    int n;              // listed tokens
-    const float* cand;  // the candidate scores (shared), mode 0
+    const float* cand;  // the candidate scores (shared)
     int ncand;
-    int mode;           // 0: cand, 1: every score above lo
     double lo;          // every candidate is > lo; every other score is <= lo <= tau
 };
 
@@ -1099,14 +1096,7 @@ template <typename Fn>
 EKV_DEV void for_candidates(const TauSrc& s, Fn&& f)
 {
     const int lane = threadIdx.x & 31;
-    if (s.mode == 0) {
-        for (int i = lane; i < s.ncand; i += 32) f(s.cand[i]);
-    } else {
-        for (int k = lane; k < s.n; k += 32) {
-            const float v = __ldcg(s.x + k);
-            if ((double)v > s.lo) f(v);
-        }
-    }
+    for (int i = lane; i < s.ncand; i += 32) f(s.cand[i]);
 }
 
 // Lower bound of tau from one split's chunk maxima, by one warp.  cm: the
@@ -1245,7 +1235,7 @@ EKV_DEV int gather_candidates(const float* cval, const int* cidx, int nq, int S,
     int bounds[kFusedMaxSplits + 1];                   // prefix sums, in registers
 #pragma unroll
     for (int q = 0; q <= kFusedMaxSplits; ++q) bounds[q] = q <= S ? pre[q] : total;
-    constexpr int U = 8;
+    constexpr int U = 4;
     int n = 0;
     for (int k0 = 0; k0 < total; k0 += 32 * U) {
         float v[U];
@@ -1383,15 +1373,194 @@ EKV_DEV double solve_tau(const TauSrc& src, float M, float alpha)
     double next = 0.0;
     const double tc = closed((double)t, &next);
     if (tc == tc) return tc;
-    // float64 iteration from the bound (rounding left the float support off)
-    double tau = src.lo;
+    // float64 steps from just below the float iterate (rounding left the float
+    // support off by a value or two); should that start lie right of the root
+    // (a step that does not move right), from the bound itself
+    double tau = fmax(src.lo, (double)t - 1e-4 * fmax(1.0, fabs((double)t)));
+    bool restarted = tau == src.lo;
     for (int it = 0; it < 100; ++it) {
         const double c = closed(tau, &next);
         if (c == c) return c;
-        if (!(next != tau) || !isfinite(next)) break;
+        if (!(next > tau) || !isfinite(next)) {
+            if (restarted) break;
+            tau = src.lo;
+            restarted = true;
+            continue;
+        }
         tau = next;
     }
     return tau;
+}
+
+// tau of every head by the whole cluster, for when a head's candidates do not
+// fit the slots: each iteration every CTA sums its own split's scores of the
+// head at the current iterate (one warp per head, heads h and h + 4 on warp
+// h % 4), the S partial sums go through distributed shared memory, and every
+// CTA adds them in split order (lane q holds split q; the xor butterfly gives
+// every lane, and so every CTA, the same bits) and takes the same step, so
+// all CTAs hold the same iterates and leave the loop after the same barrier.
+//  alpha = 2 and 1.5: from the group bound, the closed form on the current
+//  support {x > t}; accepted when the support is consistent with it, else t
+//  moves to the next iterate from the left (t = (sum x - 1) / k for 2, a
+//  Newton step on sum (x - t)^2 = 1 for 1.5).
+//  Any other alpha: safeguarded Newton steps on F^(1/r) inside [bound, max].
+// x: score row of head 0 (heads xstride apart); [t0, t1): this split's
+// tokens; skip: this CTA adds nothing (it gave up on a copy); part, mm:
+// shared [2][8][3] doubles and [2][8][2] floats; pub_t, pub_m: every split's
+// bound and largest score per head (read through distributed shared memory);
+// tau_h: tau per head, out (every CTA).
+EKV_DEV void cluster_tau(const float* x, size_t xstride, int t0, int t1, const float* pub_t, const float* pub_m,
+                         int G, int S, float alpha, bool skip, double* part, float* mm, double* tau_h)
+{
+    constexpr int kMaxIt = 48;
+    constexpr int U = 8;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const bool a2 = alpha == 2.0f, a15 = alpha == 1.5f, gen = !a2 && !a15;
+    const double r = 1.0 / ((double)alpha - 1.0);
+    const float rm1 = (float)(r - 1.0);
+    double t[2], lo[2], hi[2], res[2];
+    bool dn[2];
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+        const int h = warp + 4 * k;
+        dn[k] = true;
+        t[k] = lo[k] = hi[k] = res[k] = INFINITY;
+        if (h < G) {
+            float tb = lane < S ? ld_dsmem_f32(dsmem(&pub_t[h], lane)) : -INFINITY;
+            float mx = lane < S ? ld_dsmem_f32(dsmem(&pub_m[h], lane)) : -INFINITY;
+            tb = warp_max(tb);
+            mx = warp_max(mx);
+            dn[k] = !(mx > -INFINITY);           // no scores: tau = +inf, nothing is kept
+            t[k] = lo[k] = (double)tb;
+            hi[k] = (double)mx;
+        }
+    }
+    for (int it = 0; it < kMaxIt; ++it) {
+        const int bf = it & 1;
+#pragma unroll
+        for (int k = 0; k < 2; ++k) {
+            const int h = warp + 4 * k;
+            if (h >= G) continue;
+            double v[3] = {0.0, 0.0, 0.0};
+            float mnS = INFINITY, mxN = -INFINITY;
+            if (!dn[k] && !skip) {
+                const float* xr = x + (size_t)h * xstride;
+                const double tk = t[k];
+                for (int i0 = t0; i0 < t1; i0 += 32 * U) {
+                    float f[U];
+#pragma unroll
+                    for (int u = 0; u < U; ++u) {
+                        const int i = i0 + u * 32 + lane;
+                        f[u] = i < t1 ? __ldcg(xr + i) : -INFINITY;
+                    }
+#pragma unroll
+                    for (int u = 0; u < U; ++u) {
+                        const double vd = (double)f[u];
+                        if (vd > tk) {
+                            if (gen) {
+                                const float uu = (float)(vd - tk);
+                                if (uu > 0.f) {
+                                    const float p1 = powf(uu, rm1);
+                                    v[0] += (double)(p1 * uu);
+                                    v[1] += (double)p1;
+                                }
+                            } else {
+                                v[0] += 1.0;
+                                v[1] += vd;
+                                v[2] = fma(vd, vd, v[2]);
+                                mnS = fminf(mnS, f[u]);
+                            }
+                        } else if (f[u] > -INFINITY) {
+                            mxN = fmaxf(mxN, f[u]);
+                        }
+                    }
+                }
+            }
+            warp_red5(v, mnS, mxN);
+            if (lane == 0) {
+                double* pp = part + (bf * 8 + h) * 3;
+                pp[0] = v[0];
+                pp[1] = v[1];
+                pp[2] = v[2];
+                mm[(bf * 8 + h) * 2] = mnS;
+                mm[(bf * 8 + h) * 2 + 1] = mxN;
+            }
+        }
+        __syncthreads();
+        cluster_sync();
+#pragma unroll
+        for (int k = 0; k < 2; ++k) {
+            const int h = warp + 4 * k;
+            if (h >= G || dn[k]) continue;
+            double w[3] = {0.0, 0.0, 0.0};
+            float mnS = INFINITY, mxN = -INFINITY;
+            if (lane < S) {
+                const double* pp = part + (bf * 8 + h) * 3;
+#pragma unroll
+                for (int j = 0; j < 3; ++j) w[j] = __longlong_as_double((long long)ld_dsmem_u64(dsmem(pp + j, lane)));
+                mnS = ld_dsmem_f32(dsmem(&mm[(bf * 8 + h) * 2], lane));
+                mxN = ld_dsmem_f32(dsmem(&mm[(bf * 8 + h) * 2 + 1], lane));
+            }
+            warp_red5(w, mnS, mxN);
+            const double tk = t[k];
+            if (gen) {
+                const double F = w[0], S1 = r * w[1];     // F and -dF/dt
+                if (F >= 1.0) lo[k] = tk; else hi[k] = tk;
+                if (F == 1.0 || hi[k] - lo[k] <= 1e-13 * fmax(1.0, fabs(tk))) {
+                    dn[k] = true;
+                    res[k] = tk;
+                } else {
+                    double nt = (F > 0.0 && S1 > 0.0) ? tk + r * F * (1.0 - pow(F, -1.0 / r)) / S1
+                                                      : 0.5 * (lo[k] + hi[k]);
+                    if (!(nt > lo[k] && nt < hi[k])) nt = 0.5 * (lo[k] + hi[k]);
+                    if (fabs(nt - tk) <= 1e-8 * fmax(1.0, fabs(tk))) {
+                        dn[k] = true;
+                        res[k] = nt;
+                    }
+                    t[k] = nt;
+                }
+            } else {
+                const double kk = w[0], sx = w[1], sxx = w[2];
+                if (!(kk > 0.0)) {
+                    dn[k] = true;
+                    res[k] = tk;
+                } else {
+                    double tcf, next;
+                    bool ok;
+                    if (a2) {
+                        tcf = (sx - 1.0) / kk;
+                        ok = true;
+                        next = tcf;
+                    } else {
+                        const double mean = sx / kk, msq = sxx / kk;
+                        const double disc = mean * mean - msq + 1.0 / kk;
+                        ok = disc >= 0.0;
+                        tcf = ok ? mean - sqrt(disc) : 0.0;
+                        const double s1 = sx - kk * tk;
+                        const double s2 = sxx - 2.0 * tk * sx + kk * tk * tk;
+                        next = tk + (s2 - 1.0) / (2.0 * s1);
+                    }
+                    if (ok && tcf < (double)mnS && (double)mxN <= tcf && tcf >= lo[k]) {
+                        dn[k] = true;
+                        res[k] = tcf;
+                    } else if (!(next > tk) || !isfinite(next)) {
+                        dn[k] = true;
+                        res[k] = ok ? tcf : tk;
+                    } else {
+                        t[k] = next;
+                    }
+                }
+            }
+        }
+        // the same in every CTA: every head's iterates are
+        if (__syncthreads_and(dn[0] && dn[1])) break;
+    }
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+        const int h = warp + 4 * k;
+        if (h < G && lane == 0) tau_h[h] = dn[k] ? res[k] : t[k];
+    }
+    __syncthreads();
 }
 
 // List position j of (b, g) -> physical page (and logical page in lp), read
@@ -1447,11 +1616,17 @@ __global__ void __launch_bounds__(kThreads, 2) entmax_bf16_kernel(const __grid_c
     __shared__ unsigned int vbits[kBitWords];     // weighted pages of every head
     __shared__ float tau_pub[8];                  // tau of the heads this CTA solved
     __shared__ int fb_all;
+    __shared__ int nlc_s[8];
     __shared__ int wbase[kBitWords];
     // this split's bound, largest score and candidate count per head (read by
     // the other CTAs through distributed shared memory)
     __shared__ float pub_t[8], pub_m[8];
     __shared__ int pub_n[8];
+    // the cluster-wide threshold solve: partial sums per iteration parity and head
+    __shared__ double ct_part[2 * 8 * 3];
+    __shared__ float ct_mm[2 * 8 * 2];
+    __shared__ double ct_tau[8];
+    __shared__ int over_all;
 
     const int b = blockIdx.z, g = blockIdx.y, s = blockIdx.x;   // s = rank in the cluster
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -1564,34 +1739,69 @@ __global__ void __launch_bounds__(kThreads, 2) entmax_bf16_kernel(const __grid_c
     if (tid < 8) smax[tid] = tid < a.G ? fmaxf(fmaxf(wm[0][tid], wm[1][tid]), fmaxf(wm[2][tid], wm[3][tid])) : -INFINITY;
     __syncthreads();
 
-    // ------------------------------------------------------------ local bound and candidates
+    // ------------------------------------------------------------ local bound, then candidates
+    // above the group's bound (the largest of the splits' bounds)
     const int c0 = r.start * C, c1 = r.end * C;
+    if (!abort_flag) {
+        for (int h = warp, k = 0; h < a.G; h += 4, ++k) {
+            int* lc = reinterpret_cast<int*>(smem + warp * WSCR + k * LC_CAP * 8);
+            float* lcv = reinterpret_cast<float*>(smem + warp * WSCR + k * LC_CAP * 8 + LC_CAP * 4);
+            int nlc;
+            const float t = split_bound(a.cmax + (row0h + h) * cstride, c0, c1, smax[h], rpow, a2, a15, lc, lcv,
+                                        LC_CAP, &nlc);
+            if (lane == 0) {
+                pub_t[h] = t;
+                pub_m[h] = smax[h];
+                nlc_s[h] = nlc;
+            }
+        }
+    }
+    __syncthreads();
+    cluster_sync();
     if (!abort_flag) {
         for (int h = warp, k = 0; h < a.G; h += 4, ++k) {
             const size_t row = row0h + h;
             int* lc = reinterpret_cast<int*>(smem + warp * WSCR + k * LC_CAP * 8);
             float* lcv = reinterpret_cast<float*>(smem + warp * WSCR + k * LC_CAP * 8 + LC_CAP * 4);
-            int nlc;
-            const float t = split_bound(a.cmax + row * cstride, c0, c1, smax[h], rpow, a2, a15, lc, lcv, LC_CAP, &nlc);
-            const int n = local_candidates(a.xbuf + row * xstride, a.cmax + row * cstride, c0, c1, lc, lcv, nlc,
-                                           LC_CAP, t, a.cval + row * seg + (size_t)s * kCandCap,
+            float tlb = lane < a.S ? ld_dsmem_f32(dsmem(&pub_t[h], lane)) : -INFINITY;
+            tlb = warp_max(tlb);
+            const int n = local_candidates(a.xbuf + row * xstride, a.cmax + row * cstride, c0, c1, lc, lcv, nlc_s[h],
+                                           LC_CAP, tlb, a.cval + row * seg + (size_t)s * kCandCap,
                                            a.cidx + row * seg + (size_t)s * kCandCap);
-            if (lane == 0) {
-                pub_t[h] = t;
-                pub_m[h] = smax[h];
-                pub_n[h] = n;
-            }
+            if (lane == 0) pub_n[h] = n;
         }
     }
     __threadfence();   // candidates and scores in global memory are read by the other splits
     __syncthreads();
     cluster_sync();
 
-    // ------------------------------------------------------------ threshold (one CTA per head)
-    // query head h is solved by CTA h % S, on its warp (h / S) % 4; the owner
-    // keeps tau, its fallback flag and the head's weighted pages for the others
+    // ------------------------------------------------------------ threshold
+    // Every CTA reads every split's candidate counts.  When some split's
+    // candidates of a head outgrew its slots, or a head's outgrow what one warp
+    // gathers, the whole cluster solves every head (cluster_tau; the same
+    // decision in every CTA) and the V pass takes each split's own pages.
+    // Otherwise query head h is solved by CTA h % S, on its warp (h / S) % 4;
+    // the owner keeps tau and the head's weighted pages for the others.
     const bool bitmap_ok = cnt <= kBitWords * 32;
-    if (!abort_flag) {
+    if (tid < 32) {
+        bool o = false;
+        for (int h = 0; h < a.G; ++h) {
+            const int n = lane < a.S ? ld_dsmem_s32(dsmem(&pub_n[h], lane)) : 0;
+            const int tot = warp_sum(n);
+            o = o || __any_sync(0xffffffffu, n > kCandCap) || tot > CAND_CAP;
+        }
+        if (tid == 0) over_all = o;
+    }
+    __syncthreads();
+    if (over_all) {
+        cluster_tau(a.xbuf + row0h * xstride, xstride, r.start * PS, r.end * PS, pub_t, pub_m, a.G, a.S, a.alpha,
+                    abort_flag != 0, ct_part, ct_mm, ct_tau);
+        if (tid < a.G) {
+            tau_pub[tid] = (float)ct_tau[tid];
+            if (a.tau_out && tid % a.S == s) a.tau_out[row0h + tid] = (float)ct_tau[tid];
+        }
+        if (tid == 0) fallback = 1;
+    } else if (!abort_flag) {
         float* cv = reinterpret_cast<float*>(smem + warp * WSCR);
         int* ci = reinterpret_cast<int*>(smem + warp * WSCR + CAND_CAP * 4);
         for (int h = s + warp * a.S; h < a.G; h += 4 * a.S) {
@@ -1605,32 +1815,20 @@ __global__ void __launch_bounds__(kThreads, 2) entmax_bf16_kernel(const __grid_c
             }
             M = warp_max(M);
             tlb = warp_max(tlb);
-            const bool over = __any_sync(0xffffffffu, nq > kCandCap);
-            double tau;
-            int nc = -1;
-            if (!(M > -INFINITY)) {
-                tau = INFINITY;
-                nc = 0;
-            } else {
-                if (!over)
-                    nc = gather_candidates(a.cval + row * seg, a.cidx + row * seg, nq, a.S, tlb, cv, ci, CAND_CAP,
-                                           pre[warp]);
-                if (nc >= 0) {
-                    TauSrc src{nullptr, 0, cv, nc, 0, (double)tlb};
-                    tau = solve_tau(src, M, a.alpha);
-                    // value pages holding weight: the pages of the candidates above tau
-                    if (bitmap_ok)
-                        for (int k = lane; k < nc; k += 32)
-                            if ((double)cv[k] > tau) {
-                                const int pg = ci[k] / PS;
-                                atomicOr(&bits[pg >> 5], 1u << (pg & 31));
-                            }
-                } else {
-                    // more candidates than the slots hold: every score of the head above the bound
-                    TauSrc src{a.xbuf + row * xstride, cnt * PS, nullptr, 0, 1, (double)tlb};
-                    tau = solve_tau(src, M, a.alpha);
-                    if (lane == 0) fallback = 1;
-                }
+            double tau = INFINITY;
+            if (M > -INFINITY) {
+                // at most CAND_CAP candidates in all (over_all is false)
+                const int nc = gather_candidates(a.cval + row * seg, a.cidx + row * seg, nq, a.S, tlb, cv, ci,
+                                                 CAND_CAP, pre[warp]);
+                TauSrc src{cv, max(nc, 0), (double)tlb};
+                tau = solve_tau(src, M, a.alpha);
+                // value pages holding weight: the pages of the candidates above tau
+                if (bitmap_ok)
+                    for (int k = lane; k < nc; k += 32)
+                        if ((double)cv[k] > tau) {
+                            const int pg = ci[k] / PS;
+                            atomicOr(&bits[pg >> 5], 1u << (pg & 31));
+                        }
             }
             if (lane == 0) {
                 tau_pub[h] = (float)tau;

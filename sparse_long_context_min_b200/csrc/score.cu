@@ -89,9 +89,9 @@ struct ScoreArgs {
     float* e_out;
     int32_t* status;
     // appended tokens scored in the same launch (bf16 bounding boxes): n_new
-    // tokens per sequence, written by the CTAs [nscore, nscore + B) while the
-    // others score every untouched page (n_new = 0: no append)
-    int n_new, nscore;
+    // tokens per sequence, written by the CTAs [0, napp) (napp = B, or 0 when
+    // n_new = 0) while the nscore CTAs after them score every untouched page
+    int n_new, napp, nscore;
     const uint16_t* k_new;  // [B][H_kv][n_new][d]
     const uint16_t* v_new;
     uint16_t* k_pool;       // [num_phys][H_kv][ps][d]
@@ -519,10 +519,13 @@ __global__ void __launch_bounds__(BoxWsShape<D, G>::CTA, 2) score_box16_kernel(c
     using S = BoxWsShape<D, G>;
     constexpr int NST = kWsStages;
     extern __shared__ __align__(128) uint8_t box_smem[];
-    if ((int)blockIdx.x >= a.nscore) {                   // an appending CTA: no barriers below
-        append_and_score<D, G>(a, blockIdx.x - a.nscore, box_smem);
+    // appending CTAs first, so that they start with the scoring CTAs rather
+    // than in the slots the scoring CTAs leave at the end
+    if ((int)blockIdx.x < a.napp) {                      // an appending CTA: no barriers below
+        append_and_score<D, G>(a, blockIdx.x, box_smem);
         return;
     }
+    const int cta = (int)blockIdx.x - a.napp;
     int4* info = reinterpret_cast<int4*>(box_smem + S::DATA);                     // [NST][SLOTS]
     uint64_t* full = reinterpret_cast<uint64_t*>(box_smem + S::DATA + NST * S::SLOTS * 16);
     uint64_t* empty = full + NST;
@@ -531,7 +534,7 @@ __global__ void __launch_bounds__(BoxWsShape<D, G>::CTA, 2) score_box16_kernel(c
     const long long items = (long long)a.B * a.max_pages;
     const long long nchunks = (items + PPS - 1) / PPS;
     const long long per = (nchunks + a.nscore - 1) / a.nscore;
-    const long long c0 = blockIdx.x * per;
+    const long long c0 = cta * per;
     const int K = (int)max(0ll, min(nchunks, c0 + per) - c0);   // chunks of this CTA
     const size_t vecb = (size_t)a.H_kv * S::ROWB;        // one page's block of one vector
     if (tid == 0) {
@@ -658,10 +661,13 @@ static int launch_box16(const ScoreArgs& a, cudaStream_t stream)
     }
     const int pps = S::SLOTS / a.H_kv;
     const long long chunks = ((long long)a.B * a.max_pages + pps - 1) / pps;
-    const int grid = (int)std::max<long long>(1, std::min<long long>(chunks, (long long)occ[dev] * num_sms()));
-    ScoreArgs b = a;
-    b.nscore = grid;
     const int appenders = a.n_new > 0 ? a.B : 0;
+    // every CTA resident at once where the appending CTAs leave room
+    const long long slots = std::max<long long>(1, (long long)occ[dev] * num_sms() - appenders);
+    const int grid = (int)std::max<long long>(1, std::min<long long>(chunks, slots));
+    ScoreArgs b = a;
+    b.napp = appenders;
+    b.nscore = grid;
     launch_pdl(score_box16_kernel<D, G>, dim3(grid + appenders), dim3(S::CTA), S::SMEM, stream, b);
     return cudaGetLastError() == cudaSuccess ? ENTMAXKV_OK : ENTMAXKV_CUDA_ERROR;
 }

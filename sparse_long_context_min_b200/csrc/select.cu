@@ -245,12 +245,13 @@ topk_kernel(const float* __restrict__ ub, const int32_t* __restrict__ seq_lens, 
 //         of lower rank.
 constexpr int kTopkCTAs = 8;
 constexpr int kCThreads = 512;
-constexpr int kCBins = kCThreads; // one bin per thread (each CTA reads every CTA's bins)
+constexpr int kCBins = kCThreads; // one bin per thread
 constexpr int kCCap = 1024;
 constexpr int kCRounds = 40;     // each round shrinks the range >= 512x: 40 rounds cover every float range
 
 struct TopkClusterShared {
     __align__(16) int hist[kCBins];          // this CTA's histogram of the round
+    int tot[kCBins / kTopkCTAs];             // cluster totals of this CTA's slice of the bins
     unsigned long long lc[kCCap];            // this CTA's keys of the threshold bucket
     unsigned long long mc[kCCap];            // the whole cluster's, merged
     int wsum[32];
@@ -389,11 +390,20 @@ topk_cluster_kernel(const float* __restrict__ ub, const int32_t* __restrict__ se
         for (int e = 0; e < KPT; ++e)
             if (inplay(e)) atomicAdd(&sh.hist[bucket_of(kv[e], mn, w)], 1);
         cluster_sync();
-        // thread t sums bin jb = NB - 1 - t over the cluster (thread 0 the top bin)
-        const int jb = kCBins - 1 - tid;
-        int hsum = 0;
+        // cluster totals in two steps (distributed shared memory is slow for
+        // many small reads): CTA r totals its slice of kCBins / C bins over the
+        // cluster, then thread t reads the total of bin jb = NB - 1 - t (thread
+        // 0 the top bin) from the CTA that holds it
+        constexpr int SL = kCBins / C;
+        if (tid < SL) {
+            int t = 0;
 #pragma unroll
-        for (int q = 0; q < C; ++q) hsum += ld_dsmem_s32(dsmem(&sh.hist[jb], q));
+            for (int q = 0; q < C; ++q) t += ld_dsmem_s32(dsmem(&sh.hist[r * SL + tid], q));
+            sh.tot[tid] = t;
+        }
+        cluster_sync();
+        const int jb = kCBins - 1 - tid;
+        const int hsum = ld_dsmem_s32(dsmem(&sh.tot[jb % SL], jb / SL));
         const int incl = block_scan_incl(hsum, sh.wsum);
         const int above = incl - hsum;   // keys in the bins above jb
         if (above < need && need <= above + hsum) {

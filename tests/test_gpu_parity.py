@@ -511,6 +511,52 @@ def test_any_alpha_sparse_and_full(built, alpha):
             H.compare_out(full[b, g * G:(g + 1) * G], f_ref, cfg.dtype)
 
 
+@pytest.mark.parametrize("alpha", [1.5, 2.0, 1.25, 3.0])
+def test_flat_scores_cluster_threshold(alpha):
+    """Nearly equal keys put almost every token above every split's bound --
+    more candidates than a split's slots hold -- so the threshold is solved by
+    the whole cluster over every score.  129 pages per kv head (a ragged last
+    page), every page listed; against the oracle on the same keys."""
+    gen = torch.Generator().manual_seed(4242)
+    H_kv, G, d, ps = 8, 4, 128, 64
+    L = 128 * ps + 37
+    P = (L + ps - 1) // ps
+    sigma = 1e-4 if alpha == 2.0 else 0.02      # score spread small against the support's width
+    keys = (sigma * torch.randn(H_kv, L, d, generator=gen)).to(torch.bfloat16)
+    vals = torch.randn(H_kv, L, d, generator=gen).to(torch.bfloat16)
+    q = torch.randn(1, H_kv * G, d, generator=gen)
+    pool = B.Pool.allocate(P, H_kv, ps, d, torch.bfloat16, "cuda")
+    pt = torch.arange(P, dtype=torch.int32, device="cuda").view(1, P)
+    seq_lens = torch.zeros(1, dtype=torch.int32, device="cuda")
+    st = _status()
+    B.append_metadata(pool, keys.cuda().unsqueeze(0).contiguous(), vals.cuda().unsqueeze(0).contiguous(), pt,
+                      seq_lens, st)
+    sel = torch.arange(P, dtype=torch.int32, device="cuda").view(1, 1, P).repeat(1, H_kv, 1).contiguous()
+    cnt = torch.full((1, H_kv), P, dtype=torch.int32, device="cuda")
+    ws = torch.empty(B.workspace_size(B.OP_SPARSE_ATTEND, 1, H_kv * G, H_kv, P, P, ps, d), dtype=torch.uint8,
+                     device="cuda")
+    out = torch.empty(1, H_kv * G, d, device="cuda")
+    tau = torch.empty(1, H_kv * G, device="cuda")
+    qd = q.cuda()
+    scale = float(np.float32(1.0 / math.sqrt(d)))
+    B.sparse_attend(pool, qd, pt, seq_lens, sel, cnt, alpha, scale, out, ws, st, tau_out=tau)
+    _assert_ok(st)
+    out, tau = out.cpu().numpy(), tau.cpu().numpy()
+    qn = q[0].numpy()
+    for g in range(0, H_kv, 3):
+        K, V = keys[g].float().numpy(), vals[g].float().numpy()
+        o_ref, t_ref, p = attend.entmax_attention(qn[g * G:(g + 1) * G], K, V, alpha, scale)
+        # the case is the one meant: more candidates than the slots hold (16 x 256)
+        # -- every token of the support is one; for alpha > 2 every token
+        # within 1 of the largest score is one (the bound is max - 1 there)
+        x = (alpha - 1.0) * scale * (K.astype(np.float64) @ qn[g * G:(g + 1) * G].astype(np.float64).T)
+        for h in range(G):
+            n_cand = np.count_nonzero(p[h]) if alpha <= 2.0 else np.count_nonzero(x[:, h] > x[:, h].max() - 1.0)
+            assert n_cand > 16 * 256, n_cand
+        H.compare_out(out[0, g * G:(g + 1) * G], o_ref, torch.bfloat16)
+        assert np.all(np.abs(tau[0, g * G:(g + 1) * G] - t_ref) <= 1e-5 * np.maximum(1, np.abs(t_ref)))
+
+
 def test_support_recovery_on_gpu():
     """If the kept pages hold the support, sparse == full (oracle: bitwise)."""
     wl = _wl(2, [8192 + 33])
