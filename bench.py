@@ -7,8 +7,10 @@ write + page metadata), score every page (bounding-box bound), select the top
 1/64 of pages per kv head, and run exact 1.5-entmax attention over the
 selected pages.  Workload: B=1 sequence of 2^20 tokens per GPU, 32 query / 8
 kv heads, head dim 128, pages of 64, bf16 cache (synthetic clustered keys with
-planted tokens).  L2 is flushed (a 256 MiB write) between timed steps, outside
-the per-step CUDA events.  Rank 0 prints one JSON line.
+planted tokens).  L2 is flushed between timed steps, outside the per-step
+CUDA events: a 256 MiB buffer is written, then a second 256 MiB buffer is
+read, so that the written lines are back in HBM before the step starts.  Rank
+0 prints one JSON line.
 
 --impl reference times the CPU oracle on the host cores instead (rank 0 only).
 """
@@ -36,6 +38,25 @@ HBM_NOMINAL_GBS = 8000.0
 PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
 FALLBACK_HBM_GBS = 6650.0
 MiB = 1 << 20
+
+
+class L2Flush:
+    """Evicts the step's data from L2 between timed steps: a 256 MiB write,
+    then a read of another 256 MiB buffer, so that the write's dirty lines
+    drain to HBM here rather than inside the next step (L2 is 126 MB); no
+    host synchronisation."""
+
+    def __init__(self):
+        self.w = torch.empty(256 * MiB, dtype=torch.uint8, device="cuda")
+        self.r = torch.ones(256 * MiB, dtype=torch.uint8, device="cuda")
+        self.sink = torch.zeros((), dtype=torch.int64, device="cuda")
+
+    def __call__(self, i):
+        self.w.fill_(i & 0xFF)
+        torch.sum(self.r, dim=0, dtype=torch.int64, out=self.sink)
+
+    def fill_(self, v):
+        self(v)
 
 
 def parse():
@@ -286,7 +307,7 @@ def native_line(cfg, world, K, W, mean_us, best_us, median_us, score_us, stage, 
             "global_batch": world,
             "seq_len": cfg.lengths[0],
             "parallelism": "replicas: one independent sequence per GPU" if world > 1 else "single GPU",
-            "l2": "flushed between steps (256 MiB write outside the step events)",
+            "l2": "flushed between steps outside the step events (256 MiB written, then another 256 MiB read)",
             "selected_pages_per_step": round(sel_total, 1),
             "value_pages_loaded_per_step": round(v_total, 1),
             "algorithmic_bytes_per_step": by["total"],
@@ -321,7 +342,7 @@ def native_line(cfg, world, K, W, mean_us, best_us, median_us, score_us, stage, 
 def timed_replays(gs, step, toks, warm, steps, flush, stream, stages=False):
     """`warm` + `steps` replays of a graphed step, issued back to back with no
     host synchronisation: per step the step's inputs are copied in (device to
-    device), the L2 is flushed (256 MiB write) and the replay is bracketed by
+    device), the L2 is flushed (L2Flush) and the replay is bracketed by
     CUDA events on the stream; the selected and loaded-value page counts add up
     on the device.  Returns (per-step us, mean selected page-heads, mean value
     page-heads, mean stage us or None)."""
@@ -335,7 +356,7 @@ def timed_replays(gs, step, toks, warm, steps, flush, stream, stages=False):
         gs.k.copy_(k)
         gs.v.copy_(v)
         step.v_pages.zero_()
-        flush.fill_(i & 0xFF)
+        flush(i)
         j = i - warm
         if j >= 0:
             ev[j][0].record(stream)
@@ -373,7 +394,7 @@ def run_native(args, rank, world, local):
     pool, seq_lens = build_pool(wl)
     torch.cuda.synchronize()
     stream = torch.cuda.current_stream()
-    flush = torch.empty(256 * MiB, dtype=torch.uint8, device="cuda")
+    flush = L2Flush()
 
     # ---- headline: top-k 1/64, K graphed steps bracketed by barrier + sync
     step = DecodeStep(pool, wl.page_table, seq_lens, cfg.H_q, "topk", budget_frac=1 / 64, alpha=cfg.alpha)
@@ -459,7 +480,7 @@ def run_e2e(wl, pool, seq_lens, K, W, flush):
         host.append(gs.pack_host(k, v, q))
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
     for i in range(W + K):
-        flush.fill_(i & 0xFF)
+        flush(i)
         j = i - W
         if j >= 0:
             ev[j][0].record(stream)
@@ -488,7 +509,7 @@ def run_full(wl, pool, seq_lens, flush, reps=5, warm=3):
                          dtype=torch.uint8, device="cuda")
         times = []
         for i in range(warm + reps):
-            flush.fill_(i & 0xFF)
+            flush(i)
             a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             a.record(stream)
             if op == BND.OP_FULL_ENTMAX:
@@ -538,7 +559,7 @@ def run_attend_variants(wl, pool, seq_lens, flush, reps=5, warm=3):
     for name, fn in calls.items():
         times = []
         for i in range(warm + reps):
-            flush.fill_(i & 0xFF)
+            flush(i)
             a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             a.record(stream)
             fn()
@@ -768,7 +789,7 @@ def selector_sweep(args):
     torch.cuda.set_device(0)
     W, K = args.warmup, min(args.steps, 200)
     stream = torch.cuda.current_stream()
-    flush = torch.empty(256 * MiB, dtype=torch.uint8, device="cuda")
+    flush = L2Flush()
     for ctx in (1 << 18, 1 << 19, 1 << 20):
         wl = make_workload(ctx, 0, appends=2 * (W + K) + 64)
         cfg = wl.cfg
@@ -800,11 +821,11 @@ def replay_only(args):
     st = DecodeStep(pool, wl.page_table, seq_lens, cfg.H_q, args.replay_only, budget_frac=1 / 64,
                     alpha=cfg.alpha, delta=0.5)
     gs = GraphedStep(st, append=True, stage_events=False)
-    flush = torch.empty(256 * MiB, dtype=torch.uint8, device="cuda")
+    flush = L2Flush()
     for i in range(args.steps):
         k, v, q = wl.decode_token(i)
         gs.inputs.copy_(gs.pack_host(k, v, q), non_blocking=True)
-        flush.fill_(i & 0xFF)
+        flush(i)
         gs.replay()
     torch.cuda.synchronize()
     st.check()

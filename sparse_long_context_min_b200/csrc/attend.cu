@@ -1213,16 +1213,19 @@ EKV_DEV int local_candidates(const float* x, const float* cm, int c0, int c1, in
     return nc;
 }
 
-// The group's candidates of one head above tlb, gathered by one warp from the
-// S splits' slots (global: split q's at cval + q * kCandCap, n_q of them,
-// lane q holding n_q) into (cv, ci), in split order; returns how many (-1 when
-// more than cap).  pre: per-warp shared scratch of S + 1 ints.
-EKV_DEV int gather_candidates(const float* cval, const int* cidx, int nq, int S, float tlb, float* cv, int* ci,
-                              int cap, int* pre)
+// The group's candidates of one head (every one above the group's bound),
+// gathered by one warp from the S splits' slots (global: split q's n_q of them
+// at cval + q * kCandCap, lane q holding n_q) into (cv, ci) in one round trip:
+// 16-byte asynchronous copies, split q's at the next 4-entry boundary, the up
+// to three entries past its count set to -inf (no candidate).  Returns the
+// entries written, gaps included (-1 when more than cap).  pre: per-warp
+// shared scratch of S + 1 ints.
+EKV_DEV int gather_candidates(const float* cval, const int* cidx, int nq, int S, float* cv, int* ci, int cap,
+                              int* pre)
 {
     const int lane = threadIdx.x & 31;
-    const unsigned below = (1u << lane) - 1u;
-    int incl = nq;
+    const int n4 = lane < S ? (nq + 3) & ~3 : 0;
+    int incl = n4;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
         const int t = __shfl_up_sync(0xffffffffu, incl, o);
@@ -1232,42 +1235,22 @@ EKV_DEV int gather_candidates(const float* cval, const int* cidx, int nq, int S,
     if (lane == 0) pre[0] = 0;
     const int total = __shfl_sync(0xffffffffu, incl, 31);
     __syncwarp();
-    int bounds[kFusedMaxSplits + 1];                   // prefix sums, in registers
-#pragma unroll
-    for (int q = 0; q <= kFusedMaxSplits; ++q) bounds[q] = q <= S ? pre[q] : total;
-    constexpr int U = 4;
-    int n = 0;
-    for (int k0 = 0; k0 < total; k0 += 32 * U) {
-        float v[U];
-        int p[U];
-#pragma unroll
-        for (int u = 0; u < U; ++u) {
-            const int k = k0 + u * 32 + lane;
-            int q = 0, before = 0;                     // split q holds candidates [pre[q], pre[q + 1])
-#pragma unroll
-            for (int j = 1; j <= kFusedMaxSplits; ++j)
-                if (k >= bounds[j]) {
-                    q = j;
-                    before = bounds[j];
-                }
-            const size_t off = (size_t)q * kCandCap + (k - before);
-            v[u] = k < total ? __ldcg(cval + off) : -INFINITY;
-            p[u] = k < total ? __ldcg(cidx + off) : 0;
-        }
-#pragma unroll
-        for (int u = 0; u < U; ++u) {
-            const bool keep = v[u] > tlb;
-            const unsigned m = __ballot_sync(0xffffffffu, keep);
-            const int q = n + __popc(m & below);
-            if (keep && q < cap) {
-                cv[q] = v[u];
-                ci[q] = p[u];
-            }
-            n += __popc(m);
+    if (total > cap) return -1;
+    const uint32_t vbase = smem_addr(cv), ibase = smem_addr(ci);
+    for (int q = 0; q < S; ++q) {
+        const int o = pre[q], chunks = (pre[q + 1] - o) >> 2;
+        for (int c = lane; c < chunks; c += 32) {
+            cp_async16(vbase + 4u * (uint32_t)(o + 4 * c), cval + (size_t)q * kCandCap + 4 * c);
+            cp_async16(ibase + 4u * (uint32_t)(o + 4 * c), cidx + (size_t)q * kCandCap + 4 * c);
         }
     }
+    cp_async_commit();
+    cp_async_wait<0>();
     __syncwarp();
-    return n <= cap ? n : -1;
+    if (lane < S)
+        for (int j = nq; j < n4; ++j) cv[pre[lane] + j] = -INFINITY;
+    __syncwarp();
+    return total;
 }
 
 // tau from the candidates of src, one warp, every lane returns it.
@@ -1787,7 +1770,7 @@ __global__ void __launch_bounds__(kThreads, 2) entmax_bf16_kernel(const __grid_c
         bool o = false;
         for (int h = 0; h < a.G; ++h) {
             const int n = lane < a.S ? ld_dsmem_s32(dsmem(&pub_n[h], lane)) : 0;
-            const int tot = warp_sum(n);
+            const int tot = warp_sum((n + 3) & ~3);           // as gathered: 4-entry aligned per split
             o = o || __any_sync(0xffffffffu, n > kCandCap) || tot > CAND_CAP;
         }
         if (tid == 0) over_all = o;
@@ -1817,9 +1800,9 @@ __global__ void __launch_bounds__(kThreads, 2) entmax_bf16_kernel(const __grid_c
             tlb = warp_max(tlb);
             double tau = INFINITY;
             if (M > -INFINITY) {
-                // at most CAND_CAP candidates in all (over_all is false)
-                const int nc = gather_candidates(a.cval + row * seg, a.cidx + row * seg, nq, a.S, tlb, cv, ci,
-                                                 CAND_CAP, pre[warp]);
+                // at most CAND_CAP entries in all (over_all is false)
+                const int nc = gather_candidates(a.cval + row * seg, a.cidx + row * seg, nq, a.S, cv, ci, CAND_CAP,
+                                                 pre[warp]);
                 TauSrc src{cv, max(nc, 0), (double)tlb};
                 tau = solve_tau(src, M, a.alpha);
                 // value pages holding weight: the pages of the candidates above tau

@@ -92,6 +92,24 @@ EKV_DEV uint64_t global_ns()
     return t;
 }
 
+// try_wait that lets the hardware suspend the thread until the phase
+// completes or about hint_ns elapse, so that waiting warps do not spin on the
+// issue slots the working warps of the SM need.
+EKV_DEV bool mbar_try_wait_for(uint64_t* bar, uint32_t parity, uint32_t hint_ns)
+{
+    uint32_t ok;
+    asm volatile(
+        "{\n"
+        " .reg .pred p;\n"
+        " mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n"
+        " selp.u32 %0, 1, 0, p;\n"
+        "}\n"
+        : "=r"(ok)
+        : "r"(smem_addr(bar)), "r"(parity), "r"(hint_ns)
+        : "memory");
+    return ok != 0;
+}
+
 // Bounded wait for the phase with the given parity to complete.  Returns false
 // when limit_ns elapsed first (the caller reports ENTMAXKV_TIMEOUT).
 EKV_DEV bool mbar_wait(uint64_t* bar, uint32_t parity, uint64_t limit_ns)
@@ -99,7 +117,7 @@ EKV_DEV bool mbar_wait(uint64_t* bar, uint32_t parity, uint64_t limit_ns)
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = global_ns();
     while (true) {
-        if (mbar_try_wait(bar, parity)) return true;
+        if (mbar_try_wait_for(bar, parity, 100000u)) return true;
         if (global_ns() - t0 > limit_ns) return false;
     }
 }

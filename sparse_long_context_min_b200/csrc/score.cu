@@ -278,8 +278,9 @@ score_kernel(const ScoreArgs a, const ZTable zt)
 //    PPS pages: it resolves each page (page-table entries loaded 32 at a time,
 //    ahead of use), writes (sequence, page, tokens) of the chunk's pages into
 //    the stage header and copies each page's k_min and k_max blocks (all kv
-//    heads, contiguous in the pool) with bulk copies (TMA) whose bytes
-//    complete the stage's `full` mbarrier.  It refills a stage once all
+//    heads, contiguous in the pool; one copy per run of consecutive physical
+//    pages) with bulk copies (TMA) whose bytes complete the stage's `full`
+//    mbarrier.  It refills a stage once all
 //    consumer warps have arrived on its `empty` mbarrier.
 //  * kWsConsumers consumer warps each own kWsRounds x RPW fixed (page slot,
 //    kv head) rows of every stage, all of the same kv heads, so their query
@@ -389,14 +390,26 @@ EKV_DEV void ws_produce(const ScoreArgs& a, uint8_t* data, int stageb, int slots
             pp -= a.max_pages;
             ++bb;
         }
-        const unsigned copies = __ballot_sync(0xffffffffu, lane < PPS && n > 0);
+        // one copy per run of slots whose physical pages are consecutive (the
+        // blocks of consecutive pages are contiguous in the pool and in the stage)
+        const bool mem = lane < PPS && n > 0;
+        const unsigned copies = __ballot_sync(0xffffffffu, mem);
+        const int prev = __shfl_up_sync(0xffffffffu, pt, 1);
+        const bool start = mem && (lane == 0 || !((copies >> (lane - 1)) & 1u) || pt != prev + 1);
+        const unsigned starts = __ballot_sync(0xffffffffu, start);
         __syncwarp();                                    // header writes before the arrive
         if (lane == 0) mbar_arrive_expect_tx(&full[s], (uint32_t)(__popc(copies) * 2 * vecb));
-        if (lane < PPS && n > 0) {
-            uint8_t* dst = data + (size_t)s * stageb + lane * 2 * vecb;
+        if (start) {
+            const unsigned after = starts & ~((2u << lane) - 1u);            // later run starts
+            const int stop = after ? __ffs(after) - 1 : PPS;
+            const unsigned rest = ~(copies >> lane);                         // 0 bits: members from lane on
+            const int gap = rest ? __ffs(rest) - 1 : 32 - lane;
+            const int len = min(stop - lane, gap);
+            uint8_t* dst = data + (size_t)s * stageb + (size_t)lane * vecb;
             const size_t off = (size_t)pt * vecb;
-            bulk_load(dst, static_cast<const uint8_t*>(a.row_a) + off, (uint32_t)vecb, &full[s]);
-            bulk_load(dst + vecb, static_cast<const uint8_t*>(a.row_b) + off, (uint32_t)vecb, &full[s]);
+            bulk_load(dst, static_cast<const uint8_t*>(a.row_a) + off, (uint32_t)(len * vecb), &full[s]);
+            bulk_load(dst + (size_t)PPS * vecb, static_cast<const uint8_t*>(a.row_b) + off, (uint32_t)(len * vecb),
+                      &full[s]);
         }
     }
 }
@@ -557,7 +570,9 @@ __global__ void __launch_bounds__(BoxWsShape<D, G>::CTA, 2) score_box16_kernel(c
     const int slot = warp * S::RPW + rw;                 // row of round 0; round r adds r * SET
     const int g = slot % a.H_kv, pi = slot / a.H_kv;     // kv head and page of this row (round 0)
     const int ppr = S::SET / a.H_kv;                     // pages per round (host checks H_kv | SET)
-    const uint32_t rowoff = (uint32_t)(pi * 2 * vecb + g * S::ROWB + ks * S::SW * 2);
+    // stage layout: the k_min blocks of the stage's PPS pages, then their k_max blocks
+    const uint32_t rowoff = (uint32_t)(pi * vecb + g * S::ROWB + ks * S::SW * 2);
+    const uint32_t maxoff = (uint32_t)(PPS * vecb);
     const uint32_t sbase = smem_addr(box_smem);
     uint64_t qp[S::SW];                                  // (head 0, head 1) query pairs per coordinate
     float qs[S::SW];                                     // single head (HPT == 1)
@@ -601,12 +616,12 @@ __global__ void __launch_bounds__(BoxWsShape<D, G>::CTA, 2) score_box16_kernel(c
 #pragma unroll
             for (int i = 0; i < S::HPT; ++i) acc[i] = 0.f;
             if (n > 0) {
-                const uint32_t src = sbase + (uint32_t)(s * S::STAGEB) + rowoff + (uint32_t)(r * ppr * 2 * vecb);
+                const uint32_t src = sbase + (uint32_t)(s * S::STAGEB) + rowoff + (uint32_t)(r * ppr * vecb);
                 uint64_t acc2 = pack2(0.f, 0.f);
 #pragma unroll
                 for (int c = 0; c < S::NV; ++c) {
                     const uint4 va = lds128(src + 16 * c);
-                    const uint4 vb = lds128(src + (uint32_t)vecb + 16 * c);
+                    const uint4 vb = lds128(src + maxoff + 16 * c);
                     const uint32_t wa[4] = {va.x, va.y, va.z, va.w};
                     const uint32_t wb[4] = {vb.x, vb.y, vb.z, vb.w};
 #pragma unroll

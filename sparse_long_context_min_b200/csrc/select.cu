@@ -52,7 +52,7 @@ struct TopkShared {
     int hist[kBins];
     unsigned long long cand[kRankCap];
     int wsum[32];
-    float redf[32];
+    unsigned int redk[32];
     int ncand;
     int bucket;
     int need;
@@ -85,57 +85,63 @@ topk_kernel(const float* __restrict__ ub, const int32_t* __restrict__ seq_lens, 
         return;
     }
 
-    // --- find the k-th key (thr_key, thr_idx) in the order (key desc, index asc)
-    float lo_v = -INFINITY, hi_v = INFINITY;   // current value range [lo_v, hi_v]
+    // --- find the k-th key (thr_key, thr_idx) in the order (key desc, index asc),
+    // on ordered 32-bit keys (monotone in the float order, -0 as +0, infinities
+    // included); buckets are a float multiple of the offset from the minimum
+    auto key_at = [&](int i) { return ordered_key(keys[i]); };
+    auto bmin = [&](unsigned int v) {
+        v = __reduce_min_sync(0xffffffffu, v);
+        __syncthreads();
+        if ((tid & 31) == 0) sh.redk[tid >> 5] = v;
+        __syncthreads();
+        return __reduce_min_sync(0xffffffffu, sh.redk[tid & 31]);
+    };
+    auto bmax = [&](unsigned int v) {
+        v = __reduce_max_sync(0xffffffffu, v);
+        __syncthreads();
+        if ((tid & 31) == 0) sh.redk[tid >> 5] = v;
+        __syncthreads();
+        return __reduce_max_sync(0xffffffffu, sh.redk[tid & 31]);
+    };
+    unsigned int lo_k = 0u, hi_k = 0xFFFFFFFFu;   // current key range [lo_k, hi_k]
     int need = k;
     bool done = false;
     unsigned int thr_key = 0;
     int thr_idx = 0;
     for (int round = 0; round < 8 && !done; ++round) {
-        float mn = INFINITY, mx = -INFINITY;
+        unsigned int mn = 0xFFFFFFFFu, mx = 0u;
         for (int i = tid; i < P; i += kSelThreads) {
-            float v = keys[i];
-            if (v == 0.f) v = 0.f;
-            if (v >= lo_v && v <= hi_v) { mn = fminf(mn, v); mx = fmaxf(mx, v); }
+            const unsigned int v = key_at(i);
+            if (v >= lo_k && v <= hi_k) { mn = min(mn, v); mx = max(mx, v); }
         }
-        mn = block_min(mn, sh.redf);
-        mx = block_max(mx, sh.redf);
+        mn = bmin(mn);
+        mx = bmax(mx);
         if (mn == mx) {
             // every key in range is equal: the need-th lowest index among them
-            thr_key = ordered_key(mn);
+            thr_key = mn;
             const int per = (P + kSelThreads - 1) / kSelThreads;
             const int i0 = tid * per, i1 = min(P, i0 + per);
             int c = 0;
-            for (int i = i0; i < i1; ++i) {
-                float v = keys[i];
-                if (v == 0.f) v = 0.f;
-                c += (v == mn);
-            }
+            for (int i = i0; i < i1; ++i) c += (key_at(i) == mn);
             const int incl = block_scan_incl(c, sh.wsum);
             int before = incl - c;
-            for (int i = i0; i < i1; ++i) {
-                float v = keys[i];
-                if (v == 0.f) v = 0.f;
-                if (v == mn) {
+            for (int i = i0; i < i1; ++i)
+                if (key_at(i) == mn) {
                     if (before == need - 1) sh.thr_idx = i;
                     ++before;
                 }
-            }
             __syncthreads();
             thr_idx = sh.thr_idx;
             done = true;
             break;
         }
-        const float w = (float)kBins / (mx - mn);
+        const float w = (float)kBins / ((float)(mx - mn) + 1.0f);
+        auto bucket_of = [&](unsigned int v) { return min((int)((float)(v - mn) * w), kBins - 1); };
         for (int i = tid; i < kBins; i += kSelThreads) sh.hist[i] = 0;
         __syncthreads();
         for (int i = tid; i < P; i += kSelThreads) {
-            float v = keys[i];
-            if (v == 0.f) v = 0.f;
-            if (v >= mn && v <= mx) {
-                const int bk = (int)fminf((v - mn) * w, (float)(kBins - 1));
-                atomicAdd(&sh.hist[bk], 1);
-            }
+            const unsigned int v = key_at(i);
+            if (v >= mn && v <= mx) atomicAdd(&sh.hist[bucket_of(v)], 1);
         }
         __syncthreads();
         // suffix counts: thread t owns bins kBins-1-2t and kBins-2-2t (descending)
@@ -153,31 +159,29 @@ topk_kernel(const float* __restrict__ ub, const int32_t* __restrict__ seq_lens, 
         __syncthreads();
         const int T = sh.bucket;
         need = sh.need;
-        // value range of bucket T
-        float bmn = INFINITY, bmx = -INFINITY;
+        // key range of bucket T
+        unsigned int bmn = 0xFFFFFFFFu, bmx = 0u;
         for (int i = tid; i < P; i += kSelThreads) {
-            float v = keys[i];
-            if (v == 0.f) v = 0.f;
-            if (v >= mn && v <= mx && (int)fminf((v - mn) * w, (float)(kBins - 1)) == T) {
-                bmn = fminf(bmn, v);
-                bmx = fmaxf(bmx, v);
+            const unsigned int v = key_at(i);
+            if (v >= mn && v <= mx && bucket_of(v) == T) {
+                bmn = min(bmn, v);
+                bmx = max(bmx, v);
             }
         }
-        bmn = block_min(bmn, sh.redf);
-        bmx = block_max(bmx, sh.redf);
-        lo_v = bmn;
-        hi_v = bmx;
+        bmn = bmin(bmn);
+        bmx = bmax(bmx);
+        lo_k = bmn;
+        hi_k = bmx;
         const int cnt = sh.hist[T];
         if (cnt <= kRankCap && bmn != bmx) {
             if (tid == 0) sh.ncand = 0;
             __syncthreads();
             for (int i = tid; i < P; i += kSelThreads) {
-                float v = keys[i];
-                if (v == 0.f) v = 0.f;
-                if (v >= lo_v && v <= hi_v) {
+                const unsigned int v = key_at(i);
+                if (v >= lo_k && v <= hi_k) {
                     const int slot = atomicAdd(&sh.ncand, 1);
                     if (slot < kRankCap)
-                        sh.cand[slot] = ((unsigned long long)ordered_key(v) << 32) |
+                        sh.cand[slot] = ((unsigned long long)v << 32) |
                                         (unsigned long long)(0xFFFFFFFFu - (unsigned)i);
                 }
             }
@@ -199,7 +203,7 @@ topk_kernel(const float* __restrict__ ub, const int32_t* __restrict__ seq_lens, 
         }
         __syncthreads();
     }
-    if (!done) {   // cannot happen for finite keys; keep the output well formed
+    if (!done) {   // cannot happen (a few rounds reach one value); keep the output well formed
         if (tid == 0) report(status, ENTMAXKV_DEVICE_BOUNDS);
         thr_key = 0xFFFFFFFFu;
         thr_idx = -1;
@@ -235,19 +239,22 @@ topk_kernel(const float* __restrict__ ub, const int32_t* __restrict__ seq_lens, 
 // (range, histogram, candidates, counts) in shared memory and every CTA reads
 // all of them through distributed shared memory, so all CTAs take identical
 // decisions and meet the same cluster barriers.
-//  round: [min, max] of the keys in play; if equal, the keys in play are
-//         tied and the `need` lowest indices among them are kept; otherwise
-//         a 512-bin histogram over a linear map of [min, max] gives the
+//  round: [min, max] of the keys in play (as ordered 32-bit keys); if equal,
+//         the keys in play are tied and the `need` lowest indices among them
+//         are kept; otherwise a 512-bin histogram over a linear map of
+//         [min, max] gives the
 //         bucket T holding the need-th key; if T holds at most kCCap keys
-//         they are gathered and ranked exactly, else the next round
-//         narrows to T.
+//         they are gathered and ranked exactly (all pairs compared), else
+//         the next round narrows to T.
+//  The keys are read coalesced into shared memory, then each thread takes
+//  its KPT consecutive ones.
 //  emit:  kept pages in page order, offset by the kept counts of the CTAs
 //         of lower rank.
 constexpr int kTopkCTAs = 8;
 constexpr int kCThreads = 512;
 constexpr int kCBins = kCThreads; // one bin per thread
-constexpr int kCCap = 1024;
-constexpr int kCRounds = 40;     // each round shrinks the range >= 512x: 40 rounds cover every float range
+constexpr int kCCap = 128;      // exact ranking is quadratic: larger buckets narrow once more
+constexpr int kCRounds = 40;     // each round shrinks the key range about 512-fold: a few rounds reach one value
 
 struct TopkClusterShared {
     __align__(16) int hist[kCBins];          // this CTA's histogram of the round
@@ -255,9 +262,9 @@ struct TopkClusterShared {
     unsigned long long lc[kCCap];            // this CTA's keys of the threshold bucket
     unsigned long long mc[kCCap];            // the whole cluster's, merged
     int wsum[32];
-    float redf[2][32];
-    float pub_mm[2];                         // this CTA's range of the keys in play
-    float g_mm[2];
+    unsigned int redk[2][32];
+    unsigned int pub_mm[2];                  // this CTA's range of the keys in play (ordered keys)
+    unsigned int g_mm[2];
     int lcn;                                 // entries of lc
     int pub_tie;                             // this CTA's tied keys (tie round)
     int pub_kept;                            // this CTA's kept keys
@@ -296,22 +303,29 @@ topk_cluster_kernel(const float* __restrict__ ub, const int32_t* __restrict__ se
         return;
     }
     const int i0 = (r * kCThreads + tid) * KPT;
-    float kv[KPT];
+    __shared__ unsigned int kst[kCThreads * KPT];
 #pragma unroll
     for (int e = 0; e < KPT; ++e) {
-        const int i = i0 + e;
-        float v = i < P ? __ldg(keys + i) : -INFINITY;
-        if (v == 0.f) v = 0.f;
-        kv[e] = v;
+        const int i = r * kCThreads * KPT + e * kCThreads + tid;
+        kst[e * kCThreads + tid] = i < P ? ordered_key(__ldg(keys + i)) : 0u;
     }
-    // keys in play: valid, inside [lo_v, hi_v] and in bucket pT of the previous
-    // round's map (pmn, pw); round 0 takes every valid key
-    float lo_v = -INFINITY, hi_v = INFINITY, pmn = 0.f, pw = 0.f;
+    __syncthreads();
+    unsigned int kv[KPT];                 // ordered keys (-0 as +0), page order
+#pragma unroll
+    for (int e = 0; e < KPT; ++e) kv[e] = kst[tid * KPT + e];
+    // keys in play: valid, inside [lo_k, hi_k] and in bucket pT of the previous
+    // round's map (plo, pw); round 0 takes every valid key.  Buckets are a
+    // float multiple of the ordered-key offset: monotone, so they keep the key
+    // order, and infinities need no special case.
+    unsigned int lo_k = 0u, hi_k = 0xFFFFFFFFu, plo = 0u;
+    float pw = 0.f;
     int pT = -1;
-    auto bucket_of = [](float v, float mn, float w) { return (int)fminf((v - mn) * w, (float)(kCBins - 1)); };
+    auto bucket_of = [](unsigned int v, unsigned int lo, float w) {
+        return min((int)((float)(v - lo) * w), kCBins - 1);
+    };
     auto inplay = [&](int e) {
-        if (!(i0 + e < P && kv[e] >= lo_v && kv[e] <= hi_v)) return false;
-        return pT < 0 || bucket_of(kv[e], pmn, pw) == pT;
+        if (!(i0 + e < P && kv[e] >= lo_k && kv[e] <= hi_k)) return false;
+        return pT < 0 || bucket_of(kv[e], plo, pw) == pT;
     };
     int need = k;
     int mode = 0;           // 0 searching, 1 threshold (thr_key, thr_idx), 2 tie (thr_idx per thread)
@@ -319,25 +333,23 @@ topk_cluster_kernel(const float* __restrict__ ub, const int32_t* __restrict__ se
     int thr_idx = -1;
     for (int round = 0; round < kCRounds && mode == 0; ++round) {
         // --- range of the keys in play, over the cluster
-        float mn = INFINITY, mx = -INFINITY;
+        unsigned int mn = 0xFFFFFFFFu, mx = 0u;
 #pragma unroll
         for (int e = 0; e < KPT; ++e)
             if (inplay(e)) {
-                mn = fminf(mn, kv[e]);
-                mx = fmaxf(mx, kv[e]);
+                mn = min(mn, kv[e]);
+                mx = max(mx, kv[e]);
             }
-        mn = warp_min(mn);
-        mx = warp_max(mx);
+        mn = __reduce_min_sync(0xffffffffu, mn);
+        mx = __reduce_max_sync(0xffffffffu, mx);
         if (lane == 0) {
-            sh.redf[0][warp] = mn;
-            sh.redf[1][warp] = mx;
+            sh.redk[0][warp] = mn;
+            sh.redk[1][warp] = mx;
         }
         __syncthreads();
         if (warp == 0) {
-            float a = lane < kCThreads / 32 ? sh.redf[0][lane] : INFINITY;
-            float c = lane < kCThreads / 32 ? sh.redf[1][lane] : -INFINITY;
-            a = warp_min(a);
-            c = warp_max(c);
+            const unsigned int a = __reduce_min_sync(0xffffffffu, lane < kCThreads / 32 ? sh.redk[0][lane] : 0xFFFFFFFFu);
+            const unsigned int c = __reduce_max_sync(0xffffffffu, lane < kCThreads / 32 ? sh.redk[1][lane] : 0u);
             if (lane == 0) {
                 sh.pub_mm[0] = a;
                 sh.pub_mm[1] = c;
@@ -345,10 +357,10 @@ topk_cluster_kernel(const float* __restrict__ ub, const int32_t* __restrict__ se
         }
         cluster_sync();
         if (warp == 0) {
-            float a = lane < C ? ld_dsmem_f32(dsmem(&sh.pub_mm[0], lane)) : INFINITY;
-            float c = lane < C ? ld_dsmem_f32(dsmem(&sh.pub_mm[1], lane)) : -INFINITY;
-            a = warp_min(a);
-            c = warp_max(c);
+            const unsigned int a = __reduce_min_sync(
+                0xffffffffu, lane < C ? (unsigned)ld_dsmem_s32(dsmem(&sh.pub_mm[0], lane)) : 0xFFFFFFFFu);
+            const unsigned int c =
+                __reduce_max_sync(0xffffffffu, lane < C ? (unsigned)ld_dsmem_s32(dsmem(&sh.pub_mm[1], lane)) : 0u);
             if (lane == 0) {
                 sh.g_mm[0] = a;
                 sh.g_mm[1] = c;
@@ -359,7 +371,7 @@ topk_cluster_kernel(const float* __restrict__ ub, const int32_t* __restrict__ se
         mx = sh.g_mm[1];
         if (mn == mx) {
             // every key in play equals mn: keep the `need` lowest indices of them
-            thr_key = ordered_key(mn);
+            thr_key = mn;
             int c = 0;
 #pragma unroll
             for (int e = 0; e < KPT; ++e) c += inplay(e);
@@ -383,7 +395,7 @@ topk_cluster_kernel(const float* __restrict__ ub, const int32_t* __restrict__ se
             break;
         }
         // --- histogram; this CTA's is read by the cluster after the barrier
-        const float w = (float)kCBins / (mx - mn);
+        const float w = (float)kCBins / ((float)(mx - mn) + 1.0f);
         for (int i = tid; i < kCBins; i += kCThreads) sh.hist[i] = 0;
         __syncthreads();
 #pragma unroll
@@ -423,7 +435,7 @@ topk_cluster_kernel(const float* __restrict__ ub, const int32_t* __restrict__ se
             for (int e = 0; e < KPT; ++e)
                 if (inplay(e) && bucket_of(kv[e], mn, w) == T) {
                     const int slot = atomicAdd(&sh.lcn, 1);
-                    sh.lc[slot] = ((unsigned long long)ordered_key(kv[e]) << 32) |
+                    sh.lc[slot] = ((unsigned long long)kv[e] << 32) |
                                   (unsigned long long)(0xFFFFFFFFu - (unsigned)(i0 + e));
                 }
             cluster_sync();
@@ -461,9 +473,9 @@ topk_cluster_kernel(const float* __restrict__ ub, const int32_t* __restrict__ se
             thr_idx = sh.thr_idx;
             mode = 1;
         } else {
-            lo_v = mn;
-            hi_v = mx;
-            pmn = mn;
+            lo_k = mn;
+            hi_k = mx;
+            plo = mn;
             pw = w;
             pT = T;
         }
@@ -474,7 +486,7 @@ topk_cluster_kernel(const float* __restrict__ ub, const int32_t* __restrict__ se
     int c = 0;
 #pragma unroll
     for (int e = 0; e < KPT; ++e) {
-        const unsigned kk = ordered_key(kv[e]);
+        const unsigned kk = kv[e];
         c += (i0 + e < P) && ((kk > thr_key) || (kk == thr_key && i0 + e <= thr_idx));
     }
     const int incl = block_scan_incl(c, sh.wsum);
@@ -494,7 +506,7 @@ topk_cluster_kernel(const float* __restrict__ ub, const int32_t* __restrict__ se
     int pos = sh.before + incl - c;
 #pragma unroll
     for (int e = 0; e < KPT; ++e) {
-        const unsigned kk = ordered_key(kv[e]);
+        const unsigned kk = kv[e];
         if ((i0 + e < P) && ((kk > thr_key) || (kk == thr_key && i0 + e <= thr_idx))) {
             if (pos < k_max) out[pos] = i0 + e;
             ++pos;

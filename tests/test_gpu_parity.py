@@ -240,13 +240,19 @@ def _topk_cases():
     dense = (1.0 + np.arange(3000, dtype=np.float32) * np.float32(2.0 ** -22)).astype(np.float32)
     dense[5] = -1e30
     rng.shuffle(dense)                                   # 3000 distinct keys a few ulps apart
-    wide = rng.standard_normal(60000).astype(np.float32) # several keys per thread
+    mid = rng.standard_normal(20000).astype(np.float32)  # 20 keys per thread of the one-CTA kernel
+    infs = rng.standard_normal(9000).astype(np.float32)
+    infs[rng.permutation(9000)[:2000]] = -np.inf         # empty pages bound at -inf
+    infs[rng.permutation(9000)[:5]] = np.inf
+    wide = rng.standard_normal(60000).astype(np.float32) # several keys per thread of an 8-CTA cluster
     huge = rng.standard_normal(70001).astype(np.float32) # past the cluster kernel: global-memory top-k
     huge[rng.permutation(70001)[:3000]] = 0.5            # with a large tie
-    return {"big_tie": big_tie, "outlier": outlier, "dense": dense, "wide": wide, "huge": huge}
+    huge[rng.permutation(70001)[:500]] = -np.inf         # and empty pages
+    return {"big_tie": big_tie, "outlier": outlier, "dense": dense, "mid": mid, "infs": infs, "wide": wide,
+            "huge": huge}
 
 
-@pytest.mark.parametrize("case", ["big_tie", "outlier", "dense", "wide", "huge"])
+@pytest.mark.parametrize("case", ["big_tie", "outlier", "dense", "mid", "infs", "wide", "huge"])
 def test_topk_narrowing_rounds(case):
     """Key sets whose threshold bucket holds more than the exact-rank capacity,
     so the selection narrows over several rounds (or ends in a tie round)."""
