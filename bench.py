@@ -30,10 +30,10 @@ sys.path.insert(0, ROOT)
 
 METRIC = "sparse entmax decode µs/step @1M ctx; achieved HBM GB/s vs 8 TB/s roofline"
 # DRAM bytes the scoring kernel read per (page, kv head) metadata row in an ncu
-# capture of the 2^18-token case (16,842,240 bytes for 4097 pages x 8 heads);
+# capture of the 2^18-token case (16,865,024 bytes for 4097 pages x 8 heads);
 # scaled by rows to the bench launch.  Must be re-measured when the scoring
 # kernel changes.
-SCORE_DRAM_BYTES_PER_ROW = 16842240 / (4097 * 8)
+SCORE_DRAM_BYTES_PER_ROW = 16865024 / (4097 * 8)
 HBM_NOMINAL_GBS = 8000.0
 PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
 FALLBACK_HBM_GBS = 6650.0

@@ -1057,7 +1057,8 @@ __global__ void __launch_bounds__(kThreads) pv_f32_kernel(const float* __restric
 // barrier, whatever happens (a timed-out copy only skips work).
 constexpr int kFusedStages = 5;
 constexpr int kCandCap = kFusedCandCap;   // candidate slots per (split, query head) in the workspace
-constexpr int kBitWords = 1024;           // weighted-page bitmap: lists of up to 32768 pages
+constexpr int kBitWords = 128;            // weighted-page bitmap: lists of up to 4096 pages (the clustered
+                                          // kernel's longest: 16 splits of 4096 tokens in pages of 16)
 constexpr int kFusedMaxSplitTokens = 4096; // listed tokens per split (per query head) the fused kernel takes
 
 // Warp-wide sum of three doubles and min / max of two floats (xor butterfly:
@@ -1100,7 +1101,7 @@ EKV_DEV void for_candidates(const TauSrc& s, Fn&& f)
 }
 
 // Lower bound of tau from one split's chunk maxima, by one warp.  cm: the
-// head's chunk-maximum row, own chunks [c0, c1); m_s the split's largest
+// maxima of the split's own chunks [c0, c1) (cm[c - c0]); m_s the split's largest
 // score.  Every chunk maximum is the score of a distinct token, so for any
 // subset of the head's tokens sum_i (x_i - t)_+^r >= sum over the subset's
 // chunk maxima, and the root of the latter is at or below tau.  Up to three
@@ -1125,7 +1126,7 @@ EKV_DEV float split_bound(const float* cm, int c0, int c1, float m_s, float r, b
 #pragma unroll
         for (int u = 0; u < U; ++u) {
             const int i = i0 + u * 32 + lane;
-            v[u] = i < c1 ? cm[i] : -INFINITY;
+            v[u] = i < c1 ? cm[i - c0] : -INFINITY;
         }
 #pragma unroll
         for (int u = 0; u < U; ++u) {
@@ -1167,8 +1168,8 @@ EKV_DEV float split_bound(const float* cm, int c0, int c1, float m_s, float r, b
 // returns how many there are.  The chunks to read: those of split_bound's
 // list above t (the list holds every chunk above m_s - 1 <= t), or all the
 // split's chunks [c0, c1) when the list overflowed.
-EKV_DEV int local_candidates(const float* x, const float* cm, int c0, int c1, int* lc, const float* lcv, int nlc,
-                             int cap, float t, float* oval, int* oidx)
+EKV_DEV int local_candidates(const float* x, int c0, int c1, int* lc, const float* lcv, int nlc, int cap, float t,
+                             float* oval, int* oidx)
 {
     const int lane = threadIdx.x & 31;
     const unsigned below = (1u << lane) - 1u;
@@ -1605,6 +1606,8 @@ __global__ void __launch_bounds__(kThreads, 2) entmax_bf16_kernel(const __grid_c
     // the other CTAs through distributed shared memory)
     __shared__ float pub_t[8], pub_m[8];
     __shared__ int pub_n[8];
+    // the largest score of every 16-token chunk of this split, per head
+    __shared__ float cm_s[4 * NT][kFusedMaxSplitTokens / 16];
     // the cluster-wide threshold solve: partial sums per iteration parity and head
     __shared__ double ct_part[2 * 8 * 3];
     __shared__ float ct_mm[2 * 8 * 2];
@@ -1621,7 +1624,6 @@ __global__ void __launch_bounds__(kThreads, 2) entmax_bf16_kernel(const __grid_c
     const int nst = r.end > r.start ? (r.end - r.start + PPS - 1) / PPS : 0;
     const size_t row0h = (size_t)b * a.H_q + (size_t)g * a.G;
     const size_t xstride = (size_t)a.k_max * PS;
-    const size_t cstride = (size_t)a.k_max * C;
     const uint32_t sbase = smem_addr(smem);
     const bool a2 = a.alpha == 2.0f;
     const bool a15 = a.alpha == 1.5f;
@@ -1702,8 +1704,7 @@ __global__ void __launch_bounds__(kThreads, 2) entmax_bf16_kernel(const __grid_c
                 const float m = group_lane_max(cmx[nt]);
                 run[nt] = fmaxf(run[nt], m);
                 const int head = 4 * nt + c;
-                if (gi == 0 && head < a.G)
-                    a.cmax[(row0h + head) * cstride + (size_t)idx * C + (row0 % PS) / 16] = m;
+                if (gi == 0 && head < a.G) cm_s[head][(idx - r.start) * C + (row0 % PS) / 16] = m;
             }
         }
         __syncthreads();
@@ -1730,8 +1731,7 @@ __global__ void __launch_bounds__(kThreads, 2) entmax_bf16_kernel(const __grid_c
             int* lc = reinterpret_cast<int*>(smem + warp * WSCR + k * LC_CAP * 8);
             float* lcv = reinterpret_cast<float*>(smem + warp * WSCR + k * LC_CAP * 8 + LC_CAP * 4);
             int nlc;
-            const float t = split_bound(a.cmax + (row0h + h) * cstride, c0, c1, smax[h], rpow, a2, a15, lc, lcv,
-                                        LC_CAP, &nlc);
+            const float t = split_bound(cm_s[h], c0, c1, smax[h], rpow, a2, a15, lc, lcv, LC_CAP, &nlc);
             if (lane == 0) {
                 pub_t[h] = t;
                 pub_m[h] = smax[h];
@@ -1748,8 +1748,8 @@ __global__ void __launch_bounds__(kThreads, 2) entmax_bf16_kernel(const __grid_c
             float* lcv = reinterpret_cast<float*>(smem + warp * WSCR + k * LC_CAP * 8 + LC_CAP * 4);
             float tlb = lane < a.S ? ld_dsmem_f32(dsmem(&pub_t[h], lane)) : -INFINITY;
             tlb = warp_max(tlb);
-            const int n = local_candidates(a.xbuf + row * xstride, a.cmax + row * cstride, c0, c1, lc, lcv, nlc_s[h],
-                                           LC_CAP, tlb, a.cval + row * seg + (size_t)s * kCandCap,
+            const int n = local_candidates(a.xbuf + row * xstride, c0, c1, lc, lcv, nlc_s[h], LC_CAP, tlb,
+                                           a.cval + row * seg + (size_t)s * kCandCap,
                                            a.cidx + row * seg + (size_t)s * kCandCap);
             if (lane == 0) pub_n[h] = n;
         }
@@ -1911,7 +1911,7 @@ __global__ void __launch_bounds__(kThreads, 2) entmax_bf16_kernel(const __grid_c
             __syncthreads();
             for (int it = tid; it < wn * a.G; it += kThreads) {
                 const int j = it / a.G, h = it % a.G;
-                const float* cp = a.cmax + (row0h + h) * cstride + (size_t)(w0 + j) * C;
+                const float* cp = cm_s[h] + (w0 + j - r.start) * C;
                 float m = -INFINITY;
 #pragma unroll
                 for (int k = 0; k < C; ++k) m = fmaxf(m, cp[k]);
