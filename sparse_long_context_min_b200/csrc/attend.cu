@@ -1554,10 +1554,13 @@ EKV_DEV void cluster_tau(const float* x, size_t xstride, int t0, int t1, const f
 EKV_DEV int resolve_peer(const AttnArgs& a, int b, int g, int j, int P, int per, int& lp)
 {
     const int q = j / per;
-    const int li = j - q * per;
-    if (li < ld_dsmem_s32(dsmem(&tab_n, q))) {
-        lp = ld_dsmem_s32(dsmem(&tab_lp[li], q));
-        return ld_dsmem_s32(dsmem(&tab_phys[li], q));
+    const int li = j - q * per;          // < per <= kTabCap: the three reads go out together
+    const int n = ld_dsmem_s32(dsmem(&tab_n, q));
+    const int l = ld_dsmem_s32(dsmem(&tab_lp[li], q));
+    const int ph = ld_dsmem_s32(dsmem(&tab_phys[li], q));
+    if (li < n) {
+        lp = l;
+        return ph;
     }
     return resolve_g(a, b, g, j, P, lp, true);
 }
@@ -1629,6 +1632,10 @@ __global__ void __launch_bounds__(kThreads, 2) entmax_bf16_kernel(const __grid_c
     const bool a15 = a.alpha == 1.5f;
     const float rpow = a2 ? 1.0f : (a15 ? 2.0f : 1.0f / (a.alpha - 1.0f));
     const size_t seg = (size_t)kFusedMaxSplits * kCandCap;   // candidate slots of one head row
+    // the query first: its load overlaps the page-table lookups instead of
+    // queueing behind the first key tiles
+    uint32_t bq[NT][KS][2];
+    load_q_frags<D, NT>(a, b, g, a.xscale, bq);
     tab_fill(a, b, g, r, P);
 
     // ------------------------------------------------------------ K pass
@@ -1652,8 +1659,6 @@ __global__ void __launch_bounds__(kThreads, 2) entmax_bf16_kernel(const __grid_c
     float run[NT];
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt) run[nt] = -INFINITY;
-    uint32_t bq[NT][KS][2];
-    load_q_frags<D, NT>(a, b, g, a.xscale, bq);
     __syncthreads();
     int kst = 0;
     for (; kst < nst; ++kst) {
@@ -1767,11 +1772,14 @@ __global__ void __launch_bounds__(kThreads, 2) entmax_bf16_kernel(const __grid_c
     // the owner keeps tau and the head's weighted pages for the others.
     const bool bitmap_ok = cnt <= kBitWords * 32;
     if (tid < 32) {
+        int nh[8];                                            // every read goes out before the first use
+#pragma unroll
+        for (int h = 0; h < 8; ++h) nh[h] = h < a.G && lane < a.S ? ld_dsmem_s32(dsmem(&pub_n[h], lane)) : 0;
         bool o = false;
-        for (int h = 0; h < a.G; ++h) {
-            const int n = lane < a.S ? ld_dsmem_s32(dsmem(&pub_n[h], lane)) : 0;
-            const int tot = warp_sum((n + 3) & ~3);           // as gathered: 4-entry aligned per split
-            o = o || __any_sync(0xffffffffu, n > kCandCap) || tot > CAND_CAP;
+#pragma unroll
+        for (int h = 0; h < 8; ++h) {
+            const int tot = warp_sum((nh[h] + 3) & ~3);       // as gathered: 4-entry aligned per split
+            o = o || __any_sync(0xffffffffu, nh[h] > kCandCap) || tot > CAND_CAP;
         }
         if (tid == 0) over_all = o;
     }
@@ -1834,8 +1842,12 @@ __global__ void __launch_bounds__(kThreads, 2) entmax_bf16_kernel(const __grid_c
         }
         if (bitmap_ok)
             for (int w = tid; w < words; w += kThreads) {
+                unsigned v[8];                   // owners <= 8: every read goes out before the first use
+#pragma unroll
+                for (int q = 0; q < 8; ++q) v[q] = q < owners ? (unsigned)ld_dsmem_s32(dsmem(&bits[w], q)) : 0u;
                 unsigned u = 0;
-                for (int q = 0; q < owners; ++q) u |= (unsigned)ld_dsmem_s32(dsmem(&bits[w], q));
+#pragma unroll
+                for (int q = 0; q < 8; ++q) u |= v[q];
                 vbits[w] = u;
             }
     }
@@ -2055,8 +2067,12 @@ __global__ void __launch_bounds__(kThreads, 2) entmax_bf16_kernel(const __grid_c
     const int per = (E + a.S - 1) / a.S;
     for (int e = s * per + tid; e < min(E, (s + 1) * per); e += kThreads) {
         const int head = e / D, dd = e % D;
-        float sum = 0.f;
-        for (int q = 0; q < a.S; ++q) sum += ld_dsmem_f32(dsmem(part + e, q));
+        float v[kFusedMaxSplits];            // every read goes out before the first add
+#pragma unroll
+        for (int q = 0; q < kFusedMaxSplits; ++q) v[q] = q < a.S ? ld_dsmem_f32(dsmem(part + e, q)) : 0.f;
+        float sum = 0.f;                     // in CTA order; the +0 of absent splits changes nothing
+#pragma unroll
+        for (int q = 0; q < kFusedMaxSplits; ++q) sum += v[q];
         a.out[(row0h + head) * D + dd] = sum;
     }
     cluster_sync();       // no CTA leaves while another may still read its shared memory

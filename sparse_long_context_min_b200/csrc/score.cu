@@ -579,6 +579,31 @@ __global__ void __launch_bounds__(BoxWsShape<D, G>::CTA, 2) score_box16_kernel(c
     uint32_t sel[S::HPT][S::WPS];                        // byte-permute selectors
     int qb = -1;
     const float scale = a.scale;
+    auto load_q = [&](int b) {
+        const float* qg = a.q + ((size_t)b * a.H_q + (size_t)g * G + hs * S::HPT) * D + ks * S::SW;
+        float qv[S::HPT][S::SW];
+#pragma unroll
+        for (int i = 0; i < S::HPT; ++i)
+#pragma unroll
+            for (int e = 0; e < S::SW; e += 4) {
+                const float4 f = __ldg(reinterpret_cast<const float4*>(qg + (size_t)i * D + e));
+                qv[i][e] = f.x; qv[i][e + 1] = f.y; qv[i][e + 2] = f.z; qv[i][e + 3] = f.w;
+            }
+#pragma unroll
+        for (int i = 0; i < S::HPT; ++i)
+#pragma unroll
+            for (int kk = 0; kk < S::WPS; ++kk)   // k_max (second operand) where q >= 0, else k_min
+                sel[i][kk] = (qv[i][2 * kk] >= 0.f ? 0x0054u : 0x0010u) | (qv[i][2 * kk + 1] >= 0.f ? 0x7600u : 0x3200u);
+#pragma unroll
+        for (int e = 0; e < S::SW; ++e) {
+            if (S::HPT == 2) qp[e] = pack2(qv[0][e], qv[S::HPT - 1][e]);
+            else qs[e] = qv[0][e];
+        }
+        qb = b;
+    };
+    // the query of the CTA's first sequence before the first chunk arrives: a
+    // load issued after the chunk copies would queue behind them
+    if (K > 0 && c0 * PPS < items) load_q((int)(c0 * PPS / a.max_pages));
     for (int k = 0; k < K; ++k) {
         const int s = k % NST;
         const bool ok = mbar_wait(&full[s], (k / NST) & 1, kWaitLimitNs);
@@ -590,28 +615,7 @@ __global__ void __launch_bounds__(BoxWsShape<D, G>::CTA, 2) score_box16_kernel(c
         for (int r = 0; r < kWsRounds; ++r) {
             const int4 inf = info[s * S::SLOTS + pi + r * ppr];
             const int b = inf.x, p = inf.y, n = inf.z;
-            if (b >= 0 && b != qb) {
-                const float* qg = a.q + ((size_t)b * a.H_q + (size_t)g * G + hs * S::HPT) * D + ks * S::SW;
-                float qv[S::HPT][S::SW];
-#pragma unroll
-                for (int i = 0; i < S::HPT; ++i)
-#pragma unroll
-                    for (int e = 0; e < S::SW; e += 4) {
-                        const float4 f = __ldg(reinterpret_cast<const float4*>(qg + (size_t)i * D + e));
-                        qv[i][e] = f.x; qv[i][e + 1] = f.y; qv[i][e + 2] = f.z; qv[i][e + 3] = f.w;
-                    }
-#pragma unroll
-                for (int i = 0; i < S::HPT; ++i)
-#pragma unroll
-                    for (int kk = 0; kk < S::WPS; ++kk)   // k_max (second operand) where q >= 0, else k_min
-                        sel[i][kk] = (qv[i][2 * kk] >= 0.f ? 0x0054u : 0x0010u) | (qv[i][2 * kk + 1] >= 0.f ? 0x7600u : 0x3200u);
-#pragma unroll
-                for (int e = 0; e < S::SW; ++e) {
-                    if (S::HPT == 2) qp[e] = pack2(qv[0][e], qv[S::HPT - 1][e]);
-                    else qs[e] = qv[0][e];
-                }
-                qb = b;
-            }
+            if (b >= 0 && b != qb) load_q(b);
             float acc[S::HPT];
 #pragma unroll
             for (int i = 0; i < S::HPT; ++i) acc[i] = 0.f;

@@ -357,10 +357,10 @@ topk_cluster_kernel(const float* __restrict__ ub, const int32_t* __restrict__ se
         }
         cluster_sync();
         if (warp == 0) {
-            const unsigned int a = __reduce_min_sync(
-                0xffffffffu, lane < C ? (unsigned)ld_dsmem_s32(dsmem(&sh.pub_mm[0], lane)) : 0xFFFFFFFFu);
-            const unsigned int c =
-                __reduce_max_sync(0xffffffffu, lane < C ? (unsigned)ld_dsmem_s32(dsmem(&sh.pub_mm[1], lane)) : 0u);
+            const unsigned int va = lane < C ? (unsigned)ld_dsmem_s32(dsmem(&sh.pub_mm[0], lane)) : 0xFFFFFFFFu;
+            const unsigned int vc = lane < C ? (unsigned)ld_dsmem_s32(dsmem(&sh.pub_mm[1], lane)) : 0u;
+            const unsigned int a = __reduce_min_sync(0xffffffffu, va);
+            const unsigned int c = __reduce_max_sync(0xffffffffu, vc);
             if (lane == 0) {
                 sh.g_mm[0] = a;
                 sh.g_mm[1] = c;
@@ -408,9 +408,12 @@ topk_cluster_kernel(const float* __restrict__ ub, const int32_t* __restrict__ se
         // 0 the top bin) from the CTA that holds it
         constexpr int SL = kCBins / C;
         if (tid < SL) {
+            int v[C];                        // every read goes out before the first add
+#pragma unroll
+            for (int q = 0; q < C; ++q) v[q] = ld_dsmem_s32(dsmem(&sh.hist[r * SL + tid], q));
             int t = 0;
 #pragma unroll
-            for (int q = 0; q < C; ++q) t += ld_dsmem_s32(dsmem(&sh.hist[r * SL + tid], q));
+            for (int q = 0; q < C; ++q) t += v[q];
             sh.tot[tid] = t;
         }
         cluster_sync();
@@ -451,14 +454,14 @@ topk_cluster_kernel(const float* __restrict__ ub, const int32_t* __restrict__ se
                 if (lane == 0) sh.mc_off[0] = 0;
             }
             __syncthreads();
-#pragma unroll 1
-            for (int q = 0; q < C; ++q) {
-                const int o = sh.mc_off[q], n = sh.mc_off[q + 1] - o;
-                const uint32_t base = dsmem(&sh.lc[0], q);
-                for (int j = tid; j < n; j += kCThreads) sh.mc[o + j] = ld_dsmem_u64(base + 8u * (uint32_t)j);
+            const int nc = sh.mc_off[C];
+            for (int j = tid; j < nc; j += kCThreads) {   // one read per thread, all at once
+                int q = 0;
+#pragma unroll
+                for (int u = 1; u < C; ++u) q += j >= sh.mc_off[u];
+                sh.mc[j] = ld_dsmem_u64(dsmem(&sh.lc[j - sh.mc_off[q]], q));
             }
             __syncthreads();
-            const int nc = sh.mc_off[C];
             for (int j = tid; j < nc; j += kCThreads) {
                 const unsigned long long me = sh.mc[j];
                 int rank = 0;
