@@ -183,7 +183,7 @@ static int num_splits(int B, int H_kv, int list_pages)
 
 struct AttnLayout {
     int S;
-    size_t xbuf, cmax, opart, mlpart, lmax, tau, counters, lbound, ccnt, cval, cidx, total;
+    size_t xbuf, cmax, opart, mlpart, lmax, tau, counters, cval, cidx, total;
 };
 
 // attention ops over a caller's page list / with softmax weights
@@ -211,12 +211,8 @@ static AttnLayout attn_layout(int op, int B, int H_q, int H_kv, int max_pages, i
     off += round256((size_t)B * H_q * sizeof(float));
     L.counters = off;
     off += round256((size_t)B * H_kv * sizeof(int32_t));
-    // threshold bounds and candidates of the fused bf16 entmax kernel
+    // candidate slots of the clustered bf16 entmax kernel
     const size_t rows = soft ? 0 : (size_t)B * H_q * kFusedMaxSplits;
-    L.lbound = off;
-    off += round256(rows * sizeof(float));
-    L.ccnt = off;
-    off += round256(rows * sizeof(int32_t));
     L.cval = off;
     off += round256(rows * kFusedCandCap * sizeof(float));
     L.cidx = off;
@@ -277,8 +273,6 @@ static int attend_common(int op, const entmaxkv_pool* pool, const float* q, int 
     a.vpages = v_pages;
     a.tau = reinterpret_cast<float*>(ws + lay.tau);
     a.counters = reinterpret_cast<int32_t*>(ws + lay.counters);
-    a.lbound = reinterpret_cast<float*>(ws + lay.lbound);
-    a.ccnt = reinterpret_cast<int32_t*>(ws + lay.ccnt);
     a.cval = reinterpret_cast<float*>(ws + lay.cval);
     a.cidx = reinterpret_cast<int32_t*>(ws + lay.cidx);
     a.out = out;

@@ -39,8 +39,6 @@ struct AttnArgs {
     float* lmax;                   // [B][H_q][S] largest score of each split (K pass)
     int32_t* vpages;               // [B][H_kv] value pages loaded (V pass adds), or NULL
     int32_t* counters;             // [B][H_kv] arrival counters of the split reduction
-    float* lbound;                 // [B][H_q][S] each split's lower bound of tau (fused bf16 kernel)
-    int32_t* ccnt;                 // [B][H_q][S] each split's candidate count (fused bf16 kernel)
     float* cval;                   // [B][H_q][S][kFusedCandCap] candidate scores (fused bf16 kernel)
     int32_t* cidx;                 // [B][H_q][S][kFusedCandCap] their list positions (fused bf16 kernel)
     float* out;                    // [B][H_q][d]

@@ -219,11 +219,22 @@ def test_head_and_page_shapes(shape):
     step.check()
     ub, sel, cnt = step.ub.cpu().numpy(), step.sel.cpu().numpy(), step.sel_count.cpu().numpy()
     out = step.out.cpu().numpy()
+    # the Gaussian page model of the same shape (role-split moments kernel where the layout allows)
+    st = _status()
+    gshape = (cfg.B, cfg.H_q, wl.max_pages)
+    gm, gv, ge = (torch.empty(gshape, device="cuda") for _ in range(3))
+    B.score_pages(pool, wl.q, wl.page_table, seq_lens, B.SCORE_GAUSS, H.scale32(cfg), st, m=gm, v=gv, est_max=ge)
+    _assert_ok(st)
+    gm, gv, ge = gm.cpu().numpy(), gv.cpu().numpy(), ge.cpu().numpy()
     G = cfg.G
     for b in range(cfg.B):
         o = H.OracleSeq(wl, b)
         P = cfg.pages(b)
         for g in range(cfg.H_kv):
+            rm, rv, re = o.gauss(g)
+            sl = slice(g * G, (g + 1) * G)
+            assert np.array_equal(gm[b, sl, :P], rm) and np.array_equal(gv[b, sl, :P], rv), (b, g)
+            assert np.array_equal(ge[b, sl, :P], re) and np.all(ge[b, sl, P:] == -np.inf), (b, g)
             assert np.array_equal(ub[b, g, :P], o.ubg(g)), (b, g)
             ref = o.topk(g, -1, 1 / 8)
             assert np.array_equal(sel[b, g, :cnt[b, g]], ref), (b, g)
@@ -561,6 +572,54 @@ def test_flat_scores_cluster_threshold(alpha):
             assert n_cand > 16 * 256, n_cand
         H.compare_out(out[0, g * G:(g + 1) * G], o_ref, torch.bfloat16)
         assert np.all(np.abs(tau[0, g * G:(g + 1) * G] - t_ref) <= 1e-5 * np.maximum(1, np.abs(t_ref)))
+
+
+def test_clustered_attention_longest_list():
+    """The clustered kernel at its longest list: pages of 16 tokens, 4096
+    listed pages per kv head (16 splits of 4096 tokens, the weighted-page
+    bitmap full to its last word), a few planted tokens spread over the list
+    (the first and the last page among them) carrying the support.  Output
+    and tau against the oracle over every token, and the value pages loaded
+    equal to the pages holding weight."""
+    gen = torch.Generator().manual_seed(777)
+    H_kv, G, d, ps, P = 2, 4, 128, 16, 4096
+    L = P * ps
+    keys = 0.1 * torch.randn(H_kv, L, d, generator=gen)
+    vals = torch.randn(H_kv, L, d, generator=gen).to(torch.bfloat16)
+    q = torch.randn(1, H_kv * G, d, generator=gen)
+    plant = [3, 16 * 700 + 5, 16 * 2047 + 9, L - 2]          # tokens on pages 0, 700, 2047 and 4095
+    for g in range(H_kv):
+        for j, t in enumerate(plant):
+            h = g * G + j % G
+            keys[g, t] = 4.0 * q[0, h] / q[0, h].norm()
+    keys = keys.to(torch.bfloat16)
+    pool = B.Pool.allocate(P, H_kv, ps, d, torch.bfloat16, "cuda")
+    pt = torch.arange(P, dtype=torch.int32, device="cuda").view(1, P)
+    seq_lens = torch.zeros(1, dtype=torch.int32, device="cuda")
+    st = _status()
+    B.append_metadata(pool, keys.cuda().unsqueeze(0).contiguous(), vals.cuda().unsqueeze(0).contiguous(), pt,
+                      seq_lens, st)
+    sel = torch.arange(P, dtype=torch.int32, device="cuda").view(1, 1, P).repeat(1, H_kv, 1).contiguous()
+    cnt = torch.full((1, H_kv), P, dtype=torch.int32, device="cuda")
+    ws = torch.empty(B.workspace_size(B.OP_SPARSE_ATTEND, 1, H_kv * G, H_kv, P, P, ps, d), dtype=torch.uint8,
+                     device="cuda")
+    out = torch.empty(1, H_kv * G, d, device="cuda")
+    tau = torch.empty(1, H_kv * G, device="cuda")
+    vp = torch.zeros(1, H_kv, dtype=torch.int32, device="cuda")
+    scale = float(np.float32(1.0 / math.sqrt(d)))
+    alpha = 1.5
+    B.sparse_attend(pool, q.cuda(), pt, seq_lens, sel, cnt, alpha, scale, out, ws, st, tau_out=tau, v_pages=vp)
+    _assert_ok(st)
+    out, tau, vp = out.cpu().numpy(), tau.cpu().numpy(), vp.cpu().numpy()
+    qn = q[0].numpy()
+    for g in range(H_kv):
+        K, V = keys[g].float().numpy(), vals[g].float().numpy()
+        o_ref, t_ref, p = attend.entmax_attention(qn[g * G:(g + 1) * G], K, V, alpha, scale)
+        H.compare_out(out[0, g * G:(g + 1) * G], o_ref, torch.bfloat16)
+        assert np.all(np.abs(tau[0, g * G:(g + 1) * G] - t_ref) <= 1e-5 * np.maximum(1, np.abs(t_ref)))
+        weighted = np.unique(np.nonzero(np.any(p > 0, axis=0))[0] // ps)
+        assert 0 in weighted and P - 1 in weighted
+        assert vp[0, g] == len(weighted), (vp[0, g], len(weighted))
 
 
 def test_support_recovery_on_gpu():
