@@ -1263,43 +1263,48 @@ EKV_DEV int gather_candidates(const float* cval, const int* cidx, int nq, int S,
 //  one at or below).  Should rounding in float leave the support
 //  inconsistent, the same iteration runs in float64.
 //  Any other alpha: safeguarded Newton steps on F^(1/r) inside [src.lo, M].
+// Any other alpha: safeguarded Newton steps on F^(1/r) inside [src.lo, M]
+// (kept out of line: the alpha = 1.5 and 2 path does not fetch its code).
+__device__ __noinline__ double solve_tau_general(const TauSrc src, float M, float alpha)
+{
+    // Newton on G(t) = F(t)^(1/r) - 1 inside [lo, hi] (F(lo) >= 1 > F(M) = 0),
+    // bisection where a step leaves it; terms in float (powf), sums in float64
+    double tau = src.lo;
+    const double r = 1.0 / ((double)alpha - 1.0);
+    const float rf = (float)r;
+    double lo = src.lo, hi = (double)M;
+    for (int it = 0; it < 100; ++it) {
+        double v[3] = {0.0, 0.0, 0.0};
+        float u0 = INFINITY, u1 = -INFINITY;
+        for_candidates(src, [&](float f) {
+            const double vd = (double)f;
+            if (vd > tau) {
+                const float u = (float)(vd - tau);
+                const float pu = powf(u, rf);
+                v[0] += (double)pu;
+                v[1] += (double)pu / (double)u;
+            }
+        });
+        warp_red5(v, u0, u1);
+        const double F = v[0], S1 = r * v[1];
+        if (F >= 1.0) lo = tau; else hi = tau;
+        if (F == 1.0 || hi - lo <= 1e-13 * fmax(1.0, fabs(tau))) break;
+        double nt = (F > 0.0 && S1 > 0.0) ? tau + r * F * (1.0 - pow(F, -1.0 / r)) / S1 : 0.5 * (lo + hi);
+        if (!(nt > lo && nt < hi)) nt = 0.5 * (lo + hi);
+        if (fabs(nt - tau) <= 1e-8 * fmax(1.0, fabs(tau))) {
+            tau = nt;
+            break;
+        }
+        tau = nt;
+    }
+    return tau;
+}
+
 EKV_DEV double solve_tau(const TauSrc& src, float M, float alpha)
 {
     const bool a2 = alpha == 2.0f;
     const bool a15 = alpha == 1.5f;
-    if (!a2 && !a15) {
-        // Newton on G(t) = F(t)^(1/r) - 1 inside [lo, hi] (F(lo) >= 1 > F(M) = 0),
-        // bisection where a step leaves it; terms in float (powf), sums in float64
-        double tau = src.lo;
-        const double r = 1.0 / ((double)alpha - 1.0);
-        const float rf = (float)r;
-        double lo = src.lo, hi = (double)M;
-        for (int it = 0; it < 100; ++it) {
-            double v[3] = {0.0, 0.0, 0.0};
-            float u0 = INFINITY, u1 = -INFINITY;
-            for_candidates(src, [&](float f) {
-                const double vd = (double)f;
-                if (vd > tau) {
-                    const float u = (float)(vd - tau);
-                    const float pu = powf(u, rf);
-                    v[0] += (double)pu;
-                    v[1] += (double)pu / (double)u;
-                }
-            });
-            warp_red5(v, u0, u1);
-            const double F = v[0], S1 = r * v[1];
-            if (F >= 1.0) lo = tau; else hi = tau;
-            if (F == 1.0 || hi - lo <= 1e-13 * fmax(1.0, fabs(tau))) break;
-            double nt = (F > 0.0 && S1 > 0.0) ? tau + r * F * (1.0 - pow(F, -1.0 / r)) / S1 : 0.5 * (lo + hi);
-            if (!(nt > lo && nt < hi)) nt = 0.5 * (lo + hi);
-            if (fabs(nt - tau) <= 1e-8 * fmax(1.0, fabs(tau))) {
-                tau = nt;
-                break;
-            }
-            tau = nt;
-        }
-        return tau;
-    }
+    if (!a2 && !a15) return solve_tau_general(src, M, alpha);
     // exact closed form on the support {x > t}, float64; NaN when inconsistent
     auto closed = [&](double t, double* next) -> double {
         double v[3] = {0.0, 0.0, 0.0};
@@ -1393,7 +1398,8 @@ EKV_DEV double solve_tau(const TauSrc& src, float M, float alpha)
 // shared [2][8][3] doubles and [2][8][2] floats; pub_t, pub_m: every split's
 // bound and largest score per head (read through distributed shared memory);
 // tau_h: tau per head, out (every CTA).
-EKV_DEV void cluster_tau(const float* x, size_t xstride, int t0, int t1, const float* pub_t, const float* pub_m,
+__device__ __noinline__ void cluster_tau(const float* x, size_t xstride, int t0, int t1, const float* pub_t,
+                                        const float* pub_m,
                          int G, int S, float alpha, bool skip, double* part, float* mm, double* tau_h)
 {
     constexpr int kMaxIt = 48;
