@@ -1254,17 +1254,50 @@ EKV_DEV int gather_candidates(const float* cval, const int* cidx, int nq, int S,
     return total;
 }
 
-// tau from the candidates of src, one warp, every lane returns it.
-//  alpha = 2 and 1.5: steps in float from the bound src.lo -- Newton on
-//  sum (x - t)^2 = 1 for 1.5, the fixed point t = (sum x - 1) / k for 2, both
-//  from the left over the current support {x > t} -- until the support holds
-//  for a step; then the closed form on that support in float64, accepted when
-//  the support is consistent with it (every kept value above, every dropped
-//  one at or below).  Should rounding in float leave the support
-//  inconsistent, the same iteration runs in float64.
-//  Any other alpha: safeguarded Newton steps on F^(1/r) inside [src.lo, M].
-// Any other alpha: safeguarded Newton steps on F^(1/r) inside [src.lo, M]
-// (kept out of line: the alpha = 1.5 and 2 path does not fetch its code).
+// The exact closed form of tau on the support {x > t} of the candidates
+// (float64, one warp, every lane the same): alpha = 2 gives (sum x - 1) / k,
+// alpha = 1.5 the smaller root of sum (x - tau)^2 = 1.  NaN unless the support
+// is consistent with it (every kept value above, every dropped one at or
+// below, and at least the bound); *next: the next iterate from t (the fixed
+// point for 2, a Newton step on sum (x - t)^2 = 1 for 1.5).
+EKV_DEV double closed_form(const TauSrc& src, bool a2, double t, double* next)
+{
+    double v[3] = {0.0, 0.0, 0.0};
+    float minS = INFINITY, maxN = -INFINITY;
+    for_candidates(src, [&](float f) {
+        const double vd = (double)f;
+        if (vd > t) {
+            v[0] += 1.0;
+            v[1] += vd;
+            v[2] = fma(vd, vd, v[2]);
+            minS = fminf(minS, f);
+        } else {
+            maxN = fmaxf(maxN, f);
+        }
+    });
+    warp_red5(v, minS, maxN);
+    const double k = v[0], sx = v[1], sxx = v[2];
+    double tcf;
+    bool ok;
+    if (a2) {
+        tcf = (sx - 1.0) / k;
+        ok = true;
+        *next = tcf;
+    } else {
+        const double mean = sx / k, msq = sxx / k;
+        const double disc = mean * mean - msq + 1.0 / k;
+        ok = disc >= 0.0;
+        tcf = ok ? mean - sqrt(disc) : 0.0;
+        const double s1 = sx - k * t;
+        const double s2 = sxx - 2.0 * t * sx + k * t * t;
+        *next = t + (s2 - 1.0) / (2.0 * s1);
+    }
+    return (ok && tcf < (double)minS && (double)maxN <= tcf && tcf >= src.lo) ? tcf : NAN;
+}
+
+// tau of solve_tau for any alpha other than 1.5 and 2: safeguarded Newton
+// steps on F^(1/r) inside [src.lo, M] (kept out of line: the alpha = 1.5 and
+// 2 path does not fetch its code).
 __device__ __noinline__ double solve_tau_general(const TauSrc src, float M, float alpha)
 {
     // Newton on G(t) = F(t)^(1/r) - 1 inside [lo, hi] (F(lo) >= 1 > F(M) = 0),
@@ -1300,45 +1333,22 @@ __device__ __noinline__ double solve_tau_general(const TauSrc src, float M, floa
     return tau;
 }
 
+__device__ __noinline__ double solve_tau_refine(const TauSrc src, bool a2, float t);
+
+// tau from the candidates of src, one warp, every lane returns it.
+//  alpha = 2 and 1.5: steps in float from the bound src.lo -- Newton on
+//  sum (x - t)^2 = 1 for 1.5, the fixed point t = (sum x - 1) / k for 2, both
+//  from the left over the current support {x > t} -- until the support holds
+//  for a step; then the closed form on that support in float64, accepted when
+//  the support is consistent with it (every kept value above, every dropped
+//  one at or below).  Should rounding in float leave the support
+//  inconsistent, the same iteration runs in float64 (solve_tau_refine).
+//  Any other alpha: solve_tau_general.
 EKV_DEV double solve_tau(const TauSrc& src, float M, float alpha)
 {
     const bool a2 = alpha == 2.0f;
     const bool a15 = alpha == 1.5f;
     if (!a2 && !a15) return solve_tau_general(src, M, alpha);
-    // exact closed form on the support {x > t}, float64; NaN when inconsistent
-    auto closed = [&](double t, double* next) -> double {
-        double v[3] = {0.0, 0.0, 0.0};
-        float minS = INFINITY, maxN = -INFINITY;
-        for_candidates(src, [&](float f) {
-            const double vd = (double)f;
-            if (vd > t) {
-                v[0] += 1.0;
-                v[1] += vd;
-                v[2] = fma(vd, vd, v[2]);
-                minS = fminf(minS, f);
-            } else {
-                maxN = fmaxf(maxN, f);
-            }
-        });
-        warp_red5(v, minS, maxN);
-        const double k = v[0], sx = v[1], sxx = v[2];
-        double tcf;
-        bool ok;
-        if (a2) {
-            tcf = (sx - 1.0) / k;
-            ok = true;
-            *next = tcf;
-        } else {
-            const double mean = sx / k, msq = sxx / k;
-            const double disc = mean * mean - msq + 1.0 / k;
-            ok = disc >= 0.0;
-            tcf = ok ? mean - sqrt(disc) : 0.0;
-            const double s1 = sx - k * t;
-            const double s2 = sxx - 2.0 * t * sx + k * t * t;
-            *next = t + (s2 - 1.0) / (2.0 * s1);
-        }
-        return (ok && tcf < (double)minS && (double)maxN <= tcf && tcf >= src.lo) ? tcf : NAN;
-    };
     // float iteration to the support
     float t = (float)src.lo;
     float kprev = -1.f;
@@ -1360,15 +1370,23 @@ EKV_DEV double solve_tau(const TauSrc& src, float M, float alpha)
         t = nt;
     }
     double next = 0.0;
-    const double tc = closed((double)t, &next);
+    const double tc = closed_form(src, a2, (double)t, &next);
     if (tc == tc) return tc;
+    return solve_tau_refine(src, a2, t);
+}
+
+// The float64 iteration of solve_tau for when the float iterate's support was
+// not consistent with its closed form (kept out of line: rarely taken).
+__device__ __noinline__ double solve_tau_refine(const TauSrc src, bool a2, float t)
+{
+    double next = 0.0;
     // float64 steps from just below the float iterate (rounding left the float
     // support off by a value or two); should that start lie right of the root
     // (a step that does not move right), from the bound itself
     double tau = fmax(src.lo, (double)t - 1e-4 * fmax(1.0, fabs((double)t)));
     bool restarted = tau == src.lo;
     for (int it = 0; it < 100; ++it) {
-        const double c = closed(tau, &next);
+        const double c = closed_form(src, a2, tau, &next);
         if (c == c) return c;
         if (!(next > tau) || !isfinite(next)) {
             if (restarted) break;
