@@ -34,6 +34,11 @@ METRIC = "sparse entmax decode µs/step @1M ctx; achieved HBM GB/s vs 8 TB/s roo
 # scaled by rows to the bench launch.  Must be re-measured when the scoring
 # kernel changes.
 SCORE_DRAM_BYTES_PER_ROW = 16865024 / (4097 * 8)
+# DRAM bytes (read + write) of one fused attention launch of the 2^20-token
+# top-k 1/64 workload in an ncu capture (the first graph replay); reported as
+# that launch's traffic beside the mean algorithmic bytes.  Must be re-measured
+# when the attention kernel changes.
+ATTEND_DRAM_BYTES_1M = 37660000 + 39170   # 37.66 MB read, 39.17 KB written (ncu rounding)
 HBM_NOMINAL_GBS = 8000.0
 PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
 FALLBACK_HBM_GBS = 6650.0
@@ -264,7 +269,7 @@ def score_bytes(cfg, mode):
     return algorithmic_bytes(cfg, 0, 0, mode)["score"]
 
 
-N_LAUNCH = 4   # per step: append (one token, advances the length itself), score, top-k, fused attention
+N_LAUNCH = 4   # per step: scoring with the token append, the length advance, top-k, fused attention
 
 
 def roofline_entry(kernel, nbytes, us, peak, traffic=None, note=None):
@@ -281,7 +286,7 @@ def roofline_entry(kernel, nbytes, us, peak, traffic=None, note=None):
 
 
 def native_line(cfg, world, K, W, mean_us, best_us, median_us, score_us, stage, sel_total, v_total, extra, e2e,
-                clk, cpu, peak, attend_us=None):
+                clk, cpu, peak, attend_us):
     """The native arm's JSON line from the measured numbers (times are the
     max over ranks; e2e = (us per step, H2D bytes, D2H bytes); peak = (GB/s,
     "measured" or "fallback"))."""
@@ -320,19 +325,24 @@ def native_line(cfg, world, K, W, mean_us, best_us, median_us, score_us, stage, 
             "stage_note": "stage_us from a graph with event nodes between stages (no overlap across them)",
             **extra,
         },
-        "roofline": roofline_entry("score_box16_kernel (entmaxkv_score_pages, bbox, bf16)", by["score"], score_us,
-                                   peak, round(SCORE_DRAM_BYTES_PER_ROW * sum(cfg.pages(b) for b in range(cfg.B))
-                                               * cfg.H_kv),
-                                   "ncu dram__bytes_read+write of the 2^18-token case scaled by rows"),
+        "roofline_score": roofline_entry(
+            "score_box16_kernel (entmaxkv_append_score_pages, bbox, bf16)", by["score"], score_us, peak,
+            round(SCORE_DRAM_BYTES_PER_ROW * sum(cfg.pages(b) for b in range(cfg.B)) * cfg.H_kv),
+            "ncu dram__bytes_read+write of the 2^18-token case scaled by rows"),
         "e2e": {"value": round(e2e_us, 2), "unit": "us/step", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h},
         "gpu_launches": N_LAUNCH * K,
         "clocks": clk,
     }
-    if attend_us:
-        line["roofline_attend"] = roofline_entry(
-            "entmax_bf16_kernel (entmaxkv_sparse_attend: K pass, threshold, V pass)", by["attend"], attend_us, peak,
-            None, "keys of the selected page-heads plus values of those holding weight")
+    # the dominant kernel (the largest share of the step's kernel time): the
+    # fused attention, on the bytes it must read (keys of the selected
+    # page-heads, values of those holding weight)
+    one_m = cfg.B == 1 and cfg.lengths[0] == 1 << 20
+    line["roofline"] = roofline_entry(
+        "entmax_bf16_kernel (entmaxkv_sparse_attend: K pass, threshold, V pass)", by["attend"], attend_us, peak,
+        ATTEND_DRAM_BYTES_1M if one_m else None,
+        "algorithmic bytes: keys of the selected page-heads plus values of those holding weight (mean over the "
+        "timed steps); traffic: ncu dram__bytes_read+write of one launch of this workload")
     if cpu is not None:
         line["cpu_baseline"] = cpu
     return line

@@ -175,20 +175,25 @@ def test_native_line_carries_the_contract():
             "cpu_baseline"} <= set(line)
     assert line["value"] == 88.19 and line["higher_is_better"] is False and line["scaling"] == "weak"
     assert line["gpu_launches"] == 4 * 20 and line["config"]["x"] == 1
-    r = line["roofline"]
+    r = line["roofline"]                         # the dominant kernel: the fused attention, on the bytes it must read
     assert {"bound", "achieved", "peak", "unit", "frac", "traffic"} <= set(r)
     by = bench.algorithmic_bytes(cfg, 2056, 278.2, "topk")
-    assert abs(r["achieved"] - by["score"] / 28.78e-6 / 1e9) < 0.1
+    assert abs(r["achieved"] - by["attend"] / 21.5e-6 / 1e9) < 0.1
     assert abs(r["frac"] - r["achieved"] / 6528.7) < 1e-3
-    assert r["traffic"] == round(bench.SCORE_DRAM_BYTES_PER_ROW * 16384 * 8)
-    ra = line["roofline_attend"]                 # the fused attention kernel on the bytes it must read
-    assert abs(ra["achieved"] - by["attend"] / 21.5e-6 / 1e9) < 0.1
-    assert abs(ra["frac_of_8tbs"] - ra["achieved"] / 8000.0) < 1e-3 and ra["traffic"] is None
+    assert abs(r["frac_of_8tbs"] - r["achieved"] / 8000.0) < 1e-3
+    assert r["traffic"] == bench.ATTEND_DRAM_BYTES_1M and r["bytes_per_launch"] == by["attend"]
+    rs = line["roofline_score"]                  # the scoring kernel with the token append
+    assert abs(rs["achieved"] - by["score"] / 28.78e-6 / 1e9) < 0.1
+    assert rs["traffic"] == round(bench.SCORE_DRAM_BYTES_PER_ROW * 16384 * 8)
     assert line["e2e"] == {"value": 100.91, "unit": "us/step", "h2d_bytes_per_step": 20480,
                            "d2h_bytes_per_step": 16384}
     assert line["config"]["step_us_best"] == 86.0 and line["config"]["workload"] == bench.workload_name(1 << 20)
-    assert "cpu_baseline" not in bench.native_line(cfg, 2, 20, 5, 88.19, 86.0, 88.0, 28.78, stage, 2056, 278.2,
-                                                   {}, (100.91, 20480, 16384), clk, None, (6650.0, "fallback"))
+    other = bench.native_line(cfg, 2, 20, 5, 88.19, 86.0, 88.0, 28.78, stage, 2056, 278.2,
+                              {}, (100.91, 20480, 16384), clk, None, (6650.0, "fallback"), 21.5)
+    assert "cpu_baseline" not in other and other["roofline"]["peak_kind"] == "fallback"
+    short = dataclasses.replace(cfg, lengths=[1 << 18])   # the ncu traffic figure is of the 2^20 launch only
+    assert bench.native_line(short, 1, 20, 5, 60.0, 58.0, 60.0, 10.0, stage, 520, 159.0, {},
+                             (70.0, 20480, 16384), clk, None, (6528.7, "measured"), 15.0)["roofline"]["traffic"] is None
 
 
 def test_oracle_leg_on_the_host_cores():
