@@ -103,6 +103,37 @@ EKV_DEV void tab_fill(const AttnArgs& a, int b, int g, Range r, int P)
     __syncthreads();
 }
 
+// tab_fill for a split whose first list entries were loaded ahead (thread t
+// holds entry rs.start + t and its page-table entry, or -1): used where the
+// split is the one they were loaded for, with the same checks as resolve_g.
+EKV_DEV void tab_fill_ahead(const AttnArgs& a, int b, int g, Range r, int P, Range rs, int ahead_lp,
+                            int ahead_phys)
+{
+    const int n = r.end > r.start ? r.end - r.start : 0;
+    if (threadIdx.x == 0) {
+        tab_base = r.start;
+        tab_n = n <= kTabCap ? n : 0;
+    }
+    const bool same = a.sel != nullptr && r.start == rs.start && r.end == rs.end;
+    if (n <= kTabCap)
+        for (int i = threadIdx.x; i < n; i += blockDim.x) {
+            int lp, ph;
+            if (same && i == (int)threadIdx.x) {
+                lp = ahead_lp;
+                ph = ahead_phys;
+                if (lp < 0 || lp >= P || ph < 0 || ph >= a.num_phys) {
+                    report(a.status, ENTMAXKV_DEVICE_BOUNDS);
+                    ph = -1;
+                }
+            } else {
+                ph = resolve_g(a, b, g, r.start + i, P, lp, true);
+            }
+            tab_phys[i] = ph;
+            tab_lp[i] = lp;
+        }
+    __syncthreads();
+}
+
 EKV_DEV int resolve(const AttnArgs& a, int b, int g, int idx, int P, int& lp, bool rep)
 {
     const int j = idx - tab_base;
@@ -1643,7 +1674,15 @@ __global__ void __launch_bounds__(kThreads, 2) entmax_bf16_kernel(const __grid_c
 
     const int b = blockIdx.z, g = blockIdx.y, s = blockIdx.x;   // s = rank in the cluster
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    // A full list (every top-k list once the sequence has k_max pages) fixes
+    // this split's range before its count arrives: its first entries and their
+    // page-table entries load together with the length and the count.
+    const Range rs = split_range(a.k_max, a.S, s);
+    const bool ahead = a.sel != nullptr && tid < rs.end - rs.start;
     const int L = a.seq_lens[b];
+    const int ahead_lp = ahead ? a.sel[((size_t)b * a.H_kv + g) * a.k_max + rs.start + tid] : -1;
+    const int ahead_phys =
+        ahead_lp >= 0 && ahead_lp < a.max_pages ? a.page_table[(size_t)b * a.max_pages + ahead_lp] : -1;
     const int P = pages_of(L, PS, a.max_pages, a.status);
     const int cnt = list_count(a, b, g, P);
     const Range r = split_range(cnt, a.S, s);
@@ -1660,7 +1699,7 @@ __global__ void __launch_bounds__(kThreads, 2) entmax_bf16_kernel(const __grid_c
     // queueing behind the first key tiles
     uint32_t bq[NT][KS][2];
     load_q_frags<D, NT>(a, b, g, a.xscale, bq);
-    tab_fill(a, b, g, r, P);
+    tab_fill_ahead(a, b, g, r, P, rs, ahead_lp, ahead_phys);
 
     // ------------------------------------------------------------ K pass
     if (tid == 0) {
