@@ -2105,6 +2105,41 @@ __global__ void __launch_bounds__(kThreads, 2) entmax_bf16_kernel(const __grid_c
         __syncthreads();   // act and nact are rebuilt by the next window
     }
     if (tid == 0 && a.vpages) atomicAdd(&a.vpages[(size_t)b * a.H_kv + g], loaded);
+    const int E = a.G * D;
+    const int per = (E + a.S - 1) / a.S;     // output elements [s per, (s + 1) per) are added by CTA s
+    if (balanced) {
+        // Every CTA stores its partial of each output element straight into the
+        // shared memory of the element's owner, received as rb[split][element -
+        // owner's first] in the chunk maxima (unused on this path after the
+        // bounds); one cluster barrier, then each owner adds its elements'
+        // partials locally in split order.  Nothing reads another CTA's shared
+        // memory after that barrier, so no CTA waits for the others to leave.
+        static_assert(4 * NT * (kFusedMaxSplitTokens / 16) >= 4 * NT * D + kFusedMaxSplits,
+                      "the received partials fit the chunk-maximum array");
+        float* rb = &cm_s[0][0];
+        const int c = lane & 3, gi = lane >> 2;
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+            const int head = 4 * nt + c;
+            if (head >= a.G) continue;
+#pragma unroll
+            for (int m = 0; m < MTW; ++m) {
+                const int e0 = head * D + 16 * (warp * MTW + m) + gi, e1 = e0 + 8;
+                const int o0 = e0 / per, o1 = e1 / per;
+                st_dsmem_f32(dsmem(rb + s * per + (e0 - o0 * per), o0), acc[nt][m][0] + acc[nt][m][1]);
+                st_dsmem_f32(dsmem(rb + s * per + (e1 - o1 * per), o1), acc[nt][m][2] + acc[nt][m][3]);
+            }
+        }
+        cluster_sync();   // every split's partials have landed at their owners
+        for (int e = s * per + tid; e < min(E, (s + 1) * per); e += kThreads) {
+            const int j = e - s * per;
+            float sum = 0.f;                     // in CTA order, as the loads below
+            for (int q = 0; q < a.S; ++q) sum += rb[q * per + j];
+            if (a.S < kFusedMaxSplits) sum += 0.f;   // the absent splits' +0 (turns a -0 sum into +0)
+            a.out[(row0h + e / D) * D + e % D] = sum;
+        }
+        return;
+    }
     // partial output of this CTA into shared memory (every copy has landed or
     // been waited out above): part[head 4nt + c][d]
     __syncthreads();
@@ -2126,8 +2161,6 @@ __global__ void __launch_bounds__(kThreads, 2) entmax_bf16_kernel(const __grid_c
     cluster_sync();
 
     // ------------------------------------------------------------ merge
-    const int E = a.G * D;
-    const int per = (E + a.S - 1) / a.S;
     for (int e = s * per + tid; e < min(E, (s + 1) * per); e += kThreads) {
         const int head = e / D, dd = e % D;
         float v[kFusedMaxSplits];            // every read goes out before the first add

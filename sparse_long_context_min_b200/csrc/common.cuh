@@ -329,6 +329,10 @@ EKV_DEV uint32_t dsmem(const void* p, uint32_t rank)
     asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(smem_addr(p)), "r"(rank));
     return r;
 }
+EKV_DEV void st_dsmem_f32(uint32_t a, float v)
+{
+    asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(a), "f"(v) : "memory");
+}
 EKV_DEV float ld_dsmem_f32(uint32_t a)
 {
     float v;
