@@ -1664,6 +1664,10 @@ __global__ void __launch_bounds__(kThreads, 2) entmax_bf16_kernel(const __grid_c
     // the other CTAs through distributed shared memory)
     __shared__ float pub_t[8], pub_m[8];
     __shared__ int pub_n[8];
+    // every split's bound, largest score and candidate count per head, as the
+    // splits stored them into this CTA before the barriers (read locally)
+    __shared__ float all_t[kFusedMaxSplits][8], all_m[kFusedMaxSplits][8];
+    __shared__ int all_n[kFusedMaxSplits][8];
     // the largest score of every 16-token chunk of this split, per head
     __shared__ float cm_s[4 * NT][kFusedMaxSplitTokens / 16];
     // the cluster-wide threshold solve: partial sums per iteration parity and head
@@ -1808,13 +1812,18 @@ __global__ void __launch_bounds__(kThreads, 2) entmax_bf16_kernel(const __grid_c
         }
     }
     __syncthreads();
+    if (tid < a.S * 8) {   // this split's bound and largest score per head into every CTA
+        const int q = tid >> 3, h = tid & 7;
+        st_dsmem_f32(dsmem(&all_t[s][h], q), pub_t[h]);
+        st_dsmem_f32(dsmem(&all_m[s][h], q), pub_m[h]);
+    }
     cluster_sync();
     if (!abort_flag) {
         for (int h = warp, k = 0; h < a.G; h += 4, ++k) {
             const size_t row = row0h + h;
             int* lc = reinterpret_cast<int*>(smem + warp * WSCR + k * LC_CAP * 8);
             float* lcv = reinterpret_cast<float*>(smem + warp * WSCR + k * LC_CAP * 8 + LC_CAP * 4);
-            float tlb = lane < a.S ? ld_dsmem_f32(dsmem(&pub_t[h], lane)) : -INFINITY;
+            float tlb = lane < a.S ? all_t[lane][h] : -INFINITY;
             tlb = warp_max(tlb);
             const int n = local_candidates(a.xbuf + row * xstride, c0, c1, lc, lcv, nlc_s[h], LC_CAP, tlb,
                                            a.cval + row * seg + (size_t)s * kCandCap,
@@ -1824,6 +1833,8 @@ __global__ void __launch_bounds__(kThreads, 2) entmax_bf16_kernel(const __grid_c
     }
     __threadfence();   // candidates and scores in global memory are read by the other splits
     __syncthreads();
+    if (tid < a.S * 8)     // this split's candidate count per head into every CTA
+        st_dsmem_s32(dsmem(&all_n[s][tid & 7], tid >> 3), pub_n[tid & 7]);
     cluster_sync();
 
     // ------------------------------------------------------------ threshold
@@ -1837,7 +1848,7 @@ __global__ void __launch_bounds__(kThreads, 2) entmax_bf16_kernel(const __grid_c
     if (tid < 32) {
         int nh[8];                                            // every read goes out before the first use
 #pragma unroll
-        for (int h = 0; h < 8; ++h) nh[h] = h < a.G && lane < a.S ? ld_dsmem_s32(dsmem(&pub_n[h], lane)) : 0;
+        for (int h = 0; h < 8; ++h) nh[h] = h < a.G && lane < a.S ? all_n[lane][h] : 0;
         bool o = false;
 #pragma unroll
         for (int h = 0; h < 8; ++h) {
@@ -1863,9 +1874,9 @@ __global__ void __launch_bounds__(kThreads, 2) entmax_bf16_kernel(const __grid_c
             float M = -INFINITY, tlb = -INFINITY;
             int nq = 0;
             if (lane < a.S) {
-                M = ld_dsmem_f32(dsmem(&pub_m[h], lane));
-                tlb = ld_dsmem_f32(dsmem(&pub_t[h], lane));
-                nq = ld_dsmem_s32(dsmem(&pub_n[h], lane));
+                M = all_m[lane][h];
+                tlb = all_t[lane][h];
+                nq = all_n[lane][h];
             }
             M = warp_max(M);
             tlb = warp_max(tlb);

@@ -333,6 +333,10 @@ EKV_DEV void st_dsmem_f32(uint32_t a, float v)
 {
     asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(a), "f"(v) : "memory");
 }
+EKV_DEV void st_dsmem_s32(uint32_t a, int v)
+{
+    asm volatile("st.shared::cluster.s32 [%0], %1;" ::"r"(a), "r"(v) : "memory");
+}
 EKV_DEV float ld_dsmem_f32(uint32_t a)
 {
     float v;
